@@ -1,0 +1,198 @@
+"""Pins of the oracle's NABLA selection, AR composition and attention (CPU only)."""
+import itertools
+import math
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+import oracle as O
+from tests._golden import load
+
+
+# ----------------------------------------------------------------- pooling
+
+def test_pool_mean_over_valid_tokens_only():
+    x = np.zeros((1, 8, 1, 2))
+    x[0, :, 0, 0] = np.arange(8)
+    x[0, :, 0, 1] = 1.0
+    # n_valid = 6: block 0 = tokens 0..3, block 1 = tokens 4, 5 (6, 7 are padding)
+    x[0, 6:] = 123.0
+    out = O.nabla_pool(x, 4, 6)
+    assert np.allclose(out[0, 0, 0], [1.5, 1.0])
+    assert np.allclose(out[0, 0, 1], [4.5, 1.0])
+
+
+# ----------------------------------------------------------------- top-p selection
+
+def _brute_min_cardinality(probs, p):
+    n = len(probs)
+    for k in range(1, n + 1):
+        best = max(sum(probs[list(c)]) for c in itertools.combinations(range(n), k))
+        if best >= p:
+            return k
+    return n
+
+
+@pytest.mark.parametrize("seed", range(6))
+@pytest.mark.parametrize("p", [0.3, 0.7, 0.9, 0.97])
+def test_select_is_minimal_and_covers_p_brute_force(seed, p):
+    rng = np.random.default_rng(seed)
+    n = 9
+    z = rng.normal(0, 1.5, n)
+    probs = scipy.special.softmax(z)
+    kept, cum, k_star, _ = O.nabla_select_row(probs, p)
+    assert len(kept) == k_star == _brute_min_cardinality(probs, p)
+    assert probs[kept].sum() >= p                       # coverage
+    top = np.sort(probs)[::-1]
+    assert top[:k_star - 1].sum() < p                   # minimality
+    # the kept set is a top set: nothing dropped is larger than anything kept
+    dropped = np.setdiff1d(np.arange(n), kept)
+    if dropped.size:
+        assert probs[dropped].max() <= probs[kept].min()
+
+
+def test_select_uniform_keeps_ceil_p_lowest_indices():
+    kb = 40
+    probs = np.full(kb, 1.0 / kb)
+    for p in (0.1, 0.5, 0.9, 0.925):
+        kept, _, k_star, _ = O.nabla_select_row(probs, p)
+        expect = math.ceil(round(p * kb, 9))
+        assert k_star == expect
+        assert sorted(kept.tolist()) == list(range(expect))
+
+
+def test_select_small_p_is_argmax_and_p_one_keeps_all():
+    probs = scipy.special.softmax(np.array([0.1, 2.0, -1.0, 1.9]))
+    kept, _, _, _ = O.nabla_select_row(probs, 1e-9)
+    assert kept.tolist() == [1]
+    kept, _, k_star, _ = O.nabla_select_row(probs, 1.0)
+    assert k_star == 4
+
+
+def test_nabla_mask_dominant_block_and_constant_queries():
+    rng = np.random.default_rng(7)
+    Bn, H, QB, KB, D = 1, 2, 3, 16, 8
+    qbar = np.zeros((Bn, H, QB, D))
+    qbar[..., 0] = 10.0
+    qbar[..., 1:] = rng.normal(size=(Bn, H, QB, D - 1)) * 0.01
+    kbar = rng.normal(size=(Bn, H, KB, D)) * 0.01
+    # head 0: key block 5 has logit 10 * 5 * sqrt(D) / sqrt(D) = +50 against every query
+    kbar[0, 0, 5] = 0.0
+    kbar[0, 0, 5, 0] = 5.0 * math.sqrt(D)
+    mask, near = O.nabla_mask(qbar, kbar, 0.9, 1.0 / math.sqrt(D))
+    for qb in range(QB):
+        assert mask[0, 0, qb].tolist() == [1 if c == 5 else 0 for c in range(KB)]
+    # head 1: identical pooled keys -> uniform -> ceil(0.9 * 16) = 15 lowest blocks
+    kbar[0, 1] = 0.3
+    mask, near = O.nabla_mask(qbar, kbar, 0.9, 1.0 / math.sqrt(D))
+    assert np.all(mask[0, 1, :, :15] == 1) and np.all(mask[0, 1, :, 15] == 0)
+
+
+def test_nabla_mask_range_and_forced_outside():
+    rng = np.random.default_rng(9)
+    qbar = rng.normal(size=(1, 1, 4, 8))
+    kbar = rng.normal(size=(1, 1, 20, 8))
+    mask, _ = O.nabla_mask(qbar, kbar, 0.8, 0.35, kb_begin=3, kb_end=15, force_outside=1)
+    assert np.all(mask[..., :3] == 1) and np.all(mask[..., 15:] == 1)
+    # middle range: softmax renormalised over blocks 3..14 only
+    z = (qbar[0, 0] @ kbar[0, 0, 3:15].T) * 0.35
+    probs = scipy.special.softmax(z, axis=1)
+    for qb in range(4):
+        kept = np.nonzero(mask[0, 0, qb, 3:15])[0]
+        assert probs[qb, kept].sum() >= 0.8
+        assert np.sort(probs[qb])[::-1][:len(kept) - 1].sum() < 0.8
+
+
+def test_ar_ranges_match_the_decode_workload():
+    # 60 frames of 30x52 = 1560 tokens, 64-token blocks, 3 anchor frames, last 6 dense
+    a_end, r_begin = O.ar_block_ranges(60 * 1560, 1560, 64, 3, 6)
+    kb = math.ceil(60 * 1560 / 64)
+    assert kb == 1463
+    assert a_end == 74                   # blocks touching tokens [0, 4680)
+    assert kb - r_begin == 147           # blocks touching tokens [84240, 93600)
+
+
+def test_near_threshold_flag():
+    probs_z = np.log(np.array([0.5, 0.4, 0.1]))
+    qbar = np.zeros((1, 1, 1, 1))
+    kbar = np.zeros((1, 1, 3, 1))
+    # z = qbar.kbar * scale: encode the logits in kbar with qbar = 1
+    qbar[...] = 1.0
+    kbar[0, 0, :, 0] = probs_z
+    _, near = O.nabla_mask(qbar, kbar, 0.9, 1.0)       # 0.5 + 0.4 == 0.9 exactly
+    assert near[0, 0, 0]
+    _, near = O.nabla_mask(qbar, kbar, 0.8, 1.0)
+    assert not near[0, 0, 0]
+
+
+# ----------------------------------------------------------------- attention
+
+def test_attention_golden_two_keys():
+    q, k0, k1, v0, v1, o, lse = load("attention_two_keys.txt")[0]
+    out, l = O.dense_masked_attention(np.array([[q]]), np.array([[k0], [k1]]),
+                                      np.array([[v0], [v1]]), np.ones((1, 2), bool), 1.0)
+    assert abs(out[0, 0] - o) < 1e-12 and abs(l[0] - lse) < 1e-12
+
+
+def _rand_qkv(Bn, nq, nk, H, D, seed):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((Bn, nq, H, D)), rng.standard_normal((Bn, nk, H, D)),
+            rng.standard_normal((Bn, nk, H, D)))
+
+
+def test_all_ones_mask_equals_sdpa_float64():
+    q, k, v = _rand_qkv(2, 130, 200, 3, 16, 1)
+    mask = np.ones((1, math.ceil(130 / 64), math.ceil(200 / 64)), np.uint8)
+    o, lse = O.block_sparse_attention(q, k, v, mask, 64, 64)
+    tq, tk, tv = (torch.from_numpy(a).permute(0, 2, 1, 3) for a in (q, k, v))
+    ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv).permute(0, 2, 1, 3).numpy()
+    assert np.max(np.abs(o - ref)) < 1e-12
+    s = np.einsum("bihd,bjhd->bhij", q, k) / 4.0
+    assert np.max(np.abs(lse - scipy.special.logsumexp(s, axis=-1))) < 1e-12
+
+
+@pytest.mark.parametrize("bq,bk", [(64, 64), (128, 64), (64, 128), (384, 384)])
+def test_block_mask_equals_token_level_definition(bq, bk):
+    Bn, H, D = 1, 2, 8
+    nq, nk = 3 * bq - 17, 4 * bk - 5                    # ragged last blocks
+    q, k, v = _rand_qkv(Bn, nq, nk, H, D, 2)
+    QB, KB = math.ceil(nq / bq), math.ceil(nk / bk)
+    rng = np.random.default_rng(4)
+    mask = (rng.random((Bn * H, QB, KB)) < 0.5).astype(np.uint8)
+    mask[1, 1] = 0                                      # an empty row
+    o, lse = O.block_sparse_attention(q, k, v, mask, bq, bk)
+    for h in range(H):
+        allowed = O.token_mask_from_blocks(mask[h], nq, nk, bq, bk)
+        ro, rl = O.dense_masked_attention(q[0, :, h], k[0, :, h], v[0, :, h], allowed,
+                                          1 / math.sqrt(D))
+        assert np.allclose(o[0, :, h], ro, atol=1e-12, rtol=0)
+        assert np.array_equal(np.isneginf(lse[0, h]), np.isneginf(rl))
+        fin = np.isfinite(rl)
+        assert np.allclose(lse[0, h][fin], rl[fin], atol=1e-12)
+    rows = np.arange(bq, 2 * bq)
+    assert np.all(o[0, rows, 1] == 0) and np.all(np.isneginf(lse[0, 1, rows]))
+
+
+def test_single_kept_block_is_softmax_over_that_block_and_lse_normalises():
+    Bn, H, D, blk = 1, 1, 16, 64
+    q, k, v = _rand_qkv(Bn, 128, 256, H, D, 5)
+    mask = np.zeros((1, 2, 4), np.uint8)
+    mask[0, 0, 2] = 1
+    mask[0, 1, 3] = 1
+    o, lse = O.block_sparse_attention(q, k, v, mask, blk, blk)
+    s = q[0, :64, 0] @ k[0, 128:192, 0].T / 4.0
+    w = scipy.special.softmax(s, axis=1)
+    assert np.allclose(o[0, :64, 0], w @ v[0, 128:192, 0], atol=1e-12)
+    assert np.allclose(np.exp(s - lse[0, 0, :64, None]).sum(axis=1), 1.0, atol=1e-12)
+
+
+def test_sampled_rows_match_full_evaluation():
+    q, k, v = _rand_qkv(1, 300, 300, 2, 8, 6)
+    mask = (np.random.default_rng(1).random((1, 5, 5)) < 0.6).astype(np.uint8)
+    o, lse = O.block_sparse_attention(q, k, v, mask, 64, 64)
+    rows = np.array([0, 63, 64, 200, 299])
+    o2, lse2 = O.block_sparse_attention(q, k, v, mask, 64, 64, rows=rows)
+    assert np.allclose(o[:, rows], o2[:, rows], atol=1e-13, rtol=0)
+    assert np.allclose(lse[..., rows], lse2[..., rows], atol=1e-13, rtol=0)
