@@ -1,0 +1,360 @@
+#!/usr/bin/env python3
+"""Benchmark of the block-sparse video attention path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step = one pass of the whole path over one batch of synthetic input already
+resident in HBM: tile permute of Q, K, V -> block mask -> CSR compaction ->
+block-sparse attention forward -> inverse permute of O.  The default workload is
+the Sliding-Tile 720p DiT shape (1 x 24 heads x 128, 30x48x80 tokens, 6x8x8
+tiles of 384 tokens, 3x3x5-tile window).  Metric: effective TFLOP/s =
+4 * head_dim * (query, key) pairs inside kept blocks / time.
+
+Under torchrun (N > 1) every rank runs its own batch of the same shape (the path
+shards by batch/head with no collective): weak scaling, value = all ranks' work
+divided by the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def attn_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("attn_fwd.cu", "bsa_common.cuh", "tmem_io.cuh"):
+        with open(os.path.join(ROOT, "block_sparse_attention_tokens_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per attention launch from the committed ncu summary, if that
+    summary was taken on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", f"attn_fwd_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    s = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
+    if not m or not s or s.group(1) != attn_source_hash():
+        return None
+    return float(m.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.samples = []
+        if self.proc is None:
+            return
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.samples.append(parts)
+
+    def summary(self):
+        if not getattr(self, "samples", None):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        mx = [float(s[2]) for s in self.samples if s[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for s in self.samples:
+            for n, val in zip(names, s[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(self.samples)}
+
+
+def cpu_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def oracle_sample_rate(w, q, k, v, budget_s: float):
+    """Times the CPU oracle on whole query blocks of the workload (all heads),
+    adding blocks until ~budget_s of work; returns (effective TFLOP/s, sample text)."""
+    import numpy as np
+    import oracle as O
+
+    D = w.head_dim
+    if w.tile is not None:
+        perm = O.tile_order(w.grid, w.tile)
+        n_pad = math.ceil(w.n_tokens / w.block) * w.block
+        tg = tuple(math.ceil(g / t) for g, t in zip(w.grid, w.tile))
+    rng = np.random.default_rng(7)
+    QB = math.ceil(w.nq / w.block)
+    order = rng.permutation(QB)
+    t0 = time.perf_counter()
+    if w.mask == "sta":
+        mask = O.sta_tile_mask(tg, w.window)[None]
+    elif w.mask == "radial":
+        mask = O.radial_block_mask_fast(w.nk, w.tokens_per_frame, w.block)[None]
+    else:
+        raise ValueError("cpu baseline implemented for static-mask workloads")
+    heads64 = []
+    for h in range(w.heads):
+        qh = q[:, :, h:h + 1].double().numpy()
+        kh = k[:, :, h:h + 1].double().numpy()
+        vh = v[:, :, h:h + 1].double().numpy()
+        if w.tile is not None:
+            qh = O.tile_permute(qh, perm, n_pad)[:, :w.nq]
+            kh = O.tile_permute(kh, perm, n_pad)[:, :w.nk]
+            vh = O.tile_permute(vh, perm, n_pad)[:, :w.nk]
+        heads64.append((qh, kh, vh))
+    prep = time.perf_counter() - t0
+    flops = 0.0
+    done = 0
+    t1 = time.perf_counter()
+    for qb in order:
+        rows = np.arange(qb * w.block, min((qb + 1) * w.block, w.nq))
+        for qh, kh, vh in heads64:
+            O.block_sparse_attention(qh, kh, vh, mask, w.block, w.block, rows=rows)
+        kept = np.nonzero(mask[0, qb])[0]
+        nkeys = sum(min((kb + 1) * w.block, w.nk) - kb * w.block for kb in kept)
+        flops += 4.0 * D * len(rows) * nkeys * w.heads
+        done += 1
+        if time.perf_counter() - t1 > budget_s:
+            break
+    el = time.perf_counter() - t1
+    sample = (f"{done} random query blocks x {w.heads} heads of {w.name} "
+              f"({flops / 1e12:.4f} effective TFLOP), float64 oracle, {el:.1f} s "
+              f"(+{prep:.1f} s mask/permute/upcast setup, untimed)")
+    return flops / el / 1e12, sample
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from block_sparse_attention_tokens_b200 import synth
+    q, k, v, _ = synth.workload_inputs(w)
+    budget = max(2.0, min(20.0, 60.0 / max(1, args.steps + args.warmup)))
+    vals = []
+    sample = ""
+    for i in range(args.warmup + args.steps):
+        val, sample = oracle_sample_rate(w, q, k, v, budget)
+        if i >= args.warmup:
+            vals.append(val)
+    value = statistics.median(vals)
+    line = {"impl": "reference", "metric": "block-sparse attention effective TFLOP/s (path step)",
+            "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": True, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(w),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_cores(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+def workload_config(w):
+    cfg = {"workload": w.name, "batch": w.batch, "heads": w.heads, "head_dim": w.head_dim,
+           "grid_thw": list(w.grid), "block": w.block, "mask": w.mask}
+    if w.tile:
+        cfg["tile"] = list(w.tile)
+    if w.window:
+        cfg["window_tiles"] = list(w.window)
+    if w.p is not None:
+        cfg["p"] = w.p
+    cfg["l2"] = "inputs larger than L2 (no flush between steps)"
+    return cfg
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="sta_720p")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0,
+                    help="seconds of oracle work for the cpu_baseline field")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+
+    from block_sparse_attention_tokens_b200 import configs
+    w = configs.get(args.workload)
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import torch
+    import torch.distributed as dist
+    from block_sparse_attention_tokens_b200 import binding as B
+    from block_sparse_attention_tokens_b200 import synth
+    from block_sparse_attention_tokens_b200.pipeline import Plan, effective_flops
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    # inputs (the same seeded batch on every rank: each rank owns one batch of work)
+    q_h, k_h, v_h, _ = synth.workload_inputs(w)
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    plan = Plan(w, dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(max(3, args.warmup)):
+        plan.step(q, k, v)
+    barrier()
+    flops = effective_flops(plan.mask, plan.nq, plan.nk, w.block, w.head_dim,
+                            w.batch * w.heads)
+    if B.bsa_read_status(plan.attn_ws) != 0:
+        raise RuntimeError("attention kernel reported a device-side error")
+
+    # ---- timed region: K whole-path steps, attention launches bracketed by events
+    stream = torch.cuda.current_stream()
+    ev_a = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index)
+    barrier()
+    with sampler:
+        start.record(stream)
+        for i in range(args.steps):
+            plan._q, plan._k, plan._v = q, k, v
+            if plan.permuted:
+                plan.permute_inputs(q, k, v)
+            plan.build_mask()
+            plan.compact()
+            ev_a[i][0].record(stream)
+            plan.attention()
+            ev_a[i][1].record(stream)
+            if plan.permuted:
+                plan.untile()
+        end.record(stream)
+        barrier()
+    ms_total = start.elapsed_time(end)
+    attn_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_a)
+    t = torch.tensor([ms_total, attn_ms], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_total, attn_ms = t.tolist()
+    ms_per_step = ms_total / args.steps
+    value = flops * world / (ms_per_step * 1e-3) / 1e12
+
+    # ---- end to end through the public API: pinned host inputs in, O back to host
+    e2e = None
+    if not args.no_e2e:
+        qp, kp, vp = (t_.pin_memory() for t_ in (q_h, k_h, v_h))
+        o_host = torch.empty(plan.o.shape, dtype=plan.o.dtype).pin_memory()
+        qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        e2e_steps = max(3, args.steps // 2)
+        for it in range(2 + e2e_steps):
+            if it == 2:
+                barrier()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+            qd.copy_(qp, non_blocking=True)
+            kd.copy_(kp, non_blocking=True)
+            vd.copy_(vp, non_blocking=True)
+            o, _ = plan.step(qd, kd, vd)
+            o_host.copy_(o, non_blocking=True)
+        e1.record(stream)
+        barrier()
+        e_ms = torch.tensor([e0.elapsed_time(e1) / e2e_steps], device=dev, dtype=torch.float64)
+        if world > 1:
+            dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
+        h2d = sum(t_.numel() * t_.element_size() for t_ in (q_h, k_h, v_h))
+        d2h = o_host.numel() * o_host.element_size()
+        e2e = {"value": flops * world / (e_ms.item() * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": e_ms.item(), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    peaks, peak_kind = load_peaks()
+    achieved = flops / (attn_ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    traffic = profiled_traffic(w.name)
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": traffic,
+                "kernel": "attn_fwd_kernel<128>", "attn_ms": attn_ms,
+                "peak_note": f"{peak_kind} sustained bf16 (kernel timed inside back-to-back steps)",
+                "frac_of_burst": achieved / peaks["bf16_tflops"]}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        val, sample = oracle_sample_rate(w, q_h, k_h, v_h, args.cpu_budget)
+        cpu = {"value": val, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+               "sample": sample}
+
+    if rank == 0:
+        line = {"metric": "block-sparse attention effective TFLOP/s (path step)",
+                "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+                "warmup": max(3, args.warmup), "ms_per_step": ms_per_step,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic", "config": workload_config(w),
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "clocks": sampler.summary(),
+                "gpu_launches": plan.kernel_launches_per_step() * args.steps,
+                "effective_tflop_per_step": flops / 1e12}
+        print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,244 @@
+"""Thin Python binding of libbsa.so (argument marshalling only).
+
+Every function here has the name of the C entry point it wraps (see
+``include/bsa.h``), takes torch tensors where the C ABI takes device pointers,
+passes the current torch CUDA stream, and raises ``BsaError`` on a non-OK
+status.  All arithmetic happens in the library's CUDA kernels; when the shared
+library is missing the import fails loudly -- there is no other code path.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libbsa.so")
+
+STATUS = {0: "BSA_OK", 1: "BSA_ERR_INVALID_ARG", 2: "BSA_ERR_UNSUPPORTED", 3: "BSA_ERR_WORKSPACE",
+          4: "BSA_ERR_CUDA", 5: "BSA_ERR_TIMEOUT"}
+
+EXPORTS = [
+    "bsa_status_string", "bsa_last_error_message", "bsa_version", "bsa_tile_permute",
+    "bsa_tile_untile", "bsa_sta_mask", "bsa_radial_mask", "bsa_nabla_workspace_size",
+    "bsa_nabla_mask", "bsa_mask_compact", "bsa_attn_workspace_size", "bsa_attn_fwd",
+    "bsa_read_status",
+]
+
+
+class BsaError(RuntimeError):
+    def __init__(self, code: int, where: str, detail: str = ""):
+        self.code = code
+        super().__init__(f"{where}: {STATUS.get(code, code)}" + (f" ({detail})" if detail else ""))
+
+
+_lib = None
+
+
+def load_library(path: str = _LIB_PATH) -> ctypes.CDLL:
+    """Loads libbsa.so once.  Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"libbsa.so not found at {path}; build it with "
+                          f"`python -m block_sparse_attention_tokens_b200.build`")
+    lib = ctypes.CDLL(path)
+    c_int, c_void, c_size, c_float = ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_float
+    sig = {
+        "bsa_status_string": (ctypes.c_char_p, [c_int]),
+        "bsa_last_error_message": (ctypes.c_char_p, []),
+        "bsa_version": (c_int, []),
+        "bsa_tile_permute": (c_int, [c_void, c_void] + [c_int] * 9 + [c_void]),
+        "bsa_tile_untile": (c_int, [c_void, c_void] + [c_int] * 9 + [c_void]),
+        "bsa_sta_mask": (c_int, [c_int] * 7 + [c_void, c_void]),
+        "bsa_radial_mask": (c_int, [c_int] * 3 + [c_void, c_void]),
+        "bsa_nabla_workspace_size": (c_size, [c_int] * 6),
+        "bsa_nabla_mask": (c_int, [c_void, c_void] + [c_int] * 6 + [c_float, c_float] + [c_int] * 3
+                           + [c_void, c_void, c_void, c_size, c_void]),
+        "bsa_mask_compact": (c_int, [c_void, c_int, c_int, c_void, c_void, c_void]),
+        "bsa_attn_workspace_size": (c_size, [c_int] * 7),
+        "bsa_attn_fwd": (c_int, [c_void, c_void, c_void] + [c_int] * 7 + [c_void, c_void, c_int,
+                                                                           c_float, c_void, c_void,
+                                                                           c_void, c_size, c_void]),
+        "bsa_read_status": (c_int, [c_void, ctypes.POINTER(c_int), c_void]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _check(code: int, where: str):
+    if code != 0:
+        detail = load_library().bsa_last_error_message().decode() if code == 4 else ""
+        raise BsaError(code, where, detail)
+
+
+def _cuda(t: torch.Tensor, name: str):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+# --------------------------------------------------------------------------- (a)
+
+def bsa_tile_permute(x: torch.Tensor, grid: Tuple[int, int, int], tile: Tuple[int, int, int],
+                     n_pad: int, y: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """x [B, N, ...] raster order -> y [B, n_pad, ...] tile order with a zero tail."""
+    _cuda(x, "x")
+    B, N = x.shape[0], x.shape[1]
+    row_bytes = x[0, 0].numel() * x.element_size()
+    if y is None:
+        y = torch.empty((B, n_pad) + tuple(x.shape[2:]), dtype=x.dtype, device=x.device)
+    _check(load_library().bsa_tile_permute(_ptr(x), _ptr(y), B, *grid, *tile, row_bytes, n_pad,
+                                           _stream()), "bsa_tile_permute")
+    return y
+
+
+def bsa_tile_untile(y: torch.Tensor, grid: Tuple[int, int, int], tile: Tuple[int, int, int],
+                    x: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """y [B, n_pad, ...] tile order -> x [B, N, ...] raster order."""
+    _cuda(y, "y")
+    B, n_pad = y.shape[0], y.shape[1]
+    N = grid[0] * grid[1] * grid[2]
+    row_bytes = y[0, 0].numel() * y.element_size()
+    if x is None:
+        x = torch.empty((B, N) + tuple(y.shape[2:]), dtype=y.dtype, device=y.device)
+    _check(load_library().bsa_tile_untile(_ptr(y), _ptr(x), B, *grid, *tile, row_bytes, n_pad,
+                                          _stream()), "bsa_tile_untile")
+    return x
+
+
+# --------------------------------------------------------------------------- (b)
+
+def bsa_sta_mask(tile_grid: Tuple[int, int, int], window: Tuple[int, int, int], shift: int = 0,
+                 mask: Optional[torch.Tensor] = None, device="cuda") -> torch.Tensor:
+    n = tile_grid[0] * tile_grid[1] * tile_grid[2]
+    if mask is None:
+        mask = torch.empty((n, n), dtype=torch.uint8, device=device)
+    _check(load_library().bsa_sta_mask(*tile_grid, *window, int(shift), _ptr(mask), _stream()),
+           "bsa_sta_mask")
+    return mask
+
+
+def bsa_radial_mask(n_tokens: int, tokens_per_frame: int, block: int,
+                    mask: Optional[torch.Tensor] = None, device="cuda") -> torch.Tensor:
+    nb = -(-n_tokens // block)
+    if mask is None:
+        mask = torch.empty((nb, nb), dtype=torch.uint8, device=device)
+    _check(load_library().bsa_radial_mask(n_tokens, tokens_per_frame, block, _ptr(mask),
+                                          _stream()), "bsa_radial_mask")
+    return mask
+
+
+def bsa_nabla_workspace_size(batch, heads, nq, nk, head_dim, block) -> int:
+    return int(load_library().bsa_nabla_workspace_size(batch, heads, nq, nk, head_dim, block))
+
+
+def bsa_nabla_mask(q: torch.Tensor, k: torch.Tensor, block: int, p: float, scale: float = 0.0,
+                   kb_begin: int = 0, kb_end: Optional[int] = None, force_outside: int = 0,
+                   nq: Optional[int] = None, nk: Optional[int] = None,
+                   mask: Optional[torch.Tensor] = None, near_count: Optional[torch.Tensor] = None,
+                   ws: Optional[torch.Tensor] = None):
+    """NABLA block mask [B, H, QB, KB] (uint8) from q, k [B, N, H, D] (bf16).
+
+    nq / nk: number of valid tokens (default: the tensors' lengths).
+    Returns (mask, near_count tensor).
+    """
+    _cuda(q, "q")
+    _cuda(k, "k")
+    B, _, H, D = q.shape
+    nq = q.shape[1] if nq is None else nq
+    nk = k.shape[1] if nk is None else nk
+    QB, KB = -(-nq // block), -(-nk // block)
+    kb_end = KB if kb_end is None else kb_end
+    if mask is None:
+        mask = torch.empty((B, H, QB, KB), dtype=torch.uint8, device=q.device)
+    if near_count is None:
+        near_count = torch.zeros(1, dtype=torch.int32, device=q.device)
+    if ws is None:
+        ws = torch.empty(bsa_nabla_workspace_size(B, H, nq, nk, D, block), dtype=torch.uint8,
+                         device=q.device)
+    _check(load_library().bsa_nabla_mask(_ptr(q), _ptr(k), B, H, nq, nk, D, block, float(p),
+                                         float(scale), kb_begin, kb_end, int(force_outside),
+                                         _ptr(mask), _ptr(near_count), _ptr(ws), ws.numel(),
+                                         _stream()), "bsa_nabla_mask")
+    return mask, near_count
+
+
+# --------------------------------------------------------------------------- (c)
+
+def bsa_mask_compact(mask: torch.Tensor, row_ptr: Optional[torch.Tensor] = None,
+                     col_idx: Optional[torch.Tensor] = None):
+    """uint8 mask [..., KB] (rows = product of leading dims) -> (row_ptr, col_idx) int32."""
+    _cuda(mask, "mask")
+    KB = mask.shape[-1]
+    rows = mask.numel() // KB
+    if row_ptr is None:
+        row_ptr = torch.empty(rows + 1, dtype=torch.int32, device=mask.device)
+    if col_idx is None:
+        col_idx = torch.empty(rows * KB, dtype=torch.int32, device=mask.device)
+    _check(load_library().bsa_mask_compact(_ptr(mask), rows, KB, _ptr(row_ptr), _ptr(col_idx),
+                                           _stream()), "bsa_mask_compact")
+    return row_ptr, col_idx
+
+
+# --------------------------------------------------------------------------- (d)
+
+def bsa_attn_workspace_size(batch, heads, nq, nk, block_q, block_k, list_heads) -> int:
+    return int(load_library().bsa_attn_workspace_size(batch, heads, nq, nk, block_q, block_k,
+                                                      list_heads))
+
+
+def bsa_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, row_ptr: torch.Tensor,
+                 col_idx: torch.Tensor, block_q: int, block_k: int, list_heads: int,
+                 nq: Optional[int] = None, nk: Optional[int] = None, scale: float = 0.0,
+                 o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                 ws: Optional[torch.Tensor] = None):
+    """Block-sparse attention forward.  Returns (o [B, nq_rows, H, D] bf16, lse [B, H, nq])."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (row_ptr, "row_ptr"), (col_idx, "col_idx")):
+        _cuda(t, n)
+    B, _, H, D = q.shape
+    nq = q.shape[1] if nq is None else nq
+    nk = k.shape[1] if nk is None else nk
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, nq), dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = torch.empty(bsa_attn_workspace_size(B, H, nq, nk, block_q, block_k, list_heads),
+                         dtype=torch.uint8, device=q.device)
+    _check(load_library().bsa_attn_fwd(_ptr(q), _ptr(k), _ptr(v), B, H, nq, nk, D, block_q,
+                                       block_k, _ptr(row_ptr), _ptr(col_idx), list_heads,
+                                       float(scale), _ptr(o), _ptr(lse), _ptr(ws), ws.numel(),
+                                       _stream()), "bsa_attn_fwd")
+    return o, lse, ws
+
+
+def bsa_read_status(ws: torch.Tensor) -> int:
+    out = ctypes.c_int(0)
+    _check(load_library().bsa_read_status(_ptr(ws), ctypes.byref(out), _stream()),
+           "bsa_read_status")
+    return out.value
+
+
+def bsa_status_string(code: int) -> str:
+    return load_library().bsa_status_string(code).decode()
+
+
+def bsa_version() -> int:
+    return int(load_library().bsa_version())

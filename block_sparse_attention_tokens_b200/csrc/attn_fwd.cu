@@ -1,0 +1,638 @@
+// Block-sparse attention forward on sm_100a: tcgen05 tensor cores with TMEM
+// accumulators, TMA-fed K/V ring indexed by per-q-tile kept lists.
+//
+// Sources: "Fast Video Generation with Sliding Tile Attention" explainer
+// (aibr.jp/archives/60739), section 3 (attention restricted to kept tiles with a
+// hardware-aware kernel); SPADE summary (gist.science/ja/paper/2608.03335),
+// solution part 3 (head-wise sparse attention); NABLA explainer
+// (aibr.jp/archives/124678), section 3 (block mask applied at block level).
+// The arithmetic is softmax(Q K^T * scale + M) V with M = -inf outside kept
+// block pairs, evaluated with an online (running max / running sum) softmax.
+//
+// Design (one persistent CTA per SM, 320 threads):
+//   warps 0-3  softmax for q-tile slot 0 (thread = query row = TMEM lane)
+//   warps 4-7  softmax for q-tile slot 1
+//   warp  8    TMA producer: Q tiles, K/V tiles into an NSTAGE ring
+//   warp  9    MMA issuer (one thread), also owns the TMEM allocation
+// Each CTA processes "units" of two 128-row q-tiles (slots) in lock-step rounds:
+//   round r:  S_0 = Q_0 K_0r^T, S_1 = Q_1 K_1r^T, O_0 += P_0 V_0r, O_1 += P_1 V_1r
+// so that while one slot's softmax runs on the CUDA cores the tensor core works
+// on the other slot.  TMEM (512 columns): S_0 | S_1 | O_0 | O_1, 128 columns
+// each; P (bf16) is written over the first half of its slot's S columns and is
+// the TMEM A operand of the P.V MMA.  The K/V ring stages are released by
+// tcgen05.commit when the MMA that read them completes.
+// Lazy rescaling: the running max used for the exponentials only moves when a
+// row's new max exceeds it by more than 8 (log2 units), so O in TMEM is rarely
+// touched by the softmax warps.
+// All mbarrier waits are bounded; on expiry BSA_ERR_TIMEOUT is recorded in the
+// workspace status word and every role leaves its loop.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "bsa_common.cuh"
+#include "tmem_io.cuh"
+
+namespace bsa {
+namespace {
+
+constexpr int kBM = 128;          // query rows per tile (= TMEM lanes)
+constexpr int kBN = 128;          // keys per K/V tile
+constexpr int kThreads = 320;
+constexpr int kLoadWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+template <int D>
+struct Cfg {
+  static constexpr int KCH = D / 64;                  // 128-byte swizzle chunks per row
+  static constexpr int CHUNK_BYTES = kBM * 128;       // one chunk of a 128-row tile
+  static constexpr int TILE_BYTES = KCH * CHUNK_BYTES;
+  static constexpr int NSTAGE = D == 128 ? 5 : 10;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_RING = 2 * TILE_BYTES;
+  static constexpr int OFF_BAR = OFF_RING + NSTAGE * TILE_BYTES;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM = OFF_BAR + BAR_BYTES + 1024;  // + alignment slack
+};
+
+struct AttnParams {
+  int B, H, nq, nk, QT;
+  int block_q, block_k, QB, LR, list_heads, expand;
+  int total_items, total_units;
+  float scale_log2;
+  const int* row_ptr;
+  const int* cnt;
+  const uint32_t* entries;
+  __nv_bfloat16* o;
+  float* lse;
+  int* status;
+  unsigned long long timeout_ns;
+};
+
+struct Item {
+  int b, h, qt, n;  // n < 0: no item; n == 0: empty kept list
+  const uint32_t* ent;
+};
+
+__device__ __forceinline__ Item get_item(const AttnParams& p, int it) {
+  Item r;
+  r.n = -1;
+  r.ent = nullptr;
+  r.b = r.h = r.qt = 0;
+  if (it >= p.total_items) return r;
+  r.qt = it % p.QT;
+  const int bh = it / p.QT;
+  r.h = bh % p.H;
+  r.b = bh / p.H;
+  const int mh = p.list_heads == 1 ? 0 : bh;
+  const int lr = p.block_q >= 128 ? (r.qt * kBM) / p.block_q : r.qt;
+  const int first_qb = p.block_q >= 128 ? lr : 2 * lr;
+  r.n = p.cnt[mh * p.LR + lr];
+  r.ent = p.entries + static_cast<long long>(p.row_ptr[mh * p.QB + first_qb]) * p.expand;
+  return r;
+}
+
+// ---------------------------------------------------------------------------
+// Per-q-tile step lists.  One thread per list row (a q-block when block_q >= 128,
+// a 128-row q-tile made of two 64-row q-blocks otherwise).  Entry = k-tile index
+// (bits 0-27) | quadrant bits << 28, bit (q_half * 2 + k_half) set when the
+// 64x64 quadrant is kept.  Lists are written at the offset the block CSR gives
+// the list row's first block row (times the k expansion), which bounds their
+// length without a scan.  Malformed CSR rows are reported and left empty.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void emit(uint32_t* out, int& n, int kt, uint32_t bits) {
+  if (n > 0 && static_cast<int>(out[n - 1] & 0x0FFFFFFFu) == kt) {
+    out[n - 1] |= bits << 28;
+  } else {
+    out[n++] = static_cast<uint32_t>(kt) | (bits << 28);
+  }
+}
+
+__global__ void build_lists_kernel(const int* __restrict__ row_ptr, const int* __restrict__ col_idx,
+                                   int list_heads, int QB, int KB, int LR, int block_q,
+                                   int block_k, int expand, long long nnz_cap,
+                                   int* __restrict__ cnt, uint32_t* __restrict__ entries,
+                                   int* status) {
+  const long long g = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (g >= static_cast<long long>(list_heads) * LR) return;
+  const int mh = static_cast<int>(g / LR), lr = static_cast<int>(g - static_cast<long long>(mh) * LR);
+  const int nrows = block_q >= 128 ? 1 : ((2 * lr + 1 < QB) ? 2 : 1);
+  const int first_qb = block_q >= 128 ? lr : 2 * lr;
+  const int* rp = row_ptr + static_cast<long long>(mh) * QB + first_qb;
+  // validate the CSR rows this list reads
+  for (int r = 0; r < nrows; ++r) {
+    if (rp[r] < 0 || rp[r] > rp[r + 1] || rp[r + 1] > nnz_cap) {
+      set_status(status, BSA_ERR_INVALID_ARG);
+      cnt[g] = 0;
+      return;
+    }
+    for (int i = rp[r]; i < rp[r + 1]; ++i) {
+      const int c = col_idx[i];
+      if (c < 0 || c >= KB || (i > rp[r] && c <= col_idx[i - 1])) {
+        set_status(status, BSA_ERR_INVALID_ARG);
+        cnt[g] = 0;
+        return;
+      }
+    }
+  }
+  uint32_t* out = entries + static_cast<long long>(rp[0]) * expand;
+  int n = 0;
+  int i0 = rp[0], e0 = rp[1];
+  int i1 = nrows == 2 ? rp[1] : 0, e1 = nrows == 2 ? rp[2] : 0;
+  const bool single = nrows == 1;
+  while (i0 < e0 || i1 < e1) {
+    // next k-block from the two sorted rows (ties: both)
+    int kb;
+    uint32_t qh;  // bit 0: q-half 0 wants it, bit 1: q-half 1 wants it
+    const int c0 = i0 < e0 ? col_idx[i0] : 0x7fffffff;
+    const int c1 = i1 < e1 ? col_idx[i1] : 0x7fffffff;
+    if (c0 <= c1) {
+      kb = c0;
+      qh = single ? (block_q >= 128 ? 0x3u : 0x1u) : 0x1u;
+      ++i0;
+      if (c1 == c0) { qh |= 0x2u; ++i1; }
+    } else {
+      kb = c1;
+      qh = 0x2u;
+      ++i1;
+    }
+    if (block_k >= 128) {
+      uint32_t bits = 0;
+      if (qh & 1u) bits |= 0x3u;  // q-half 0, both k-halves
+      if (qh & 2u) bits |= 0xCu;  // q-half 1, both k-halves
+      for (int t = 0; t < expand; ++t) emit(out, n, kb * expand + t, bits);
+    } else {  // 64-token key blocks: one k-half of tile kb/2
+      const uint32_t kh = static_cast<uint32_t>(kb & 1);
+      uint32_t bits = 0;
+      if (qh & 1u) bits |= 1u << (0 + kh);
+      if (qh & 2u) bits |= 1u << (2 + kh);
+      emit(out, n, kb >> 1, bits);
+    }
+  }
+  cnt[g] = n;
+}
+
+// ---------------------------------------------------------------------------
+// The attention kernel.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sQ = sbase + C::OFF_Q;
+  const uint32_t sRing = sbase + C::OFF_RING;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  // barrier slots
+  const uint32_t bar0 = smem_u32(bars);
+  auto FULL = [&](int i) { return bar0 + 8u * i; };
+  auto EMPTY = [&](int i) { return bar0 + 8u * (C::NSTAGE + i); };
+  auto QFULL = [&](int s) { return bar0 + 8u * (2 * C::NSTAGE + s); };
+  auto QEMPTY = [&](int s) { return bar0 + 8u * (2 * C::NSTAGE + 2 + s); };
+  auto SFULL = [&](int s) { return bar0 + 8u * (2 * C::NSTAGE + 4 + s); };
+  auto PREADY = [&](int s) { return bar0 + 8u * (2 * C::NSTAGE + 6 + s); };
+  auto ODONE = [&](int s) { return bar0 + 8u * (2 * C::NSTAGE + 8 + s); };
+  const uint32_t FINAL = bar0 + 8u * (2 * C::NSTAGE + 10);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + 8 * (2 * C::NSTAGE + 11));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::NSTAGE; ++i) {
+      mbar_init(FULL(i), 1);
+      mbar_init(EMPTY(i), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(QFULL(s), 1);
+      mbar_init(QEMPTY(s), 1);
+      mbar_init(SFULL(s), 1);
+      mbar_init(PREADY(s), 4);
+      mbar_init(ODONE(s), 1);
+    }
+    mbar_init(FINAL, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == kMmaWarp) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(512)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  if (warp == kLoadWarp && lane == 0) {
+    prefetch_tensormap(&tmQ);
+    prefetch_tensormap(&tmK);
+    prefetch_tensormap(&tmV);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == kLoadWarp) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int st = 0;
+      uint32_t ph = 0;
+      uint32_t qph[2] = {0, 0};
+      int last_fill_stage_phase[C::NSTAGE];
+      for (int i = 0; i < C::NSTAGE; ++i) last_fill_stage_phase[i] = -1;
+      int q_filled[2] = {-1, -1};
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.total_units && ok; u += gridDim.x) {
+        Item it[2] = {get_item(p, 2 * u), get_item(p, 2 * u + 1)};
+        for (int s = 0; s < 2 && ok; ++s) {
+          if (it[s].n <= 0) continue;
+          ok = mbar_wait(QEMPTY(s), qph[s] ^ 1u, abort_flag, p.status, p.timeout_ns);
+          if (!ok) break;
+          q_filled[s] = static_cast<int>(qph[s]);
+          qph[s] ^= 1u;
+          mbar_expect_tx(QFULL(s), C::TILE_BYTES);
+          for (int c = 0; c < C::KCH; ++c)
+            tma_load_4d(sQ + s * C::TILE_BYTES + c * C::CHUNK_BYTES, &tmQ, QFULL(s), 64 * c,
+                        it[s].h, it[s].qt * kBM, it[s].b);
+        }
+        const int R = max(it[0].n, it[1].n);
+        for (int r = 0; r < R && ok; ++r) {
+          for (int kv = 0; kv < 2 && ok; ++kv) {
+            for (int s = 0; s < 2; ++s) {
+              if (r >= it[s].n) continue;
+              ok = mbar_wait(EMPTY(st), ph ^ 1u, abort_flag, p.status, p.timeout_ns);
+              if (!ok) break;
+              const int kt = static_cast<int>(__ldg(it[s].ent + r) & 0x0FFFFFFFu);
+              mbar_expect_tx(FULL(st), C::TILE_BYTES);
+              const CUtensorMap* map = kv == 0 ? &tmK : &tmV;
+              for (int c = 0; c < C::KCH; ++c)
+                tma_load_4d(sRing + st * C::TILE_BYTES + c * C::CHUNK_BYTES, map, FULL(st),
+                            64 * c, it[s].h, kt * kBN, it[s].b);
+              last_fill_stage_phase[st] = static_cast<int>(ph);
+              if (++st == C::NSTAGE) { st = 0; ph ^= 1u; }
+            }
+          }
+        }
+      }
+      // Do not leave the CTA while a TMA copy into its shared memory may be in flight.
+      for (int i = 0; i < C::NSTAGE; ++i)
+        if (last_fill_stage_phase[i] >= 0)
+          mbar_wait_drain(FULL(i), static_cast<uint32_t>(last_fill_stage_phase[i]), p.status,
+                          p.timeout_ns);
+      for (int s = 0; s < 2; ++s)
+        if (q_filled[s] >= 0)
+          mbar_wait_drain(QFULL(s), static_cast<uint32_t>(q_filled[s]), p.status, p.timeout_ns);
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, 0, 0);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, 0, 1);
+      int st = 0;
+      uint32_t ph = 0;
+      uint32_t qph[2] = {0, 0}, pph[2] = {0, 0};
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.total_units && ok; u += gridDim.x) {
+        Item it[2] = {get_item(p, 2 * u), get_item(p, 2 * u + 1)};
+        const int R = max(it[0].n, it[1].n);
+        for (int r = 0; r < R && ok; ++r) {
+          for (int s = 0; s < 2; ++s) {  // S_s = Q_s K^T
+            if (r >= it[s].n) continue;
+            if (r == 0) {
+              ok = mbar_wait(QFULL(s), qph[s], abort_flag, p.status, p.timeout_ns);
+              if (!ok) break;
+              qph[s] ^= 1u;
+            }
+            ok = mbar_wait(FULL(st), ph, abort_flag, p.status, p.timeout_ns);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t qa = sQ + s * C::TILE_BYTES;
+            const uint32_t kb = sRing + st * C::TILE_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * C::CHUNK_BYTES + (kk & 3) * 32;
+              mma_ss(tmem + s * 128, smem_desc_sw128(qa + off, 16, 1024),
+                     smem_desc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(EMPTY(st));
+            mma_commit(SFULL(s));
+            if (r == it[s].n - 1) mma_commit(QEMPTY(s));
+            if (++st == C::NSTAGE) { st = 0; ph ^= 1u; }
+          }
+          for (int s = 0; s < 2 && ok; ++s) {  // O_s += P_s V
+            if (r >= it[s].n) continue;
+            ok = mbar_wait(FULL(st), ph, abort_flag, p.status, p.timeout_ns);
+            if (!ok) break;
+            ok = mbar_wait(PREADY(s), pph[s], abort_flag, p.status, p.timeout_ns);
+            if (!ok) break;
+            pph[s] ^= 1u;
+            tc_fence_after();
+            const uint32_t vb = sRing + st * C::TILE_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < kBN / 16; ++kk) {
+              mma_ts(tmem + 256 + s * 128, tmem + s * 128 + kk * 8,
+                     smem_desc_sw128(vb + kk * 16 * 128, C::CHUNK_BYTES, 1024), idesc_pv,
+                     (r > 0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit(EMPTY(st));
+            if (r == it[s].n - 1) mma_commit(ODONE(s));
+            if (++st == C::NSTAGE) { st = 0; ph ^= 1u; }
+          }
+        }
+      }
+      // Every MMA of this CTA has finished before TMEM is released.
+      mma_commit(FINAL);
+      mbar_wait_drain(FINAL, 0, p.status, p.timeout_ns);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax (8 warps)
+    const int s = warp >> 2;                 // slot
+    const int row = threadIdx.x & 127;       // query row within the tile = TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_base + s * 128;
+    const uint32_t tO = tmem + lane_base + 256 + s * 128;
+    const float sl2 = p.scale_log2;
+    uint32_t sph = 0, oph = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.total_units && ok; u += gridDim.x) {
+      const Item me = get_item(p, 2 * u + s);
+      if (me.n < 0) continue;
+      const int qrow = me.qt * kBM + row;
+      float m_used = -INFINITY, l = 0.f;
+      const int qh = row >> 6;
+      for (int j = 0; j < me.n; ++j) {
+        ok = mbar_wait(SFULL(s), sph, abort_flag, p.status, p.timeout_ns);
+        if (!ok) break;
+        sph ^= 1u;
+        tc_fence_after();
+        uint32_t sr[kBN];
+        tmem_ld32x32b_x128(tS, sr);
+        float sv[kBN];
+#pragma unroll
+        for (int c = 0; c < kBN; ++c) sv[c] = __uint_as_float(sr[c]);
+        const uint32_t ent = __ldg(me.ent + j);
+        const int kt = static_cast<int>(ent & 0x0FFFFFFFu);
+        const uint32_t bits = ent >> 28;
+        const int kvalid = p.nk - kt * kBN;  // keys of this tile that exist
+        if (bits != 0xFu || kvalid < kBN) {
+          const bool lo_ok = (bits >> (qh * 2)) & 1u, hi_ok = (bits >> (qh * 2 + 1)) & 1u;
+#pragma unroll
+          for (int c = 0; c < kBN; ++c) {
+            const bool keep = (c < 64 ? lo_ok : hi_ok) && c < kvalid;
+            if (!keep) sv[c] = -INFINITY;
+          }
+        }
+        float mt = sv[0];
+#pragma unroll
+        for (int c = 1; c < kBN; ++c) mt = fmaxf(mt, sv[c]);
+        mt *= sl2;
+        const float m_new = fmaxf(m_used, mt);
+        if (j == 0) {
+          m_used = m_new;
+        } else {
+          const bool need = m_new > m_used + kRescaleThreshold;
+          const bool has_o = m_used != -INFINITY;
+          if (__any_sync(0xffffffffu, need && has_o)) {
+            const float alpha = (need && has_o) ? fast_exp2(m_used - m_new) : 1.0f;
+#pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 32) {
+              uint32_t ov[32];
+              tmem_ld32x32b_x32(tO + c0, ov);
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+              tmem_st32x32b_x32(tO + c0, ov);
+            }
+            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+            l *= alpha;
+          }
+          if (need) m_used = m_new;
+        }
+        const float msub = m_used == -INFINITY ? 0.f : m_used;
+#pragma unroll
+        for (int c0 = 0; c0 < kBN; c0 += 32) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float p0 = fast_exp2(fmaf(sv[c0 + 2 * i], sl2, -msub));
+            const float p1 = fast_exp2(fmaf(sv[c0 + 2 * i + 1], sl2, -msub));
+            l += p0 + p1;
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+            pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+          }
+          tmem_st32x32b_x16(tS + c0 / 2, pk);
+        }
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(PREADY(s));
+      }
+      if (!ok) break;
+      __nv_bfloat16* orow = p.o + ((static_cast<long long>(me.b) * p.nq + qrow) * p.H + me.h) * D;
+      float* lrow = p.lse + (static_cast<long long>(me.b) * p.H + me.h) * p.nq + qrow;
+      if (me.n == 0) {
+        if (qrow < p.nq) {
+          uint4 z = make_uint4(0, 0, 0, 0);
+#pragma unroll
+          for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(orow)[c] = z;
+          *lrow = -INFINITY;
+        }
+        continue;
+      }
+      ok = mbar_wait(ODONE(s), oph, abort_flag, p.status, p.timeout_ns);
+      if (!ok) break;
+      oph ^= 1u;
+      tc_fence_after();
+      const float inv = l > 0.f ? 1.0f / l : 0.f;
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t ov[32];
+        tmem_ld32x32b_x32(tO + c0, ov);
+        if (qrow < p.nq) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(ov[2 * i]) * inv,
+                                                      __uint_as_float(ov[2 * i + 1]) * inv);
+            pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+          }
+          uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          dst[2] = make_uint4(pk[8], pk[9], pk[10], pk[11]);
+          dst[3] = make_uint4(pk[12], pk[13], pk[14], pk[15]);
+        }
+      }
+      if (qrow < p.nq) *lrow = l > 0.f ? (m_used + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+      // O is read out; the next item's first P.V may overwrite it once P is ready
+      tc_fence_before();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kMmaWarp) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512)
+                 : "memory");
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// 4D map over [B, N, H, D] bf16 (D contiguous), dimensions listed innermost first as
+// (D, H, N, B); box 64 x 1 x 128 x 1 = 128 token rows of 128 bytes, 128-byte swizzle.
+int make_map(CUtensorMap* map, const void* base, int B, int N, int H, int D) {
+  auto fn = get_encode_fn();
+  if (!fn) return BSA_ERR_CUDA;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
+                        static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2,
+                           static_cast<cuuint64_t>(N) * H * D * 2};
+  cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(kBM), 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? BSA_OK : BSA_ERR_CUDA;
+}
+
+bool block_ok(int blk) { return blk == 64 || (blk >= 128 && blk % 128 == 0); }
+
+struct Geometry {
+  int QB, KB, QT, LR, expand;
+  long long nnz_cap, entries_cap;
+  size_t cnt_off, ent_off, total;
+};
+
+Geometry geometry(int batch, int heads, int nq, int nk, int block_q, int block_k, int list_heads) {
+  Geometry g;
+  g.QB = ceil_div(nq, block_q);
+  g.KB = ceil_div(nk, block_k);
+  g.QT = ceil_div(nq, kBM);
+  g.LR = block_q >= 128 ? g.QB : g.QT;
+  g.expand = block_k >= 128 ? block_k / 128 : 1;
+  g.nnz_cap = static_cast<long long>(list_heads) * g.QB * g.KB;
+  g.entries_cap = g.nnz_cap * g.expand;
+  g.cnt_off = kStatusBytes;
+  g.ent_off = g.cnt_off + ((sizeof(int) * static_cast<size_t>(list_heads) * g.LR + 255) & ~size_t(255));
+  g.total = g.ent_off + sizeof(uint32_t) * static_cast<size_t>(g.entries_cap);
+  (void)batch;
+  (void)heads;
+  return g;
+}
+
+template <int D>
+int launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                const AttnParams& p, cudaStream_t st) {
+  using C = Cfg<D>;
+  static bool attr_done[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || !attr_done[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return record_cuda_error(e);
+    if (dev >= 0 && dev < 64) attr_done[dev] = true;
+  }
+  int grid = device_sm_count();
+  if (grid > p.total_units) grid = p.total_units;
+  attn_fwd_kernel<D><<<grid, kThreads, C::SMEM, st>>>(mq, mk, mv, p);
+  return check_launch();
+}
+
+}  // namespace
+}  // namespace bsa
+
+extern "C" size_t bsa_attn_workspace_size(int batch, int heads, int nq, int nk, int block_q,
+                                          int block_k, int list_heads) {
+  if (batch < 1 || heads < 1 || nq < 1 || nk < 1 || !bsa::block_ok(block_q) ||
+      !bsa::block_ok(block_k) || list_heads < 1)
+    return 0;
+  return bsa::geometry(batch, heads, nq, nk, block_q, block_k, list_heads).total;
+}
+
+extern "C" int bsa_attn_fwd(const void* q, const void* k, const void* v, int batch, int heads,
+                            int nq, int nk, int head_dim, int block_q, int block_k,
+                            const int* row_ptr, const int* col_idx, int list_heads, float scale,
+                            void* o, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  using namespace bsa;
+  if (!q || !k || !v || !o || !lse || !row_ptr || !col_idx || !ws) return BSA_ERR_INVALID_ARG;
+  if (batch < 1 || heads < 1 || nq < 1 || nk < 1) return BSA_ERR_INVALID_ARG;
+  if (list_heads != 1 && list_heads != batch * heads) return BSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(ws))
+    return BSA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return BSA_ERR_UNSUPPORTED;
+  if (!block_ok(block_q) || !block_ok(block_k)) return BSA_ERR_UNSUPPORTED;
+  const Geometry g = geometry(batch, heads, nq, nk, block_q, block_k, list_heads);
+  if (ws_bytes < g.total) return BSA_ERR_WORKSPACE;
+  if (g.nnz_cap > 0x7fffffffLL || static_cast<long long>(ceil_div(nk, kBN)) >= (1LL << 28) ||
+      static_cast<long long>(batch) * heads * g.QT > 0x3fffffffLL)
+    return BSA_ERR_UNSUPPORTED;
+  if (scale <= 0.0f) scale = 1.0f / sqrtf(static_cast<float>(head_dim));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  CUtensorMap mq, mk, mv;
+  if (make_map(&mq, q, batch, nq, heads, head_dim) != BSA_OK ||
+      make_map(&mk, k, batch, nk, heads, head_dim) != BSA_OK ||
+      make_map(&mv, v, batch, nk, heads, head_dim) != BSA_OK)
+    return BSA_ERR_CUDA;
+
+  char* wsb = static_cast<char*>(ws);
+  int* status = reinterpret_cast<int*>(wsb);
+  int* cnt = reinterpret_cast<int*>(wsb + g.cnt_off);
+  uint32_t* entries = reinterpret_cast<uint32_t*>(wsb + g.ent_off);
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), st);
+  if (e != cudaSuccess) return record_cuda_error(e);
+
+  const long long lists = static_cast<long long>(list_heads) * g.LR;
+  build_lists_kernel<<<static_cast<int>(ceil_div<long long>(lists, 128)), 128, 0, st>>>(
+      row_ptr, col_idx, list_heads, g.QB, g.KB, g.LR, block_q, block_k, g.expand, g.nnz_cap, cnt,
+      entries, status);
+  int rc = check_launch();
+  if (rc != BSA_OK) return rc;
+
+  AttnParams p;
+  p.B = batch;
+  p.H = heads;
+  p.nq = nq;
+  p.nk = nk;
+  p.QT = g.QT;
+  p.block_q = block_q;
+  p.block_k = block_k;
+  p.QB = g.QB;
+  p.LR = g.LR;
+  p.list_heads = list_heads;
+  p.expand = g.expand;
+  p.total_items = batch * heads * g.QT;
+  p.total_units = (p.total_items + 1) / 2;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.row_ptr = row_ptr;
+  p.cnt = cnt;
+  p.entries = entries;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.status = status;
+  p.timeout_ns = 2000000000ULL;
+  return head_dim == 128 ? launch_attn<128>(mq, mk, mv, p, st) : launch_attn<64>(mq, mk, mv, p, st);
+}

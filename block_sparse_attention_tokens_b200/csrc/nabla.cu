@@ -1,0 +1,283 @@
+// NABLA dynamic block mask: block mean-pooling of Q and K, then a per-row
+// softmax over the pooled logits and the smallest top set reaching mass p.
+//
+// Source: "NABLA (Neighborhood Adaptive Block-Level Attention)" explainer
+// (aibr.jp/archives/124678), section 3 -- Q and K are average-pooled per block,
+// full attention is computed on the pooled tokens, each row is thresholded by its
+// cumulative distribution and the binary result is applied at block level.
+// Forced key ranges (anchors / recent frames): "Sparse Forcing" summary
+// (gist.science/ja/paper/2604.21221), part 2.
+//
+// Kernels
+//   pool   : HBM-bound column sums.  One CTA per (tensor, batch, block, 1024-column
+//            chunk); each thread owns 8 adjacent bf16 columns (one 16-byte vector
+//            per token row) and accumulates in fp32 over the block's valid rows.
+//   select : one CTA per (batch, head, 8 query blocks).  Pooled keys stream
+//            through shared memory in tiles of 32 blocks; every thread forms one
+//            logit per tile.  Each warp then owns one query row: softmax
+//            statistics, a 32-step radix search over the order-preserving integer
+//            image of the fp32 logits for the cut, ties resolved to the lower
+//            block index, and the row of mask bytes.
+#include "bsa_common.cuh"
+
+namespace bsa {
+namespace {
+
+constexpr int kPoolThreads = 128;          // threads per pooling CTA
+constexpr int kPoolCols = kPoolThreads * 8;  // bf16 columns per pooling CTA
+constexpr int kSelRows = 8;                // query rows per select CTA (one per warp)
+constexpr int kSelTile = 32;               // key blocks per shared-memory tile
+
+__device__ __forceinline__ void add_bf16x8(float* acc, const uint4& v) {
+  const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 f = __bfloat1622float2(p[i]);
+    acc[2 * i] += f.x;
+    acc[2 * i + 1] += f.y;
+  }
+}
+
+// grid: x = block index, y = column chunk, z = batch * 2 + tensor (0 = q, 1 = k)
+__global__ void __launch_bounds__(kPoolThreads) nabla_pool_kernel(
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k, int heads,
+    int head_dim, int nq, int nk, int block, int qb_count, int kb_count,
+    float* __restrict__ qbar, float* __restrict__ kbar) {
+  const int which = blockIdx.z & 1;
+  const int b = blockIdx.z >> 1;
+  const int nblk = which ? kb_count : qb_count;
+  const int blk = blockIdx.x;
+  if (blk >= nblk) return;
+  const int n = which ? nk : nq;
+  const __nv_bfloat16* src = which ? k : q;
+  float* dst = which ? kbar : qbar;
+  const int C = heads * head_dim;
+  const int col = blockIdx.y * kPoolCols + threadIdx.x * 8;
+  if (col >= C) return;
+  const int r0 = blk * block;
+  const int r1 = min(r0 + block, n);
+  const uint4* base =
+      reinterpret_cast<const uint4*>(src + (static_cast<long long>(b) * n + r0) * C + col);
+  const long long stride = C / 8;  // uint4 per token row
+  float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  int r = r0;
+  for (; r + 4 <= r1; r += 4) {
+    const uint4* p = base + static_cast<long long>(r - r0) * stride;
+    uint4 v0 = __ldg(p), v1 = __ldg(p + stride), v2 = __ldg(p + 2 * stride),
+          v3 = __ldg(p + 3 * stride);
+    add_bf16x8(acc, v0);
+    add_bf16x8(acc, v1);
+    add_bf16x8(acc, v2);
+    add_bf16x8(acc, v3);
+  }
+  for (; r < r1; ++r) add_bf16x8(acc, __ldg(base + static_cast<long long>(r - r0) * stride));
+  const float inv = 1.0f / static_cast<float>(r1 - r0);
+  const int h = col / head_dim, j = col - h * head_dim;
+  float4* out = reinterpret_cast<float4*>(
+      dst + ((static_cast<long long>(b) * heads + h) * nblk + blk) * head_dim + j);
+  out[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+  out[1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
+}
+
+__device__ __forceinline__ uint32_t order_key(float z) {
+  const uint32_t u = __float_as_uint(z);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ int warp_isum(int v) {
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// grid: x = ceil(QB / kSelRows), y = heads, z = batch; 256 threads.
+// dynamic smem: qs[kSelRows][D] + ks[kSelTile][D+1] + z[kSelRows][nr] + e[kSelRows][nr]
+template <int D>
+__global__ void __launch_bounds__(256) nabla_select_kernel(
+    const float* __restrict__ qbar, const float* __restrict__ kbar, int heads, int qb_count,
+    int kb_count, int kb_begin, int kb_end, float p, float scale, int force_outside,
+    uint8_t* __restrict__ mask, int* __restrict__ near_count) {
+  extern __shared__ float smem[];
+  const int nr = kb_end - kb_begin;
+  float* qs = smem;
+  float* ks = qs + kSelRows * D;
+  float* zs = ks + kSelTile * (D + 1);
+  float* es = zs + kSelRows * nr;
+  const int b = blockIdx.z, h = blockIdx.y;
+  const int q0 = blockIdx.x * kSelRows;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const float* qsrc = qbar + (static_cast<long long>(b) * heads + h) * qb_count * D;
+  const float* ksrc = kbar + (static_cast<long long>(b) * heads + h) * kb_count * D;
+
+  for (int i = tid; i < kSelRows * D; i += blockDim.x) {
+    const int r = i / D;
+    qs[i] = (q0 + r < qb_count) ? qsrc[static_cast<long long>(q0 + r) * D + (i - r * D)] : 0.f;
+  }
+  // logits z[r][c] = qbar[r] . kbar[kb_begin + c] * scale
+  for (int t0 = 0; t0 < nr; t0 += kSelTile) {
+    __syncthreads();
+    for (int i = tid; i < kSelTile * D; i += blockDim.x) {
+      const int c = i / D, j = i - c * D;
+      ks[c * (D + 1) + j] =
+          (t0 + c < nr) ? ksrc[static_cast<long long>(kb_begin + t0 + c) * D + j] : 0.f;
+    }
+    __syncthreads();
+    const float* qrow = qs + warp * D;
+    const float* krow = ks + lane * (D + 1);
+    float acc = 0.f;
+#pragma unroll 8
+    for (int j = 0; j < D; ++j) acc = fmaf(qrow[j], krow[j], acc);
+    if (t0 + lane < nr) zs[warp * nr + t0 + lane] = acc * scale;
+  }
+  __syncthreads();
+
+  const int qb = q0 + warp;
+  if (qb >= qb_count) return;
+  uint8_t* mrow = mask + ((static_cast<long long>(b) * heads + h) * qb_count + qb) * kb_count;
+  const uint8_t fo = force_outside ? 1 : 0;
+  for (int c = lane; c < kb_begin; c += 32) mrow[c] = fo;
+  for (int c = kb_end + lane; c < kb_count; c += 32) mrow[c] = fo;
+  if (nr <= 0) return;
+
+  float* z = zs + warp * nr;
+  float* e = es + warp * nr;
+  float m = -INFINITY;
+  for (int c = lane; c < nr; c += 32) m = fmaxf(m, z[c]);
+  m = warp_max(m);
+  float tot = 0.f;
+  for (int c = lane; c < nr; c += 32) {
+    const float v = __expf(z[c] - m);
+    e[c] = v;
+    tot += v;
+  }
+  tot = warp_sum(tot);
+  __syncwarp();
+
+  if (p >= 1.0f) {
+    for (int c = lane; c < nr; c += 32) mrow[kb_begin + c] = 1;
+    return;
+  }
+  const float target = p * tot;
+  // largest v with F(v) = sum_{key_c >= v} e_c >= target
+  uint32_t v = 0;
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t cand = v | (1u << bit);
+    float f = 0.f;
+    for (int c = lane; c < nr; c += 32)
+      if (order_key(z[c]) >= cand) f += e[c];
+    f = warp_sum(f);
+    if (f >= target) v = cand;
+  }
+  // mass strictly above the cut, the tied value, and the largest value below it
+  float f_gt = 0.f, e_eq = 0.f, e_below = 0.f;
+  int n_eq = 0;
+  for (int c = lane; c < nr; c += 32) {
+    const uint32_t key = order_key(z[c]);
+    if (key > v) f_gt += e[c];
+    else if (key == v) { e_eq = e[c]; ++n_eq; }
+    else e_below = fmaxf(e_below, e[c]);
+  }
+  f_gt = warp_sum(f_gt);
+  e_eq = warp_max(e_eq);
+  e_below = warp_max(e_below);
+  n_eq = warp_isum(n_eq);
+  int t = 1;
+  float cum = f_gt + e_eq;
+  while (cum < target && t < n_eq) {
+    ++t;
+    cum += e_eq;
+  }
+  // kept: key > v, plus the first t tied entries in index order
+  int ties_seen = 0;
+  for (int c0 = 0; c0 < nr; c0 += 32) {
+    const int c = c0 + lane;
+    uint32_t key = 0;
+    if (c < nr) key = order_key(z[c]);
+    const bool tie = c < nr && key == v;
+    const uint32_t bal = __ballot_sync(0xffffffffu, tie);
+    const int rank = ties_seen + __popc(bal & ((1u << lane) - 1u));
+    ties_seen += __popc(bal);
+    if (c < nr) mrow[kb_begin + c] = (key > v || (tie && rank < t)) ? 1 : 0;
+  }
+  if (lane == 0 && near_count) {
+    const float c_last = cum / tot, c_prev = (cum - e_eq) / tot;
+    bool near = fabsf(c_last - p) < 1e-5f || fabsf(c_prev - p) < 1e-5f;
+    if (t == n_eq && e_below > 0.f && e_below >= e_eq * (1.0f - 1e-5f)) near = true;
+    if (near) atomicAdd(near_count, 1);
+  }
+}
+
+size_t nabla_ws_bytes(int batch, int heads, int nq, int nk, int head_dim, int block) {
+  const size_t qb = ceil_div(nq, block), kb = ceil_div(nk, block);
+  return kStatusBytes + sizeof(float) * static_cast<size_t>(batch) * heads * head_dim * (qb + kb);
+}
+
+}  // namespace
+}  // namespace bsa
+
+extern "C" size_t bsa_nabla_workspace_size(int batch, int heads, int nq, int nk, int head_dim,
+                                           int block) {
+  if (batch < 1 || heads < 1 || nq < 1 || nk < 1 || head_dim < 1 || block < 1) return 0;
+  return bsa::nabla_ws_bytes(batch, heads, nq, nk, head_dim, block);
+}
+
+extern "C" int bsa_nabla_mask(const void* q, const void* k, int batch, int heads, int nq, int nk,
+                              int head_dim, int block, float p, float scale, int kb_begin,
+                              int kb_end, int force_outside, uint8_t* mask, int* near_count,
+                              void* ws, size_t ws_bytes, void* stream) {
+  using namespace bsa;
+  if (!q || !k || !mask || !ws) return BSA_ERR_INVALID_ARG;
+  if (batch < 1 || heads < 1 || nq < 1 || nk < 1 || block < 16 || block > 1024 ||
+      (block % 16) != 0 || !(p > 0.0f))
+    return BSA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return BSA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(ws)) return BSA_ERR_INVALID_ARG;
+  const int qb = ceil_div(nq, block), kb = ceil_div(nk, block);
+  if (kb_begin < 0 || kb_end > kb || kb_begin > kb_end) return BSA_ERR_INVALID_ARG;
+  if (ws_bytes < nabla_ws_bytes(batch, heads, nq, nk, head_dim, block)) return BSA_ERR_WORKSPACE;
+  if (scale <= 0.0f) scale = 1.0f / sqrtf(static_cast<float>(head_dim));
+  const int nr = kb_end - kb_begin;
+  const size_t smem = sizeof(float) * (static_cast<size_t>(kSelRows) * head_dim +
+                                       static_cast<size_t>(kSelTile) * (head_dim + 1) +
+                                       2 * static_cast<size_t>(kSelRows) * nr);
+  if (smem > 200 * 1024) return BSA_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* qbar = reinterpret_cast<float*>(static_cast<char*>(ws) + kStatusBytes);
+  float* kbar = qbar + static_cast<size_t>(batch) * heads * qb * head_dim;
+  if (near_count) {
+    cudaError_t e = cudaMemsetAsync(near_count, 0, sizeof(int), st);
+    if (e != cudaSuccess) return record_cuda_error(e);
+  }
+  const int C = heads * head_dim;
+  dim3 pgrid(qb > kb ? qb : kb, ceil_div(C, kPoolCols), batch * 2);
+  nabla_pool_kernel<<<pgrid, kPoolThreads, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), heads,
+      head_dim, nq, nk, block, qb, kb, qbar, kbar);
+  int rc = check_launch();
+  if (rc != BSA_OK) return rc;
+  dim3 sgrid(ceil_div(qb, kSelRows), heads, batch);
+  cudaError_t e;
+  if (head_dim == 128) {
+    e = cudaFuncSetAttribute(nabla_select_kernel<128>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return record_cuda_error(e);
+    nabla_select_kernel<128><<<sgrid, 256, smem, st>>>(qbar, kbar, heads, qb, kb, kb_begin,
+                                                       kb_end, p, scale, force_outside, mask,
+                                                       near_count);
+  } else {
+    e = cudaFuncSetAttribute(nabla_select_kernel<64>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return record_cuda_error(e);
+    nabla_select_kernel<64><<<sgrid, 256, smem, st>>>(qbar, kbar, heads, qb, kb, kb_begin,
+                                                      kb_end, p, scale, force_outside, mask,
+                                                      near_count);
+  }
+  return check_launch();
+}

@@ -1,0 +1,199 @@
+/*
+ * bsa.h -- C ABI of libbsa.so: block-sparse 3D spatio-temporal attention for
+ * video-DiT tokens on NVIDIA B200 (sm_100a).
+ *
+ * The library computes the data-parallel path the sparse video-attention pages
+ * describe:
+ *   (a) a 3D tile permute of a T x H x W token grid (and its inverse),
+ *   (b) block masks: the static Sliding-Tile window, the static radial
+ *       (energy-decay) mask, and the dynamic per-head NABLA top-p mask,
+ *   (c) compaction of a block mask into per-row kept-block lists, and
+ *   (d) the attention forward that visits only kept (query block, key block)
+ *       pairs, with an online softmax, producing O and the log-sum-exp.
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     never allocates, frees or retains them and keeps no per-call state.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream).  A return of BSA_OK means the work was enqueued.
+ *   - Arguments are validated on the host before anything is enqueued.  Invalid
+ *     arguments return BSA_ERR_INVALID_ARG, shapes outside what the kernels
+ *     implement return BSA_ERR_UNSUPPORTED; neither enqueues work.  There is no
+ *     fallback path of any kind.
+ *   - Token tensors are bfloat16, layout [B, N, heads, head_dim] with
+ *     head_dim contiguous (one token row = heads * head_dim elements), 16-byte
+ *     aligned base addresses.
+ *   - Masks are uint8, one byte per (query block, key block), 0 = dropped,
+ *     nonzero = kept, row-major [rows][KB].
+ *   - Errors never abort the process.  Errors detected on the device (a
+ *     malformed kept list, a pipeline wait that ran out of time) are recorded
+ *     in the workspace's status word; read it with bsa_read_status().
+ */
+#ifndef BSA_H_
+#define BSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BSA_OK = 0,
+  BSA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size, bad kept list */
+  BSA_ERR_UNSUPPORTED = 2,   /* valid request outside the implemented shapes   */
+  BSA_ERR_WORKSPACE = 3,     /* workspace smaller than the *_workspace_size()   */
+  BSA_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed      */
+  BSA_ERR_TIMEOUT = 5        /* a device-side pipeline wait ran out of time      */
+} bsa_status;
+
+/* Human-readable name of a status code (static string). */
+const char* bsa_status_string(int status);
+
+/* Text of the last CUDA error seen by this thread inside the library ("" if none). */
+const char* bsa_last_error_message(void);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int bsa_version(void);
+
+/* ---------------------------------------------------------------------------
+ * (a) Tile permute.
+ * Source: "Fast Video Generation with Sliding Tile Attention" explainer
+ * (aibr.jp/archives/60739), section 3: the video latent is a 3D
+ * (time, height, width) token grid and the work is organised in 3D tiles.
+ *
+ * The grid T x H x W (raster order: w fastest) is cut into tT x tH x tW tiles.
+ * The permuted sequence lists the tiles in raster order over the tile grid and,
+ * inside each tile, its tokens in raster order.  Edge tiles may be smaller
+ * (ragged); they are not padded.  Positions N .. n_pad-1 (N = T*H*W) of the
+ * output are written with zeros so the sequence fills whole blocks.
+ *
+ *   x    : [batch, N, row_bytes] input rows in raster order (any element type)
+ *   y    : [batch, n_pad, row_bytes] output rows in tile order
+ *   row_bytes : bytes per token row (heads * head_dim * 2 for bf16), multiple of 16
+ *   n_pad >= N.  x and y must not overlap.
+ * bsa_tile_untile is the inverse: reads y (tile order, n_pad rows), writes the
+ * N raster-order rows of x; the zero tail of y is not read.
+ * ------------------------------------------------------------------------- */
+int bsa_tile_permute(const void* x, void* y, int batch, int T, int H, int W,
+                     int tT, int tH, int tW, int row_bytes, int n_pad, void* stream);
+int bsa_tile_untile(const void* y, void* x, int batch, int T, int H, int W,
+                    int tT, int tH, int tW, int row_bytes, int n_pad, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * (b1) Sliding Tile Attention mask.
+ * Source: STA explainer (aibr.jp/archives/60739), sections 2-3: each query tile
+ * attends to a window of neighbouring tiles; the window is counted in tiles.
+ *
+ * Tile grid nT x nH x nW (tiles in raster order = blocks of the permuted
+ * sequence when the block size equals the tile volume), window wT x wH x wW
+ * tiles.  shift = 0: the window covers offsets -floor((w-1)/2)..+ceil((w-1)/2)
+ * around the query tile on each axis, clipped at the grid edge.  shift = 1:
+ * the window keeps its full width and slides inward at the edges.
+ *   mask : [n_tiles][n_tiles] uint8, n_tiles = nT*nH*nW, written completely.
+ * ------------------------------------------------------------------------- */
+int bsa_sta_mask(int nT, int nH, int nW, int wT, int wH, int wW, int shift,
+                 uint8_t* mask, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * (b2) Radial (energy-decay) mask.
+ * Source: "Radial Attention" explainer (aibr.jp/archives/112136), sections 1-3:
+ * a static mask, dense for temporally close tokens, whose spatial window shrinks
+ * as the temporal distance grows, for O(n log n) kept pairs.
+ *
+ * Tokens in raster order, S = tokens_per_frame, token i is (frame i / S,
+ * in-frame index i % S).  Token pair (query, key) at frame distance d and
+ * in-frame distance ds is kept iff d <= 1, or, with r = floor(log2 d):
+ *   if S >= block * 2^r : ds < S / 2^(r+1)
+ *   else                : d % 2^c == 0 and ds < block / 2,
+ *                         c = smallest integer with S * 2^c >= block * 2^r.
+ * A block pair is kept iff any of its token pairs is kept.
+ *   mask : [NB][NB] uint8, NB = ceil(n_tokens / block), written completely.
+ * ------------------------------------------------------------------------- */
+int bsa_radial_mask(int n_tokens, int tokens_per_frame, int block, uint8_t* mask,
+                    void* stream);
+
+/* ---------------------------------------------------------------------------
+ * (b3) NABLA dynamic mask (optionally with forced-on key ranges).
+ * Source: "NABLA" explainer (aibr.jp/archives/124678), section 3: mean-pool Q
+ * and K per block, compute full attention on the pooled tokens, threshold each
+ * row by its cumulative distribution, apply the binary mask at block level.
+ * Forced ranges: "Sparse Forcing" summary (gist.science/ja/paper/2604.21221),
+ * part 2 -- persistent anchor frames and recent frames kept, sparse selection
+ * elsewhere.
+ *
+ *   q : [batch, nq, heads, head_dim] bf16 (tile order); k : [batch, nk, ...]
+ *   Blocks of `block` tokens; the last block of q / k may be partial and is
+ *   averaged over its valid tokens only.  QB = ceil(nq/block), KB = ceil(nk/block).
+ *   Row (b, h, qb): logits z_c = mean_q . mean_k[c] * scale (scale <= 0 means
+ *   1/sqrt(head_dim)) over key blocks c in [kb_begin, kb_end); softmax over that
+ *   range; the kept set is the smallest set of largest probabilities (ties to the
+ *   lower index) whose sum reaches p (p >= 1 keeps the whole range).  Key blocks
+ *   outside [kb_begin, kb_end) are written as force_outside (0 or 1).
+ *   mask : [batch][heads][QB][KB] uint8, written completely.
+ *   near_count : device int, overwritten with the number of rows whose cut lies
+ *                within 1e-5 of p (rows a float64 evaluation may decide
+ *                differently); may be NULL.
+ *   ws : device workspace of at least bsa_nabla_workspace_size() bytes.
+ *   head_dim in {64, 128}; block a multiple of 16 in [16, 1024].
+ * ------------------------------------------------------------------------- */
+size_t bsa_nabla_workspace_size(int batch, int heads, int nq, int nk, int head_dim, int block);
+int bsa_nabla_mask(const void* q, const void* k, int batch, int heads, int nq, int nk,
+                   int head_dim, int block, float p, float scale, int kb_begin, int kb_end,
+                   int force_outside, uint8_t* mask, int* near_count, void* ws,
+                   size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * (c) Mask compaction into per-row kept-block lists (CSR).
+ *   mask    : [rows][KB] uint8
+ *   row_ptr : [rows + 1] int32, written; row_ptr[rows] = number of kept blocks
+ *   col_idx : int32 with room for rows*KB entries (worst case), written with the
+ *             kept key-block indices of each row in ascending order.
+ * ------------------------------------------------------------------------- */
+int bsa_mask_compact(const uint8_t* mask, int rows, int KB, int* row_ptr, int* col_idx,
+                     void* stream);
+
+/* ---------------------------------------------------------------------------
+ * (d) Block-sparse attention forward.
+ * Sources: STA explainer section 3 (hardware-aware tile attention kernel),
+ * SPADE summary (gist.science/ja/paper/2608.03335), solution part 3 (head-wise
+ * sparse attention), NABLA explainer section 3 (mask applied at block level).
+ *
+ *   O[b, i, h, :] = softmax_j( Q[b,i,h,:] . K[b,j,h,:] * scale ) V[b, j, h, :]
+ *   over keys j < nk whose block pair (i / block_q, j / block_k) is kept in the
+ *   list of mask head m = (list_heads == 1 ? 0 : b * heads + h).
+ *   LSE[b, h, i] = natural-log sum of exp(scores) over the same keys.
+ *   A row with no kept key gets O = 0 and LSE = -inf.
+ *
+ *   q : [batch, nq, heads, head_dim] bf16; k, v : [batch, nk, heads, head_dim]
+ *   o : [batch, nq, heads, head_dim] bf16 (rows >= nq are never written)
+ *   lse : [batch, heads, nq] float32
+ *   row_ptr, col_idx : CSR over rows m * QB + qb (QB = ceil(nq/block_q)),
+ *                      col_idx ascending within a row, values < KB = ceil(nk/block_k)
+ *                      (as written by bsa_mask_compact).  Malformed lists set
+ *                      BSA_ERR_INVALID_ARG in the status word and are skipped.
+ *   list_heads : 1 (one list for every batch and head) or batch * heads
+ *   scale : <= 0 means 1/sqrt(head_dim)
+ *   head_dim in {64, 128}; block_q, block_k each 64 or a multiple of 128.
+ *   ws : device workspace of at least bsa_attn_workspace_size() bytes; its
+ *        status word is cleared at the start of every call.
+ * ------------------------------------------------------------------------- */
+size_t bsa_attn_workspace_size(int batch, int heads, int nq, int nk, int block_q, int block_k,
+                               int list_heads);
+int bsa_attn_fwd(const void* q, const void* k, const void* v, int batch, int heads, int nq,
+                 int nk, int head_dim, int block_q, int block_k, const int* row_ptr,
+                 const int* col_idx, int list_heads, float scale, void* o, float* lse,
+                 void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Device status word of a workspace (attention or NABLA): synchronises `stream`,
+ * copies the word to *status (a bsa_status value) and clears it.
+ * ------------------------------------------------------------------------- */
+int bsa_read_status(void* ws, int* status, void* stream);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* BSA_H_ */
