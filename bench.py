@@ -217,7 +217,7 @@ def workload_config(w):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="sta_720p")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -225,10 +225,15 @@ def main():
                     help="seconds of oracle work for the cpu_baseline field")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="override the head count (smaller cases for profiler captures)")
     args = ap.parse_args()
 
     from block_sparse_attention_tokens_b200 import configs
+    import dataclasses
     w = configs.get(args.workload)
+    if args.heads > 0:
+        w = dataclasses.replace(w, heads=args.heads)
     if args.impl == "reference":
         return run_reference(args, w)
 
@@ -273,6 +278,7 @@ def main():
     sampler = ClockSampler(dev.index)
     barrier()
     with sampler:
+        time.sleep(0.5)          # let nvidia-smi start sampling before the timed region
         start.record(stream)
         for i in range(args.steps):
             plan._q, plan._k, plan._v = q, k, v
