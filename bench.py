@@ -123,56 +123,62 @@ def cpu_cores() -> int:
         return os.cpu_count() or 1
 
 
-def oracle_sample_rate(w, q, k, v, budget_s: float):
-    """Times the CPU oracle on whole query blocks of the workload (all heads),
-    adding blocks until ~budget_s of work; returns (effective TFLOP/s, sample text)."""
-    import numpy as np
-    import oracle as O
+class OracleSample:
+    """The CPU oracle on whole query blocks of the workload (all heads).
 
-    D = w.head_dim
-    if w.tile is not None:
-        perm = O.tile_order(w.grid, w.tile)
-        n_pad = math.ceil(w.n_tokens / w.block) * w.block
-        tg = tuple(math.ceil(g / t) for g, t in zip(w.grid, w.tile))
-    rng = np.random.default_rng(7)
-    QB = math.ceil(w.nq / w.block)
-    order = rng.permutation(QB)
-    t0 = time.perf_counter()
-    if w.mask == "sta":
-        mask = O.sta_tile_mask(tg, w.window)[None]
-    elif w.mask == "radial":
-        mask = O.radial_block_mask_fast(w.nk, w.tokens_per_frame, w.block)[None]
-    else:
-        raise ValueError("cpu baseline implemented for static-mask workloads")
-    heads64 = []
-    for h in range(w.heads):
-        qh = q[:, :, h:h + 1].double().numpy()
-        kh = k[:, :, h:h + 1].double().numpy()
-        vh = v[:, :, h:h + 1].double().numpy()
+    Setup (untimed): the oracle's own mask and float64, tile-ordered copies of
+    Q, K, V per head.  ``run(budget_s)`` evaluates random query blocks until about
+    budget_s seconds of oracle work and returns (effective TFLOP/s, sample text).
+    """
+
+    def __init__(self, w, q, k, v):
+        import numpy as np
+        import oracle as O
+        self.w, self.O, self.np = w, O, np
+        t0 = time.perf_counter()
         if w.tile is not None:
-            qh = O.tile_permute(qh, perm, n_pad)[:, :w.nq]
-            kh = O.tile_permute(kh, perm, n_pad)[:, :w.nk]
-            vh = O.tile_permute(vh, perm, n_pad)[:, :w.nk]
-        heads64.append((qh, kh, vh))
-    prep = time.perf_counter() - t0
-    flops = 0.0
-    done = 0
-    t1 = time.perf_counter()
-    for qb in order:
-        rows = np.arange(qb * w.block, min((qb + 1) * w.block, w.nq))
-        for qh, kh, vh in heads64:
-            O.block_sparse_attention(qh, kh, vh, mask, w.block, w.block, rows=rows)
-        kept = np.nonzero(mask[0, qb])[0]
-        nkeys = sum(min((kb + 1) * w.block, w.nk) - kb * w.block for kb in kept)
-        flops += 4.0 * D * len(rows) * nkeys * w.heads
-        done += 1
-        if time.perf_counter() - t1 > budget_s:
-            break
-    el = time.perf_counter() - t1
-    sample = (f"{done} random query blocks x {w.heads} heads of {w.name} "
-              f"({flops / 1e12:.4f} effective TFLOP), float64 oracle, {el:.1f} s "
-              f"(+{prep:.1f} s mask/permute/upcast setup, untimed)")
-    return flops / el / 1e12, sample
+            perm = O.tile_order(w.grid, w.tile)
+            n_pad = math.ceil(w.n_tokens / w.block) * w.block
+            tg = tuple(math.ceil(g / t) for g, t in zip(w.grid, w.tile))
+        if w.mask == "sta":
+            self.mask = O.sta_tile_mask(tg, w.window)[None]
+        elif w.mask == "radial":
+            self.mask = O.radial_block_mask_fast(w.nk, w.tokens_per_frame, w.block)[None]
+        else:
+            raise ValueError("cpu baseline implemented for static-mask workloads")
+        self.heads64 = []
+        for h in range(w.heads):
+            qh = q[:, :, h:h + 1].double().numpy()
+            kh = k[:, :, h:h + 1].double().numpy()
+            vh = v[:, :, h:h + 1].double().numpy()
+            if w.tile is not None:
+                qh = O.tile_permute(qh, perm, n_pad)[:, :w.nq]
+                kh = O.tile_permute(kh, perm, n_pad)[:, :w.nk]
+                vh = O.tile_permute(vh, perm, n_pad)[:, :w.nk]
+            self.heads64.append((qh, kh, vh))
+        self.setup_s = time.perf_counter() - t0
+        self.rng = np.random.default_rng(7)
+
+    def run(self, budget_s: float):
+        w, O, np = self.w, self.O, self.np
+        QB = math.ceil(w.nq / w.block)
+        flops, done = 0.0, 0
+        t1 = time.perf_counter()
+        for qb in self.rng.permutation(QB):
+            rows = np.arange(qb * w.block, min((qb + 1) * w.block, w.nq))
+            for qh, kh, vh in self.heads64:
+                O.block_sparse_attention(qh, kh, vh, self.mask, w.block, w.block, rows=rows)
+            kept = np.nonzero(self.mask[0, qb])[0]
+            nkeys = sum(min((kb + 1) * w.block, w.nk) - kb * w.block for kb in kept)
+            flops += 4.0 * w.head_dim * len(rows) * nkeys * w.heads
+            done += 1
+            if time.perf_counter() - t1 > budget_s:
+                break
+        el = time.perf_counter() - t1
+        sample = (f"{done} random query blocks x {w.heads} heads of {w.name} "
+                  f"({flops / 1e12:.4f} effective TFLOP), float64 oracle, {el:.1f} s "
+                  f"(+{self.setup_s:.1f} s untimed setup: oracle mask, tile permute, upcast)")
+        return flops / el / 1e12, sample
 
 
 def run_reference(args, w):
@@ -181,20 +187,22 @@ def run_reference(args, w):
         return 0
     from block_sparse_attention_tokens_b200 import synth
     q, k, v, _ = synth.workload_inputs(w)
-    budget = max(2.0, min(20.0, 60.0 / max(1, args.steps + args.warmup)))
+    sampler = OracleSample(w, q, k, v)
+    n = max(1, args.steps + args.warmup)
+    budget = max(0.5, min(10.0, 90.0 / n))
     vals = []
     sample = ""
-    for i in range(args.warmup + args.steps):
-        val, sample = oracle_sample_rate(w, q, k, v, budget)
+    for i in range(n):
+        val, sample = sampler.run(budget)
         if i >= args.warmup:
             vals.append(val)
-    value = statistics.median(vals)
+    value = statistics.median(vals) if vals else val
     line = {"impl": "reference", "metric": "block-sparse attention effective TFLOP/s (path step)",
             "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "higher_is_better": True, "dtype": "f64",
             "data": "synthetic", "config": workload_config(w),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_cores(),
-                             "kind": "oracle", "sample": sample},
+                             "kind": "oracle", "sample": f"per step: {sample}"},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
@@ -342,7 +350,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        val, sample = oracle_sample_rate(w, q_h, k_h, v_h, args.cpu_budget)
+        val, sample = OracleSample(w, q_h, k_h, v_h).run(args.cpu_budget)
         cpu = {"value": val, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
                "sample": sample}
 
