@@ -14,10 +14,10 @@
 //   warps 4-7  softmax for q-tile slot 1
 //   warp  8    TMA producer: Q tiles, K/V tiles into an NSTAGE ring
 //   warp  9    MMA issuer (one thread), also owns the TMEM allocation
-// Each CTA processes "units" of two 128-row q-tiles (slots) in lock-step rounds:
-//   round r:  S_0 = Q_0 K_0r^T, S_1 = Q_1 K_1r^T, O_0 += P_0 V_0r, O_1 += P_1 V_1r
-// so that while one slot's softmax runs on the CUDA cores the tensor core works
-// on the other slot.  TMEM (512 columns): S_0 | S_1 | O_0 | O_1, 128 columns
+// Each CTA processes "units" of two 128-row q-tiles (slots) in lock-step rounds;
+// the MMA warp issues, per round r and slot s, O_s += P_s V_s,r then
+// S_s = Q_s K_s,r+1^T, alternating slots, so that while one slot's softmax runs
+// on the CUDA cores the tensor core works on the other slot.  TMEM (512 columns): S_0 | S_1 | O_0 | O_1, 128 columns
 // each; P (bf16) is written over the first half of its slot's S columns and is
 // the TMEM A operand of the P.V MMA.  The K/V ring stages are released by
 // tcgen05.commit when the MMA that read them completes.
@@ -239,14 +239,28 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kLoadWarp) {
     // ------------------------------------------------------------ producer
+    // Ring order (must match the MMA issuer): per unit, K of step 0 for each slot,
+    // then per round r and slot s: V(s, r) followed by K(s, r + 1).
     if (lane == 0) {
       int st = 0;
       uint32_t ph = 0;
       uint32_t qph[2] = {0, 0};
-      int last_fill_stage_phase[C::NSTAGE];
-      for (int i = 0; i < C::NSTAGE; ++i) last_fill_stage_phase[i] = -1;
+      uint32_t filled = 0, fill_phase = 0;  // per stage: ever filled / phase of the last fill
       int q_filled[2] = {-1, -1};
       bool ok = true;
+      auto load_tile = [&](const CUtensorMap* map, const Item& itm, int step) -> bool {
+        if (!mbar_wait(EMPTY(st), ph ^ 1u, abort_flag, p.status, p.timeout_ns)) return false;
+        const int kt = static_cast<int>(__ldg(itm.ent + step) & 0x0FFFFFFFu);
+        mbar_expect_tx(FULL(st), C::TILE_BYTES);
+#pragma unroll
+        for (int c = 0; c < C::KCH; ++c)
+          tma_load_4d(sRing + st * C::TILE_BYTES + c * C::CHUNK_BYTES, map, FULL(st), 64 * c,
+                      itm.h, kt * kBN, itm.b);
+        filled |= 1u << st;
+        fill_phase = (fill_phase & ~(1u << st)) | (ph << st);
+        if (++st == C::NSTAGE) { st = 0; ph ^= 1u; }
+        return true;
+      };
       for (int u = blockIdx.x; u < p.total_units && ok; u += gridDim.x) {
         Item it[2] = {get_item(p, 2 * u), get_item(p, 2 * u + 1)};
         for (int s = 0; s < 2 && ok; ++s) {
@@ -260,36 +274,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_4d(sQ + s * C::TILE_BYTES + c * C::CHUNK_BYTES, &tmQ, QFULL(s), 64 * c,
                         it[s].h, it[s].qt * kBM, it[s].b);
         }
+        for (int s = 0; s < 2 && ok; ++s)
+          if (it[s].n > 0) ok = load_tile(&tmK, it[s], 0);
         const int R = max(it[0].n, it[1].n);
         for (int r = 0; r < R && ok; ++r) {
-          for (int kv = 0; kv < 2 && ok; ++kv) {
-            for (int s = 0; s < 2; ++s) {
-              if (r >= it[s].n) continue;
-              ok = mbar_wait(EMPTY(st), ph ^ 1u, abort_flag, p.status, p.timeout_ns);
-              if (!ok) break;
-              const int kt = static_cast<int>(__ldg(it[s].ent + r) & 0x0FFFFFFFu);
-              mbar_expect_tx(FULL(st), C::TILE_BYTES);
-              const CUtensorMap* map = kv == 0 ? &tmK : &tmV;
-              for (int c = 0; c < C::KCH; ++c)
-                tma_load_4d(sRing + st * C::TILE_BYTES + c * C::CHUNK_BYTES, map, FULL(st),
-                            64 * c, it[s].h, kt * kBN, it[s].b);
-              last_fill_stage_phase[st] = static_cast<int>(ph);
-              if (++st == C::NSTAGE) { st = 0; ph ^= 1u; }
-            }
+          for (int s = 0; s < 2 && ok; ++s) {
+            if (r >= it[s].n) continue;
+            ok = load_tile(&tmV, it[s], r);
+            if (ok && r + 1 < it[s].n) ok = load_tile(&tmK, it[s], r + 1);
           }
         }
       }
       // Do not leave the CTA while a TMA copy into its shared memory may be in flight.
       for (int i = 0; i < C::NSTAGE; ++i)
-        if (last_fill_stage_phase[i] >= 0)
-          mbar_wait_drain(FULL(i), static_cast<uint32_t>(last_fill_stage_phase[i]), p.status,
-                          p.timeout_ns);
+        if (filled & (1u << i))
+          mbar_wait_drain(FULL(i), (fill_phase >> i) & 1u, p.status, p.timeout_ns);
       for (int s = 0; s < 2; ++s)
         if (q_filled[s] >= 0)
           mbar_wait_drain(QFULL(s), static_cast<uint32_t>(q_filled[s]), p.status, p.timeout_ns);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
+    // Per slot the tensor core alternates P.V of step r and Q.K^T of step r + 1, the
+    // two slots interleaved: while slot A's softmax runs, slot B's P.V and next
+    // Q.K^T execute, and the reverse.
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, 0, 1);
@@ -297,51 +305,55 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t ph = 0;
       uint32_t qph[2] = {0, 0}, pph[2] = {0, 0};
       bool ok = true;
+      auto issue_qk = [&](int s, int step, int n) -> bool {
+        if (!mbar_wait(FULL(st), ph, abort_flag, p.status, p.timeout_ns)) return false;
+        tc_fence_after();
+        const uint32_t qa = sQ + s * C::TILE_BYTES;
+        const uint32_t kb = sRing + st * C::TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::CHUNK_BYTES + (kk & 3) * 32;
+          mma_ss(tmem + s * 128, smem_desc_sw128(qa + off, 16, 1024),
+                 smem_desc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(EMPTY(st));
+        mma_commit(SFULL(s));
+        if (step == n - 1) mma_commit(QEMPTY(s));
+        if (++st == C::NSTAGE) { st = 0; ph ^= 1u; }
+        return true;
+      };
+      auto issue_pv = [&](int s, int step, int n) -> bool {
+        if (!mbar_wait(FULL(st), ph, abort_flag, p.status, p.timeout_ns)) return false;
+        if (!mbar_wait(PREADY(s), pph[s], abort_flag, p.status, p.timeout_ns)) return false;
+        pph[s] ^= 1u;
+        tc_fence_after();
+        const uint32_t vb = sRing + st * C::TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          mma_ts(tmem + 256 + s * 128, tmem + s * 128 + kk * 8,
+                 smem_desc_sw128(vb + kk * 16 * 128, C::CHUNK_BYTES, 1024), idesc_pv,
+                 (step > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(EMPTY(st));
+        if (step == n - 1) mma_commit(ODONE(s));
+        if (++st == C::NSTAGE) { st = 0; ph ^= 1u; }
+        return true;
+      };
       for (int u = blockIdx.x; u < p.total_units && ok; u += gridDim.x) {
         Item it[2] = {get_item(p, 2 * u), get_item(p, 2 * u + 1)};
+        for (int s = 0; s < 2 && ok; ++s) {
+          if (it[s].n <= 0) continue;
+          ok = mbar_wait(QFULL(s), qph[s], abort_flag, p.status, p.timeout_ns);
+          if (!ok) break;
+          qph[s] ^= 1u;
+          ok = issue_qk(s, 0, it[s].n);
+        }
         const int R = max(it[0].n, it[1].n);
         for (int r = 0; r < R && ok; ++r) {
-          for (int s = 0; s < 2; ++s) {  // S_s = Q_s K^T
+          for (int s = 0; s < 2 && ok; ++s) {
             if (r >= it[s].n) continue;
-            if (r == 0) {
-              ok = mbar_wait(QFULL(s), qph[s], abort_flag, p.status, p.timeout_ns);
-              if (!ok) break;
-              qph[s] ^= 1u;
-            }
-            ok = mbar_wait(FULL(st), ph, abort_flag, p.status, p.timeout_ns);
-            if (!ok) break;
-            tc_fence_after();
-            const uint32_t qa = sQ + s * C::TILE_BYTES;
-            const uint32_t kb = sRing + st * C::TILE_BYTES;
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t off = (kk >> 2) * C::CHUNK_BYTES + (kk & 3) * 32;
-              mma_ss(tmem + s * 128, smem_desc_sw128(qa + off, 16, 1024),
-                     smem_desc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
-            }
-            mma_commit(EMPTY(st));
-            mma_commit(SFULL(s));
-            if (r == it[s].n - 1) mma_commit(QEMPTY(s));
-            if (++st == C::NSTAGE) { st = 0; ph ^= 1u; }
-          }
-          for (int s = 0; s < 2 && ok; ++s) {  // O_s += P_s V
-            if (r >= it[s].n) continue;
-            ok = mbar_wait(FULL(st), ph, abort_flag, p.status, p.timeout_ns);
-            if (!ok) break;
-            ok = mbar_wait(PREADY(s), pph[s], abort_flag, p.status, p.timeout_ns);
-            if (!ok) break;
-            pph[s] ^= 1u;
-            tc_fence_after();
-            const uint32_t vb = sRing + st * C::TILE_BYTES;
-#pragma unroll
-            for (int kk = 0; kk < kBN / 16; ++kk) {
-              mma_ts(tmem + 256 + s * 128, tmem + s * 128 + kk * 8,
-                     smem_desc_sw128(vb + kk * 16 * 128, C::CHUNK_BYTES, 1024), idesc_pv,
-                     (r > 0 || kk > 0) ? 1u : 0u);
-            }
-            mma_commit(EMPTY(st));
-            if (r == it[s].n - 1) mma_commit(ODONE(s));
-            if (++st == C::NSTAGE) { st = 0; ph ^= 1u; }
+            ok = issue_pv(s, r, it[s].n);
+            if (ok && r + 1 < it[s].n) ok = issue_qk(s, r + 1, it[s].n);
           }
         }
       }
@@ -365,68 +377,156 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int qrow = me.qt * kBM + row;
       float m_used = -INFINITY, l = 0.f;
       const int qh = row >> 6;
+      uint32_t ent_next = me.n > 0 ? __ldg(me.ent) : 0u;
       for (int j = 0; j < me.n; ++j) {
+        const uint32_t ent = ent_next;
+        if (j + 1 < me.n) ent_next = __ldg(me.ent + j + 1);
         ok = mbar_wait(SFULL(s), sph, abort_flag, p.status, p.timeout_ns);
         if (!ok) break;
         sph ^= 1u;
         tc_fence_after();
-        uint32_t sr[kBN];
-        tmem_ld32x32b_x128(tS, sr);
-        float sv[kBN];
-#pragma unroll
-        for (int c = 0; c < kBN; ++c) sv[c] = __uint_as_float(sr[c]);
-        const uint32_t ent = __ldg(me.ent + j);
         const int kt = static_cast<int>(ent & 0x0FFFFFFFu);
         const uint32_t bits = ent >> 28;
         const int kvalid = p.nk - kt * kBN;  // keys of this tile that exist
-        if (bits != 0xFu || kvalid < kBN) {
-          const bool lo_ok = (bits >> (qh * 2)) & 1u, hi_ok = (bits >> (qh * 2 + 1)) & 1u;
-#pragma unroll
-          for (int c = 0; c < kBN; ++c) {
-            const bool keep = (c < 64 ? lo_ok : hi_ok) && c < kvalid;
-            if (!keep) sv[c] = -INFINITY;
+        const bool ragged = kvalid < kBN;
+        // Quadrant mask of 64-token blocks: each warp's 32 rows lie in one q-half, so
+        // whether a 64-column half is kept is uniform across the warp.
+        const bool lo_ok = (bits >> (qh * 2)) & 1u, hi_ok = (bits >> (qh * 2 + 1)) & 1u;
+        float lsum = 0.f;
+        bool done = false;
+        // Fast path (every tile after the first, running max finite, no ragged tail):
+        // one pass over S against the running max, next 32 columns loading while the
+        // current ones are exponentiated; P stays in registers until it is known
+        // that no score exceeds the running max by more than the threshold.
+        if (j > 0 && !ragged && __all_sync(0xffffffffu, m_used != -INFINITY)) {
+          uint32_t pk[64];
+          float lp[4] = {0.f, 0.f, 0.f, 0.f};
+          float xmax = -INFINITY;
+          uint32_t ra[32], rb[32];
+          if (lo_ok) {
+            tmem_ld32x32b_x32_nowait(tS, ra);
+            tmem_wait_ld_x32(ra);
           }
-        }
-        float mt = sv[0];
 #pragma unroll
-        for (int c = 1; c < kBN; ++c) mt = fmaxf(mt, sv[c]);
-        mt *= sl2;
-        const float m_new = fmaxf(m_used, mt);
-        if (j == 0) {
-          m_used = m_new;
-        } else {
-          const bool need = m_new > m_used + kRescaleThreshold;
-          const bool has_o = m_used != -INFINITY;
-          if (__any_sync(0xffffffffu, need && has_o)) {
-            const float alpha = (need && has_o) ? fast_exp2(m_used - m_new) : 1.0f;
+          for (int c = 0; c < 4; ++c) {
+            const bool cur_ok = c < 2 ? lo_ok : hi_ok;
+            const bool nxt_ok = c + 1 < 2 ? lo_ok : hi_ok;
+            uint32_t* cur = (c & 1) ? rb : ra;
+            uint32_t* nxt = (c & 1) ? ra : rb;
+            if (c < 3 && nxt_ok) tmem_ld32x32b_x32_nowait(tS + (c + 1) * 32, nxt);
+            if (cur_ok) {
 #pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 32) {
-              uint32_t ov[32];
-              tmem_ld32x32b_x32(tO + c0, ov);
+              for (int i = 0; i < 16; ++i) {
+                const float x0 = fmaf(__uint_as_float(cur[2 * i]), sl2, -m_used);
+                const float x1 = fmaf(__uint_as_float(cur[2 * i + 1]), sl2, -m_used);
+                xmax = fmaxf(xmax, fmaxf(x0, x1));
+                const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+                lp[(2 * i) & 3] += p0;
+                lp[(2 * i + 1) & 3] += p1;
+                __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+                pk[c * 16 + i] = *reinterpret_cast<uint32_t*>(&h2);
+              }
+            } else {
 #pragma unroll
-              for (int i = 0; i < 32; ++i)
-                ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-              tmem_st32x32b_x32(tO + c0, ov);
+              for (int i = 0; i < 16; ++i) pk[c * 16 + i] = 0u;
             }
-            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-            l *= alpha;
+            if (c < 3 && nxt_ok) tmem_wait_ld_x32(nxt);
           }
-          if (need) m_used = m_new;
-        }
-        const float msub = m_used == -INFINITY ? 0.f : m_used;
+          if (!__any_sync(0xffffffffu, xmax > kRescaleThreshold)) {
 #pragma unroll
-        for (int c0 = 0; c0 < kBN; c0 += 32) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float p0 = fast_exp2(fmaf(sv[c0 + 2 * i], sl2, -msub));
-            const float p1 = fast_exp2(fmaf(sv[c0 + 2 * i + 1], sl2, -msub));
-            l += p0 + p1;
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-            pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+            for (int c = 0; c < 4; ++c) tmem_st32x32b_x16(tS + c * 16, pk + c * 16);
+            lsum = (lp[0] + lp[1]) + (lp[2] + lp[3]);
+            done = true;
           }
-          tmem_st32x32b_x16(tS + c0 / 2, pk);
         }
+        float alpha = 1.0f;
+        bool rescale_o = false;
+        if (!done) {
+          // General path: pass 1 takes the tile's row max, then the running max is
+          // moved lazily (only when it grew by more than the threshold; O in TMEM and
+          // l are then scaled by alpha -- O holds data only once a finite base has
+          // been used), pass 2 writes P.  Handles the first tile, masked quadrants,
+          // the ragged key tail and rows whose max jumped.
+          float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+          for (int c0 = 0; c0 < kBN; c0 += 64) {
+            const bool half_ok = c0 < 64 ? lo_ok : hi_ok;
+            if (!half_ok) continue;
+            uint32_t sr[64];
+            tmem_ld32x32b_x64(tS + c0, sr);
+            if (!ragged) {
+#pragma unroll
+              for (int i = 0; i < 64; ++i) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(sr[i]));
+            } else {
+#pragma unroll
+              for (int i = 0; i < 64; ++i)
+                if (c0 + i < kvalid) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(sr[i]));
+            }
+          }
+          const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
+          const float m_new = fmaxf(m_used, mt);
+          if (j == 0) {
+            m_used = m_new;
+          } else if (m_new > m_used + kRescaleThreshold) {
+            if (m_used != -INFINITY) {
+              alpha = fast_exp2(m_used - m_new);
+              rescale_o = true;
+            }
+            m_used = m_new;
+          }
+          const float msub = m_used == -INFINITY ? 0.f : m_used;
+          float lp[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int c0 = 0; c0 < kBN; c0 += 32) {
+            const bool half_ok = c0 < 64 ? lo_ok : hi_ok;
+            uint32_t pk[16];
+            if (!half_ok) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) pk[i] = 0u;
+            } else {
+              uint32_t sr[32];
+              tmem_ld32x32b_x32(tS + c0, sr);
+              if (!ragged) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                  const float p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * i]), sl2, -msub));
+                  const float p1 = fast_exp2(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -msub));
+                  lp[(2 * i) & 3] += p0;
+                  lp[(2 * i + 1) & 3] += p1;
+                  __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+                  pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+                }
+              } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                  const int c = c0 + 2 * i;
+                  const float p0 =
+                      c < kvalid ? fast_exp2(fmaf(__uint_as_float(sr[2 * i]), sl2, -msub)) : 0.f;
+                  const float p1 = c + 1 < kvalid
+                                       ? fast_exp2(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -msub))
+                                       : 0.f;
+                  lp[(2 * i) & 3] += p0;
+                  lp[(2 * i + 1) & 3] += p1;
+                  __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+                  pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+                }
+              }
+            }
+            tmem_st32x32b_x16(tS + c0 / 2, pk);
+          }
+          lsum = (lp[0] + lp[1]) + (lp[2] + lp[3]);
+        }
+        if (__any_sync(0xffffffffu, rescale_o)) {  // rare: O is idle until P is signalled
+#pragma unroll 1
+          for (int c0 = 0; c0 < D; c0 += 16) {
+            uint32_t ov[16];
+            tmem_ld32x32b_x16(tO + c0, ov);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+            tmem_st32x32b_x16(tO + c0, ov);
+          }
+        }
+        l = fmaf(l, alpha, lsum);
         asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
         tc_fence_before();
         __syncwarp();

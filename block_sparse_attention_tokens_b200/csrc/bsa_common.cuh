@@ -184,6 +184,23 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, in
          | (static_cast<uint32_t>(M >> 4) << 24);// M / 16
 }
 
+// 2^x on the FMA/ALU pipes (no MUFU), for finite x <= 64: Cody-Waite style
+// reduction x = n + f with n = round(x) obtained by the 1.5 * 2^23 rounding
+// constant, f in [-0.5, 0.5]; 2^f by a cubic fitted here to 2^f on [-0.5, 0.5]
+// for least maximum relative error (max rel. error 7.8e-5, below the 2^-9
+// spacing of the bfloat16 values it feeds); the exponent n is added to the bit
+// pattern.  x is clamped at -125 so the result stays a normal float (>= 2^-125.5).
+__device__ __forceinline__ float poly_exp2(float x) {
+  x = fmaxf(x, -125.0f);
+  const float round_const = 12582912.0f;  // 1.5 * 2^23
+  const float t = x + round_const;
+  const float f = x - (t - round_const);
+  float p = fmaf(0.055089012f, f, 0.24260408f);
+  p = fmaf(p, f, 0.69327617f);
+  p = fmaf(p, f, 0.99992895f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
