@@ -23,6 +23,9 @@ LIB = os.path.join(PKG, "libbsa.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-O3",
          "--expt-relaxed-constexpr", "-I" + os.path.join(ROOT, "include")]
+# Extra nvcc flags (e.g. -DBSA_POLY_EXP2=1 to route part of the attention
+# exponentials through the FMA pipe), space separated.
+EXTRA = os.environ.get("BSA_NVCC_FLAGS", "").split()
 
 
 def nvcc() -> str:
@@ -54,7 +57,7 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
         o = os.path.join(BUILD, os.path.basename(s)[:-3] + ".o")
         objs.append(o)
         if force or verbose_ptxas or not _newer(o, [s] + headers):
-            cmd = [nvcc()] + ARCH + FLAGS + (["-Xptxas", "-v"] if verbose_ptxas else []) + \
+            cmd = [nvcc()] + ARCH + FLAGS + EXTRA + (["-Xptxas", "-v"] if verbose_ptxas else []) + \
                 ["-c", s, "-o", o]
             jobs.append(cmd)
     with cf.ThreadPoolExecutor(max_workers=max(1, min(len(jobs), os.cpu_count() or 4))) as ex:

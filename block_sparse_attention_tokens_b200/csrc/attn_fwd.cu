@@ -42,6 +42,14 @@ constexpr int kThreads = 320;
 constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// The fast path keeps the running max while a tile's P sum stays <= 2^12.
+constexpr float kFastSumLimit = 4096.0f;
+// Software 2^x (FMA pipe) for a quarter of the fast-path exponentials, relieving
+// the MUFU, which carries one exponential per 512 tensor FLOPs at head_dim 128.
+#ifndef BSA_POLY_EXP2
+#define BSA_POLY_EXP2 0
+#endif
+constexpr bool kPolyExp2 = BSA_POLY_EXP2 != 0;
 
 template <int D>
 struct Cfg {
@@ -395,13 +403,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         float lsum = 0.f;
         bool done = false;
         // Fast path (every tile after the first, running max finite, no ragged tail):
-        // one pass over S against the running max, next 32 columns loading while the
-        // current ones are exponentiated; P stays in registers until it is known
-        // that no score exceeds the running max by more than the threshold.
+        // one pass over S against the running max, the next 32 columns loading while
+        // the current ones are exponentiated; P stays in registers until the tile's
+        // P sum is known to be <= kFastSumLimit, which bounds every P (an overflow
+        // to inf fails the test too).  Otherwise the general path below redoes the
+        // tile from S, which is still intact in TMEM.
         if (j > 0 && !ragged && __all_sync(0xffffffffu, m_used != -INFINITY)) {
           uint32_t pk[64];
-          float lp[4] = {0.f, 0.f, 0.f, 0.f};
-          float xmax = -INFINITY;
+          float2 lpa = make_float2(0.f, 0.f), lpb = make_float2(0.f, 0.f);
+          const float2 sl2x2 = make_float2(sl2, sl2);
+          const float2 negm = make_float2(-m_used, -m_used);
           uint32_t ra[32], rb[32];
           if (lo_ok) {
             tmem_ld32x32b_x32_nowait(tS, ra);
@@ -417,13 +428,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (cur_ok) {
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
-                const float x0 = fmaf(__uint_as_float(cur[2 * i]), sl2, -m_used);
-                const float x1 = fmaf(__uint_as_float(cur[2 * i + 1]), sl2, -m_used);
-                xmax = fmaxf(xmax, fmaxf(x0, x1));
-                const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-                lp[(2 * i) & 3] += p0;
-                lp[(2 * i + 1) & 3] += p1;
-                __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+                const float2 x = ffma2(make_float2(__uint_as_float(cur[2 * i]),
+                                                   __uint_as_float(cur[2 * i + 1])),
+                                       sl2x2, negm);
+                float2 pp;
+                if (kPolyExp2 && (i & 3) == 3) {
+                  pp.x = poly_exp2(x.x);
+                  pp.y = poly_exp2(x.y);
+                } else {
+                  pp.x = fast_exp2(x.x);
+                  pp.y = fast_exp2(x.y);
+                }
+                if (i & 1) lpb = fadd2(lpb, pp); else lpa = fadd2(lpa, pp);
+                __nv_bfloat162 h2 = __floats2bfloat162_rn(pp.x, pp.y);
                 pk[c * 16 + i] = *reinterpret_cast<uint32_t*>(&h2);
               }
             } else {
@@ -432,10 +449,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (c < 3 && nxt_ok) tmem_wait_ld_x32(nxt);
           }
-          if (!__any_sync(0xffffffffu, xmax > kRescaleThreshold)) {
+          const float tile_sum = (lpa.x + lpa.y) + (lpb.x + lpb.y);
+          if (__all_sync(0xffffffffu, tile_sum <= kFastSumLimit)) {
 #pragma unroll
             for (int c = 0; c < 4; ++c) tmem_st32x32b_x16(tS + c * 16, pk + c * 16);
-            lsum = (lp[0] + lp[1]) + (lp[2] + lp[3]);
+            lsum = tile_sum;
             done = true;
           }
         }
