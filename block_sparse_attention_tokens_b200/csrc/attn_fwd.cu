@@ -51,6 +51,20 @@ constexpr float kFastSumLimit = 4096.0f;
 #endif
 constexpr bool kPolyExp2 = BSA_POLY_EXP2 != 0;
 
+// Optional phase timestamps (SM clock) of CTA 0 for latency analysis; compiled
+// only with -DBSA_TRACE and read back with bsa_trace_dump().
+#ifdef BSA_TRACE
+__device__ unsigned long long g_bsa_trace[1 << 16];
+#define BSA_TRACE_AT(idx) \
+  do {                    \
+    if (blockIdx.x == 0 && (idx) < (1 << 16)) g_bsa_trace[(idx)] = clock64(); \
+  } while (0)
+#else
+#define BSA_TRACE_AT(idx) \
+  do {                    \
+  } while (0)
+#endif
+
 template <int D>
 struct Cfg {
   static constexpr int KCH = D / 64;                  // 128-byte swizzle chunks per row
@@ -99,6 +113,11 @@ __device__ __forceinline__ Item get_item(const AttnParams& p, int it) {
   r.n = p.cnt[mh * p.LR + lr];
   r.ent = p.entries + static_cast<long long>(p.row_ptr[mh * p.QB + first_qb]) * p.expand;
   return r;
+}
+
+// Both slots of a unit read the same K/V stream: same batch, head and kept list.
+__device__ __forceinline__ bool shares_kv(const Item& a, const Item& b) {
+  return a.n > 0 && b.n == a.n && a.ent == b.ent && a.b == b.b && a.h == b.h;
 }
 
 // ---------------------------------------------------------------------------
@@ -256,8 +275,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t filled = 0, fill_phase = 0;  // per stage: ever filled / phase of the last fill
       int q_filled[2] = {-1, -1};
       bool ok = true;
+      int gld = 0;
+      (void)gld;
       auto load_tile = [&](const CUtensorMap* map, const Item& itm, int step) -> bool {
+        const int tix = 32768 + min(gld++, 8191) * 2;
+        BSA_TRACE_AT(tix + 0);
         if (!mbar_wait(EMPTY(st), ph ^ 1u, abort_flag, p.status, p.timeout_ns)) return false;
+        BSA_TRACE_AT(tix + 1);
         const int kt = static_cast<int>(__ldg(itm.ent + step) & 0x0FFFFFFFu);
         mbar_expect_tx(FULL(st), C::TILE_BYTES);
 #pragma unroll
@@ -281,6 +305,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < C::KCH; ++c)
             tma_load_4d(sQ + s * C::TILE_BYTES + c * C::CHUNK_BYTES, &tmQ, QFULL(s), 64 * c,
                         it[s].h, it[s].qt * kBM, it[s].b);
+        }
+        if (shares_kv(it[0], it[1])) {  // one K/V stream read by both slots
+          const int n = it[0].n;
+          ok = ok && load_tile(&tmK, it[0], 0);
+          for (int r = 0; r < n && ok; ++r) {
+            ok = load_tile(&tmV, it[0], r);
+            if (ok && r + 1 < n) ok = load_tile(&tmK, it[0], r + 1);
+          }
+          continue;
         }
         for (int s = 0; s < 2 && ok; ++s)
           if (it[s].n > 0) ok = load_tile(&tmK, it[s], 0);
@@ -313,55 +346,117 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t ph = 0;
       uint32_t qph[2] = {0, 0}, pph[2] = {0, 0};
       bool ok = true;
-      auto issue_qk = [&](int s, int step, int n) -> bool {
+      int gop = 0;
+      (void)gop;
+      // Descriptors are built once; per MMA only the 14-bit start-address field
+      // (16-byte units, shared memory < 256 KB so no carry) moves by a constant.
+      const uint64_t dq0 = smem_desc_sw128(sQ, 16, 1024);
+      const uint64_t dk0 = smem_desc_sw128(sRing, 16, 1024);
+      const uint64_t dv0 = smem_desc_sw128(sRing, C::CHUNK_BYTES, 1024);
+      constexpr uint32_t kTileUnits = C::TILE_BYTES >> 4;
+      // Wait for the next ring stage in fill order and return its index.
+      auto acquire = [&](int& stage) -> bool {
+        const int tix = 16384 + min(gop++, 4095) * 4;
+        BSA_TRACE_AT(tix + 0);
         if (!mbar_wait(FULL(st), ph, abort_flag, p.status, p.timeout_ns)) return false;
-        tc_fence_after();
-        const uint32_t qa = sQ + s * C::TILE_BYTES;
-        const uint32_t kb = sRing + st * C::TILE_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::CHUNK_BYTES + (kk & 3) * 32;
-          mma_ss(tmem + s * 128, smem_desc_sw128(qa + off, 16, 1024),
-                 smem_desc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(EMPTY(st));
-        mma_commit(SFULL(s));
-        if (step == n - 1) mma_commit(QEMPTY(s));
+        BSA_TRACE_AT(tix + 1);
+        stage = st;
         if (++st == C::NSTAGE) { st = 0; ph ^= 1u; }
         return true;
       };
-      auto issue_pv = [&](int s, int step, int n) -> bool {
-        if (!mbar_wait(FULL(st), ph, abort_flag, p.status, p.timeout_ns)) return false;
+      // S_s = Q_s K^T, K in ring stage `stage`.
+      auto qk = [&](int s, int stage) {
+        tc_fence_after();
+        const uint64_t da = dq0 + static_cast<uint64_t>(s * kTileUnits);
+        const uint64_t db = dk0 + static_cast<uint64_t>(stage * kTileUnits);
+        const uint32_t dt = tmem + s * 128;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t off =
+              static_cast<uint64_t>((((kk >> 2) * C::CHUNK_BYTES) + (kk & 3) * 32) >> 4);
+          mma_ss(dt, da + off, db + off, idesc_qk, kk > 0 ? 1u : 0u);
+        }
+      };
+      // O_s (+)= P_s V once slot s's softmax has published P.
+      auto pv = [&](int s, int stage, int step) -> bool {
         if (!mbar_wait(PREADY(s), pph[s], abort_flag, p.status, p.timeout_ns)) return false;
         pph[s] ^= 1u;
         tc_fence_after();
-        const uint32_t vb = sRing + st * C::TILE_BYTES;
+        const uint64_t db = dv0 + static_cast<uint64_t>(stage * kTileUnits);
+        const uint32_t dt = tmem + 256 + s * 128;
+        const uint32_t ta = tmem + s * 128;
+        const uint32_t acc0 = step > 0 ? 1u : 0u;
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          mma_ts(tmem + 256 + s * 128, tmem + s * 128 + kk * 8,
-                 smem_desc_sw128(vb + kk * 16 * 128, C::CHUNK_BYTES, 1024), idesc_pv,
-                 (step > 0 || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(EMPTY(st));
-        if (step == n - 1) mma_commit(ODONE(s));
-        if (++st == C::NSTAGE) { st = 0; ph ^= 1u; }
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          mma_ts(dt, ta + kk * 8, db + static_cast<uint64_t>(kk * (16 * 128 / 16)), idesc_pv,
+                 kk > 0 ? 1u : acc0);
         return true;
       };
       for (int u = blockIdx.x; u < p.total_units && ok; u += gridDim.x) {
         Item it[2] = {get_item(p, 2 * u), get_item(p, 2 * u + 1)};
+        if (shares_kv(it[0], it[1])) {
+          const int n = it[0].n;
+          int ks = 0, vs = 0;
+          for (int s = 0; s < 2 && ok; ++s) {
+            ok = mbar_wait(QFULL(s), qph[s], abort_flag, p.status, p.timeout_ns);
+            qph[s] ^= 1u;
+          }
+          if (!ok || !acquire(ks)) { ok = false; break; }
+          qk(0, ks);
+          mma_commit(SFULL(0));
+          qk(1, ks);
+          mma_commit(EMPTY(ks));
+          mma_commit(SFULL(1));
+          if (n == 1) { mma_commit(QEMPTY(0)); mma_commit(QEMPTY(1)); }
+          for (int r = 0; r < n && ok; ++r) {
+            const bool more = r + 1 < n;
+            if (!acquire(vs) || !pv(0, vs, r)) { ok = false; break; }
+            if (r == n - 1) mma_commit(ODONE(0));
+            if (more) {
+              if (!acquire(ks)) { ok = false; break; }
+              qk(0, ks);
+              mma_commit(SFULL(0));
+              if (r + 1 == n - 1) mma_commit(QEMPTY(0));
+            }
+            if (!pv(1, vs, r)) { ok = false; break; }
+            mma_commit(EMPTY(vs));
+            if (r == n - 1) mma_commit(ODONE(1));
+            if (more) {
+              qk(1, ks);
+              mma_commit(EMPTY(ks));
+              mma_commit(SFULL(1));
+              if (r + 1 == n - 1) mma_commit(QEMPTY(1));
+            }
+          }
+          continue;
+        }
         for (int s = 0; s < 2 && ok; ++s) {
           if (it[s].n <= 0) continue;
-          ok = mbar_wait(QFULL(s), qph[s], abort_flag, p.status, p.timeout_ns);
+          int ks = 0;
+          ok = mbar_wait(QFULL(s), qph[s], abort_flag, p.status, p.timeout_ns) && acquire(ks);
           if (!ok) break;
           qph[s] ^= 1u;
-          ok = issue_qk(s, 0, it[s].n);
+          qk(s, ks);
+          mma_commit(EMPTY(ks));
+          mma_commit(SFULL(s));
+          if (it[s].n == 1) mma_commit(QEMPTY(s));
         }
         const int R = max(it[0].n, it[1].n);
         for (int r = 0; r < R && ok; ++r) {
           for (int s = 0; s < 2 && ok; ++s) {
-            if (r >= it[s].n) continue;
-            ok = issue_pv(s, r, it[s].n);
-            if (ok && r + 1 < it[s].n) ok = issue_qk(s, r + 1, it[s].n);
+            const int n = it[s].n;
+            if (r >= n) continue;
+            int vs = 0, ks = 0;
+            if (!acquire(vs) || !pv(s, vs, r)) { ok = false; break; }
+            mma_commit(EMPTY(vs));
+            if (r == n - 1) mma_commit(ODONE(s));
+            if (r + 1 < n) {
+              if (!acquire(ks)) { ok = false; break; }
+              qk(s, ks);
+              mma_commit(EMPTY(ks));
+              mma_commit(SFULL(s));
+              if (r + 1 == n - 1) mma_commit(QEMPTY(s));
+            }
           }
         }
       }
@@ -378,6 +473,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tO = tmem + lane_base + 256 + s * 128;
     const float sl2 = p.scale_log2;
     uint32_t sph = 0, oph = 0;
+    int gstep = 0;
+    (void)gstep;
     bool ok = true;
     for (int u = blockIdx.x; u < p.total_units && ok; u += gridDim.x) {
       const Item me = get_item(p, 2 * u + s);
@@ -389,7 +486,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < me.n; ++j) {
         const uint32_t ent = ent_next;
         if (j + 1 < me.n) ent_next = __ldg(me.ent + j + 1);
+        const int tix = (warp & 3) == 0 && lane == 0 ? s * 8192 + min(gstep, 1023) * 8 : (1 << 16);
+        BSA_TRACE_AT(tix + 0);
         ok = mbar_wait(SFULL(s), sph, abort_flag, p.status, p.timeout_ns);
+        BSA_TRACE_AT(tix + 1);
+        ++gstep;
         if (!ok) break;
         sph ^= 1u;
         tc_fence_after();
@@ -418,6 +519,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_ld32x32b_x32_nowait(tS, ra);
             tmem_wait_ld_x32(ra);
           }
+          BSA_TRACE_AT(tix + 4);
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             const bool cur_ok = c < 2 ? lo_ok : hi_ok;
@@ -433,8 +535,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                        sl2x2, negm);
                 float2 pp;
                 if (kPolyExp2 && (i & 3) == 3) {
-                  pp.x = poly_exp2(x.x);
-                  pp.y = poly_exp2(x.y);
+                  pp = poly_exp2x2(x);
                 } else {
                   pp.x = fast_exp2(x.x);
                   pp.y = fast_exp2(x.y);
@@ -449,10 +550,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (c < 3 && nxt_ok) tmem_wait_ld_x32(nxt);
           }
+          BSA_TRACE_AT(tix + 5);
           const float tile_sum = (lpa.x + lpa.y) + (lpb.x + lpb.y);
           if (__all_sync(0xffffffffu, tile_sum <= kFastSumLimit)) {
 #pragma unroll
             for (int c = 0; c < 4; ++c) tmem_st32x32b_x16(tS + c * 16, pk + c * 16);
+            BSA_TRACE_AT(tix + 6);
             lsum = tile_sum;
             done = true;
           }
@@ -545,10 +648,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         l = fmaf(l, alpha, lsum);
+        BSA_TRACE_AT(tix + 2);
         asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(PREADY(s));
+        BSA_TRACE_AT(tix + 3);
       }
       if (!ok) break;
       __nv_bfloat16* orow = p.o + ((static_cast<long long>(me.b) * p.nq + qrow) * p.H + me.h) * D;
@@ -682,6 +787,14 @@ int launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap&
 
 }  // namespace
 }  // namespace bsa
+
+#ifdef BSA_TRACE
+extern "C" int bsa_trace_dump(void* host, size_t bytes) {
+  if (bytes > sizeof(unsigned long long) * (1 << 16)) bytes = sizeof(unsigned long long) * (1 << 16);
+  cudaError_t e = cudaMemcpyFromSymbol(host, bsa::g_bsa_trace, bytes);
+  return e == cudaSuccess ? BSA_OK : bsa::record_cuda_error(e);
+}
+#endif
 
 extern "C" size_t bsa_attn_workspace_size(int batch, int heads, int nq, int nk, int block_q,
                                           int block_k, int list_heads) {

@@ -222,6 +222,31 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
   return d;
 }
 
+__device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// poly_exp2 on two lanes with packed f32x2 arithmetic.
+__device__ __forceinline__ float2 poly_exp2x2(float2 x) {
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  const float2 rc = make_float2(12582912.0f, 12582912.0f);  // 1.5 * 2^23
+  const float2 t = fadd2(x, rc);
+  const float2 f = fsub2(x, fsub2(t, rc));
+  float2 p = ffma2(make_float2(0.055089012f, 0.055089012f), f,
+                   make_float2(0.24260408f, 0.24260408f));
+  p = ffma2(p, f, make_float2(0.69327617f, 0.69327617f));
+  p = ffma2(p, f, make_float2(0.99992895f, 0.99992895f));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
