@@ -24,7 +24,7 @@ EXPORTS = [
     "bsa_status_string", "bsa_last_error_message", "bsa_version", "bsa_tile_permute",
     "bsa_tile_untile", "bsa_sta_mask", "bsa_radial_mask", "bsa_nabla_workspace_size",
     "bsa_nabla_mask", "bsa_mask_compact", "bsa_attn_workspace_size", "bsa_attn_fwd",
-    "bsa_read_status",
+    "bsa_attn_fwd_noalloc", "bsa_read_status",
 ]
 
 
@@ -63,6 +63,9 @@ def load_library(path: str = _LIB_PATH) -> ctypes.CDLL:
         "bsa_attn_fwd": (c_int, [c_void, c_void, c_void] + [c_int] * 7 + [c_void, c_void, c_int,
                                                                            c_float, c_void, c_void,
                                                                            c_void, c_size, c_void]),
+        "bsa_attn_fwd_noalloc": (c_int, [c_void, c_void, c_void] + [c_int] * 7
+                                 + [c_void, c_void, c_int, c_float, c_void, c_void, c_void,
+                                    c_void]),
         "bsa_read_status": (c_int, [c_void, ctypes.POINTER(c_int), c_void]),
     }
     for name, (res, args) in sig.items():
@@ -83,7 +86,7 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
 
 def _check(code: int, where: str):
     if code != 0:
-        detail = load_library().bsa_last_error_message().decode() if code == 4 else ""
+        detail = load_library().bsa_last_error_message().decode() if code in (3, 4) else ""
         raise BsaError(code, where, detail)
 
 
@@ -227,6 +230,33 @@ def bsa_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, row_ptr: tor
                                        float(scale), _ptr(o), _ptr(lse), _ptr(ws), ws.numel(),
                                        _stream()), "bsa_attn_fwd")
     return o, lse, ws
+
+
+def bsa_attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                         row_ptr: torch.Tensor, col_idx: torch.Tensor, block_q: int, block_k: int,
+                         list_heads: int, nq: Optional[int] = None, nk: Optional[int] = None,
+                         scale: float = 0.0, o: Optional[torch.Tensor] = None,
+                         lse: Optional[torch.Tensor] = None,
+                         device_status: Optional[torch.Tensor] = None):
+    """bsa_attn_fwd without a workspace argument: the library's fixed per-device
+    scratch array is used instead (for callers that may not allocate device
+    memory; see include/bsa.h).  Outputs are passed in or created here by the
+    caller-side wrapper.  Returns (o, lse)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (row_ptr, "row_ptr"), (col_idx, "col_idx")):
+        _cuda(t, n)
+    B, _, H, D = q.shape
+    nq = q.shape[1] if nq is None else nq
+    nk = k.shape[1] if nk is None else nk
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, nq), dtype=torch.float32, device=q.device)
+    _check(load_library().bsa_attn_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), B, H, nq, nk, D,
+                                               block_q, block_k, _ptr(row_ptr), _ptr(col_idx),
+                                               list_heads, float(scale), _ptr(o), _ptr(lse),
+                                               _ptr(device_status), _stream()),
+           "bsa_attn_fwd_noalloc")
+    return o, lse
 
 
 def bsa_read_status(ws: torch.Tensor) -> int:

@@ -14,6 +14,11 @@ int record_cuda_error(cudaError_t err) {
   return BSA_ERR_CUDA;
 }
 
+int record_error_message(const char* msg) {
+  std::snprintf(g_last_error, sizeof(g_last_error), "%s", msg);
+  return 0;
+}
+
 int device_sm_count() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;

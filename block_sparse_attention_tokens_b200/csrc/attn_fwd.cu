@@ -868,3 +868,68 @@ extern "C" int bsa_attn_fwd(const void* q, const void* k, const void* v, int bat
   p.timeout_ns = 2000000000ULL;
   return head_dim == 128 ? launch_attn<128>(mq, mk, mv, p, st) : launch_attn<64>(mq, mk, mv, p, st);
 }
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of bsa_attn_fwd.
+//
+// Some callers cannot hand the library a workspace: a host framework that owns
+// every device byte through its own pre-reserved pool and forbids extra CUDA
+// allocations, or a latency-critical serving loop where a cudaMalloc (which may
+// synchronise the device) is not allowed.  For them, the attention workspace
+// lives in a fixed device array that every GPU loading this library holds until
+// the process exits (kNoAllocScratchBytes per device).
+// ---------------------------------------------------------------------------
+namespace bsa {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB per device
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch for the current device, resolved on the
+// first call made with that device current (the host-side name of a __device__
+// array is only a stand-in, never a device address).
+int noalloc_scratch(void** out) {
+  static std::mutex mu;
+  static void* addr[64] = {nullptr};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return record_cuda_error(e);
+  if (dev < 0 || dev >= 64) return BSA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return record_cuda_error(e);
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return BSA_OK;
+}
+
+}  // namespace
+}  // namespace bsa
+
+extern "C" int bsa_attn_fwd_noalloc(const void* q, const void* k, const void* v, int batch,
+                                    int heads, int nq, int nk, int head_dim, int block_q,
+                                    int block_k, const int* row_ptr, const int* col_idx,
+                                    int list_heads, float scale, void* o, float* lse,
+                                    int* device_status, void* stream) {
+  using namespace bsa;
+  const size_t need =
+      bsa_attn_workspace_size(batch, heads, nq, nk, block_q, block_k, list_heads);
+  if (need == 0) return BSA_ERR_INVALID_ARG;
+  if (need > kNoAllocScratchBytes) {
+    record_error_message("bsa_attn_fwd_noalloc: this shape needs a larger workspace than the "
+                         "library's fixed 8 MiB scratch; use bsa_attn_fwd with a caller workspace");
+    return BSA_ERR_WORKSPACE;
+  }
+  void* scratch = nullptr;
+  int rc = noalloc_scratch(&scratch);
+  if (rc != BSA_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  rc = bsa_attn_fwd(q, k, v, batch, heads, nq, nk, head_dim, block_q, block_k, row_ptr, col_idx,
+                    list_heads, scale, o, lse, scratch, kNoAllocScratchBytes, stream);
+  if (rc != BSA_OK || device_status == nullptr) return rc;
+  cudaError_t e = cudaMemcpyAsync(device_status, scratch, sizeof(int), cudaMemcpyDeviceToDevice, st);
+  return e == cudaSuccess ? BSA_OK : record_cuda_error(e);
+}

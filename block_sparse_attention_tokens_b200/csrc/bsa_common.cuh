@@ -19,6 +19,9 @@ namespace bsa {
 // Records the CUDA error text for bsa_last_error_message() and maps it to BSA_ERR_CUDA.
 int record_cuda_error(cudaError_t err);
 
+// Stores a library-side error text for bsa_last_error_message().
+int record_error_message(const char* msg);
+
 // Checks the launch that was just enqueued.
 inline int check_launch() {
   cudaError_t e = cudaGetLastError();

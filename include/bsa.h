@@ -187,6 +187,35 @@ int bsa_attn_fwd(const void* q, const void* k, const void* v, int batch, int hea
                  void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * (d') Block-sparse attention forward that allocates nothing.
+ * No counterpart in the pages: this is a library convenience, not part of the
+ * method.
+ *
+ * For callers that cannot provide or allocate a workspace -- e.g. code running
+ * inside a host framework that owns every device allocation through its own
+ * pre-reserved pool, or a serving loop where a cudaMalloc (which may
+ * synchronise the device) is not permitted.  Same arguments and results as
+ * bsa_attn_fwd, without ws / ws_bytes: the workspace is a fixed 8 MiB device
+ * array inside libbsa.so, which every GPU that loads the library holds until
+ * the process exits.
+ *   - Shapes whose bsa_attn_workspace_size() exceeds 8 MiB are rejected with
+ *     BSA_ERR_WORKSPACE (see bsa_last_error_message()) before any work.
+ *   - The first call made with a given device current looks up that device's
+ *     array address (cudaGetSymbolAddress); make that first call before any
+ *     stream capture.
+ *   - All calls share the one array per device: calls that can overlap on the
+ *     GPU (different streams without ordering) race and must be serialised by
+ *     the caller.  Everything the call needs zeroed is cleared by the call.
+ *   - device_status (optional device int, may be NULL) receives the call's
+ *     device-side status word (a bsa_status value) when the work completes.
+ *   The library itself calls no allocator in this entry point.
+ * ------------------------------------------------------------------------- */
+int bsa_attn_fwd_noalloc(const void* q, const void* k, const void* v, int batch, int heads,
+                         int nq, int nk, int head_dim, int block_q, int block_k,
+                         const int* row_ptr, const int* col_idx, int list_heads, float scale,
+                         void* o, float* lse, int* device_status, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Device status word of a workspace (attention or NABLA): synchronises `stream`,
  * copies the word to *status (a bsa_status value) and clears it.
  * ------------------------------------------------------------------------- */
