@@ -515,40 +515,58 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float2 sl2x2 = make_float2(sl2, sl2);
           const float2 negm = make_float2(-m_used, -m_used);
           uint32_t ra[32], rb[32];
-          if (lo_ok) {
+          auto exp_chunk = [&](const uint32_t* cur, uint32_t* out) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float2 x = ffma2(make_float2(__uint_as_float(cur[2 * i]),
+                                                 __uint_as_float(cur[2 * i + 1])),
+                                     sl2x2, negm);
+              float2 pp;
+              if (kPolyExp2 && (i & 3) == 3) {
+                pp = poly_exp2x2(x);
+              } else {
+                pp.x = fast_exp2(x.x);
+                pp.y = fast_exp2(x.y);
+              }
+              if (i & 1) lpb = fadd2(lpb, pp); else lpa = fadd2(lpa, pp);
+              __nv_bfloat162 h2 = __floats2bfloat162_rn(pp.x, pp.y);
+              out[i] = *reinterpret_cast<uint32_t*>(&h2);
+            }
+          };
+          if (lo_ok && hi_ok) {
+            // Whole tile kept (every Sliding-Tile / radial step): no per-chunk tests.
             tmem_ld32x32b_x32_nowait(tS, ra);
             tmem_wait_ld_x32(ra);
-          }
-          BSA_TRACE_AT(tix + 4);
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const bool cur_ok = c < 2 ? lo_ok : hi_ok;
-            const bool nxt_ok = c + 1 < 2 ? lo_ok : hi_ok;
-            uint32_t* cur = (c & 1) ? rb : ra;
-            uint32_t* nxt = (c & 1) ? ra : rb;
-            if (c < 3 && nxt_ok) tmem_ld32x32b_x32_nowait(tS + (c + 1) * 32, nxt);
-            if (cur_ok) {
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                const float2 x = ffma2(make_float2(__uint_as_float(cur[2 * i]),
-                                                   __uint_as_float(cur[2 * i + 1])),
-                                       sl2x2, negm);
-                float2 pp;
-                if (kPolyExp2 && (i & 3) == 3) {
-                  pp = poly_exp2x2(x);
-                } else {
-                  pp.x = fast_exp2(x.x);
-                  pp.y = fast_exp2(x.y);
-                }
-                if (i & 1) lpb = fadd2(lpb, pp); else lpa = fadd2(lpa, pp);
-                __nv_bfloat162 h2 = __floats2bfloat162_rn(pp.x, pp.y);
-                pk[c * 16 + i] = *reinterpret_cast<uint32_t*>(&h2);
-              }
-            } else {
-#pragma unroll
-              for (int i = 0; i < 16; ++i) pk[c * 16 + i] = 0u;
+            tmem_ld32x32b_x32_nowait(tS + 32, rb);
+            exp_chunk(ra, pk);
+            tmem_wait_ld_x32(rb);
+            tmem_ld32x32b_x32_nowait(tS + 64, ra);
+            exp_chunk(rb, pk + 16);
+            tmem_wait_ld_x32(ra);
+            tmem_ld32x32b_x32_nowait(tS + 96, rb);
+            exp_chunk(ra, pk + 32);
+            tmem_wait_ld_x32(rb);
+            exp_chunk(rb, pk + 48);
+          } else {
+            if (lo_ok) {
+              tmem_ld32x32b_x32_nowait(tS, ra);
+              tmem_wait_ld_x32(ra);
             }
-            if (c < 3 && nxt_ok) tmem_wait_ld_x32(nxt);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const bool cur_ok = c < 2 ? lo_ok : hi_ok;
+              const bool nxt_ok = c + 1 < 2 ? lo_ok : hi_ok;
+              uint32_t* cur = (c & 1) ? rb : ra;
+              uint32_t* nxt = (c & 1) ? ra : rb;
+              if (c < 3 && nxt_ok) tmem_ld32x32b_x32_nowait(tS + (c + 1) * 32, nxt);
+              if (cur_ok) {
+                exp_chunk(cur, pk + c * 16);
+              } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) pk[c * 16 + i] = 0u;
+              }
+              if (c < 3 && nxt_ok) tmem_wait_ld_x32(nxt);
+            }
           }
           BSA_TRACE_AT(tix + 5);
           const float tile_sum = (lpa.x + lpa.y) + (lpb.x + lpb.y);
