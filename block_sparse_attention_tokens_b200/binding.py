@@ -24,7 +24,7 @@ EXPORTS = [
     "bsa_status_string", "bsa_last_error_message", "bsa_version", "bsa_tile_permute",
     "bsa_tile_untile", "bsa_sta_mask", "bsa_radial_mask", "bsa_nabla_workspace_size",
     "bsa_nabla_mask", "bsa_mask_compact", "bsa_attn_workspace_size", "bsa_attn_fwd",
-    "bsa_attn_fwd_noalloc", "bsa_read_status",
+    "bsa_attn_fwd_noalloc", "bsa_read_status", "bsa_tile_permute_pool", "bsa_nabla_select",
 ]
 
 
@@ -67,6 +67,9 @@ def load_library(path: str = _LIB_PATH) -> ctypes.CDLL:
                                  + [c_void, c_void, c_int, c_float, c_void, c_void, c_void,
                                     c_void]),
         "bsa_read_status": (c_int, [c_void, ctypes.POINTER(c_int), c_void]),
+        "bsa_tile_permute_pool": (c_int, [c_void, c_void] + [c_int] * 11 + [c_void, c_void]),
+        "bsa_nabla_select": (c_int, [c_void, c_void] + [c_int] * 5 + [c_float, c_float]
+                             + [c_int] * 3 + [c_void, c_void, c_void, c_void]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -126,6 +129,24 @@ def bsa_tile_untile(y: torch.Tensor, grid: Tuple[int, int, int], tile: Tuple[int
     return x
 
 
+def bsa_tile_permute_pool(x: torch.Tensor, grid: Tuple[int, int, int],
+                          tile: Tuple[int, int, int], n_pad: int, block: int,
+                          y: Optional[torch.Tensor] = None,
+                          pooled: Optional[torch.Tensor] = None):
+    """x [B, N, H, D] bf16 raster -> (y [B, n_pad, H, D] tile order,
+    pooled [B, H, n_pad / block, D] fp32 block means)."""
+    _cuda(x, "x")
+    B, N, H, D = x.shape
+    if y is None:
+        y = torch.empty((B, n_pad, H, D), dtype=x.dtype, device=x.device)
+    if pooled is None:
+        pooled = torch.empty((B, H, n_pad // block, D), dtype=torch.float32, device=x.device)
+    _check(load_library().bsa_tile_permute_pool(_ptr(x), _ptr(y), B, *grid, *tile, H, D, n_pad,
+                                                block, _ptr(pooled), _stream()),
+           "bsa_tile_permute_pool")
+    return y, pooled
+
+
 # --------------------------------------------------------------------------- (b)
 
 def bsa_sta_mask(tile_grid: Tuple[int, int, int], window: Tuple[int, int, int], shift: int = 0,
@@ -180,6 +201,29 @@ def bsa_nabla_mask(q: torch.Tensor, k: torch.Tensor, block: int, p: float, scale
                                          float(scale), kb_begin, kb_end, int(force_outside),
                                          _ptr(mask), _ptr(near_count), _ptr(ws), ws.numel(),
                                          _stream()), "bsa_nabla_mask")
+    return mask, near_count
+
+
+def bsa_nabla_select(qbar: torch.Tensor, kbar: torch.Tensor, p: float, scale: float = 0.0,
+                     kb_begin: int = 0, kb_end: Optional[int] = None, force_outside: int = 0,
+                     base_mask: Optional[torch.Tensor] = None,
+                     mask: Optional[torch.Tensor] = None,
+                     near_count: Optional[torch.Tensor] = None):
+    """NABLA selection from pooled means qbar [B, H, QB, D], kbar [B, H, KB, D] (fp32),
+    optionally OR-ed with a head-shared base mask [QB, KB].  Returns (mask, near_count)."""
+    _cuda(qbar, "qbar")
+    _cuda(kbar, "kbar")
+    B, H, QB, D = qbar.shape
+    KB = kbar.shape[2]
+    kb_end = KB if kb_end is None else kb_end
+    if mask is None:
+        mask = torch.empty((B, H, QB, KB), dtype=torch.uint8, device=qbar.device)
+    if near_count is None:
+        near_count = torch.zeros(1, dtype=torch.int32, device=qbar.device)
+    _check(load_library().bsa_nabla_select(_ptr(qbar), _ptr(kbar), B, H, QB, KB, D, float(p),
+                                           float(scale), kb_begin, kb_end, int(force_outside),
+                                           _ptr(base_mask), _ptr(mask), _ptr(near_count),
+                                           _stream()), "bsa_nabla_select")
     return mask, near_count
 
 

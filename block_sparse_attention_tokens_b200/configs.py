@@ -87,7 +87,16 @@ WORKLOADS = [
              recent_frames=6),
 ]
 
-BY_NAME = {w.name: w for w in WORKLOADS}
+# Extra parity cases (not benchmark lines).
+EXTRA = [
+    # NABLA united with a Sliding-Tile window on a 480p-like grid whose 4x4x4 tiles
+    # coincide with the 64-token blocks (20x32x52 = 520 blocks).
+    Workload(name="nabla_sta_480p", index=5, batch=1, heads=40, head_dim=128,
+             grid=(20, 32, 52), block=64, mask="nabla_sta", tile=(4, 4, 4), window=(3, 3, 5),
+             p=0.9, strength_range=(0.5, 3.0)),
+]
+
+BY_NAME = {w.name: w for w in WORKLOADS + EXTRA}
 
 
 def get(name_or_index) -> Workload:

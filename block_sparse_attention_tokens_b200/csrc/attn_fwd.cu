@@ -121,83 +121,104 @@ __device__ __forceinline__ bool shares_kv(const Item& a, const Item& b) {
 }
 
 // ---------------------------------------------------------------------------
-// Per-q-tile step lists.  One thread per list row (a q-block when block_q >= 128,
+// Per-q-tile step lists.  One list per list row (a q-block when block_q >= 128,
 // a 128-row q-tile made of two 64-row q-blocks otherwise).  Entry = k-tile index
 // (bits 0-27) | quadrant bits << 28, bit (q_half * 2 + k_half) set when the
 // 64x64 quadrant is kept.  Lists are written at the offset the block CSR gives
 // the list row's first block row (times the k expansion), which bounds their
 // length without a scan.  Malformed CSR rows are reported and left empty.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void emit(uint32_t* out, int& n, int kt, uint32_t bits) {
-  if (n > 0 && static_cast<int>(out[n - 1] & 0x0FFFFFFFu) == kt) {
-    out[n - 1] |= bits << 28;
-  } else {
-    out[n++] = static_cast<uint32_t>(kt) | (bits << 28);
-  }
-}
+constexpr int kListThreads = 256;
 
-__global__ void build_lists_kernel(const int* __restrict__ row_ptr, const int* __restrict__ col_idx,
-                                   int list_heads, int QB, int KB, int LR, int block_q,
-                                   int block_k, int expand, long long nnz_cap,
-                                   int* __restrict__ cnt, uint32_t* __restrict__ entries,
-                                   int* status) {
-  const long long g = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (g >= static_cast<long long>(list_heads) * LR) return;
-  const int mh = static_cast<int>(g / LR), lr = static_cast<int>(g - static_cast<long long>(mh) * LR);
+// One CTA per list row.  The kept blocks of the (one or two) CSR rows are OR-ed
+// into a shared-memory map holding one 4-bit quadrant mask per 128-key tile
+// (eight tiles per 32-bit word); a block-wide ordered compaction then writes the
+// non-empty tiles in ascending order.  Dynamic shared memory: 4 * ceil(KT / 8) bytes.
+__global__ void __launch_bounds__(kListThreads) build_lists_kernel(
+    const int* __restrict__ row_ptr, const int* __restrict__ col_idx, int QB, int KB, int KT,
+    int LR, int block_q, int block_k, int expand, long long nnz_cap, int* __restrict__ cnt,
+    uint32_t* __restrict__ entries, int* status) {
+  extern __shared__ uint32_t quad[];
+  __shared__ int warp_sums[kListThreads / 32];
+  const int g = blockIdx.x;
+  const int mh = g / LR, lr = g - mh * LR;
   const int nrows = block_q >= 128 ? 1 : ((2 * lr + 1 < QB) ? 2 : 1);
   const int first_qb = block_q >= 128 ? lr : 2 * lr;
   const int* rp = row_ptr + static_cast<long long>(mh) * QB + first_qb;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   // validate the CSR rows this list reads
+  bool bad = false;
   for (int r = 0; r < nrows; ++r) {
-    if (rp[r] < 0 || rp[r] > rp[r + 1] || rp[r + 1] > nnz_cap) {
+    const int b0 = rp[r], b1 = rp[r + 1];
+    if (b0 < 0 || b0 > b1 || b1 > nnz_cap) {
+      bad = true;
+      break;
+    }
+    for (int i = b0 + tid; i < b1; i += kListThreads) {
+      const int c = col_idx[i];
+      if (c < 0 || c >= KB || (i > b0 && c <= col_idx[i - 1])) bad = true;
+    }
+  }
+  if (__syncthreads_or(bad)) {
+    if (tid == 0) {
       set_status(status, BSA_ERR_INVALID_ARG);
       cnt[g] = 0;
-      return;
     }
-    for (int i = rp[r]; i < rp[r + 1]; ++i) {
-      const int c = col_idx[i];
-      if (c < 0 || c >= KB || (i > rp[r] && c <= col_idx[i - 1])) {
-        set_status(status, BSA_ERR_INVALID_ARG);
-        cnt[g] = 0;
-        return;
+    return;
+  }
+  const int words = (KT + 7) / 8;
+  for (int w = tid; w < words; w += kListThreads) quad[w] = 0u;
+  __syncthreads();
+  for (int r = 0; r < nrows; ++r) {
+    // q-half bits of this row: a block of >= 128 rows covers both halves
+    const uint32_t qbits = block_q >= 128 ? 0x3u : (r == 0 ? 0x1u : 0x2u);
+    for (int i = rp[r] + tid; i < rp[r + 1]; i += kListThreads) {
+      const int kb = col_idx[i];
+      if (block_k >= 128) {
+        uint32_t bits = 0;
+        if (qbits & 1u) bits |= 0x3u;
+        if (qbits & 2u) bits |= 0xCu;
+        for (int t = 0; t < expand; ++t) {
+          const int kt = kb * expand + t;
+          atomicOr(&quad[kt >> 3], bits << (4 * (kt & 7)));
+        }
+      } else {
+        const int kt = kb >> 1, kh = kb & 1;
+        uint32_t bits = 0;
+        if (qbits & 1u) bits |= 1u << kh;
+        if (qbits & 2u) bits |= 1u << (2 + kh);
+        atomicOr(&quad[kt >> 3], bits << (4 * (kt & 7)));
       }
     }
   }
+  __syncthreads();
+  // ordered compaction: thread t owns words [t*per, (t+1)*per)
+  const int per = (words + kListThreads - 1) / kListThreads;
+  const int w0 = min(words, tid * per), w1 = min(words, w0 + per);
+  int mine = 0;
+  for (int w = w0; w < w1; ++w) {
+    const uint32_t q = quad[w];
+    for (int j = 0; j < 8; ++j) mine += ((q >> (4 * j)) & 0xFu) != 0u;
+  }
+  int incl = mine;
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  int base = 0;
+  for (int w = 0; w < warp; ++w) base += warp_sums[w];
+  int pos = base + incl - mine;
   uint32_t* out = entries + static_cast<long long>(rp[0]) * expand;
-  int n = 0;
-  int i0 = rp[0], e0 = rp[1];
-  int i1 = nrows == 2 ? rp[1] : 0, e1 = nrows == 2 ? rp[2] : 0;
-  const bool single = nrows == 1;
-  while (i0 < e0 || i1 < e1) {
-    // next k-block from the two sorted rows (ties: both)
-    int kb;
-    uint32_t qh;  // bit 0: q-half 0 wants it, bit 1: q-half 1 wants it
-    const int c0 = i0 < e0 ? col_idx[i0] : 0x7fffffff;
-    const int c1 = i1 < e1 ? col_idx[i1] : 0x7fffffff;
-    if (c0 <= c1) {
-      kb = c0;
-      qh = single ? (block_q >= 128 ? 0x3u : 0x1u) : 0x1u;
-      ++i0;
-      if (c1 == c0) { qh |= 0x2u; ++i1; }
-    } else {
-      kb = c1;
-      qh = 0x2u;
-      ++i1;
-    }
-    if (block_k >= 128) {
-      uint32_t bits = 0;
-      if (qh & 1u) bits |= 0x3u;  // q-half 0, both k-halves
-      if (qh & 2u) bits |= 0xCu;  // q-half 1, both k-halves
-      for (int t = 0; t < expand; ++t) emit(out, n, kb * expand + t, bits);
-    } else {  // 64-token key blocks: one k-half of tile kb/2
-      const uint32_t kh = static_cast<uint32_t>(kb & 1);
-      uint32_t bits = 0;
-      if (qh & 1u) bits |= 1u << (0 + kh);
-      if (qh & 2u) bits |= 1u << (2 + kh);
-      emit(out, n, kb >> 1, bits);
+  for (int w = w0; w < w1; ++w) {
+    const uint32_t q = quad[w];
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t bits = (q >> (4 * j)) & 0xFu;
+      if (bits) out[pos++] = static_cast<uint32_t>(w * 8 + j) | (bits << 28);
     }
   }
-  cnt[g] = n;
+  if (tid == kListThreads - 1) cnt[g] = pos;
 }
 
 // ---------------------------------------------------------------------------
@@ -856,8 +877,17 @@ extern "C" int bsa_attn_fwd(const void* q, const void* k, const void* v, int bat
   if (e != cudaSuccess) return record_cuda_error(e);
 
   const long long lists = static_cast<long long>(list_heads) * g.LR;
-  build_lists_kernel<<<static_cast<int>(ceil_div<long long>(lists, 128)), 128, 0, st>>>(
-      row_ptr, col_idx, list_heads, g.QB, g.KB, g.LR, block_q, block_k, g.expand, g.nnz_cap, cnt,
+  const int KT = ceil_div(nk, kBN);
+  const size_t list_smem = sizeof(uint32_t) * static_cast<size_t>((KT + 7) / 8);
+  if (list_smem > 200 * 1024 || lists > 0x7fffffffLL) return BSA_ERR_UNSUPPORTED;
+  if (list_smem > 48 * 1024) {
+    cudaError_t ea = cudaFuncSetAttribute(build_lists_kernel,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          static_cast<int>(list_smem));
+    if (ea != cudaSuccess) return record_cuda_error(ea);
+  }
+  build_lists_kernel<<<static_cast<int>(lists), kListThreads, list_smem, st>>>(
+      row_ptr, col_idx, g.QB, g.KB, KT, g.LR, block_q, block_k, g.expand, g.nnz_cap, cnt,
       entries, status);
   int rc = check_launch();
   if (rc != BSA_OK) return rc;

@@ -103,7 +103,8 @@ template <int D>
 __global__ void __launch_bounds__(256) nabla_select_kernel(
     const float* __restrict__ qbar, const float* __restrict__ kbar, int heads, int qb_count,
     int kb_count, int kb_begin, int kb_end, float p, float scale, int force_outside,
-    uint8_t* __restrict__ mask, int* __restrict__ near_count) {
+    const uint8_t* __restrict__ base_mask, uint8_t* __restrict__ mask,
+    int* __restrict__ near_count) {
   extern __shared__ float smem[];
   const int nr = kb_end - kb_begin;
   float* qs = smem;
@@ -141,9 +142,11 @@ __global__ void __launch_bounds__(256) nabla_select_kernel(
   const int qb = q0 + warp;
   if (qb >= qb_count) return;
   uint8_t* mrow = mask + ((static_cast<long long>(b) * heads + h) * qb_count + qb) * kb_count;
+  // optional head-shared mask OR-ed into the result (e.g. a Sliding-Tile window)
+  const uint8_t* brow = base_mask ? base_mask + static_cast<long long>(qb) * kb_count : nullptr;
   const uint8_t fo = force_outside ? 1 : 0;
-  for (int c = lane; c < kb_begin; c += 32) mrow[c] = fo;
-  for (int c = kb_end + lane; c < kb_count; c += 32) mrow[c] = fo;
+  for (int c = lane; c < kb_begin; c += 32) mrow[c] = fo | (brow ? (brow[c] != 0) : 0);
+  for (int c = kb_end + lane; c < kb_count; c += 32) mrow[c] = fo | (brow ? (brow[c] != 0) : 0);
   if (nr <= 0) return;
 
   float* z = zs + warp * nr;
@@ -204,7 +207,8 @@ __global__ void __launch_bounds__(256) nabla_select_kernel(
     const uint32_t bal = __ballot_sync(0xffffffffu, tie);
     const int rank = ties_seen + __popc(bal & ((1u << lane) - 1u));
     ties_seen += __popc(bal);
-    if (c < nr) mrow[kb_begin + c] = (key > v || (tie && rank < t)) ? 1 : 0;
+    if (c < nr)
+      mrow[kb_begin + c] = ((key > v || (tie && rank < t)) || (brow && brow[kb_begin + c] != 0)) ? 1 : 0;
   }
   if (lane == 0 && near_count) {
     const float c_last = cum / tot, c_prev = (cum - e_eq) / tot;
@@ -228,6 +232,59 @@ extern "C" size_t bsa_nabla_workspace_size(int batch, int heads, int nq, int nk,
   return bsa::nabla_ws_bytes(batch, heads, nq, nk, head_dim, block);
 }
 
+namespace bsa {
+namespace {
+
+int launch_select(const float* qbar, const float* kbar, int batch, int heads, int qb, int kb,
+                  int head_dim, float p, float scale, int kb_begin, int kb_end, int force_outside,
+                  const uint8_t* base_mask, uint8_t* mask, int* near_count, cudaStream_t st) {
+  const int nr = kb_end - kb_begin;
+  const size_t smem = sizeof(float) * (static_cast<size_t>(kSelRows) * head_dim +
+                                       static_cast<size_t>(kSelTile) * (head_dim + 1) +
+                                       2 * static_cast<size_t>(kSelRows) * nr);
+  if (smem > 200 * 1024) return BSA_ERR_UNSUPPORTED;
+  if (scale <= 0.0f) scale = 1.0f / sqrtf(static_cast<float>(head_dim));
+  if (near_count) {
+    cudaError_t e = cudaMemsetAsync(near_count, 0, sizeof(int), st);
+    if (e != cudaSuccess) return record_cuda_error(e);
+  }
+  dim3 sgrid(ceil_div(qb, kSelRows), heads, batch);
+  cudaError_t e;
+  if (head_dim == 128) {
+    e = cudaFuncSetAttribute(nabla_select_kernel<128>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return record_cuda_error(e);
+    nabla_select_kernel<128><<<sgrid, 256, smem, st>>>(qbar, kbar, heads, qb, kb, kb_begin, kb_end,
+                                                       p, scale, force_outside, base_mask, mask,
+                                                       near_count);
+  } else {
+    e = cudaFuncSetAttribute(nabla_select_kernel<64>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return record_cuda_error(e);
+    nabla_select_kernel<64><<<sgrid, 256, smem, st>>>(qbar, kbar, heads, qb, kb, kb_begin, kb_end,
+                                                      p, scale, force_outside, base_mask, mask,
+                                                      near_count);
+  }
+  return check_launch();
+}
+
+}  // namespace
+}  // namespace bsa
+
+extern "C" int bsa_nabla_select(const float* qbar, const float* kbar, int batch, int heads,
+                                int QB, int KB, int head_dim, float p, float scale, int kb_begin,
+                                int kb_end, int force_outside, const uint8_t* base_mask,
+                                uint8_t* mask, int* near_count, void* stream) {
+  using namespace bsa;
+  if (!qbar || !kbar || !mask) return BSA_ERR_INVALID_ARG;
+  if (batch < 1 || heads < 1 || QB < 1 || KB < 1 || !(p > 0.0f)) return BSA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return BSA_ERR_UNSUPPORTED;
+  if (kb_begin < 0 || kb_end > KB || kb_begin > kb_end) return BSA_ERR_INVALID_ARG;
+  return launch_select(qbar, kbar, batch, heads, QB, KB, head_dim, p, scale, kb_begin, kb_end,
+                       force_outside, base_mask, mask, near_count,
+                       static_cast<cudaStream_t>(stream));
+}
+
 extern "C" int bsa_nabla_mask(const void* q, const void* k, int batch, int heads, int nq, int nk,
                               int head_dim, int block, float p, float scale, int kb_begin,
                               int kb_end, int force_outside, uint8_t* mask, int* near_count,
@@ -242,19 +299,9 @@ extern "C" int bsa_nabla_mask(const void* q, const void* k, int batch, int heads
   const int qb = ceil_div(nq, block), kb = ceil_div(nk, block);
   if (kb_begin < 0 || kb_end > kb || kb_begin > kb_end) return BSA_ERR_INVALID_ARG;
   if (ws_bytes < nabla_ws_bytes(batch, heads, nq, nk, head_dim, block)) return BSA_ERR_WORKSPACE;
-  if (scale <= 0.0f) scale = 1.0f / sqrtf(static_cast<float>(head_dim));
-  const int nr = kb_end - kb_begin;
-  const size_t smem = sizeof(float) * (static_cast<size_t>(kSelRows) * head_dim +
-                                       static_cast<size_t>(kSelTile) * (head_dim + 1) +
-                                       2 * static_cast<size_t>(kSelRows) * nr);
-  if (smem > 200 * 1024) return BSA_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   float* qbar = reinterpret_cast<float*>(static_cast<char*>(ws) + kStatusBytes);
   float* kbar = qbar + static_cast<size_t>(batch) * heads * qb * head_dim;
-  if (near_count) {
-    cudaError_t e = cudaMemsetAsync(near_count, 0, sizeof(int), st);
-    if (e != cudaSuccess) return record_cuda_error(e);
-  }
   const int C = heads * head_dim;
   dim3 pgrid(qb > kb ? qb : kb, ceil_div(C, kPoolCols), batch * 2);
   nabla_pool_kernel<<<pgrid, kPoolThreads, 0, st>>>(
@@ -262,22 +309,6 @@ extern "C" int bsa_nabla_mask(const void* q, const void* k, int batch, int heads
       head_dim, nq, nk, block, qb, kb, qbar, kbar);
   int rc = check_launch();
   if (rc != BSA_OK) return rc;
-  dim3 sgrid(ceil_div(qb, kSelRows), heads, batch);
-  cudaError_t e;
-  if (head_dim == 128) {
-    e = cudaFuncSetAttribute(nabla_select_kernel<128>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return record_cuda_error(e);
-    nabla_select_kernel<128><<<sgrid, 256, smem, st>>>(qbar, kbar, heads, qb, kb, kb_begin,
-                                                       kb_end, p, scale, force_outside, mask,
-                                                       near_count);
-  } else {
-    e = cudaFuncSetAttribute(nabla_select_kernel<64>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return record_cuda_error(e);
-    nabla_select_kernel<64><<<sgrid, 256, smem, st>>>(qbar, kbar, heads, qb, kb, kb_begin,
-                                                      kb_end, p, scale, force_outside, mask,
-                                                      near_count);
-  }
-  return check_launch();
+  return launch_select(qbar, kbar, batch, heads, qb, kb, head_dim, p, scale, kb_begin, kb_end,
+                       force_outside, nullptr, mask, near_count, st);
 }

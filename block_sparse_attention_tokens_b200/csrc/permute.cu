@@ -79,6 +79,85 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(const uint4* __restri
   }
 }
 
+// Inverse of tile_position: raster token index of tile-order position p (p < N).
+__device__ __forceinline__ int tile_token(long long p, const PermGeo& g) {
+  const long long hw = static_cast<long long>(g.H) * g.W;
+  const long long slab = static_cast<long long>(g.tT) * hw;       // full frame slab
+  const int a = static_cast<int>(p / slab);
+  long long rem = p - a * slab;
+  const int lt = min(g.tT, g.T - a * g.tT);
+  const long long rowslab = static_cast<long long>(lt) * g.tH * g.W;
+  const int b = static_cast<int>(rem / rowslab);
+  rem -= b * rowslab;
+  const int lh = min(g.tH, g.H - b * g.tH);
+  const long long tilesz = static_cast<long long>(lt) * lh * g.tW;
+  const int c = static_cast<int>(rem / tilesz);
+  rem -= c * tilesz;
+  const int lw = min(g.tW, g.W - c * g.tW);
+  const int in = static_cast<int>(rem);
+  const int t = in / (lh * lw), h = (in / lw) % lh, w = in % lw;
+  return ((a * g.tT + t) * g.H + (b * g.tH + h)) * g.W + (c * g.tW + w);
+}
+
+// Tile permute fused with the per-block mean of the permuted rows (the pooling
+// step of the NABLA mask): one CTA per (batch, block of `block` output rows).
+// Each thread owns 8 adjacent bf16 columns, gathers its column slice of every row
+// of the block, stores it in tile order and sums it in fp32.  Rows past N are the
+// zero tail and are not averaged.  pooled: [B, heads, NB, head_dim] fp32.
+__global__ void __launch_bounds__(128) permute_pool_kernel(
+    const uint4* __restrict__ src, uint4* __restrict__ dst, int n, int n_pad, int vpr,
+    int head_dim, int heads, int block, PermGeo g, float* __restrict__ pooled) {
+  const int blk = blockIdx.x, b = blockIdx.y;
+  const int nb = n_pad / block;
+  const long long p0 = static_cast<long long>(blk) * block;
+  const int rows_valid =
+      static_cast<int>(max(0LL, min(static_cast<long long>(block), n - p0)));
+  __shared__ int src_row[1024];
+  for (int r = threadIdx.x; r < block; r += blockDim.x)
+    src_row[r] = (p0 + r < n) ? tile_token(p0 + r, g) : -1;
+  __syncthreads();
+  const uint4* sb = src + static_cast<long long>(b) * n * vpr;
+  uint4* db = dst + (static_cast<long long>(b) * n_pad + p0) * vpr;
+  for (int v = threadIdx.x; v < vpr; v += blockDim.x) {
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    int r = 0;
+    for (; r + 8 <= rows_valid; r += 8) {
+      uint4 x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) x[u] = __ldg(sb + static_cast<long long>(src_row[r + u]) * vpr + v);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        db[static_cast<long long>(r + u) * vpr + v] = x[u];
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&x[u]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(h2[e]);
+          acc[2 * e] += f.x;
+          acc[2 * e + 1] += f.y;
+        }
+      }
+    }
+    for (; r < rows_valid; ++r) {
+      const uint4 x = __ldg(sb + static_cast<long long>(src_row[r]) * vpr + v);
+      db[static_cast<long long>(r) * vpr + v] = x;
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&x);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(h2[e]);
+        acc[2 * e] += f.x;
+        acc[2 * e + 1] += f.y;
+      }
+    }
+    for (; r < block; ++r) db[static_cast<long long>(r) * vpr + v] = make_uint4(0, 0, 0, 0);
+    const float inv = rows_valid > 0 ? 1.0f / static_cast<float>(rows_valid) : 0.f;
+    const int col = v * 8, h = col / head_dim, j = col - h * head_dim;
+    float4* out = reinterpret_cast<float4*>(
+        pooled + ((static_cast<long long>(b) * heads + h) * nb + blk) * head_dim + j);
+    out[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+    out[1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
+  }
+}
+
 int permute_common(bool forward, const void* src, void* dst, int batch, int T, int H, int W,
                    int tT, int tH, int tW, int row_bytes, int n_pad, void* stream) {
   if (!src || !dst) return BSA_ERR_INVALID_ARG;
@@ -115,6 +194,30 @@ int permute_common(bool forward, const void* src, void* dst, int batch, int T, i
 
 }  // namespace
 }  // namespace bsa
+
+extern "C" int bsa_tile_permute_pool(const void* x, void* y, int batch, int T, int H, int W,
+                                     int tT, int tH, int tW, int heads, int head_dim, int n_pad,
+                                     int block, float* pooled, void* stream) {
+  using namespace bsa;
+  if (!x || !y || !pooled) return BSA_ERR_INVALID_ARG;
+  if (batch < 1 || T < 1 || H < 1 || W < 1 || tT < 1 || tH < 1 || tW < 1 || heads < 1 ||
+      head_dim < 8 || (head_dim % 8) != 0 || block < 1 || block > 1024)
+    return BSA_ERR_INVALID_ARG;
+  const long long n = static_cast<long long>(T) * H * W;
+  if (n > 0x7fffffffLL || n_pad < n || (n_pad % block) != 0) return BSA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y) || !aligned16(pooled)) return BSA_ERR_INVALID_ARG;
+  const long long row_bytes = static_cast<long long>(heads) * head_dim * 2;
+  const char* s0 = static_cast<const char*>(x);
+  const char* d0 = static_cast<const char*>(y);
+  if (s0 < d0 + batch * n_pad * row_bytes && d0 < s0 + batch * n * row_bytes)
+    return BSA_ERR_INVALID_ARG;
+  PermGeo g{T, H, W, tT, tH, tW};
+  dim3 grid(n_pad / block, batch);
+  permute_pool_kernel<<<grid, 128, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(x), static_cast<uint4*>(y), static_cast<int>(n), n_pad,
+      static_cast<int>(row_bytes / 16), head_dim, heads, block, g, pooled);
+  return check_launch();
+}
 
 extern "C" int bsa_tile_permute(const void* x, void* y, int batch, int T, int H, int W, int tT,
                                 int tH, int tW, int row_bytes, int n_pad, void* stream) {

@@ -55,9 +55,14 @@ class Plan:
             self.list_heads = Bt * Hh
             self.mask = torch.empty((Bt, Hh, self.QB, self.KB), dtype=torch.uint8, device=device)
             self.near = torch.zeros(1, dtype=torch.int32, device=device)
+        if w.mask == "ar":
             self.nabla_ws = torch.empty(
                 B.bsa_nabla_workspace_size(Bt, Hh, self.nq, self.nk, D, w.block),
                 dtype=torch.uint8, device=device)
+        if w.mask in ("nabla", "nabla_sta"):
+            # block means come out of the fused permute of Q and K
+            self.qbar = torch.empty((Bt, Hh, self.QB, D), dtype=torch.float32, device=device)
+            self.kbar = torch.empty((Bt, Hh, self.KB, D), dtype=torch.float32, device=device)
         rows = self.list_heads * self.QB
         self.row_ptr = torch.empty(rows + 1, dtype=torch.int32, device=device)
         self.col_idx = torch.empty(rows * self.KB, dtype=torch.int32, device=device)
@@ -69,6 +74,8 @@ class Plan:
         if w.tile is not None:
             g, t = w.grid, w.tile
             self.tile_grid = (ceil_div(g[0], t[0]), ceil_div(g[1], t[1]), ceil_div(g[2], t[2]))
+        if w.mask == "nabla_sta":
+            self.base_mask = torch.empty((self.QB, self.KB), dtype=torch.uint8, device=device)
         if w.mask == "ar":
             self.kb_range = ar_block_ranges(self.nk, w.tokens_per_frame, w.block, w.anchor_frames,
                                             w.recent_frames)
@@ -76,6 +83,14 @@ class Plan:
     # --- individual stages (each one or a few libbsa launches) ---
     def permute_inputs(self, q, k, v):
         w = self.w
+        if w.mask in ("nabla", "nabla_sta"):
+            # NABLA pools Q and K per block while they are permuted
+            B.bsa_tile_permute_pool(q, w.grid, w.tile, self.n_pad, w.block, y=self.qp,
+                                    pooled=self.qbar)
+            B.bsa_tile_permute_pool(k, w.grid, w.tile, self.n_pad, w.block, y=self.kp,
+                                    pooled=self.kbar)
+            B.bsa_tile_permute(v, w.grid, w.tile, self.n_pad, y=self.vp)
+            return
         for src, dst in ((q, self.qp), (k, self.kp), (v, self.vp)):
             B.bsa_tile_permute(src, w.grid, w.tile, self.n_pad, y=dst)
 
@@ -86,8 +101,11 @@ class Plan:
         elif w.mask == "radial":
             B.bsa_radial_mask(self.nk, w.tokens_per_frame, w.block, mask=self.mask)
         elif w.mask == "nabla":
-            B.bsa_nabla_mask(self.qp, self.kp, w.block, w.p, 0.0, 0, self.KB, 0, nq=self.nq,
-                             nk=self.nk, mask=self.mask, near_count=self.near, ws=self.nabla_ws)
+            B.bsa_nabla_select(self.qbar, self.kbar, w.p, mask=self.mask, near_count=self.near)
+        elif w.mask == "nabla_sta":
+            B.bsa_sta_mask(self.tile_grid, w.window, 0, mask=self.base_mask)
+            B.bsa_nabla_select(self.qbar, self.kbar, w.p, base_mask=self.base_mask,
+                               mask=self.mask, near_count=self.near)
         elif w.mask == "ar":
             a_end, r_begin = self.kb_range
             B.bsa_nabla_mask(self._q, self._k, w.block, w.p, 0.0, a_end, r_begin, 1, nq=self.nq,
@@ -125,7 +143,7 @@ class Plan:
         n = 0
         if self.permuted:
             n += 3 + 1                   # permute Q, K, V and untile O
-        n += 2 if self.w.mask in ("nabla", "ar") else 1   # pool + select, or one static mask
+        n += {"nabla": 1, "nabla_sta": 2, "ar": 2}.get(self.w.mask, 1)   # mask kernels
         n += 3                           # compact: count, scan, fill
         n += 2                           # kept-list build + attention
         return n

@@ -82,6 +82,22 @@ int bsa_tile_untile(const void* y, void* x, int batch, int T, int H, int W,
                     int tT, int tH, int tW, int row_bytes, int n_pad, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * (a') Tile permute fused with per-block mean pooling.
+ * Sources: STA explainer section 3 (tile order) and the NABLA explainer
+ * (aibr.jp/archives/124678), section 3 (Q and K are mean-pooled per block).
+ *
+ * Same permutation as bsa_tile_permute for bf16 rows of heads * head_dim
+ * elements, with n_pad a multiple of `block` (1..1024).  While the rows are
+ * moved, the mean of every `block` consecutive output rows is taken per head over
+ * the rows that hold tokens (the zero tail is excluded), so the NABLA mask needs
+ * no second pass over Q and K.
+ *   pooled : [batch, heads, n_pad / block, head_dim] float32, written completely.
+ * ------------------------------------------------------------------------- */
+int bsa_tile_permute_pool(const void* x, void* y, int batch, int T, int H, int W, int tT,
+                          int tH, int tW, int heads, int head_dim, int n_pad, int block,
+                          float* pooled, void* stream);
+
+/* ---------------------------------------------------------------------------
  * (b1) Sliding Tile Attention mask.
  * Source: STA explainer (aibr.jp/archives/60739), sections 2-3: each query tile
  * attends to a window of neighbouring tiles; the window is counted in tiles.
@@ -143,6 +159,25 @@ int bsa_nabla_mask(const void* q, const void* k, int batch, int heads, int nq, i
                    int head_dim, int block, float p, float scale, int kb_begin, int kb_end,
                    int force_outside, uint8_t* mask, int* near_count, void* ws,
                    size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * (b4) NABLA selection from pooled means, optionally united with a fixed mask.
+ * Sources: NABLA explainer section 3 (softmax over pooled logits, CDF cut);
+ * sections 1-2 (NABLA combines with Sliding Tile Attention and other sparse
+ * patterns); Sparse Forcing summary part 2 (forced anchor / recent ranges).
+ *
+ * The selection step of bsa_nabla_mask on caller-provided means:
+ *   qbar : [batch, heads, QB, head_dim] float32, kbar : [batch, heads, KB, head_dim]
+ * (as written by bsa_tile_permute_pool or by the pooling of bsa_nabla_mask).
+ * Semantics of p, scale, kb_begin, kb_end, force_outside, mask and near_count
+ * as for bsa_nabla_mask.  base_mask (may be NULL): [QB][KB] uint8 shared by all
+ * batches and heads, OR-ed into every row of the result -- with a Sliding-Tile
+ * mask this gives the NABLA-plus-window hybrid.  head_dim in {64, 128}.
+ * ------------------------------------------------------------------------- */
+int bsa_nabla_select(const float* qbar, const float* kbar, int batch, int heads, int QB, int KB,
+                     int head_dim, float p, float scale, int kb_begin, int kb_end,
+                     int force_outside, const uint8_t* base_mask, uint8_t* mask,
+                     int* near_count, void* stream);
 
 /* ---------------------------------------------------------------------------
  * (c) Mask compaction into per-row kept-block lists (CSR).

@@ -377,6 +377,15 @@ def ar_mask(qbar, kbar, p, scale, n_tokens_k, tokens_per_frame, block, anchor_fr
     return nabla_mask(qbar, kbar, p, scale, a_end, r_begin, force_outside=1)
 
 
+def nabla_sta_mask(qbar, kbar, p, scale, sta_mask):
+    """NABLA selection united with a Sliding-Tile window (NABLA explainer,
+    sections 1-2: NABLA is combined with STA and other sparse patterns).
+    READING: the union of the two block masks, the NABLA cut taken over all key
+    blocks as usual; the window mask is shared by every batch and head."""
+    m, near = nabla_mask(qbar, kbar, p, scale)
+    return (m | (sta_mask[None, None] != 0)).astype(np.uint8), near
+
+
 # ---------------------------------------------------------------------------
 # 6. Compaction of a block mask into per-row kept lists
 # ---------------------------------------------------------------------------

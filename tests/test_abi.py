@@ -75,3 +75,21 @@ def test_workspace_sizes(lib):
     assert ws >= 300 * 300 * 3 * 4
     assert lib.bsa_attn_workspace_size(1, 1, 1, 1, 96, 128, 1) == 0
     assert lib.bsa_nabla_workspace_size(1, 40, 32760, 32760, 128, 64) == 256 + 4 * 40 * 128 * 1024
+
+
+def declared_prototypes():
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    protos = {}
+    for m in re.finditer(r"\b(bsa_[a-z0-9_]+)\s*\(([^)]*)\)\s*;", text):
+        params = [p.strip() for p in m.group(2).split(",") if p.strip() and p.strip() != "void"]
+        protos[m.group(1)] = params
+    return protos
+
+
+def test_binding_argument_counts_match_the_header(lib):
+    protos = declared_prototypes()
+    assert protos, "no prototypes parsed"
+    for name, params in protos.items():
+        f = getattr(lib, name)
+        assert f.argtypes is not None, name
+        assert len(f.argtypes) == len(params), (name, len(f.argtypes), len(params))

@@ -131,3 +131,39 @@ def test_nabla_p_one_keeps_everything():
     mask, _ = B.bsa_nabla_mask(q, k, 64, 1.0)
     torch.cuda.synchronize()
     assert torch.all(mask == 1)
+
+
+@pytest.mark.parametrize("grid,tile,block,heads,d", [((21, 30, 52), (4, 4, 4), 64, 3, 128),
+                                                     ((5, 7, 3), (2, 3, 2), 16, 2, 64),
+                                                     ((20, 32, 52), (4, 4, 4), 64, 2, 128)])
+def test_tile_permute_pool_bit_exact_rows_and_means(grid, tile, block, heads, d):
+    n = grid[0] * grid[1] * grid[2]
+    n_pad = math.ceil(n / block) * block
+    x = torch.randn(2, n, heads, d).to(torch.bfloat16)
+    perm = O.tile_order(grid, tile)
+    y, pooled = B.bsa_tile_permute_pool(x.cuda(), grid, tile, n_pad, block)
+    torch.cuda.synchronize()
+    assert np.array_equal(_bits(y), O.tile_permute(_bits(x), perm, n_pad))
+    ref = O.nabla_pool(O.tile_permute(x.double().numpy(), perm, n_pad), block, n)
+    got = pooled.cpu().double().numpy()
+    assert got.shape == ref.shape
+    assert np.max(np.abs(got - ref)) < 2e-5        # fp32 sums of <= block bf16 values
+
+
+def test_nabla_select_with_sta_base_mask_matches_oracle():
+    w_grid, tile, block, window = (8, 16, 16), (4, 4, 4), 64, (3, 3, 3)
+    n = w_grid[0] * w_grid[1] * w_grid[2]
+    q, k, _, _ = synth.generate(1, 3, 128, w_grid, seed=31, strength_range=(0.5, 3.0))
+    perm = O.tile_order(w_grid, tile)
+    qp, qbar = B.bsa_tile_permute_pool(q.cuda(), w_grid, tile, n, block)
+    kp, kbar = B.bsa_tile_permute_pool(k.cuda(), w_grid, tile, n, block)
+    tg = tuple(g // t for g, t in zip(w_grid, tile))
+    base = B.bsa_sta_mask(tg, window)
+    mask, _ = B.bsa_nabla_select(qbar, kbar, 0.7, base_mask=base)
+    torch.cuda.synchronize()
+    rq = O.nabla_pool(O.tile_permute(q.double().numpy(), perm, n), block, n)
+    rk = O.nabla_pool(O.tile_permute(k.double().numpy(), perm, n), block, n)
+    ref, near = O.nabla_sta_mask(rq, rk, 0.7, 1 / math.sqrt(128), O.sta_tile_mask(tg, window))
+    _assert_nabla_equal(mask, ref, near)
+    m = mask.cpu().numpy()
+    assert np.all(m >= O.sta_tile_mask(tg, window)[None, None])

@@ -41,7 +41,7 @@ def oracle_mask(w, plan, q, k):
         return O.radial_block_mask_fast(w.nk, w.tokens_per_frame, w.block)[None], None
     D = w.head_dim
     scale = 1.0 / math.sqrt(D)
-    if w.mask == "nabla":
+    if w.mask in ("nabla", "nabla_sta"):
         perm = O.tile_order(w.grid, w.tile)
         qbar = np.zeros((w.batch, w.heads, plan.QB, D))
         kbar = np.zeros((w.batch, w.heads, plan.KB, D))
@@ -50,7 +50,11 @@ def oracle_mask(w, plan, q, k):
             kh = O.tile_permute(to64(k[:, :, h:h + 1]), perm, plan.n_pad)
             qbar[:, h] = O.nabla_pool(qh, w.block, w.nq)[:, 0]
             kbar[:, h] = O.nabla_pool(kh, w.block, w.nk)[:, 0]
-        m, near = O.nabla_mask(qbar, kbar, w.p, scale)
+        if w.mask == "nabla":
+            m, near = O.nabla_mask(qbar, kbar, w.p, scale)
+        else:
+            m, near = O.nabla_sta_mask(qbar, kbar, w.p, scale,
+                                       O.sta_tile_mask(plan.tile_grid, w.window))
     else:  # ar
         QBp, KBp = plan.QB * w.block, plan.KB * w.block
         qbar = np.zeros((w.batch, w.heads, plan.QB, D))
@@ -67,7 +71,7 @@ def oracle_mask(w, plan, q, k):
     return m.reshape(-1, plan.QB, plan.KB), near.reshape(-1, plan.QB)
 
 
-@pytest.mark.parametrize("name", [w.name for w in configs.WORKLOADS])
+@pytest.mark.parametrize("name", [w.name for w in configs.WORKLOADS + configs.EXTRA])
 def test_workload_path(name):
     w = configs.get(name)
     q, k, v, _ = synth.workload_inputs(w)

@@ -105,6 +105,17 @@ def test_nabla_mask_range_and_forced_outside():
         assert np.sort(probs[qb])[::-1][:len(kept) - 1].sum() < 0.8
 
 
+def test_nabla_sta_union_contains_both_masks():
+    rng = np.random.default_rng(12)
+    qbar = rng.normal(size=(1, 2, 12, 8))
+    kbar = rng.normal(size=(1, 2, 12, 8))
+    sta = O.sta_tile_mask((1, 3, 4), (1, 3, 3))
+    m, near = O.nabla_sta_mask(qbar, kbar, 0.6, 0.35, sta)
+    alone, _ = O.nabla_mask(qbar, kbar, 0.6, 0.35)
+    assert np.all(m >= alone) and np.all(m >= sta[None, None])
+    assert np.array_equal(m, np.maximum(alone, sta[None, None]))
+
+
 def test_ar_ranges_match_the_decode_workload():
     # 60 frames of 30x52 = 1560 tokens, 64-token blocks, 3 anchor frames, last 6 dense
     a_end, r_begin = O.ar_block_ranges(60 * 1560, 1560, 64, 3, 6)
