@@ -209,6 +209,23 @@ def run_reference(args, w):
     return 0
 
 
+def max_over_ranks(values, device=None):
+    """Element-wise maximum of a list of floats over all ranks (identity when not
+    distributed).  Every rank must call it at the same point."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def weak_scaling_value(flops_per_rank, world, ms_per_step):
+    """Whole-job throughput (TFLOP/s): every rank processes its own batch of the
+    same shape, the slowest rank's time bounds the step."""
+    return flops_per_rank * world / (ms_per_step * 1e-3) / 1e12
+
+
 def workload_config(w):
     cfg = {"workload": w.name, "batch": w.batch, "heads": w.heads, "head_dim": w.head_dim,
            "grid_thw": list(w.grid), "block": w.block, "mask": w.mask}
@@ -303,12 +320,9 @@ def main():
         barrier()
     ms_total = start.elapsed_time(end)
     attn_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_a)
-    t = torch.tensor([ms_total, attn_ms], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_total, attn_ms = t.tolist()
+    ms_total, attn_ms = max_over_ranks([ms_total, attn_ms], dev)
     ms_per_step = ms_total / args.steps
-    value = flops * world / (ms_per_step * 1e-3) / 1e12
+    value = weak_scaling_value(flops, world, ms_per_step)
 
     # ---- end to end through the public API: pinned host inputs in, O back to host.
     # Steps are pipelined the way a serving loop would run them: the host->device
@@ -367,12 +381,11 @@ def main():
         e1.record(stream)
         barrier()
         # time from the start of step 2 to the end of the last output copy, per step
-        e_ms = torch.tensor([e0.elapsed_time(e1) / e2e_steps], device=dev, dtype=torch.float64)
-        if world > 1:
-            dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
+        e_ms = torch.tensor(max_over_ranks([e0.elapsed_time(e1) / e2e_steps], dev),
+                            dtype=torch.float64)
         h2d_bytes = sum(t_.numel() * t_.element_size() for t_ in (q_h, k_h, v_h))
         d2h_bytes = o_host.numel() * o_host.element_size()
-        e2e = {"value": flops * world / (e_ms.item() * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": weak_scaling_value(flops, world, e_ms.item()), "unit": "TFLOP/s",
                "ms_per_step": e_ms.item(), "h2d_bytes_per_step": h2d_bytes,
                "d2h_bytes_per_step": d2h_bytes,
                "note": "pinned host buffers; copies of neighbouring steps overlap compute"}

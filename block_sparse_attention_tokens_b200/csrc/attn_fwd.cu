@@ -14,7 +14,11 @@
 //   warps 4-7  softmax for q-tile slot 1
 //   warp  8    TMA producer: Q tiles, K/V tiles into an NSTAGE ring
 //   warp  9    MMA issuer (one thread), also owns the TMEM allocation
-// Each CTA processes "units" of two 128-row q-tiles (slots) in lock-step rounds;
+// Units of two 128-row q-tiles are handed out dynamically: the producer warp takes
+// the next unit index from a global counter (so all CTAs stay on a compact window
+// of q-tiles, which keeps the K/V they read in L2, and the tail is balanced) and
+// publishes it through a 4-entry shared-memory ring to the MMA and softmax warps.
+// Each CTA processes a unit's two q-tiles (slots) in lock-step rounds;
 // the MMA warp issues, per round r and slot s, O_s += P_s V_s,r then
 // S_s = Q_s K_s,r+1^T, alternating slots, so that while one slot's softmax runs
 // on the CUDA cores the tensor core works on the other slot.  TMEM (512 columns): S_0 | S_1 | O_0 | O_1, 128 columns
@@ -74,7 +78,7 @@ struct Cfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_RING = 2 * TILE_BYTES;
   static constexpr int OFF_BAR = OFF_RING + NSTAGE * TILE_BYTES;
-  static constexpr int BAR_BYTES = 256;
+  static constexpr int BAR_BYTES = 512;
   static constexpr int SMEM = OFF_BAR + BAR_BYTES + 1024;  // + alignment slack
 };
 
@@ -89,6 +93,7 @@ struct AttnParams {
   __nv_bfloat16* o;
   float* lse;
   int* status;
+  int* unit_counter;  // next unit to hand out (zeroed before the launch)
   unsigned long long timeout_ns;
 };
 
@@ -246,8 +251,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto PREADY = [&](int s) { return bar0 + 8u * (2 * C::NSTAGE + 6 + s); };
   auto ODONE = [&](int s) { return bar0 + 8u * (2 * C::NSTAGE + 8 + s); };
   const uint32_t FINAL = bar0 + 8u * (2 * C::NSTAGE + 10);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + 8 * (2 * C::NSTAGE + 11));
+  // unit hand-off ring: the producer takes units from the global counter and
+  // publishes them to the MMA thread and the softmax warps
+  auto UFULL = [&](int i) { return bar0 + 8u * (2 * C::NSTAGE + 11 + i); };
+  auto UEMPTY = [&](int i) { return bar0 + 8u * (2 * C::NSTAGE + 15 + i); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + 8 * (2 * C::NSTAGE + 19));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* unit_ring = reinterpret_cast<volatile int*>(tmem_slot + 2);
+  constexpr int kUnitConsumers = 1 + 8;  // MMA thread + one arrival per softmax warp
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -264,6 +275,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(ODONE(s), 1);
     }
     mbar_init(FINAL, 1);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(UFULL(i), 1);
+      mbar_init(UEMPTY(i), kUnitConsumers);
+    }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -314,7 +329,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (++st == C::NSTAGE) { st = 0; ph ^= 1u; }
         return true;
       };
-      for (int u = blockIdx.x; u < p.total_units && ok; u += gridDim.x) {
+      for (int uk = 0; ok; ++uk) {
+        // take the next unit and publish it to the other roles
+        const int slot = uk & 3;
+        if (!mbar_wait(UEMPTY(slot), ((uk >> 2) & 1) ^ 1u, abort_flag, p.status, p.timeout_ns)) {
+          ok = false;
+          break;
+        }
+        const int u = atomicAdd(p.unit_counter, 1);
+        unit_ring[slot] = u;
+        mbar_arrive(UFULL(slot));
+        if (u >= p.total_units) break;
         Item it[2] = {get_item(p, 2 * u), get_item(p, 2 * u + 1)};
         for (int s = 0; s < 2 && ok; ++s) {
           if (it[s].n <= 0) continue;
@@ -413,7 +438,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                  kk > 0 ? 1u : acc0);
         return true;
       };
-      for (int u = blockIdx.x; u < p.total_units && ok; u += gridDim.x) {
+      for (int uk = 0; ok; ++uk) {
+        const int slot = uk & 3;
+        if (!mbar_wait(UFULL(slot), (uk >> 2) & 1, abort_flag, p.status, p.timeout_ns)) {
+          ok = false;
+          break;
+        }
+        const int u = unit_ring[slot];
+        mbar_arrive(UEMPTY(slot));
+        if (u >= p.total_units) break;
         Item it[2] = {get_item(p, 2 * u), get_item(p, 2 * u + 1)};
         if (shares_kv(it[0], it[1])) {
           const int n = it[0].n;
@@ -497,7 +530,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     int gstep = 0;
     (void)gstep;
     bool ok = true;
-    for (int u = blockIdx.x; u < p.total_units && ok; u += gridDim.x) {
+    for (int uk = 0; ok; ++uk) {
+      const int slot = uk & 3;
+      if (!mbar_wait(UFULL(slot), (uk >> 2) & 1, abort_flag, p.status, p.timeout_ns)) {
+        ok = false;
+        break;
+      }
+      const int u = unit_ring[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(UEMPTY(slot));
+      if (u >= p.total_units) break;
       const Item me = get_item(p, 2 * u + s);
       if (me.n < 0) continue;
       const int qrow = me.qt * kBM + row;
@@ -873,7 +915,7 @@ extern "C" int bsa_attn_fwd(const void* q, const void* k, const void* v, int bat
   int* status = reinterpret_cast<int*>(wsb);
   int* cnt = reinterpret_cast<int*>(wsb + g.cnt_off);
   uint32_t* entries = reinterpret_cast<uint32_t*>(wsb + g.ent_off);
-  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), st);
+  cudaError_t e = cudaMemsetAsync(status, 0, 2 * sizeof(int), st);  // status word + unit counter
   if (e != cudaSuccess) return record_cuda_error(e);
 
   const long long lists = static_cast<long long>(list_heads) * g.LR;
@@ -913,6 +955,7 @@ extern "C" int bsa_attn_fwd(const void* q, const void* k, const void* v, int bat
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.status = status;
+  p.unit_counter = status + 1;
   p.timeout_ns = 2000000000ULL;
   return head_dim == 128 ? launch_attn<128>(mq, mk, mv, p, st) : launch_attn<64>(mq, mk, mv, p, st);
 }

@@ -100,14 +100,15 @@ __device__ __forceinline__ int tile_token(long long p, const PermGeo& g) {
 }
 
 // Tile permute fused with the per-block mean of the permuted rows (the pooling
-// step of the NABLA mask): one CTA per (batch, block of `block` output rows).
-// Each thread owns 8 adjacent bf16 columns, gathers its column slice of every row
-// of the block, stores it in tile order and sums it in fp32.  Rows past N are the
-// zero tail and are not averaged.  pooled: [B, heads, NB, head_dim] fp32.
+// step of the NABLA mask): one CTA per (block of `block` output rows, 1024-column
+// slice, batch).  Each thread owns 8 adjacent bf16 columns, gathers its column
+// slice of every row of the block (8 rows in flight), stores it in tile order and
+// sums it in fp32.  Rows past N are the zero tail and are not averaged.
+// pooled: [B, heads, NB, head_dim] fp32.
 __global__ void __launch_bounds__(128) permute_pool_kernel(
     const uint4* __restrict__ src, uint4* __restrict__ dst, int n, int n_pad, int vpr,
     int head_dim, int heads, int block, PermGeo g, float* __restrict__ pooled) {
-  const int blk = blockIdx.x, b = blockIdx.y;
+  const int blk = blockIdx.x, b = blockIdx.z;
   const int nb = n_pad / block;
   const long long p0 = static_cast<long long>(blk) * block;
   const int rows_valid =
@@ -118,7 +119,8 @@ __global__ void __launch_bounds__(128) permute_pool_kernel(
   __syncthreads();
   const uint4* sb = src + static_cast<long long>(b) * n * vpr;
   uint4* db = dst + (static_cast<long long>(b) * n_pad + p0) * vpr;
-  for (int v = threadIdx.x; v < vpr; v += blockDim.x) {
+  for (int v = blockIdx.y * blockDim.x + threadIdx.x; v < vpr && v < (blockIdx.y + 1) * blockDim.x;
+       v += blockDim.x) {
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     int r = 0;
     for (; r + 8 <= rows_valid; r += 8) {
@@ -212,10 +214,11 @@ extern "C" int bsa_tile_permute_pool(const void* x, void* y, int batch, int T, i
   if (s0 < d0 + batch * n_pad * row_bytes && d0 < s0 + batch * n * row_bytes)
     return BSA_ERR_INVALID_ARG;
   PermGeo g{T, H, W, tT, tH, tW};
-  dim3 grid(n_pad / block, batch);
+  const int vpr = static_cast<int>(row_bytes / 16);
+  dim3 grid(n_pad / block, ceil_div(vpr, 128), batch);
   permute_pool_kernel<<<grid, 128, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const uint4*>(x), static_cast<uint4*>(y), static_cast<int>(n), n_pad,
-      static_cast<int>(row_bytes / 16), head_dim, heads, block, g, pooled);
+      static_cast<const uint4*>(x), static_cast<uint4*>(y), static_cast<int>(n), n_pad, vpr,
+      head_dim, heads, block, g, pooled);
   return check_launch();
 }
 
