@@ -25,6 +25,7 @@ EXPORTS = [
     "bsa_tile_untile", "bsa_sta_mask", "bsa_radial_mask", "bsa_nabla_workspace_size",
     "bsa_nabla_mask", "bsa_mask_compact", "bsa_attn_workspace_size", "bsa_attn_fwd",
     "bsa_attn_fwd_noalloc", "bsa_read_status", "bsa_tile_permute_pool", "bsa_nabla_select",
+    "bsa_wait_selftest",
 ]
 
 
@@ -67,6 +68,7 @@ def load_library(path: str = _LIB_PATH) -> ctypes.CDLL:
                                  + [c_void, c_void, c_int, c_float, c_void, c_void, c_void,
                                     c_void]),
         "bsa_read_status": (c_int, [c_void, ctypes.POINTER(c_int), c_void]),
+        "bsa_wait_selftest": (c_int, [c_void, ctypes.c_ulonglong, c_void]),
         "bsa_tile_permute_pool": (c_int, [c_void, c_void] + [c_int] * 11 + [c_void, c_void]),
         "bsa_nabla_select": (c_int, [c_void, c_void] + [c_int] * 5 + [c_float, c_float]
                              + [c_int] * 3 + [c_void, c_void, c_void, c_void]),
@@ -308,6 +310,17 @@ def bsa_read_status(ws: torch.Tensor) -> int:
     _check(load_library().bsa_read_status(_ptr(ws), ctypes.byref(out), _stream()),
            "bsa_read_status")
     return out.value
+
+
+def bsa_wait_selftest(timeout_ns: int, device_status: Optional[torch.Tensor] = None) -> int:
+    """Runs the bounded-wait self-test and returns the status it recorded
+    (BSA_ERR_TIMEOUT = 5 when the wait gave up as designed)."""
+    if device_status is None:
+        device_status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    _check(load_library().bsa_wait_selftest(_ptr(device_status), int(timeout_ns), _stream()),
+           "bsa_wait_selftest")
+    torch.cuda.synchronize()
+    return int(device_status.item())
 
 
 def bsa_status_string(code: int) -> str:

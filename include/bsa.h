@@ -251,6 +251,16 @@ int bsa_attn_fwd_noalloc(const void* q, const void* k, const void* v, int batch,
                          void* o, float* lse, int* device_status, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Self-test of the bounded device-side waits (failure detection).
+ * No counterpart in the pages.  Launches one thread that waits, through the
+ * same bounded wait the attention pipeline uses, on a barrier phase that never
+ * completes; after timeout_ns (1 ns .. 10 s) it writes BSA_ERR_TIMEOUT to
+ * *device_status (a device int, cleared first) and returns.  Used by the tests
+ * to show that a stuck pipeline ends with a status instead of hanging the GPU.
+ * ------------------------------------------------------------------------- */
+int bsa_wait_selftest(int* device_status, unsigned long long timeout_ns, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Device status word of a workspace (attention or NABLA): synchronises `stream`,
  * copies the word to *status (a bsa_status value) and clears it.
  * ------------------------------------------------------------------------- */
