@@ -474,3 +474,50 @@ def block_sparse_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, mask: np
                 o[b, sel, h] = (e @ v[b, cols, h]) / l
                 lse[b, h, sel] = (mx + np.log(l))[:, 0]
     return o, lse
+
+
+# ---------------------------------------------------------------------------
+# 8. Backward of the block-sparse attention (training)
+# ---------------------------------------------------------------------------
+
+def block_sparse_attention_backward(q, k, v, do, mask, block_q, block_k, scale=None):
+    """Gradients of O = softmax(Q K^T * scale + M) V with respect to Q, K, V.
+
+    The Radial explainer (section 4, training cost), the NABLA explainer
+    (section 4, training and inference speed-up) and the Sparse Forcing summary
+    (trainable sparse attention) train through the sparse attention; the
+    gradients are those of the same masked softmax, written out per row:
+        P = softmax(S),  dV = P^T dO,  dP = dO V^T,
+        dS = P * (dP - rowsum(dO * O)),  dQ = dS K * scale,  dK = dS^T Q * scale,
+    evaluated over each row's kept key blocks only (masked entries have P = 0).
+    q: [B, Nq, H, D]; k, v: [B, Nk, H, D]; do: [B, Nq, H, D]; mask: [Hm, QB, KB].
+    Returns (dq, dk, dv) with the shapes of q, k, v.
+    """
+    Bn, nq, H, D = q.shape
+    nk = k.shape[1]
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for b in range(Bn):
+        for h in range(H):
+            m = mask[0 if mask.shape[0] == 1 else b * H + h]
+            for qb in range(m.shape[0]):
+                rows = np.arange(qb * block_q, min((qb + 1) * block_q, nq))
+                kept = np.nonzero(m[qb])[0]
+                if kept.size == 0 or rows.size == 0:
+                    continue
+                cols = np.concatenate([np.arange(kb * block_k, min((kb + 1) * block_k, nk))
+                                       for kb in kept])
+                s = (q[b, rows, h] @ k[b, cols, h].T) * scale
+                s = s - s.max(axis=1, keepdims=True)
+                p = np.exp(s)
+                p /= p.sum(axis=1, keepdims=True)
+                o = p @ v[b, cols, h]
+                g = do[b, rows, h]
+                dv[b, cols, h] += p.T @ g
+                dp = g @ v[b, cols, h].T
+                ds = p * (dp - (g * o).sum(axis=1, keepdims=True))
+                dq[b, rows, h] += (ds @ k[b, cols, h]) * scale
+                dk[b, cols, h] += (ds.T @ q[b, rows, h]) * scale
+    return dq, dk, dv

@@ -207,3 +207,30 @@ def test_sampled_rows_match_full_evaluation():
     o2, lse2 = O.block_sparse_attention(q, k, v, mask, 64, 64, rows=rows)
     assert np.allclose(o[:, rows], o2[:, rows], atol=1e-13, rtol=0)
     assert np.allclose(lse[..., rows], lse2[..., rows], atol=1e-13, rtol=0)
+
+
+# ----------------------------------------------------------------- backward
+
+@pytest.mark.parametrize("bq,bk", [(64, 64), (128, 64), (384, 384)])
+def test_backward_matches_autograd_float64(bq, bk):
+    Bn, H, D = 1, 2, 16
+    nq, nk = 2 * bq + 9, 3 * bk - 7
+    q, k, v = _rand_qkv(Bn, nq, nk, H, D, 21)
+    do = np.random.default_rng(22).standard_normal((Bn, nq, H, D))
+    QB, KB = math.ceil(nq / bq), math.ceil(nk / bk)
+    mask = (np.random.default_rng(23).random((Bn * H, QB, KB)) < 0.6).astype(np.uint8)
+    mask[0, 1] = 0                                      # a row without kept blocks
+    dq, dk, dv = O.block_sparse_attention_backward(q, k, v, do, mask, bq, bk)
+    tq, tk, tv = (torch.tensor(a, requires_grad=True) for a in (q, k, v))
+    out = []
+    for h in range(H):
+        allowed = torch.from_numpy(O.token_mask_from_blocks(mask[h], nq, nk, bq, bk))
+        s = (tq[0, :, h] @ tk[0, :, h].T) / math.sqrt(D)
+        s = s.masked_fill(~allowed, float("-inf"))
+        pr = torch.softmax(s, dim=1)
+        pr = torch.nan_to_num(pr, nan=0.0)              # rows with nothing allowed
+        out.append(pr @ tv[0, :, h])
+    o = torch.stack(out, dim=1)[None]
+    o.backward(torch.from_numpy(do))
+    for got, ref in ((dq, tq.grad), (dk, tk.grad), (dv, tv.grad)):
+        assert np.max(np.abs(got - ref.numpy())) < 1e-12
