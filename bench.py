@@ -44,7 +44,7 @@ def load_peaks():
 
 def attn_source_hash() -> str:
     h = hashlib.sha256()
-    for f in ("attn_fwd.cu", "bsa_common.cuh", "tmem_io.cuh"):
+    for f in ("attn_fwd.cu", "attn_common.cuh", "bsa_common.cuh", "tmem_io.cuh"):
         with open(os.path.join(ROOT, "block_sparse_attention_tokens_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]

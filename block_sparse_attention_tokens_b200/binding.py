@@ -25,7 +25,7 @@ EXPORTS = [
     "bsa_tile_untile", "bsa_sta_mask", "bsa_radial_mask", "bsa_nabla_workspace_size",
     "bsa_nabla_mask", "bsa_mask_compact", "bsa_attn_workspace_size", "bsa_attn_fwd",
     "bsa_attn_fwd_noalloc", "bsa_read_status", "bsa_tile_permute_pool", "bsa_nabla_select",
-    "bsa_wait_selftest",
+    "bsa_wait_selftest", "bsa_attn_bwd_workspace_size", "bsa_attn_bwd",
 ]
 
 
@@ -67,6 +67,9 @@ def load_library(path: str = _LIB_PATH) -> ctypes.CDLL:
         "bsa_attn_fwd_noalloc": (c_int, [c_void, c_void, c_void] + [c_int] * 7
                                  + [c_void, c_void, c_int, c_float, c_void, c_void, c_void,
                                     c_void]),
+        "bsa_attn_bwd_workspace_size": (c_size, [c_int] * 7),
+        "bsa_attn_bwd": (c_int, [c_void] * 6 + [c_int] * 7 + [c_void, c_void, c_int, c_float]
+                         + [c_void] * 4 + [c_size, c_void]),
         "bsa_read_status": (c_int, [c_void, ctypes.POINTER(c_int), c_void]),
         "bsa_wait_selftest": (c_int, [c_void, ctypes.c_ulonglong, c_void]),
         "bsa_tile_permute_pool": (c_int, [c_void, c_void] + [c_int] * 11 + [c_void, c_void]),
@@ -303,6 +306,38 @@ def bsa_attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                                                _ptr(device_status), _stream()),
            "bsa_attn_fwd_noalloc")
     return o, lse
+
+
+def bsa_attn_bwd_workspace_size(batch, heads, nq, nk, block_q, block_k, list_heads) -> int:
+    return int(load_library().bsa_attn_bwd_workspace_size(batch, heads, nq, nk, block_q, block_k,
+                                                          list_heads))
+
+
+def bsa_attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
+                 dout: torch.Tensor, lse: torch.Tensor, row_ptr: torch.Tensor,
+                 col_idx: torch.Tensor, block_q: int, block_k: int, list_heads: int,
+                 nq: Optional[int] = None, nk: Optional[int] = None, scale: float = 0.0,
+                 dq: Optional[torch.Tensor] = None, dk: Optional[torch.Tensor] = None,
+                 dv: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None):
+    """Block-sparse attention backward.  Returns (dq, dk, dv, ws)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout"), (lse, "lse"),
+                 (row_ptr, "row_ptr"), (col_idx, "col_idx")):
+        _cuda(t, n)
+    B, _, H, D = q.shape
+    nq = q.shape[1] if nq is None else nq
+    nk = k.shape[1] if nk is None else nk
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if ws is None:
+        ws = torch.empty(bsa_attn_bwd_workspace_size(B, H, nq, nk, block_q, block_k, list_heads),
+                         dtype=torch.uint8, device=q.device)
+    _check(load_library().bsa_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
+                                       B, H, nq, nk, D, block_q, block_k, _ptr(row_ptr),
+                                       _ptr(col_idx), list_heads, float(scale), _ptr(dq),
+                                       _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(), _stream()),
+           "bsa_attn_bwd")
+    return dq, dk, dv, ws
 
 
 def bsa_read_status(ws: torch.Tensor) -> int:

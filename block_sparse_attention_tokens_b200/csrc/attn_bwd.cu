@@ -1,0 +1,704 @@
+// Block-sparse attention backward on sm_100a: dQ, dK, dV over the kept block pairs.
+//
+// Sources: the Radial explainer (aibr.jp/archives/112136), section 4 (training cost
+// cut by the sparse mask), the NABLA explainer (aibr.jp/archives/124678), section 4
+// (training and inference speed-up) and the Sparse Forcing summary
+// (gist.science/ja/paper/2604.21221): the sparse attention is trained through.
+// With P = softmax(S), S = Q K^T * scale restricted to kept block pairs and
+// D = rowsum(dO * O):
+//     dV = P^T dO,  dP = dO V^T,  dS = P * (dP - D),  dQ = dS K * scale,  dK = dS^T Q * scale.
+// P is recomputed from the forward's log-sum-exp, so nothing else is stored.
+//
+// Two passes of one kernel template, no atomics:
+//   kDKV : one CTA per 128-key tile; iterates the q-tiles that keep it (transposed
+//          kept list).  S^T = K Q^T and dP^T = V dO^T (SS MMAs) -> P, dS in registers
+//          (thread = key row = TMEM lane) -> bf16 into TMEM -> dV += P dO and
+//          dK += dS Q (TS MMAs, A operand from TMEM).
+//   kDQ  : one CTA per 128-row q-tile; iterates its kept list.  S = Q K^T and
+//          dP = dO V^T -> dS -> dQ += dS K.
+// TMEM: S | dP | accA (dK or dQ) | accB (dV), 128 columns each; P and dS in bf16
+// over the first half of S and dP.  Warps 0-3 compute, warp 4 feeds a ring of
+// (tile, tile) pairs with TMA, warp 5 issues the MMAs.  Units are handed out from a
+// global counter through a shared-memory ring as in the forward kernel.  All waits
+// are bounded.
+#include "bsa_common.cuh"
+#include "tmem_io.cuh"
+#include "attn_common.cuh"
+
+namespace bsa {
+namespace {
+
+constexpr int kBwdThreads = 192;
+constexpr int kBwdLoadWarp = 4;
+constexpr int kBwdMmaWarp = 5;
+
+template <int D>
+struct BwdCfg {
+  static constexpr int KCH = D / 64;
+  static constexpr int CHUNK_BYTES = kBM * 128;
+  static constexpr int TILE_BYTES = KCH * CHUNK_BYTES;   // 128 rows x D bf16
+  static constexpr int NSTAGE = D == 128 ? 2 : 4;        // ring of tile pairs
+  static constexpr int OFF_ROW = 0;                      // the two row-operand tiles
+  static constexpr int OFF_RING = 2 * TILE_BYTES;
+  // per compute warp, double-buffered: (LSE2, D) x 128 floats
+  static constexpr int OFF_VEC = OFF_RING + NSTAGE * 2 * TILE_BYTES;
+  static constexpr int OFF_BAR = OFF_VEC + 4 * 2 * 2 * 128 * 4;
+  static constexpr int SMEM = OFF_BAR + 512 + 1024;
+};
+
+struct BwdParams {
+  int B, H, nq, nk, QT, KT;
+  int list_heads, LR, QB, expand, block_q;
+  int total_items;
+  float scale, scale_log2;
+  const int* row_ptr;
+  const int* cnt;
+  const uint32_t* entries;   // forward per-q-tile lists
+  const int* tcnt;
+  const uint32_t* tentries;  // transposed per-k-tile lists, stride QT
+  const float* lse2;         // [B*H][QT*128]: LSE * log2(e), +inf past nq / for empty rows
+  const float* dvec;         // [B*H][QT*128]: rowsum(dO * O), 0 past nq
+  __nv_bfloat16* outA;       // dK (kDKV) or dQ (kDQ)
+  __nv_bfloat16* outB;       // dV (kDKV)
+  int* status;
+  int* unit_counter;
+  unsigned long long timeout_ns;
+};
+
+struct BItem {
+  int b, h, row_tile, n;     // n < 0: none
+  const uint32_t* ent;
+};
+
+template <bool kDKV>
+__device__ __forceinline__ BItem get_bitem(const BwdParams& p, int it) {
+  BItem r;
+  r.n = -1;
+  r.ent = nullptr;
+  r.b = r.h = r.row_tile = 0;
+  if (it >= p.total_items) return r;
+  const int per = kDKV ? p.KT : p.QT;
+  r.row_tile = it % per;
+  const int bh = it / per;
+  r.h = bh % p.H;
+  r.b = bh / p.H;
+  const int mh = p.list_heads == 1 ? 0 : bh;
+  if (kDKV) {
+    const long long g = static_cast<long long>(mh) * p.KT + r.row_tile;
+    r.n = p.tcnt[g];
+    r.ent = p.tentries + g * p.QT;
+  } else {
+    const int lr = p.block_q >= 128 ? (r.row_tile * kBM) / p.block_q : r.row_tile;
+    const int first_qb = p.block_q >= 128 ? lr : 2 * lr;
+    r.n = p.cnt[mh * p.LR + lr];
+    r.ent = p.entries + static_cast<long long>(p.row_ptr[mh * p.QB + first_qb]) * p.expand;
+  }
+  return r;
+}
+
+// rowA / rowB: the item's fixed operands (kDKV: K, V; kDQ: Q, dO) over N_row tokens.
+// colA / colB: the per-step operands (kDKV: Q, dO; kDQ: K, V).
+template <int D, bool kDKV>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    attn_bwd_kernel(const __grid_constant__ CUtensorMap tmRowA, const __grid_constant__ CUtensorMap tmRowB,
+                    const __grid_constant__ CUtensorMap tmColA, const __grid_constant__ CUtensorMap tmColB,
+                    const BwdParams p) {
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sRow = sbase + C::OFF_ROW;
+  const uint32_t sRing = sbase + C::OFF_RING;
+  float* svec = reinterpret_cast<float*>(smem + C::OFF_VEC);
+  const uint32_t bar0 = smem_u32(smem + C::OFF_BAR);
+  auto FULL = [&](int i) { return bar0 + 8u * i; };
+  auto EMPTY = [&](int i) { return bar0 + 8u * (C::NSTAGE + i); };
+  const uint32_t ROWFULL = bar0 + 8u * (2 * C::NSTAGE + 0);
+  const uint32_t ROWEMPTY = bar0 + 8u * (2 * C::NSTAGE + 1);
+  const uint32_t SFULL = bar0 + 8u * (2 * C::NSTAGE + 2);
+  const uint32_t PREADY = bar0 + 8u * (2 * C::NSTAGE + 3);
+  const uint32_t DONE = bar0 + 8u * (2 * C::NSTAGE + 4);
+  const uint32_t FINAL = bar0 + 8u * (2 * C::NSTAGE + 5);
+  auto UFULL = [&](int i) { return bar0 + 8u * (2 * C::NSTAGE + 6 + i); };
+  auto UEMPTY = [&](int i) { return bar0 + 8u * (2 * C::NSTAGE + 10 + i); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + 8 * (2 * C::NSTAGE + 14));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* unit_ring = reinterpret_cast<volatile int*>(tmem_slot + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::NSTAGE; ++i) {
+      mbar_init(FULL(i), 1);
+      mbar_init(EMPTY(i), 1);
+    }
+    mbar_init(ROWFULL, 1);
+    mbar_init(ROWEMPTY, 1);
+    mbar_init(SFULL, 1);
+    mbar_init(PREADY, 4);
+    mbar_init(DONE, 1);
+    mbar_init(FINAL, 1);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(UFULL(i), 1);
+      mbar_init(UEMPTY(i), 1 + 4);  // MMA thread + 4 compute warps
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == kBwdMmaWarp) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(512)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == kBwdLoadWarp) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int st = 0;
+      uint32_t ph = 0, rph = 0;
+      uint32_t filled = 0, fill_phase = 0;
+      int row_filled = -1;
+      bool ok = true;
+      for (int uk = 0; ok; ++uk) {
+        const int slot = uk & 3;
+        if (!mbar_wait(UEMPTY(slot), ((uk >> 2) & 1) ^ 1u, abort_flag, p.status, p.timeout_ns)) {
+          ok = false;
+          break;
+        }
+        const int u = atomicAdd(p.unit_counter, 1);
+        unit_ring[slot] = u;
+        mbar_arrive(UFULL(slot));
+        if (u >= p.total_items) break;
+        const BItem it = get_bitem<kDKV>(p, u);
+        if (it.n <= 0) continue;
+        if (!mbar_wait(ROWEMPTY, rph ^ 1u, abort_flag, p.status, p.timeout_ns)) {
+          ok = false;
+          break;
+        }
+        row_filled = static_cast<int>(rph);
+        rph ^= 1u;
+        mbar_expect_tx(ROWFULL, 2 * C::TILE_BYTES);
+        for (int c = 0; c < C::KCH; ++c) {
+          tma_load_4d(sRow + c * C::CHUNK_BYTES, &tmRowA, ROWFULL, 64 * c, it.h,
+                      it.row_tile * kBM, it.b);
+          tma_load_4d(sRow + C::TILE_BYTES + c * C::CHUNK_BYTES, &tmRowB, ROWFULL, 64 * c, it.h,
+                      it.row_tile * kBM, it.b);
+        }
+        for (int j = 0; j < it.n && ok; ++j) {
+          if (!mbar_wait(EMPTY(st), ph ^ 1u, abort_flag, p.status, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          const int ct = static_cast<int>(__ldg(it.ent + j) & 0x0FFFFFFFu);
+          mbar_expect_tx(FULL(st), 2 * C::TILE_BYTES);
+          const uint32_t dst = sRing + st * 2 * C::TILE_BYTES;
+          for (int c = 0; c < C::KCH; ++c) {
+            tma_load_4d(dst + c * C::CHUNK_BYTES, &tmColA, FULL(st), 64 * c, it.h, ct * kBM, it.b);
+            tma_load_4d(dst + C::TILE_BYTES + c * C::CHUNK_BYTES, &tmColB, FULL(st), 64 * c, it.h,
+                        ct * kBM, it.b);
+          }
+          filled |= 1u << st;
+          fill_phase = (fill_phase & ~(1u << st)) | (ph << st);
+          if (++st == C::NSTAGE) { st = 0; ph ^= 1u; }
+        }
+      }
+      for (int i = 0; i < C::NSTAGE; ++i)
+        if (filled & (1u << i))
+          mbar_wait_drain(FULL(i), (fill_phase >> i) & 1u, p.status, p.timeout_ns);
+      if (row_filled >= 0)
+        mbar_wait_drain(ROWFULL, static_cast<uint32_t>(row_filled), p.status, p.timeout_ns);
+    }
+  } else if (warp == kBwdMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_ss = idesc_bf16_f32(kBM, kBN, 0, 0);
+      constexpr uint32_t idesc_ts = idesc_bf16_f32(kBM, D, 0, 1);
+      constexpr uint32_t kTileUnits = C::TILE_BYTES >> 4;
+      const uint64_t dRowK = smem_desc_sw128(sRow, 16, 1024);
+      const uint64_t dColK = smem_desc_sw128(sRing, 16, 1024);
+      const uint64_t dColMN = smem_desc_sw128(sRing, C::CHUNK_BYTES, 1024);
+      int st = 0;
+      uint32_t ph = 0, rph = 0, pph = 0;
+      bool ok = true;
+      auto acquire = [&](int& stage) -> bool {
+        if (!mbar_wait(FULL(st), ph, abort_flag, p.status, p.timeout_ns)) return false;
+        stage = st;
+        if (++st == C::NSTAGE) { st = 0; ph ^= 1u; }
+        return true;
+      };
+      // S-like (rowA colA^T) into TMEM [0,128), dP-like (rowB colB^T) into [128,256)
+      auto mma_sd = [&](int stage) {
+        tc_fence_after();
+        const uint64_t dcol = dColK + static_cast<uint64_t>(stage * 2 * kTileUnits);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t off =
+              static_cast<uint64_t>((((kk >> 2) * C::CHUNK_BYTES) + (kk & 3) * 32) >> 4);
+          mma_ss(tmem, dRowK + off, dcol + off, idesc_ss, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t off =
+              static_cast<uint64_t>((((kk >> 2) * C::CHUNK_BYTES) + (kk & 3) * 32) >> 4);
+          mma_ss(tmem + 128, dRowK + kTileUnits + off, dcol + kTileUnits + off, idesc_ss,
+                 kk > 0 ? 1u : 0u);
+        }
+      };
+      // accA (+)= dS colA ; accB (+)= P colB (kDKV only); A operands from TMEM
+      auto mma_acc = [&](int stage, int step) {
+        tc_fence_after();
+        const uint64_t dA = dColMN + static_cast<uint64_t>(stage * 2 * kTileUnits);
+        const uint64_t dB = dA + kTileUnits;
+        const uint32_t acc0 = step > 0 ? 1u : 0u;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          mma_ts(tmem + 256, tmem + 128 + kk * 8, dA + static_cast<uint64_t>(kk * 128), idesc_ts,
+                 kk > 0 ? 1u : acc0);
+        if (kDKV) {
+#pragma unroll
+          for (int kk = 0; kk < kBN / 16; ++kk)
+            mma_ts(tmem + 384, tmem + kk * 8, dB + static_cast<uint64_t>(kk * 128), idesc_ts,
+                   kk > 0 ? 1u : acc0);
+        }
+      };
+      for (int uk = 0; ok; ++uk) {
+        const int slot = uk & 3;
+        if (!mbar_wait(UFULL(slot), (uk >> 2) & 1, abort_flag, p.status, p.timeout_ns)) {
+          ok = false;
+          break;
+        }
+        const int u = unit_ring[slot];
+        mbar_arrive(UEMPTY(slot));
+        if (u >= p.total_items) break;
+        const BItem it = get_bitem<kDKV>(p, u);
+        if (it.n <= 0) continue;
+        if (!mbar_wait(ROWFULL, rph, abort_flag, p.status, p.timeout_ns)) {
+          ok = false;
+          break;
+        }
+        rph ^= 1u;
+        int cur = 0;
+        if (!acquire(cur)) { ok = false; break; }
+        mma_sd(cur);
+        mma_commit(SFULL);
+        if (it.n == 1) mma_commit(ROWEMPTY);
+        for (int j = 0; j < it.n && ok; ++j) {
+          if (!mbar_wait(PREADY, pph, abort_flag, p.status, p.timeout_ns)) { ok = false; break; }
+          pph ^= 1u;
+          mma_acc(cur, j);
+          mma_commit(EMPTY(cur));
+          if (j == it.n - 1) {
+            mma_commit(DONE);
+          } else {
+            int nxt = 0;
+            if (!acquire(nxt)) { ok = false; break; }
+            mma_sd(nxt);
+            mma_commit(SFULL);
+            if (j + 1 == it.n - 1) mma_commit(ROWEMPTY);
+            cur = nxt;
+          }
+        }
+      }
+      mma_commit(FINAL);
+      mbar_wait_drain(FINAL, 0, p.status, p.timeout_ns);
+    }
+  } else {
+    // ------------------------------------------------------------ compute (4 warps)
+    const int row = threadIdx.x;  // 0..127 = TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_base;
+    const uint32_t tP = tmem + lane_base + 128;
+    const uint32_t tA = tmem + lane_base + 256;
+    const uint32_t tB = tmem + lane_base + 384;
+    const int rh = row >> 6;  // which 64-row half of the row tile
+    const float sl2 = p.scale_log2;
+    uint32_t sph = 0, dph = 0;
+    bool ok = true;
+    int vstep = 0;  // steps taken (selects the smem vector buffer in kDKV)
+    for (int uk = 0; ok; ++uk) {
+      const int slot = uk & 3;
+      if (!mbar_wait(UFULL(slot), (uk >> 2) & 1, abort_flag, p.status, p.timeout_ns)) {
+        ok = false;
+        break;
+      }
+      const int u = unit_ring[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(UEMPTY(slot));
+      if (u >= p.total_items) break;
+      const BItem it = get_bitem<kDKV>(p, u);
+      if (it.n < 0) continue;
+      const long long bh = static_cast<long long>(it.b) * p.H + it.h;
+      const int grow = it.row_tile * kBM + row;          // global row of this thread
+      float lse_row = 0.f, d_row = 0.f;
+      if (!kDKV) {
+        lse_row = p.lse2[bh * (p.QT * kBM) + grow];
+        d_row = p.dvec[bh * (p.QT * kBM) + grow];
+      }
+      for (int j = 0; j < it.n; ++j) {
+        const uint32_t ent = __ldg(it.ent + j);
+        const int ct = static_cast<int>(ent & 0x0FFFFFFFu);
+        const uint32_t bits = ent >> 28;
+        // this step's per-column LSE2 and D (128 query columns) into this warp's own
+        // shared-memory copy (double-buffered; __syncwarp orders writes and reads)
+        float* vbuf = svec + ((warp & 3) * 2 + (vstep & 1)) * 256;
+        if (kDKV) {
+          const float* l2 = p.lse2 + bh * (p.QT * kBM) + ct * kBM;
+          const float* dv2 = p.dvec + bh * (p.QT * kBM) + ct * kBM;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            vbuf[lane + 32 * i] = __ldg(l2 + lane + 32 * i);
+            vbuf[128 + lane + 32 * i] = __ldg(dv2 + lane + 32 * i);
+          }
+          __syncwarp();
+        }
+        ++vstep;
+        ok = mbar_wait(SFULL, sph, abort_flag, p.status, p.timeout_ns);
+        if (!ok) break;
+        sph ^= 1u;
+        tc_fence_after();
+        // quadrant mask: bit (row_half * 2 + column_half); the ragged column tail of
+        // the dQ pass (keys past nk) is masked per column
+        const bool lo_ok = (bits >> (rh * 2)) & 1u, hi_ok = (bits >> (rh * 2 + 1)) & 1u;
+        const int cvalid = kDKV ? kBN : p.nk - ct * kBN;
+#pragma unroll 1
+        for (int c0 = 0; c0 < kBN; c0 += 32) {
+          uint32_t sr[32], dr[32];
+          tmem_ld32x32b_x32(tS + c0, sr);
+          tmem_ld32x32b_x32(tP + c0, dr);
+          const bool half_ok = c0 < 64 ? lo_ok : hi_ok;
+          uint32_t ppk[16], dpk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float pv[2], dsv[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int c = c0 + 2 * i + e;
+              const float lse = kDKV ? vbuf[c] : lse_row;
+              const float dd = kDKV ? vbuf[128 + c] : d_row;
+              float pr = fast_exp2(fmaf(__uint_as_float(sr[2 * i + e]), sl2, -lse));
+              if (!half_ok || c >= cvalid) pr = 0.f;
+              pv[e] = pr;
+              dsv[e] = pr * (__uint_as_float(dr[2 * i + e]) - dd);
+            }
+            __nv_bfloat162 hp = __floats2bfloat162_rn(pv[0], pv[1]);
+            __nv_bfloat162 hd = __floats2bfloat162_rn(dsv[0], dsv[1]);
+            ppk[i] = *reinterpret_cast<uint32_t*>(&hp);
+            dpk[i] = *reinterpret_cast<uint32_t*>(&hd);
+          }
+          if (kDKV) tmem_st32x32b_x16(tS + c0 / 2, ppk);
+          tmem_st32x32b_x16(tP + c0 / 2, dpk);
+        }
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(PREADY);
+      }
+      if (!ok) break;
+      // epilogue: accA * scale -> outA, accB -> outB (rows past the tensor end skipped)
+      const int nrows = kDKV ? p.nk : p.nq;
+      __nv_bfloat16* rowA = p.outA + ((static_cast<long long>(it.b) * nrows + grow) * p.H + it.h) * D;
+      __nv_bfloat16* rowB =
+          kDKV ? p.outB + ((static_cast<long long>(it.b) * nrows + grow) * p.H + it.h) * D : nullptr;
+      if (it.n > 0) {
+        ok = mbar_wait(DONE, dph, abort_flag, p.status, p.timeout_ns);
+        if (!ok) break;
+        dph ^= 1u;
+        tc_fence_after();
+      }
+#pragma unroll 1
+      for (int pass = 0; pass < (kDKV ? 2 : 1); ++pass) {
+        const uint32_t tacc = pass == 0 ? tA : tB;
+        __nv_bfloat16* dst_row = pass == 0 ? rowA : rowB;
+        const float mul = pass == 0 ? p.scale : 1.0f;
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t ov[32];
+          if (it.n > 0) {
+            tmem_ld32x32b_x32(tacc + c0, ov);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ov[i] = 0u;
+          }
+          if (grow < nrows) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(ov[2 * i]) * mul,
+                                                        __uint_as_float(ov[2 * i + 1]) * mul);
+              pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+            }
+            uint4* d4 = reinterpret_cast<uint4*>(dst_row + c0);
+            d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            d4[2] = make_uint4(pk[8], pk[9], pk[10], pk[11]);
+            d4[3] = make_uint4(pk[12], pk[13], pk[14], pk[15]);
+          }
+        }
+      }
+      tc_fence_before();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kBwdMmaWarp) {
+    __syncwarp();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512)
+                 : "memory");
+  }
+}
+
+// LSE * log2(e) and rowsum(dO * O) per (b, h, row), padded to whole 128-row tiles:
+// rows past nq (and rows whose LSE is -inf, i.e. no kept key) get +inf / 0 so
+// their recomputed probabilities are exactly 0.
+__global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ o,
+                                const __nv_bfloat16* __restrict__ dout,
+                                const float* __restrict__ lse, int B, int H, int nq, int D,
+                                int rows_pad, float* __restrict__ lse2, float* __restrict__ dvec) {
+  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long total = static_cast<long long>(B) * H * rows_pad;
+  if (idx >= total) return;
+  const int i = static_cast<int>(idx % rows_pad);
+  const long long bh = idx / rows_pad;
+  const int h = static_cast<int>(bh % H), b = static_cast<int>(bh / H);
+  if (i >= nq) {
+    lse2[idx] = INFINITY;
+    dvec[idx] = 0.f;
+    return;
+  }
+  const float l = lse[bh * nq + i];
+  lse2[idx] = l == -INFINITY ? INFINITY : l * 1.4426950408889634f;
+  const uint4* po = reinterpret_cast<const uint4*>(o + ((static_cast<long long>(b) * nq + i) * H + h) * D);
+  const uint4* pd = reinterpret_cast<const uint4*>(dout + ((static_cast<long long>(b) * nq + i) * H + h) * D);
+  float acc = 0.f;
+  for (int c = 0; c < D / 8; ++c) {
+    const uint4 a = __ldg(po + c), g = __ldg(pd + c);
+    const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+    const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&g);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 fa = __bfloat1622float2(a2[e]), fg = __bfloat1622float2(g2[e]);
+      acc = fmaf(fa.x, fg.x, acc);
+      acc = fmaf(fa.y, fg.y, acc);
+    }
+  }
+  dvec[idx] = acc;
+}
+
+// Transposed kept lists.  Pass 1: every q-tile ORs its entries, with the quadrant
+// bits transposed (bit q_half*2 + k_half -> k_half*2 + q_half), into a dense
+// nibble map [mask head][k-tile][q-tile].  Pass 2: one CTA per (mask head, k-tile)
+// compacts its map row into an ascending list of q-tiles.
+__global__ void tmap_kernel(const int* __restrict__ row_ptr, const int* __restrict__ cnt,
+                            const uint32_t* __restrict__ entries, int QT, int KT, int LR, int QB,
+                            int block_q, int expand, int list_heads,
+                            uint32_t* __restrict__ map) {
+  const int g = blockIdx.x;  // mask head * QT + q-tile
+  const int mh = g / QT, qt = g - mh * QT;
+  if (mh >= list_heads) return;
+  const int lr = block_q >= 128 ? (qt * kBM) / block_q : qt;
+  const int first_qb = block_q >= 128 ? lr : 2 * lr;
+  const int n = cnt[mh * LR + lr];
+  const uint32_t* ent = entries + static_cast<long long>(row_ptr[mh * QB + first_qb]) * expand;
+  const int words = (QT + 7) / 8;
+  for (int j = threadIdx.x; j < n; j += blockDim.x) {
+    const uint32_t e = ent[j];
+    const int kt = static_cast<int>(e & 0x0FFFFFFFu);
+    const uint32_t b = e >> 28;
+    const uint32_t tb = (b & 1u) | ((b >> 1) & 1u) << 2 | ((b >> 2) & 1u) << 1 | ((b >> 3) & 1u) << 3;
+    atomicOr(&map[(static_cast<long long>(mh) * KT + kt) * words + (qt >> 3)], tb << (4 * (qt & 7)));
+  }
+}
+
+__global__ void __launch_bounds__(256) tcompact_kernel(const uint32_t* __restrict__ map, int QT,
+                                                       int KT, int* __restrict__ tcnt,
+                                                       uint32_t* __restrict__ tentries) {
+  __shared__ int warp_sums[8];
+  const long long g = blockIdx.x;  // mask head * KT + k-tile
+  const int words = (QT + 7) / 8;
+  const uint32_t* row = map + g * words;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int per = (words + 255) / 256;
+  const int w0 = min(words, tid * per), w1 = min(words, w0 + per);
+  int mine = 0;
+  for (int w = w0; w < w1; ++w) {
+    const uint32_t q = row[w];
+    for (int j = 0; j < 8; ++j) mine += ((q >> (4 * j)) & 0xFu) != 0u;
+  }
+  int incl = mine;
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  int base = 0;
+  for (int w = 0; w < warp; ++w) base += warp_sums[w];
+  int pos = base + incl - mine;
+  uint32_t* out = tentries + g * QT;
+  for (int w = w0; w < w1; ++w) {
+    const uint32_t q = row[w];
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t bits = (q >> (4 * j)) & 0xFu;
+      if (bits) out[pos++] = static_cast<uint32_t>(w * 8 + j) | (bits << 28);
+    }
+  }
+  if (tid == 255) tcnt[g] = pos;
+}
+
+struct BwdGeometry {
+  Geometry fwd;
+  int KT;
+  size_t tcnt_off, tent_off, map_off, lse_off, dvec_off, total;
+};
+
+BwdGeometry bwd_geometry(int batch, int heads, int nq, int nk, int block_q, int block_k,
+                         int list_heads) {
+  BwdGeometry g;
+  g.fwd = geometry(batch, heads, nq, nk, block_q, block_k, list_heads);
+  g.KT = ceil_div(nk, kBN);
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  const size_t mhk = static_cast<size_t>(list_heads) * g.KT;
+  g.tcnt_off = up(g.fwd.total);
+  g.tent_off = up(g.tcnt_off + sizeof(int) * mhk);
+  g.map_off = up(g.tent_off + sizeof(uint32_t) * mhk * g.fwd.QT);
+  g.lse_off = up(g.map_off + sizeof(uint32_t) * mhk * ((g.fwd.QT + 7) / 8));
+  const size_t vec = sizeof(float) * static_cast<size_t>(batch) * heads * g.fwd.QT * kBM;
+  g.dvec_off = up(g.lse_off + vec);
+  g.total = g.dvec_off + vec;
+  return g;
+}
+
+template <int D, bool kDKV>
+int launch_bwd(const CUtensorMap& ra, const CUtensorMap& rb, const CUtensorMap& ca,
+               const CUtensorMap& cb, const BwdParams& p, cudaStream_t st) {
+  using C = BwdCfg<D>;
+  cudaError_t e = cudaFuncSetAttribute(attn_bwd_kernel<D, kDKV>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return record_cuda_error(e);
+  int grid = device_sm_count();
+  if (grid > p.total_items) grid = p.total_items;
+  if (grid < 1) grid = 1;
+  attn_bwd_kernel<D, kDKV><<<grid, kBwdThreads, C::SMEM, st>>>(ra, rb, ca, cb, p);
+  return check_launch();
+}
+
+}  // namespace
+}  // namespace bsa
+
+extern "C" size_t bsa_attn_bwd_workspace_size(int batch, int heads, int nq, int nk, int block_q,
+                                              int block_k, int list_heads) {
+  if (batch < 1 || heads < 1 || nq < 1 || nk < 1 || !bsa::block_ok(block_q) ||
+      !bsa::block_ok(block_k) || list_heads < 1)
+    return 0;
+  return bsa::bwd_geometry(batch, heads, nq, nk, block_q, block_k, list_heads).total;
+}
+
+extern "C" int bsa_attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                            const void* dout, const float* lse, int batch, int heads, int nq,
+                            int nk, int head_dim, int block_q, int block_k, const int* row_ptr,
+                            const int* col_idx, int list_heads, float scale, void* dq, void* dk,
+                            void* dv, void* ws, size_t ws_bytes, void* stream) {
+  using namespace bsa;
+  if (!q || !k || !v || !o || !dout || !lse || !row_ptr || !col_idx || !dq || !dk || !dv || !ws)
+    return BSA_ERR_INVALID_ARG;
+  if (batch < 1 || heads < 1 || nq < 1 || nk < 1) return BSA_ERR_INVALID_ARG;
+  if (list_heads != 1 && list_heads != batch * heads) return BSA_ERR_INVALID_ARG;
+  for (const void* ptr : {q, k, v, o, dout, static_cast<const void*>(dq),
+                          static_cast<const void*>(dk), static_cast<const void*>(dv),
+                          static_cast<const void*>(ws)})
+    if (!aligned16(ptr)) return BSA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return BSA_ERR_UNSUPPORTED;
+  if (!block_ok(block_q) || !block_ok(block_k)) return BSA_ERR_UNSUPPORTED;
+  const BwdGeometry g = bwd_geometry(batch, heads, nq, nk, block_q, block_k, list_heads);
+  if (ws_bytes < g.total) return BSA_ERR_WORKSPACE;
+  if (g.fwd.nnz_cap > 0x7fffffffLL || static_cast<long long>(g.KT) >= (1LL << 28) ||
+      static_cast<long long>(batch) * heads * (g.fwd.QT > g.KT ? g.fwd.QT : g.KT) > 0x3fffffffLL)
+    return BSA_ERR_UNSUPPORTED;
+  if (scale <= 0.0f) scale = 1.0f / sqrtf(static_cast<float>(head_dim));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  CUtensorMap mq, mk, mv, mdo;
+  if (make_map(&mq, q, batch, nq, heads, head_dim) != BSA_OK ||
+      make_map(&mk, k, batch, nk, heads, head_dim) != BSA_OK ||
+      make_map(&mv, v, batch, nk, heads, head_dim) != BSA_OK ||
+      make_map(&mdo, dout, batch, nq, heads, head_dim) != BSA_OK)
+    return BSA_ERR_CUDA;
+
+  char* wsb = static_cast<char*>(ws);
+  int* status = reinterpret_cast<int*>(wsb);
+  int* cnt = reinterpret_cast<int*>(wsb + g.fwd.cnt_off);
+  uint32_t* entries = reinterpret_cast<uint32_t*>(wsb + g.fwd.ent_off);
+  int* tcnt = reinterpret_cast<int*>(wsb + g.tcnt_off);
+  uint32_t* tentries = reinterpret_cast<uint32_t*>(wsb + g.tent_off);
+  uint32_t* map = reinterpret_cast<uint32_t*>(wsb + g.map_off);
+  float* lse2 = reinterpret_cast<float*>(wsb + g.lse_off);
+  float* dvec = reinterpret_cast<float*>(wsb + g.dvec_off);
+
+  // status word + two unit counters
+  cudaError_t e = cudaMemsetAsync(status, 0, 3 * sizeof(int), st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(map, 0, g.lse_off - g.map_off, st);
+  if (e != cudaSuccess) return record_cuda_error(e);
+  int rc = launch_build_lists(row_ptr, col_idx, list_heads, g.fwd, nk, block_q, block_k, cnt,
+                              entries, status, st);
+  if (rc != BSA_OK) return rc;
+  const int rows_pad = g.fwd.QT * kBM;
+  const long long prep_total = static_cast<long long>(batch) * heads * rows_pad;
+  bwd_prep_kernel<<<static_cast<int>(ceil_div<long long>(prep_total, 256)), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, batch,
+      heads, nq, head_dim, rows_pad, lse2, dvec);
+  if ((rc = check_launch()) != BSA_OK) return rc;
+  tmap_kernel<<<list_heads * g.fwd.QT, 128, 0, st>>>(row_ptr, cnt, entries, g.fwd.QT, g.KT,
+                                                     g.fwd.LR, g.fwd.QB, block_q, g.fwd.expand,
+                                                     list_heads, map);
+  if ((rc = check_launch()) != BSA_OK) return rc;
+  tcompact_kernel<<<list_heads * g.KT, 256, 0, st>>>(map, g.fwd.QT, g.KT, tcnt, tentries);
+  if ((rc = check_launch()) != BSA_OK) return rc;
+
+  BwdParams p;
+  p.B = batch;
+  p.H = heads;
+  p.nq = nq;
+  p.nk = nk;
+  p.QT = g.fwd.QT;
+  p.KT = g.KT;
+  p.list_heads = list_heads;
+  p.LR = g.fwd.LR;
+  p.QB = g.fwd.QB;
+  p.expand = g.fwd.expand;
+  p.block_q = block_q;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.row_ptr = row_ptr;
+  p.cnt = cnt;
+  p.entries = entries;
+  p.tcnt = tcnt;
+  p.tentries = tentries;
+  p.lse2 = lse2;
+  p.dvec = dvec;
+  p.status = status;
+  p.timeout_ns = 2000000000ULL;
+  // pass 1: dK, dV (rows = key tiles, columns = q-tiles)
+  p.total_items = batch * heads * g.KT;
+  p.outA = static_cast<__nv_bfloat16*>(dk);
+  p.outB = static_cast<__nv_bfloat16*>(dv);
+  p.unit_counter = status + 1;
+  rc = head_dim == 128 ? launch_bwd<128, true>(mk, mv, mq, mdo, p, st)
+                       : launch_bwd<64, true>(mk, mv, mq, mdo, p, st);
+  if (rc != BSA_OK) return rc;
+  // pass 2: dQ (rows = q-tiles, columns = key tiles)
+  p.total_items = batch * heads * g.fwd.QT;
+  p.outA = static_cast<__nv_bfloat16*>(dq);
+  p.outB = nullptr;
+  p.unit_counter = status + 2;
+  return head_dim == 128 ? launch_bwd<128, false>(mq, mdo, mk, mv, p, st)
+                         : launch_bwd<64, false>(mq, mdo, mk, mv, p, st);
+}

@@ -222,6 +222,38 @@ int bsa_attn_fwd(const void* q, const void* k, const void* v, int batch, int hea
                  void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * (e) Block-sparse attention backward.
+ * Sources: Radial explainer (aibr.jp/archives/112136) section 4 (training cost
+ * falls with the sparse mask), NABLA explainer (aibr.jp/archives/124678)
+ * section 4 (training and inference speed-up), Sparse Forcing summary
+ * (gist.science/ja/paper/2604.21221): the sparse attention is trained through.
+ *
+ *   Gradients of bsa_attn_fwd with respect to q, k and v, for the same kept
+ *   block pairs: with P the forward's probabilities (recomputed from lse),
+ *   Delta[i] = sum_d dO[i,d] * O[i,d],
+ *     dV[j] = sum_i P[i,j] dO[i]
+ *     dS[i,j] = P[i,j] * (dO[i] . V[j] - Delta[i])
+ *     dQ[i] = scale * sum_j dS[i,j] K[j],   dK[j] = scale * sum_i dS[i,j] Q[i]
+ *   q, k, v, row_ptr, col_idx, list_heads, scale : as passed to bsa_attn_fwd
+ *   o, lse : that call's outputs; dout : dL/dO, same layout as o (bf16)
+ *   dq : [batch, nq, heads, head_dim] bf16, written (rows with no kept key: 0)
+ *   dk, dv : [batch, nk, heads, head_dim] bf16, written (keys no row keeps: 0)
+ *   head_dim in {64, 128}; block_q, block_k each 64 or a multiple of 128.
+ *   ws : device workspace of at least bsa_attn_bwd_workspace_size() bytes (its
+ *        status word, read with bsa_read_status, is cleared by every call).
+ *   Two kernel passes, no atomics: dK/dV per 128-key tile over the transposed
+ *   kept lists, then dQ per 128-query tile.  Pointer arguments must be 16-byte
+ *   aligned; errors as for bsa_attn_fwd.
+ * ------------------------------------------------------------------------- */
+size_t bsa_attn_bwd_workspace_size(int batch, int heads, int nq, int nk, int block_q,
+                                   int block_k, int list_heads);
+int bsa_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                 const float* lse, int batch, int heads, int nq, int nk, int head_dim,
+                 int block_q, int block_k, const int* row_ptr, const int* col_idx,
+                 int list_heads, float scale, void* dq, void* dk, void* dv, void* ws,
+                 size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * (d') Block-sparse attention forward that allocates nothing.
  * No counterpart in the pages: this is a library convenience, not part of the
  * method.
