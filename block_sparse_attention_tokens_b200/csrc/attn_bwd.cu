@@ -16,9 +16,10 @@
 //          dK += dS Q (TS MMAs, A operand from TMEM).
 //   kDQ  : one CTA per 128-row q-tile; iterates its kept list.  S = Q K^T and
 //          dP = dO V^T -> dS -> dQ += dS K.
-// TMEM: S | dP | accA (dK or dQ) | accB (dV), 128 columns each; P and dS in bf16
-// over the first half of S and dP.  Warps 0-3 compute, warp 4 feeds a ring of
-// (tile, tile) pairs with TMA, warp 5 issues the MMAs.  Units are handed out from a
+// TMEM: two (S | dP) half-step buffers of 64 + 64 columns, accA (dK or dQ) and
+// accB (dV) of 128 columns each; P and dS in bf16 over the S and dP columns they
+// came from.  Warps 0-7 compute (two per TMEM lane quarter, 32 columns each),
+// warp 8 feeds a ring of (half, half) pairs with TMA, warp 9 issues the MMAs.  Units are handed out from a
 // global counter through a shared-memory ring as in the forward kernel.  All waits
 // are bounded.
 #include "bsa_common.cuh"
@@ -28,21 +29,37 @@
 namespace bsa {
 namespace {
 
-constexpr int kBwdThreads = 192;
-constexpr int kBwdLoadWarp = 4;
-constexpr int kBwdMmaWarp = 5;
+// Optional per-half-step timeline of CTA 0 of the dK/dV pass (SM clock), compiled
+// only with -DBSA_TRACE and read back with bsa_btrace_dump().
+#ifdef BSA_TRACE
+__device__ unsigned long long g_bsa_btrace[1 << 16];
+#define BSA_BTRACE_AT(half, slot)                                                      \
+  do {                                                                                 \
+    if (kDKV && blockIdx.x == 0 && (half) < (1 << 13)) g_bsa_btrace[(half) * 8 + (slot)] = clock64(); \
+  } while (0)
+#else
+#define BSA_BTRACE_AT(half, slot) \
+  do {                            \
+  } while (0)
+#endif
+
+constexpr int kBwdThreads = 320;
+constexpr int kBwdLoadWarp = 8;
+constexpr int kBwdMmaWarp = 9;
 
 template <int D>
 struct BwdCfg {
   static constexpr int KCH = D / 64;
-  static constexpr int CHUNK_BYTES = kBM * 128;
-  static constexpr int TILE_BYTES = KCH * CHUNK_BYTES;   // 128 rows x D bf16
-  static constexpr int NSTAGE = D == 128 ? 2 : 4;        // ring of tile pairs
+  static constexpr int CHUNK_BYTES = kBM * 128;          // 128 rows of one 64-column chunk
+  static constexpr int TILE_BYTES = KCH * CHUNK_BYTES;   // 128 rows x D bf16 (row operands)
+  static constexpr int HCHUNK_BYTES = 64 * 128;          // 64 rows of one chunk
+  static constexpr int HALF_BYTES = KCH * HCHUNK_BYTES;  // 64 rows x D bf16 (column halves)
+  // ring of (colA, colB) half pairs: as deep as shared memory allows, since a
+  // half-step load takes several half-steps of MMA time to arrive
+  static constexpr int NSTAGE = D == 128 ? 5 : 12;
   static constexpr int OFF_ROW = 0;                      // the two row-operand tiles
   static constexpr int OFF_RING = 2 * TILE_BYTES;
-  // per compute warp, double-buffered: (LSE2, D) x 128 floats
-  static constexpr int OFF_VEC = OFF_RING + NSTAGE * 2 * TILE_BYTES;
-  static constexpr int OFF_BAR = OFF_VEC + 4 * 2 * 2 * 128 * 4;
+  static constexpr int OFF_BAR = OFF_RING + NSTAGE * 2 * HALF_BYTES;
   static constexpr int SMEM = OFF_BAR + 512 + 1024;
 };
 
@@ -56,6 +73,8 @@ struct BwdParams {
   const uint32_t* entries;   // forward per-q-tile lists
   const int* tcnt;
   const uint32_t* tentries;  // transposed per-k-tile lists, stride QT
+  const int* qhcnt;          // half-steps of each forward list (dQ pass)
+  const int* thcnt;          // half-steps of each transposed list (dK/dV pass)
   const float* lse2;         // [B*H][QT*128]: LSE * log2(e), +inf past nq / for empty rows
   const float* dvec;         // [B*H][QT*128]: rowsum(dO * O), 0 past nq
   __nv_bfloat16* outA;       // dK (kDKV) or dQ (kDQ)
@@ -67,6 +86,7 @@ struct BwdParams {
 
 struct BItem {
   int b, h, row_tile, n;     // n < 0: none
+  int nh;                    // half-steps (needed 64-column halves) of the list
   const uint32_t* ent;
 };
 
@@ -74,6 +94,7 @@ template <bool kDKV>
 __device__ __forceinline__ BItem get_bitem(const BwdParams& p, int it) {
   BItem r;
   r.n = -1;
+  r.nh = 0;
   r.ent = nullptr;
   r.b = r.h = r.row_tile = 0;
   if (it >= p.total_items) return r;
@@ -86,18 +107,30 @@ __device__ __forceinline__ BItem get_bitem(const BwdParams& p, int it) {
   if (kDKV) {
     const long long g = static_cast<long long>(mh) * p.KT + r.row_tile;
     r.n = p.tcnt[g];
+    r.nh = p.thcnt[g];
     r.ent = p.tentries + g * p.QT;
   } else {
     const int lr = p.block_q >= 128 ? (r.row_tile * kBM) / p.block_q : r.row_tile;
     const int first_qb = p.block_q >= 128 ? lr : 2 * lr;
     r.n = p.cnt[mh * p.LR + lr];
+    r.nh = p.qhcnt[mh * p.LR + lr];
     r.ent = p.entries + static_cast<long long>(p.row_ptr[mh * p.QB + first_qb]) * p.expand;
   }
   return r;
 }
 
-// rowA / rowB: the item's fixed operands (kDKV: K, V; kDQ: Q, dO) over N_row tokens.
-// colA / colB: the per-step operands (kDKV: Q, dO; kDQ: K, V).
+// Entry quadrant bits are (row_half * 2 + column_half): column half h of an entry
+// is needed when either row half keeps it.
+__device__ __forceinline__ bool half_needed(uint32_t bits, int h) {
+  return ((bits >> h) | (bits >> (2 + h))) & 1u;
+}
+
+// rowA / rowB: the item's fixed operands (kDKV: K, V; kDQ: Q, dO), 128-row tiles.
+// colA / colB: the per-step operands (kDKV: Q, dO; kDQ: K, V), loaded and consumed
+// as 64-row halves (one half-step = 64 columns of S and dP); halves that no row of
+// the tile keeps are neither loaded nor computed.  S and dP of a half-step go to one
+// of two TMEM buffers (S at 128*buf, dP at 128*buf + 64), so the tensor core works
+// on the next half-step while the compute warps turn this one into P and dS.
 template <int D, bool kDKV>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tmRowA, const __grid_constant__ CUtensorMap tmRowB,
@@ -110,19 +143,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t sbase = smem_u32(smem);
   const uint32_t sRow = sbase + C::OFF_ROW;
   const uint32_t sRing = sbase + C::OFF_RING;
-  float* svec = reinterpret_cast<float*>(smem + C::OFF_VEC);
   const uint32_t bar0 = smem_u32(smem + C::OFF_BAR);
   auto FULL = [&](int i) { return bar0 + 8u * i; };
   auto EMPTY = [&](int i) { return bar0 + 8u * (C::NSTAGE + i); };
   const uint32_t ROWFULL = bar0 + 8u * (2 * C::NSTAGE + 0);
   const uint32_t ROWEMPTY = bar0 + 8u * (2 * C::NSTAGE + 1);
-  const uint32_t SFULL = bar0 + 8u * (2 * C::NSTAGE + 2);
-  const uint32_t PREADY = bar0 + 8u * (2 * C::NSTAGE + 3);
-  const uint32_t DONE = bar0 + 8u * (2 * C::NSTAGE + 4);
-  const uint32_t FINAL = bar0 + 8u * (2 * C::NSTAGE + 5);
-  auto UFULL = [&](int i) { return bar0 + 8u * (2 * C::NSTAGE + 6 + i); };
-  auto UEMPTY = [&](int i) { return bar0 + 8u * (2 * C::NSTAGE + 10 + i); };
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + 8 * (2 * C::NSTAGE + 14));
+  auto SFULL = [&](uint32_t b) { return bar0 + 8u * (2 * C::NSTAGE + 2 + b); };
+  auto PREADY = [&](uint32_t b) { return bar0 + 8u * (2 * C::NSTAGE + 4 + b); };
+  const uint32_t DONE = bar0 + 8u * (2 * C::NSTAGE + 6);
+  const uint32_t FINAL = bar0 + 8u * (2 * C::NSTAGE + 7);
+  auto UFULL = [&](int i) { return bar0 + 8u * (2 * C::NSTAGE + 8 + i); };
+  auto UEMPTY = [&](int i) { return bar0 + 8u * (2 * C::NSTAGE + 12 + i); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + 8 * (2 * C::NSTAGE + 16));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* unit_ring = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
@@ -134,13 +166,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     mbar_init(ROWFULL, 1);
     mbar_init(ROWEMPTY, 1);
-    mbar_init(SFULL, 1);
-    mbar_init(PREADY, 4);
+    for (uint32_t b = 0; b < 2; ++b) {
+      mbar_init(SFULL(b), 1);
+      mbar_init(PREADY(b), 8);
+    }
     mbar_init(DONE, 1);
     mbar_init(FINAL, 1);
     for (int i = 0; i < 4; ++i) {
       mbar_init(UFULL(i), 1);
-      mbar_init(UEMPTY(i), 1 + 4);  // MMA thread + 4 compute warps
+      mbar_init(UEMPTY(i), 1 + 8);  // MMA thread + 8 compute warps
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -166,6 +200,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       uint32_t filled = 0, fill_phase = 0;
       int row_filled = -1;
       bool ok = true;
+      uint32_t hl = 0;  // half-steps loaded (trace index)
+      (void)hl;
       for (int uk = 0; ok; ++uk) {
         const int slot = uk & 3;
         if (!mbar_wait(UEMPTY(slot), ((uk >> 2) & 1) ^ 1u, abort_flag, p.status, p.timeout_ns)) {
@@ -191,22 +227,37 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tma_load_4d(sRow + C::TILE_BYTES + c * C::CHUNK_BYTES, &tmRowB, ROWFULL, 64 * c, it.h,
                       it.row_tile * kBM, it.b);
         }
+        // entry words read four ahead, so no load latency sits between two TMA issues
+        uint32_t pf0 = __ldg(it.ent), pf1 = it.n > 1 ? __ldg(it.ent + 1) : 0u;
+        uint32_t pf2 = it.n > 2 ? __ldg(it.ent + 2) : 0u, pf3 = it.n > 3 ? __ldg(it.ent + 3) : 0u;
         for (int j = 0; j < it.n && ok; ++j) {
-          if (!mbar_wait(EMPTY(st), ph ^ 1u, abort_flag, p.status, p.timeout_ns)) {
-            ok = false;
-            break;
+          const uint32_t ent = pf0;
+          pf0 = pf1;
+          pf1 = pf2;
+          pf2 = pf3;
+          pf3 = j + 4 < it.n ? __ldg(it.ent + j + 4) : 0u;
+          const int ct = static_cast<int>(ent & 0x0FFFFFFFu);
+          const uint32_t bits = ent >> 28;
+          for (int h = 0; h < 2; ++h) {
+            if (!half_needed(bits, h)) continue;
+            if (!mbar_wait(EMPTY(st), ph ^ 1u, abort_flag, p.status, p.timeout_ns)) {
+              ok = false;
+              break;
+            }
+            BSA_BTRACE_AT(hl, 6);
+            ++hl;
+            mbar_expect_tx(FULL(st), 2 * C::HALF_BYTES);
+            const uint32_t dst = sRing + st * 2 * C::HALF_BYTES;
+            const int r0 = ct * kBM + 64 * h;
+            for (int c = 0; c < C::KCH; ++c) {
+              tma_load_4d(dst + c * C::HCHUNK_BYTES, &tmColA, FULL(st), 64 * c, it.h, r0, it.b);
+              tma_load_4d(dst + C::HALF_BYTES + c * C::HCHUNK_BYTES, &tmColB, FULL(st), 64 * c,
+                          it.h, r0, it.b);
+            }
+            filled |= 1u << st;
+            fill_phase = (fill_phase & ~(1u << st)) | (ph << st);
+            if (++st == C::NSTAGE) { st = 0; ph ^= 1u; }
           }
-          const int ct = static_cast<int>(__ldg(it.ent + j) & 0x0FFFFFFFu);
-          mbar_expect_tx(FULL(st), 2 * C::TILE_BYTES);
-          const uint32_t dst = sRing + st * 2 * C::TILE_BYTES;
-          for (int c = 0; c < C::KCH; ++c) {
-            tma_load_4d(dst + c * C::CHUNK_BYTES, &tmColA, FULL(st), 64 * c, it.h, ct * kBM, it.b);
-            tma_load_4d(dst + C::TILE_BYTES + c * C::CHUNK_BYTES, &tmColB, FULL(st), 64 * c, it.h,
-                        ct * kBM, it.b);
-          }
-          filled |= 1u << st;
-          fill_phase = (fill_phase & ~(1u << st)) | (ph << st);
-          if (++st == C::NSTAGE) { st = 0; ph ^= 1u; }
         }
       }
       for (int i = 0; i < C::NSTAGE; ++i)
@@ -218,53 +269,60 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else if (warp == kBwdMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_ss = idesc_bf16_f32(kBM, kBN, 0, 0);
+      constexpr uint32_t idesc_ss = idesc_bf16_f32(kBM, 64, 0, 0);
       constexpr uint32_t idesc_ts = idesc_bf16_f32(kBM, D, 0, 1);
       constexpr uint32_t kTileUnits = C::TILE_BYTES >> 4;
+      constexpr uint32_t kHalfUnits = C::HALF_BYTES >> 4;
       const uint64_t dRowK = smem_desc_sw128(sRow, 16, 1024);
       const uint64_t dColK = smem_desc_sw128(sRing, 16, 1024);
-      const uint64_t dColMN = smem_desc_sw128(sRing, C::CHUNK_BYTES, 1024);
+      const uint64_t dColMN = smem_desc_sw128(sRing, C::HCHUNK_BYTES, 1024);
       int st = 0;
-      uint32_t ph = 0, rph = 0, pph = 0;
+      uint32_t ph = 0, rph = 0;
+      uint32_t hc = 0;  // half-steps whose S / dP were issued (all items)
+      uint32_t ha = 0;  // half-steps whose accumulation was issued
+      int stage_b0 = 0, stage_b1 = 0;  // ring stage held by each TMEM buffer
       bool ok = true;
-      auto acquire = [&](int& stage) -> bool {
-        if (!mbar_wait(FULL(st), ph, abort_flag, p.status, p.timeout_ns)) return false;
-        stage = st;
-        if (++st == C::NSTAGE) { st = 0; ph ^= 1u; }
-        return true;
-      };
-      // S-like (rowA colA^T) into TMEM [0,128), dP-like (rowB colB^T) into [128,256)
-      auto mma_sd = [&](int stage) {
+      // S-like (rowA colA_half^T) and dP-like (rowB colB_half^T) into TMEM buffer `buf`
+      auto sd = [&](int stage, uint32_t buf) {
         tc_fence_after();
-        const uint64_t dcol = dColK + static_cast<uint64_t>(stage * 2 * kTileUnits);
+        const uint64_t dcol = dColK + static_cast<uint64_t>(stage * 2 * kHalfUnits);
+        const uint32_t tS = tmem + 128u * buf;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t off =
+          const uint64_t offR =
               static_cast<uint64_t>((((kk >> 2) * C::CHUNK_BYTES) + (kk & 3) * 32) >> 4);
-          mma_ss(tmem, dRowK + off, dcol + off, idesc_ss, kk > 0 ? 1u : 0u);
+          const uint64_t offC =
+              static_cast<uint64_t>((((kk >> 2) * C::HCHUNK_BYTES) + (kk & 3) * 32) >> 4);
+          mma_ss(tS, dRowK + offR, dcol + offC, idesc_ss, kk > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t off =
+          const uint64_t offR =
               static_cast<uint64_t>((((kk >> 2) * C::CHUNK_BYTES) + (kk & 3) * 32) >> 4);
-          mma_ss(tmem + 128, dRowK + kTileUnits + off, dcol + kTileUnits + off, idesc_ss,
+          const uint64_t offC =
+              static_cast<uint64_t>((((kk >> 2) * C::HCHUNK_BYTES) + (kk & 3) * 32) >> 4);
+          mma_ss(tS + 64, dRowK + kTileUnits + offR, dcol + kHalfUnits + offC, idesc_ss,
                  kk > 0 ? 1u : 0u);
         }
       };
-      // accA (+)= dS colA ; accB (+)= P colB (kDKV only); A operands from TMEM
-      auto mma_acc = [&](int stage, int step) {
+      // accA (+)= dS colA_half ; accB (+)= P colB_half (kDKV); A operands from TMEM
+      auto acc = [&](int stage, uint32_t buf, bool first) {
         tc_fence_after();
-        const uint64_t dA = dColMN + static_cast<uint64_t>(stage * 2 * kTileUnits);
-        const uint64_t dB = dA + kTileUnits;
-        const uint32_t acc0 = step > 0 ? 1u : 0u;
+        const uint64_t dA = dColMN + static_cast<uint64_t>(stage * 2 * kHalfUnits);
+        const uint32_t tS = tmem + 128u * buf;
+        const uint32_t acc0 = first ? 0u : 1u;
+        // packed bf16 columns 16*kk .. 16*kk + 15 of P / dS sit at TMEM column
+        // (kk / 2) * 32 + (kk % 2) * 8 of the S / dP region (each compute warp packs
+        // its 32 columns into the first 16 of its own)
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk)
-          mma_ts(tmem + 256, tmem + 128 + kk * 8, dA + static_cast<uint64_t>(kk * 128), idesc_ts,
-                 kk > 0 ? 1u : acc0);
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ts(tmem + 256, tS + 64 + (kk >> 1) * 32 + (kk & 1) * 8,
+                 dA + static_cast<uint64_t>(kk * 128), idesc_ts, kk > 0 ? 1u : acc0);
         if (kDKV) {
 #pragma unroll
-          for (int kk = 0; kk < kBN / 16; ++kk)
-            mma_ts(tmem + 384, tmem + kk * 8, dB + static_cast<uint64_t>(kk * 128), idesc_ts,
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ts(tmem + 384, tS + (kk >> 1) * 32 + (kk & 1) * 8,
+                   dA + kHalfUnits + static_cast<uint64_t>(kk * 128), idesc_ts,
                    kk > 0 ? 1u : acc0);
         }
       };
@@ -279,49 +337,58 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (u >= p.total_items) break;
         const BItem it = get_bitem<kDKV>(p, u);
         if (it.n <= 0) continue;
+        const int nh = it.nh;  // half-steps of this item
         if (!mbar_wait(ROWFULL, rph, abort_flag, p.status, p.timeout_ns)) {
           ok = false;
           break;
         }
         rph ^= 1u;
-        int cur = 0;
-        if (!acquire(cur)) { ok = false; break; }
-        mma_sd(cur);
-        mma_commit(SFULL);
-        if (it.n == 1) mma_commit(ROWEMPTY);
-        for (int j = 0; j < it.n && ok; ++j) {
-          if (!mbar_wait(PREADY, pph, abort_flag, p.status, p.timeout_ns)) { ok = false; break; }
-          pph ^= 1u;
-          mma_acc(cur, j);
-          mma_commit(EMPTY(cur));
-          if (j == it.n - 1) {
-            mma_commit(DONE);
-          } else {
-            int nxt = 0;
-            if (!acquire(nxt)) { ok = false; break; }
-            mma_sd(nxt);
-            mma_commit(SFULL);
-            if (j + 1 == it.n - 1) mma_commit(ROWEMPTY);
-            cur = nxt;
+        int issued = 0;
+        auto issue = [&]() -> bool {
+          if (!mbar_wait(FULL(st), ph, abort_flag, p.status, p.timeout_ns)) return false;
+          BSA_BTRACE_AT(hc, 4);
+          const uint32_t buf = hc & 1u;
+          if (buf) stage_b1 = st; else stage_b0 = st;
+          sd(st, buf);
+          mma_commit(SFULL(buf));
+          BSA_BTRACE_AT(hc, 5);
+          if (++st == C::NSTAGE) { st = 0; ph ^= 1u; }
+          ++hc;
+          if (++issued == nh) mma_commit(ROWEMPTY);
+          return true;
+        };
+        ok = issue() && (issued == nh || issue());
+        for (int done = 0; ok && done < nh; ++done) {
+          const uint32_t buf = ha & 1u;
+          if (!mbar_wait(PREADY(buf), (ha >> 1) & 1u, abort_flag, p.status, p.timeout_ns)) {
+            ok = false;
+            break;
           }
+          BSA_BTRACE_AT(ha, 3);
+          const int stage = buf ? stage_b1 : stage_b0;
+          acc(stage, buf, done == 0);
+          mma_commit(EMPTY(stage));
+          ++ha;
+          if (issued < nh) ok = issue();
         }
+        if (!ok) break;
+        mma_commit(DONE);
       }
       mma_commit(FINAL);
       mbar_wait_drain(FINAL, 0, p.status, p.timeout_ns);
     }
   } else {
-    // ------------------------------------------------------------ compute (4 warps)
-    const int row = threadIdx.x;  // 0..127 = TMEM lane
-    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + lane_base;
-    const uint32_t tP = tmem + lane_base + 128;
+    // ------------------------------------------------------------ compute (8 warps)
+    const int q4 = warp & 3;            // TMEM lane quarter
+    const int cg = warp >> 2;           // column group: columns 32*cg .. +31 of each half-step
+    const int row = q4 * 32 + lane;     // 0..127 = TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
     const uint32_t tA = tmem + lane_base + 256;
     const uint32_t tB = tmem + lane_base + 384;
-    const int rh = row >> 6;  // which 64-row half of the row tile
-    const float sl2 = p.scale_log2;
-    uint32_t sph = 0, dph = 0;
+    const int rh = q4 >> 1;  // which 64-row half of the row tile (warp-uniform)
+    const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
+    uint32_t hc = 0, dph = 0;
     bool ok = true;
-    int vstep = 0;  // steps taken (selects the smem vector buffer in kDKV)
     for (int uk = 0; ok; ++uk) {
       const int slot = uk & 3;
       if (!mbar_wait(UFULL(slot), (uk >> 2) & 1, abort_flag, p.status, p.timeout_ns)) {
@@ -336,72 +403,110 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (it.n < 0) continue;
       const long long bh = static_cast<long long>(it.b) * p.H + it.h;
       const int grow = it.row_tile * kBM + row;          // global row of this thread
-      float lse_row = 0.f, d_row = 0.f;
+      const float* lse2_bh = p.lse2 + bh * (p.QT * kBM);
+      const float* dvec_bh = p.dvec + bh * (p.QT * kBM);
+      float2 nlse = make_float2(0.f, 0.f), dd = make_float2(0.f, 0.f);
       if (!kDKV) {
-        lse_row = p.lse2[bh * (p.QT * kBM) + grow];
-        d_row = p.dvec[bh * (p.QT * kBM) + grow];
+        const float l = -lse2_bh[grow];
+        const float d = dvec_bh[grow];
+        nlse = make_float2(l, l);
+        dd = make_float2(d, d);
       }
-      for (int j = 0; j < it.n; ++j) {
-        const uint32_t ent = __ldg(it.ent + j);
+      // register prefetch, one entry ahead: the entry word and (kDKV) this lane's
+      // -LSE2 / D values of column 64*h + 32*cg + lane, broadcast to the warp by
+      // shuffles when used
+      uint32_t ent_next = it.n > 0 ? __ldg(it.ent) : 0u;
+      float pl[2] = {0.f, 0.f}, pd[2] = {0.f, 0.f};
+      if (kDKV && it.n > 0) {
+        const int ct0 = static_cast<int>(ent_next & 0x0FFFFFFFu);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          pl[h] = -__ldg(lse2_bh + ct0 * kBM + 64 * h + 32 * cg + lane);
+          pd[h] = __ldg(dvec_bh + ct0 * kBM + 64 * h + 32 * cg + lane);
+        }
+      }
+      for (int j = 0; j < it.n && ok; ++j) {
+        const uint32_t ent = ent_next;
         const int ct = static_cast<int>(ent & 0x0FFFFFFFu);
         const uint32_t bits = ent >> 28;
-        // this step's per-column LSE2 and D (128 query columns) into this warp's own
-        // shared-memory copy (double-buffered; __syncwarp orders writes and reads)
-        float* vbuf = svec + ((warp & 3) * 2 + (vstep & 1)) * 256;
-        if (kDKV) {
-          const float* l2 = p.lse2 + bh * (p.QT * kBM) + ct * kBM;
-          const float* dv2 = p.dvec + bh * (p.QT * kBM) + ct * kBM;
+        if (j + 1 < it.n) ent_next = __ldg(it.ent + j + 1);
+        float cl[2] = {pl[0], pl[1]}, cd[2] = {pd[0], pd[1]};
+        if (kDKV && j + 1 < it.n) {
+          const int ctn = static_cast<int>(ent_next & 0x0FFFFFFFu);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            vbuf[lane + 32 * i] = __ldg(l2 + lane + 32 * i);
-            vbuf[128 + lane + 32 * i] = __ldg(dv2 + lane + 32 * i);
+          for (int h = 0; h < 2; ++h) {
+            pl[h] = -__ldg(lse2_bh + ctn * kBM + 64 * h + 32 * cg + lane);
+            pd[h] = __ldg(dvec_bh + ctn * kBM + 64 * h + 32 * cg + lane);
           }
-          __syncwarp();
         }
-        ++vstep;
-        ok = mbar_wait(SFULL, sph, abort_flag, p.status, p.timeout_ns);
-        if (!ok) break;
-        sph ^= 1u;
-        tc_fence_after();
-        // quadrant mask: bit (row_half * 2 + column_half); the ragged column tail of
-        // the dQ pass (keys past nk) is masked per column
-        const bool lo_ok = (bits >> (rh * 2)) & 1u, hi_ok = (bits >> (rh * 2 + 1)) & 1u;
+        // keys past nk in the dQ pass (ragged last key tile) are masked per column
         const int cvalid = kDKV ? kBN : p.nk - ct * kBN;
-#pragma unroll 1
-        for (int c0 = 0; c0 < kBN; c0 += 32) {
-          uint32_t sr[32], dr[32];
-          tmem_ld32x32b_x32(tS + c0, sr);
-          tmem_ld32x32b_x32(tP + c0, dr);
-          const bool half_ok = c0 < 64 ? lo_ok : hi_ok;
-          uint32_t ppk[16], dpk[16];
+        for (int h = 0; h < 2; ++h) {
+          if (!half_needed(bits, h)) continue;
+          const uint32_t buf = hc & 1u;
+          if (threadIdx.x == 0) BSA_BTRACE_AT(hc, 0);
+          ok = mbar_wait(SFULL(buf), (hc >> 1) & 1u, abort_flag, p.status, p.timeout_ns);
+          if (!ok) break;
+          if (threadIdx.x == 0) BSA_BTRACE_AT(hc, 1);
+          ++hc;
+          tc_fence_after();
+          // this warp's 32 columns of S and dP; P and dS are packed into the first
+          // 16 columns of the same ranges
+          const uint32_t tS = tmem + lane_base + 128u * buf + 32u * cg;
+          const bool row_ok = (bits >> (rh * 2 + h)) & 1u;
+          if (!row_ok) {
+            uint32_t z[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float pv[2], dsv[2];
+            for (int i = 0; i < 16; ++i) z[i] = 0u;
+            tmem_st32x32b_x16(tS, z);
+            tmem_st32x32b_x16(tS + 64, z);
+          } else {
+            uint32_t sr[32], dr[32];
+            tmem_ld32x32b_x32_nowait(tS, sr);
+            tmem_ld32x32b_x32_nowait(tS + 64, dr);
+            tmem_wait_ld_x32(sr);
+            tmem_wait_ld_x32(dr);
+            const int cbase = 64 * h + 32 * cg;
+            uint32_t ppk[16], dpk[16];
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int c = c0 + 2 * i + e;
-              const float lse = kDKV ? vbuf[c] : lse_row;
-              const float dd = kDKV ? vbuf[128 + c] : d_row;
-              float pr = fast_exp2(fmaf(__uint_as_float(sr[2 * i + e]), sl2, -lse));
-              if (!half_ok || c >= cvalid) pr = 0.f;
-              pv[e] = pr;
-              dsv[e] = pr * (__uint_as_float(dr[2 * i + e]) - dd);
+            for (int i = 0; i < 16; ++i) {
+              const int c = cbase + 2 * i;
+              float2 nl = nlse, dv = dd;
+              if (kDKV) {
+                const float vl = h ? cl[1] : cl[0], vd = h ? cd[1] : cd[0];
+                nl = make_float2(__shfl_sync(0xffffffffu, vl, 2 * i),
+                                 __shfl_sync(0xffffffffu, vl, 2 * i + 1));
+                dv = make_float2(__shfl_sync(0xffffffffu, vd, 2 * i),
+                                 __shfl_sync(0xffffffffu, vd, 2 * i + 1));
+              }
+              const float2 a = ffma2(make_float2(__uint_as_float(sr[2 * i]),
+                                                 __uint_as_float(sr[2 * i + 1])), sl2, nl);
+              float2 pr = make_float2(fast_exp2(a.x), fast_exp2(a.y));
+              if (!kDKV) {
+                if (c >= cvalid) pr.x = 0.f;
+                if (c + 1 >= cvalid) pr.y = 0.f;
+              }
+              const float2 ds = fmul2(pr, fsub2(make_float2(__uint_as_float(dr[2 * i]),
+                                                            __uint_as_float(dr[2 * i + 1])),
+                                                dv));
+              __nv_bfloat162 hp = __floats2bfloat162_rn(pr.x, pr.y);
+              __nv_bfloat162 hd = __floats2bfloat162_rn(ds.x, ds.y);
+              ppk[i] = *reinterpret_cast<uint32_t*>(&hp);
+              dpk[i] = *reinterpret_cast<uint32_t*>(&hd);
             }
-            __nv_bfloat162 hp = __floats2bfloat162_rn(pv[0], pv[1]);
-            __nv_bfloat162 hd = __floats2bfloat162_rn(dsv[0], dsv[1]);
-            ppk[i] = *reinterpret_cast<uint32_t*>(&hp);
-            dpk[i] = *reinterpret_cast<uint32_t*>(&hd);
+            if (kDKV) tmem_st32x32b_x16(tS, ppk);
+            tmem_st32x32b_x16(tS + 64, dpk);
           }
-          if (kDKV) tmem_st32x32b_x16(tS + c0 / 2, ppk);
-          tmem_st32x32b_x16(tP + c0 / 2, dpk);
+          asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+          tc_fence_before();
+          __syncwarp();
+          if (threadIdx.x == 0) BSA_BTRACE_AT(hc - 1, 2);
+          if (lane == 0) mbar_arrive(PREADY(buf));
         }
-        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(PREADY);
       }
       if (!ok) break;
-      // epilogue: accA * scale -> outA, accB -> outB (rows past the tensor end skipped)
+      // epilogue: accA * scale -> outA, accB -> outB (rows past the tensor end
+      // skipped); the two warps of a lane quarter take half of the D columns each
       const int nrows = kDKV ? p.nk : p.nq;
       __nv_bfloat16* rowA = p.outA + ((static_cast<long long>(it.b) * nrows + grow) * p.H + it.h) * D;
       __nv_bfloat16* rowB =
@@ -418,7 +523,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         __nv_bfloat16* dst_row = pass == 0 ? rowA : rowB;
         const float mul = pass == 0 ? p.scale : 1.0f;
 #pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 32) {
+        for (int c0 = cg * (D / 2); c0 < (cg + 1) * (D / 2); c0 += 32) {
           uint32_t ov[32];
           if (it.n > 0) {
             tmem_ld32x32b_x32(tacc + c0, ov);
@@ -520,19 +625,29 @@ __global__ void tmap_kernel(const int* __restrict__ row_ptr, const int* __restri
 
 __global__ void __launch_bounds__(256) tcompact_kernel(const uint32_t* __restrict__ map, int QT,
                                                        int KT, int* __restrict__ tcnt,
+                                                       int* __restrict__ thcnt,
                                                        uint32_t* __restrict__ tentries) {
   __shared__ int warp_sums[8];
+  __shared__ int half_total;
+  if (threadIdx.x == 0) half_total = 0;
+  __syncthreads();
   const long long g = blockIdx.x;  // mask head * KT + k-tile
   const int words = (QT + 7) / 8;
   const uint32_t* row = map + g * words;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int per = (words + 255) / 256;
   const int w0 = min(words, tid * per), w1 = min(words, w0 + per);
-  int mine = 0;
+  int mine = 0, halves = 0;
   for (int w = w0; w < w1; ++w) {
     const uint32_t q = row[w];
-    for (int j = 0; j < 8; ++j) mine += ((q >> (4 * j)) & 0xFu) != 0u;
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t b = (q >> (4 * j)) & 0xFu;
+      mine += b != 0u;
+      halves += static_cast<int>(half_needed(b, 0)) + static_cast<int>(half_needed(b, 1));
+    }
   }
+  for (int o = 16; o > 0; o >>= 1) halves += __shfl_xor_sync(0xffffffffu, halves, o);
+  if (lane == 0) atomicAdd(&half_total, halves);
   int incl = mine;
   for (int o = 1; o < 32; o <<= 1) {
     const int v = __shfl_up_sync(0xffffffffu, incl, o);
@@ -552,12 +667,38 @@ __global__ void __launch_bounds__(256) tcompact_kernel(const uint32_t* __restric
     }
   }
   if (tid == 255) tcnt[g] = pos;
+  __syncthreads();
+  if (tid == 0) thcnt[g] = half_total;
+}
+
+// Half-steps of each forward list (one CTA per list row), for the dQ pass.
+__global__ void __launch_bounds__(128) qhcount_kernel(const int* __restrict__ row_ptr,
+                                                      const int* __restrict__ cnt,
+                                                      const uint32_t* __restrict__ entries, int LR,
+                                                      int QB, int block_q, int expand,
+                                                      int* __restrict__ qhcnt) {
+  __shared__ int total;
+  const int g = blockIdx.x;  // mask head * LR + list row
+  const int mh = g / LR, lr = g - mh * LR;
+  const int first_qb = block_q >= 128 ? lr : 2 * lr;
+  const uint32_t* ent = entries + static_cast<long long>(row_ptr[mh * QB + first_qb]) * expand;
+  if (threadIdx.x == 0) total = 0;
+  __syncthreads();
+  int halves = 0;
+  for (int j = threadIdx.x; j < cnt[g]; j += blockDim.x) {
+    const uint32_t b = ent[j] >> 28;
+    halves += static_cast<int>(half_needed(b, 0)) + static_cast<int>(half_needed(b, 1));
+  }
+  for (int o = 16; o > 0; o >>= 1) halves += __shfl_xor_sync(0xffffffffu, halves, o);
+  if ((threadIdx.x & 31) == 0) atomicAdd(&total, halves);
+  __syncthreads();
+  if (threadIdx.x == 0) qhcnt[g] = total;
 }
 
 struct BwdGeometry {
   Geometry fwd;
   int KT;
-  size_t tcnt_off, tent_off, map_off, lse_off, dvec_off, total;
+  size_t tcnt_off, thcnt_off, qhcnt_off, tent_off, map_off, lse_off, dvec_off, total;
 };
 
 BwdGeometry bwd_geometry(int batch, int heads, int nq, int nk, int block_q, int block_k,
@@ -568,7 +709,9 @@ BwdGeometry bwd_geometry(int batch, int heads, int nq, int nk, int block_q, int 
   auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
   const size_t mhk = static_cast<size_t>(list_heads) * g.KT;
   g.tcnt_off = up(g.fwd.total);
-  g.tent_off = up(g.tcnt_off + sizeof(int) * mhk);
+  g.thcnt_off = up(g.tcnt_off + sizeof(int) * mhk);
+  g.qhcnt_off = up(g.thcnt_off + sizeof(int) * mhk);
+  g.tent_off = up(g.qhcnt_off + sizeof(int) * static_cast<size_t>(list_heads) * g.fwd.LR);
   g.map_off = up(g.tent_off + sizeof(uint32_t) * mhk * g.fwd.QT);
   g.lse_off = up(g.map_off + sizeof(uint32_t) * mhk * ((g.fwd.QT + 7) / 8));
   const size_t vec = sizeof(float) * static_cast<size_t>(batch) * heads * g.fwd.QT * kBM;
@@ -626,11 +769,16 @@ extern "C" int bsa_attn_bwd(const void* q, const void* k, const void* v, const v
   if (scale <= 0.0f) scale = 1.0f / sqrtf(static_cast<float>(head_dim));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-  CUtensorMap mq, mk, mv, mdo;
+  // 128-row boxes for the row operands, 64-row boxes for the column halves
+  CUtensorMap mq, mk, mv, mdo, hq, hk, hv, hdo;
   if (make_map(&mq, q, batch, nq, heads, head_dim) != BSA_OK ||
       make_map(&mk, k, batch, nk, heads, head_dim) != BSA_OK ||
       make_map(&mv, v, batch, nk, heads, head_dim) != BSA_OK ||
-      make_map(&mdo, dout, batch, nq, heads, head_dim) != BSA_OK)
+      make_map(&mdo, dout, batch, nq, heads, head_dim) != BSA_OK ||
+      make_map(&hq, q, batch, nq, heads, head_dim, 64) != BSA_OK ||
+      make_map(&hk, k, batch, nk, heads, head_dim, 64) != BSA_OK ||
+      make_map(&hv, v, batch, nk, heads, head_dim, 64) != BSA_OK ||
+      make_map(&hdo, dout, batch, nq, heads, head_dim, 64) != BSA_OK)
     return BSA_ERR_CUDA;
 
   char* wsb = static_cast<char*>(ws);
@@ -638,6 +786,8 @@ extern "C" int bsa_attn_bwd(const void* q, const void* k, const void* v, const v
   int* cnt = reinterpret_cast<int*>(wsb + g.fwd.cnt_off);
   uint32_t* entries = reinterpret_cast<uint32_t*>(wsb + g.fwd.ent_off);
   int* tcnt = reinterpret_cast<int*>(wsb + g.tcnt_off);
+  int* thcnt = reinterpret_cast<int*>(wsb + g.thcnt_off);
+  int* qhcnt = reinterpret_cast<int*>(wsb + g.qhcnt_off);
   uint32_t* tentries = reinterpret_cast<uint32_t*>(wsb + g.tent_off);
   uint32_t* map = reinterpret_cast<uint32_t*>(wsb + g.map_off);
   float* lse2 = reinterpret_cast<float*>(wsb + g.lse_off);
@@ -660,7 +810,10 @@ extern "C" int bsa_attn_bwd(const void* q, const void* k, const void* v, const v
                                                      g.fwd.LR, g.fwd.QB, block_q, g.fwd.expand,
                                                      list_heads, map);
   if ((rc = check_launch()) != BSA_OK) return rc;
-  tcompact_kernel<<<list_heads * g.KT, 256, 0, st>>>(map, g.fwd.QT, g.KT, tcnt, tentries);
+  tcompact_kernel<<<list_heads * g.KT, 256, 0, st>>>(map, g.fwd.QT, g.KT, tcnt, thcnt, tentries);
+  if ((rc = check_launch()) != BSA_OK) return rc;
+  qhcount_kernel<<<list_heads * g.fwd.LR, 128, 0, st>>>(row_ptr, cnt, entries, g.fwd.LR, g.fwd.QB,
+                                                        block_q, g.fwd.expand, qhcnt);
   if ((rc = check_launch()) != BSA_OK) return rc;
 
   BwdParams p;
@@ -681,6 +834,8 @@ extern "C" int bsa_attn_bwd(const void* q, const void* k, const void* v, const v
   p.cnt = cnt;
   p.entries = entries;
   p.tcnt = tcnt;
+  p.thcnt = thcnt;
+  p.qhcnt = qhcnt;
   p.tentries = tentries;
   p.lse2 = lse2;
   p.dvec = dvec;
@@ -691,14 +846,21 @@ extern "C" int bsa_attn_bwd(const void* q, const void* k, const void* v, const v
   p.outA = static_cast<__nv_bfloat16*>(dk);
   p.outB = static_cast<__nv_bfloat16*>(dv);
   p.unit_counter = status + 1;
-  rc = head_dim == 128 ? launch_bwd<128, true>(mk, mv, mq, mdo, p, st)
-                       : launch_bwd<64, true>(mk, mv, mq, mdo, p, st);
+  rc = head_dim == 128 ? launch_bwd<128, true>(mk, mv, hq, hdo, p, st)
+                       : launch_bwd<64, true>(mk, mv, hq, hdo, p, st);
   if (rc != BSA_OK) return rc;
   // pass 2: dQ (rows = q-tiles, columns = key tiles)
   p.total_items = batch * heads * g.fwd.QT;
   p.outA = static_cast<__nv_bfloat16*>(dq);
   p.outB = nullptr;
   p.unit_counter = status + 2;
-  return head_dim == 128 ? launch_bwd<128, false>(mq, mdo, mk, mv, p, st)
-                         : launch_bwd<64, false>(mq, mdo, mk, mv, p, st);
+  return head_dim == 128 ? launch_bwd<128, false>(mq, mdo, hk, hv, p, st)
+                         : launch_bwd<64, false>(mq, mdo, hk, hv, p, st);
 }
+
+#ifdef BSA_TRACE
+extern "C" int bsa_btrace_dump(unsigned long long* host, size_t bytes) {
+  if (bytes > sizeof(bsa::g_bsa_btrace)) bytes = sizeof(bsa::g_bsa_btrace);
+  return cudaMemcpyFromSymbol(host, bsa::g_bsa_btrace, bytes) == cudaSuccess ? 0 : 4;
+}
+#endif

@@ -132,15 +132,16 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
 }
 
 // 4D map over [B, N, H, D] bf16 (D contiguous), dimensions listed innermost first as
-// (D, H, N, B); box 64 x 1 x 128 x 1 = 128 token rows of 128 bytes, 128-byte swizzle.
-int make_map(CUtensorMap* map, const void* base, int B, int N, int H, int D) {
+// (D, H, N, B); box 64 x 1 x box_rows x 1 = box_rows token rows of 128 bytes,
+// 128-byte swizzle.
+int make_map(CUtensorMap* map, const void* base, int B, int N, int H, int D, int box_rows = kBM) {
   auto fn = get_encode_fn();
   if (!fn) return BSA_ERR_CUDA;
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
                         static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(B)};
   cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2,
                            static_cast<cuuint64_t>(N) * H * D * 2};
-  cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(kBM), 1};
+  cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,

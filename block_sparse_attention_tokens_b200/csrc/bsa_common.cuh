@@ -239,6 +239,16 @@ __device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
   return d;
 }
 
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
 // poly_exp2 on two lanes with packed f32x2 arithmetic.
 __device__ __forceinline__ float2 poly_exp2x2(float2 x) {
   x.x = fmaxf(x.x, -125.0f);
