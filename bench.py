@@ -10,6 +10,12 @@ the Sliding-Tile 720p DiT shape (1 x 24 heads x 128, 30x48x80 tokens, 6x8x8
 tiles of 384 tokens, 3x3x5-tile window).  Metric: effective TFLOP/s =
 4 * head_dim * (query, key) pairs inside kept blocks / time.
 
+``--pass bwd`` times the block-sparse attention backward instead (dQ, dK, dV from
+Q, K, V, O, LSE and dO in the path's token order, over the kept lists of the
+workload's mask), metric: effective TFLOP/s = 10 * head_dim * kept pairs / time
+(five matrix products of 2 * head_dim flops per pair: the recomputed scores, dP,
+dV, dQ and dK).
+
 Under torchrun (N > 1) every rank runs its own batch of the same shape (the path
 shards by batch/head with no collective): weak scaling, value = all ranks' work
 divided by the slowest rank's time.
@@ -42,24 +48,30 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def attn_source_hash() -> str:
+KERNEL_SOURCES = {
+    "attn_fwd": ("attn_fwd.cu", "attn_common.cuh", "bsa_common.cuh", "tmem_io.cuh"),
+    "attn_bwd": ("attn_bwd.cu", "attn_common.cuh", "bsa_common.cuh", "tmem_io.cuh"),
+}
+
+
+def attn_source_hash(kind: str = "attn_fwd") -> str:
     h = hashlib.sha256()
-    for f in ("attn_fwd.cu", "attn_common.cuh", "bsa_common.cuh", "tmem_io.cuh"):
+    for f in KERNEL_SOURCES[kind]:
         with open(os.path.join(ROOT, "block_sparse_attention_tokens_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str):
-    """DRAM bytes per attention launch from the committed ncu summary, if that
-    summary was taken on the current kernel source (else None)."""
-    path = os.path.join(ROOT, "profiles", f"attn_fwd_{workload}.md")
+def profiled_traffic(workload: str, kind: str = "attn_fwd"):
+    """DRAM bytes per launch from the committed ncu summary of `kind` on the
+    workload, if that summary was taken on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", f"{kind}_{workload}.md")
     if not os.path.exists(path):
         return None
     text = open(path).read()
     m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
     s = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
-    if not m or not s or s.group(1) != attn_source_hash():
+    if not m or not s or s.group(1) != attn_source_hash(kind):
         return None
     return float(m.group(1))
 
@@ -181,13 +193,61 @@ class OracleSample:
         return flops / el / 1e12, sample
 
 
+class BackwardOracleSample(OracleSample):
+    """The CPU oracle's backward on whole query blocks of the workload (all heads).
+
+    Each sampled query block runs the oracle's block-sparse backward with the
+    mask restricted to that block's row (the other rows keep nothing), which is
+    the backward work of those queries: 10 * head_dim flops per kept pair."""
+
+    def __init__(self, w, q, k, v, do):
+        super().__init__(w, q, k, v)
+        O = self.O
+        t0 = time.perf_counter()
+        self.do64 = []
+        for h in range(w.heads):
+            dh = do[:, :, h:h + 1].double().numpy()   # already in the path's token order
+            self.do64.append(dh)
+        self.setup_s += time.perf_counter() - t0
+
+    def run(self, budget_s: float):
+        w, O, np = self.w, self.O, self.np
+        QB = math.ceil(w.nq / w.block)
+        flops, done = 0.0, 0
+        t1 = time.perf_counter()
+        for qb in self.rng.permutation(QB):
+            m = np.zeros_like(self.mask)
+            m[0, qb] = self.mask[0, qb]
+            for (qh, kh, vh), dh in zip(self.heads64, self.do64):
+                O.block_sparse_attention_backward(qh, kh, vh, dh, m, w.block, w.block)
+            rows = min((qb + 1) * w.block, w.nq) - qb * w.block
+            kept = np.nonzero(self.mask[0, qb])[0]
+            nkeys = sum(min((kb + 1) * w.block, w.nk) - kb * w.block for kb in kept)
+            flops += 10.0 * w.head_dim * rows * nkeys * w.heads
+            done += 1
+            if time.perf_counter() - t1 > budget_s:
+                break
+        el = time.perf_counter() - t1
+        sample = (f"{done} random query blocks x {w.heads} heads of {w.name} "
+                  f"({flops / 1e12:.4f} effective TFLOP), float64 oracle backward, {el:.1f} s "
+                  f"(+{self.setup_s:.1f} s untimed setup: oracle mask, tile permute, upcast)")
+        return flops / el / 1e12, sample
+
+
+BWD_METRIC = "block-sparse attention backward effective TFLOP/s"
+FWD_METRIC = "block-sparse attention effective TFLOP/s (path step)"
+
+
 def run_reference(args, w):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     from block_sparse_attention_tokens_b200 import synth
     q, k, v, _ = synth.workload_inputs(w)
-    sampler = OracleSample(w, q, k, v)
+    if args.pass_ == "bwd":
+        sampler = BackwardOracleSample(w, q, k, v, path_order_grad(w))
+    else:
+        sampler = OracleSample(w, q, k, v)
     n = max(1, args.steps + args.warmup)
     budget = max(0.5, min(10.0, 90.0 / n))
     vals = []
@@ -197,10 +257,10 @@ def run_reference(args, w):
         if i >= args.warmup:
             vals.append(val)
     value = statistics.median(vals) if vals else val
-    line = {"impl": "reference", "metric": "block-sparse attention effective TFLOP/s (path step)",
+    line = {"impl": "reference", "metric": BWD_METRIC if args.pass_ == "bwd" else FWD_METRIC,
             "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "higher_is_better": True, "dtype": "f64",
-            "data": "synthetic", "config": workload_config(w),
+            "data": "synthetic", "config": workload_config(w, args.pass_),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_cores(),
                              "kind": "oracle", "sample": f"per step: {sample}"},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -226,9 +286,17 @@ def weak_scaling_value(flops_per_rank, world, ms_per_step):
     return flops_per_rank * world / (ms_per_step * 1e-3) / 1e12
 
 
-def workload_config(w):
+def path_order_grad(w):
+    """The seeded dL/dO of the workload, [B, nq, H, D] bf16 in the path's token order."""
+    from block_sparse_attention_tokens_b200 import synth
+    return synth.grad_output(w)
+
+
+def workload_config(w, pass_: str = "fwd"):
     cfg = {"workload": w.name, "batch": w.batch, "heads": w.heads, "head_dim": w.head_dim,
            "grid_thw": list(w.grid), "block": w.block, "mask": w.mask}
+    if pass_ == "bwd":
+        cfg["pass"] = "backward (dQ, dK, dV)"
     if w.tile:
         cfg["tile"] = list(w.tile)
     if w.window:
@@ -237,6 +305,132 @@ def workload_config(w):
         cfg["p"] = w.p
     cfg["l2"] = "inputs larger than L2 (no flush between steps)"
     return cfg
+
+
+def setup_ranks():
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return world, rank, torch.device("cuda", torch.cuda.current_device())
+
+
+def run_backward(args, w):
+    """Times bsa_attn_bwd at the workload's full size.  The forward path runs once
+    (untimed) to give O, LSE and the kept lists; each timed step is one backward
+    call (list transposition, LSE/Delta preparation and the two tcgen05 passes)."""
+    import torch
+    import torch.distributed as dist
+    from block_sparse_attention_tokens_b200 import binding as B
+    from block_sparse_attention_tokens_b200 import synth
+    from block_sparse_attention_tokens_b200.pipeline import Plan, effective_flops
+
+    world, rank, dev = setup_ranks()
+    q_h, k_h, v_h, _ = synth.workload_inputs(w)
+    do_h = path_order_grad(w)
+    plan = Plan(w, dev)
+    plan.step(q_h.to(dev), k_h.to(dev), v_h.to(dev))
+    qq, kk, vv = (plan.qp, plan.kp, plan.vp) if plan.permuted else (plan._q, plan._k, plan._v)
+    oo = plan.op if plan.permuted else plan.o
+    do = do_h.to(dev)
+    dq, dk, dv = torch.empty_like(qq), torch.empty_like(kk), torch.empty_like(vv)
+    ws = torch.empty(B.bsa_attn_bwd_workspace_size(w.batch, w.heads, plan.nq, plan.nk, w.block,
+                                                   w.block, plan.list_heads),
+                     dtype=torch.uint8, device=dev)
+
+    def bwd(q_, k_, v_, o_, do_, lse_, rp_, ci_):
+        B.bsa_attn_bwd(q_, k_, v_, o_, do_, lse_, rp_, ci_, w.block, w.block, plan.list_heads,
+                       nq=plan.nq, nk=plan.nk, dq=dq, dk=dk, dv=dv, ws=ws)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    args_dev = (qq, kk, vv, oo, do, plan.lse, plan.row_ptr, plan.col_idx)
+    for _ in range(max(3, args.warmup)):
+        bwd(*args_dev)
+    barrier()
+    if B.bsa_read_status(ws) != 0:
+        raise RuntimeError("backward kernel reported a device-side error")
+    flops = 2.5 * effective_flops(plan.mask, plan.nq, plan.nk, w.block, w.head_dim,
+                                  w.batch * w.heads)
+
+    stream = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    sampler = ClockSampler(dev.index)
+    barrier()
+    with sampler:
+        time.sleep(0.5)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            bwd(*args_dev)
+            ev[i][1].record(stream)
+        barrier()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    ms_total = sum(a.elapsed_time(b) for a, b in ev)
+    ms, ms_total = max_over_ranks([ms, ms_total], dev)
+    value = weak_scaling_value(flops, world, ms)
+
+    # end to end through the public API: every step copies its inputs from pinned
+    # host memory (Q, K, V, O, dO in the path's token order, LSE, the kept lists),
+    # runs the backward and copies dQ, dK, dV back, all on one stream
+    e2e = None
+    if not args.no_e2e:
+        host_in = [t_.detach().to("cpu").pin_memory() for t_ in args_dev]
+        dev_in = [torch.empty_like(t_) for t_ in args_dev]
+        host_out = [torch.empty(t_.shape, dtype=t_.dtype).pin_memory() for t_ in (dq, dk, dv)]
+        e_steps = max(3, args.steps // 2)
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e_steps):
+            for dst, src in zip(dev_in, host_in):
+                dst.copy_(src, non_blocking=True)
+            bwd(*dev_in)
+            for dst, src in zip(host_out, (dq, dk, dv)):
+                dst.copy_(src, non_blocking=True)
+        e1.record(stream)
+        barrier()
+        e_ms = max_over_ranks([e0.elapsed_time(e1) / e_steps], dev)[0]
+        e2e = {"value": weak_scaling_value(flops, world, e_ms), "unit": "TFLOP/s",
+               "ms_per_step": e_ms,
+               "h2d_bytes_per_step": sum(t_.numel() * t_.element_size() for t_ in host_in),
+               "d2h_bytes_per_step": sum(t_.numel() * t_.element_size() for t_ in host_out),
+               "note": "pinned host buffers; copies and the backward serialised on one stream"}
+
+    peaks, peak_kind = load_peaks()
+    achieved = flops / (ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": profiled_traffic(w.name, "attn_bwd"),
+                "kernel": "attn_bwd_kernel<128> (dK/dV pass + dQ pass) and list preparation",
+                "bwd_ms": ms,
+                "peak_note": f"{peak_kind} sustained bf16 (calls timed back to back)",
+                "frac_of_burst": achieved / peaks["bf16_tflops"]}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        val, sample = BackwardOracleSample(w, q_h, k_h, v_h, do_h).run(args.cpu_budget)
+        cpu = {"value": val, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+               "sample": sample}
+    if rank == 0:
+        line = {"metric": BWD_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+                "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic", "config": workload_config(w, "bwd"),
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "clocks": sampler.summary(), "gpu_launches": 7 * args.steps,
+                "effective_tflop_per_step": flops / 1e12}
+        print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
 
 
 def main():
@@ -252,6 +446,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--heads", type=int, default=0,
                     help="override the head count (smaller cases for profiler captures)")
+    ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "bwd"],
+                    help="fwd: the whole forward path (default); bwd: the attention backward")
     args = ap.parse_args()
 
     from block_sparse_attention_tokens_b200 import configs
@@ -261,6 +457,8 @@ def main():
         w = dataclasses.replace(w, heads=args.heads)
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.pass_ == "bwd":
+        return run_backward(args, w)
 
     import torch
     import torch.distributed as dist
@@ -268,14 +466,7 @@ def main():
     from block_sparse_attention_tokens_b200 import synth
     from block_sparse_attention_tokens_b200.pipeline import Plan, effective_flops
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        torch.cuda.set_device(local)
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    dev = torch.device("cuda", torch.cuda.current_device())
+    world, rank, dev = setup_ranks()
 
     # inputs (the same seeded batch on every rank: each rank owns one batch of work)
     q_h, k_h, v_h, _ = synth.workload_inputs(w)
@@ -407,7 +598,7 @@ def main():
                "sample": sample}
 
     if rank == 0:
-        line = {"metric": "block-sparse attention effective TFLOP/s (path step)",
+        line = {"metric": FWD_METRIC,
                 "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
                 "warmup": max(3, args.warmup), "ms_per_step": ms_per_step,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,

@@ -107,6 +107,14 @@ def workload_inputs(w: "_configs.Workload"):
                     strength_range=w.strength_range, iid=w.iid, q_token_ids=q_ids)
 
 
+def grad_output(w: "_configs.Workload", seed_offset: int = 500) -> torch.Tensor:
+    """dL/dO for a workload's backward pass: i.i.d. N(0, 1) in bfloat16, shaped like O
+    ([B, nq, H, D]) in the path's token order."""
+    rng = np.random.default_rng(w.seed + seed_offset)
+    a = rng.standard_normal((w.batch, w.nq, w.heads, w.head_dim), dtype=np.float32)
+    return _to_bf16(a)
+
+
 def random_mask(rows: int, cols: int, density: float, seed: int) -> np.ndarray:
     """Uniform random 0/1 block mask (uint8) used by parity tests of the attention kernel."""
     rng = np.random.default_rng(seed)
