@@ -20,6 +20,9 @@ Plain, slow, float64 NumPy written for reading against the pages:
   Diffusion Video Generation" summary (gist.science/ja/paper/2604.21221),
   part 2 (persistent anchors, recent frames looked at closely, sparse selection
   elsewhere).
+* SPADE summary (gist.science/ja/paper/2608.03335), solution parts 1 (a menu of
+  3D slice shapes) and 2 (scheme generation with SICS, the sum of intra-block
+  cosine similarities).
 
 Where the pages leave a step open, the reading taken is marked READING and is
 the contract the CUDA path is held to.  Parity status: every function here is
@@ -521,3 +524,72 @@ def block_sparse_attention_backward(q, k, v, do, mask, block_q, block_k, scale=N
                 dq[b, rows, h] += (ds @ k[b, cols, h]) * scale
                 dk[b, cols, h] += (ds.T @ q[b, rows, h]) * scale
     return dq, dk, dv
+
+
+# ---------------------------------------------------------------------------
+# SPADE: slice-shape menu and SICS scheme generation
+# ---------------------------------------------------------------------------
+
+def tile_tokens(grid: Tuple[int, int, int], tile: Tuple[int, int, int], index: int) -> np.ndarray:
+    """Raster token indices (ascending) of tile `index`, tiles in raster order over
+    the tile grid, ragged at the grid's far edges (the same tiling as tile_order)."""
+    T, H, W = grid
+    tT, tH, tW = tile
+    nT, nH, nW = ceil_div(T, tT), ceil_div(H, tH), ceil_div(W, tW)
+    a, rem = divmod(index, nH * nW)
+    b, c = divmod(rem, nW)
+    ts = np.arange(a * tT, min(T, a * tT + tT))
+    hs = np.arange(b * tH, min(H, b * tH + tH))
+    ws = np.arange(c * tW, min(W, c * tW + tW))
+    return ((ts[:, None, None] * H + hs[None, :, None]) * W + ws[None, None, :]).reshape(-1)
+
+
+def sics_blocks(x: np.ndarray, grid: Tuple[int, int, int], tile: Tuple[int, int, int]) -> np.ndarray:
+    """SICS of every block of one slicing (SPADE summary, solution part 2).
+
+    A block is one tile of shape `tile`; its SICS is the sum over all ordered token
+    pairs (i, j) of the block, i == j included, of the cosine similarity of the two
+    tokens' vectors, per head.  A zero vector has no direction and contributes 0
+    (READING).  x: [B, N, H, D] in raster token order.  Returns [B, H, n_tiles].
+    """
+    Bn, N, Hh, D = x.shape
+    nt = ceil_div(grid[0], tile[0]) * ceil_div(grid[1], tile[1]) * ceil_div(grid[2], tile[2])
+    out = np.zeros((Bn, Hh, nt))
+    for t in range(nt):
+        idx = tile_tokens(grid, tile, t)
+        for b in range(Bn):
+            for h in range(Hh):
+                v = x[b, idx, h, :]
+                norm = np.sqrt((v * v).sum(axis=1))
+                u = np.where(norm[:, None] > 0, v / np.where(norm > 0, norm, 1.0)[:, None], 0.0)
+                out[b, h, t] = (u @ u.T).sum()      # every pairwise cosine, summed
+    return out
+
+
+def sics_scheme(q: np.ndarray, k: np.ndarray, grid: Tuple[int, int, int],
+                shapes: Sequence[Tuple[int, int, int]]):
+    """Per-head slicing choice from a menu of block shapes (SPADE summary, parts 1-2).
+
+    READING: a slicing is better the more its blocks agree internally.  Its score for
+    head h is the mean cosine similarity over the intra-block token pairs of Q and K,
+        score = (sum_b SICS_Q(b) + sum_b SICS_K(b)) / (2 * sum_b n_b^2),
+    n_b the block's token count; the head takes the highest-scoring shape (ties: the
+    earlier menu entry).  Returns (scores [B, H, n_shapes], choice [B, H] int).
+    """
+    Bn, _, Hh, _ = q.shape
+    scores = np.zeros((Bn, Hh, len(shapes)))
+    for si, shape in enumerate(shapes):
+        nt = ceil_div(grid[0], shape[0]) * ceil_div(grid[1], shape[1]) * ceil_div(grid[2], shape[2])
+        pairs = sum(len(tile_tokens(grid, shape, t)) ** 2 for t in range(nt))
+        total = sics_blocks(q, grid, shape).sum(axis=2) + sics_blocks(k, grid, shape).sum(axis=2)
+        scores[:, :, si] = total / (2.0 * pairs)
+    choice = np.zeros((Bn, Hh), dtype=np.int64)
+    for b in range(Bn):
+        for h in range(Hh):
+            best = 0
+            for si in range(1, len(shapes)):
+                if scores[b, h, si] > scores[b, h, best]:
+                    best = si
+            choice[b, h] = best
+    return scores, choice
+
