@@ -10,6 +10,10 @@ the Sliding-Tile 720p DiT shape (1 x 24 heads x 128, 30x48x80 tokens, 6x8x8
 tiles of 384 tokens, 3x3x5-tile window).  Metric: effective TFLOP/s =
 4 * head_dim * (query, key) pairs inside kept blocks / time.
 
+``--pass sics`` times SPADE scheme generation (SICS of Q and K under every shape
+of the workload's slice-shape menu, per-head choice), metric: GB/s of Q and K read
+(one pass per shape), with its time as a fraction of the workload's attention.
+
 ``--pass bwd`` times the block-sparse attention backward instead (dQ, dK, dV from
 Q, K, V, O, LSE and dO in the path's token order, over the kept lists of the
 workload's mask), metric: effective TFLOP/s = 10 * head_dim * kept pairs / time
@@ -235,6 +239,38 @@ class BackwardOracleSample(OracleSample):
 
 
 BWD_METRIC = "block-sparse attention backward effective TFLOP/s"
+SICS_METRIC = "SPADE SICS scheme generation GB/s (Q and K read once per menu shape)"
+
+
+class SicsOracleSample:
+    """The oracle's SICS scheme generation on whole heads of the workload: each
+    sampled head runs the full menu over that head's Q and K."""
+
+    def __init__(self, w, q, k):
+        import numpy as np
+        import oracle as O
+        from block_sparse_attention_tokens_b200 import configs
+        self.w, self.O, self.np = w, O, np
+        self.q, self.k = q, k
+        self.menu = configs.sics_menu(w.block)
+        self.rng = np.random.default_rng(11)
+
+    def run(self, budget_s: float):
+        w, O = self.w, self.O
+        done, nbytes = 0, 0.0
+        t1 = time.perf_counter()
+        for h in self.rng.permutation(w.heads):
+            qh = self.q[:, :, h:h + 1].double().numpy()
+            kh = self.k[:, :, h:h + 1].double().numpy()
+            O.sics_scheme(qh, kh, w.grid, self.menu)
+            nbytes += len(self.menu) * 2 * w.batch * w.nq * w.head_dim * 2
+            done += 1
+            if time.perf_counter() - t1 > budget_s:
+                break
+        el = time.perf_counter() - t1
+        sample = (f"{done} random heads of {w.name}, full menu of {len(self.menu)} shapes, "
+                  f"float64 oracle, {el:.1f} s (bytes counted as the bf16 Q and K rows read)")
+        return nbytes / el / 1e9, sample
 FWD_METRIC = "block-sparse attention effective TFLOP/s (path step)"
 
 
@@ -246,6 +282,8 @@ def run_reference(args, w):
     q, k, v, _ = synth.workload_inputs(w)
     if args.pass_ == "bwd":
         sampler = BackwardOracleSample(w, q, k, v, path_order_grad(w))
+    elif args.pass_ == "sics":
+        sampler = SicsOracleSample(w, q, k)
     else:
         sampler = OracleSample(w, q, k, v)
     n = max(1, args.steps + args.warmup)
@@ -257,13 +295,15 @@ def run_reference(args, w):
         if i >= args.warmup:
             vals.append(val)
     value = statistics.median(vals) if vals else val
-    line = {"impl": "reference", "metric": BWD_METRIC if args.pass_ == "bwd" else FWD_METRIC,
-            "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+    metric = {"bwd": BWD_METRIC, "sics": SICS_METRIC}.get(args.pass_, FWD_METRIC)
+    unit = "GB/s" if args.pass_ == "sics" else "TFLOP/s"
+    line = {"impl": "reference", "metric": metric,
+            "value": value, "unit": unit, "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "higher_is_better": True, "dtype": "f64",
             "data": "synthetic", "config": workload_config(w, args.pass_),
-            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_cores(),
+            "cpu_baseline": {"value": value, "unit": unit, "cores": cpu_cores(),
                              "kind": "oracle", "sample": f"per step: {sample}"},
-            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
     return 0
@@ -297,6 +337,10 @@ def workload_config(w, pass_: str = "fwd"):
            "grid_thw": list(w.grid), "block": w.block, "mask": w.mask}
     if pass_ == "bwd":
         cfg["pass"] = "backward (dQ, dK, dV)"
+    if pass_ == "sics":
+        from block_sparse_attention_tokens_b200 import configs
+        cfg["pass"] = "SPADE scheme generation (SICS)"
+        cfg["menu"] = [list(sh) for sh in configs.sics_menu(w.block)]
     if w.tile:
         cfg["tile"] = list(w.tile)
     if w.window:
@@ -433,6 +477,117 @@ def run_backward(args, w):
     return 0
 
 
+def run_sics(args, w):
+    """Times bsa_sics_scheme over the workload's Q and K (raster order, resident in
+    HBM) with the workload's slice-shape menu; also times the workload's attention
+    kernel to state scheme generation as a fraction of it."""
+    import torch
+    import torch.distributed as dist
+    from block_sparse_attention_tokens_b200 import binding as B
+    from block_sparse_attention_tokens_b200 import configs, synth
+    from block_sparse_attention_tokens_b200.pipeline import Plan
+
+    world, rank, dev = setup_ranks()
+    q_h, k_h, v_h, _ = synth.workload_inputs(w)
+    q, k = q_h.to(dev), k_h.to(dev)
+    menu = configs.sics_menu(w.block)
+    scores = torch.empty((w.batch, w.heads, len(menu)), dtype=torch.float32, device=dev)
+    choice = torch.empty((w.batch, w.heads), dtype=torch.int32, device=dev)
+    ws = torch.empty(B.bsa_sics_workspace_size(w.batch, w.heads, w.grid, menu),
+                     dtype=torch.uint8, device=dev)
+
+    def scheme(q_, k_):
+        B.bsa_sics_scheme(q_, k_, w.grid, menu, scores=scores, choice=choice, ws=ws)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(max(3, args.warmup)):
+        scheme(q, k)
+    barrier()
+    nbytes = len(menu) * 2 * q.numel() * q.element_size()
+    stream = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    sampler = ClockSampler(dev.index)
+    barrier()
+    with sampler:
+        time.sleep(0.5)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            scheme(q, k)
+            ev[i][1].record(stream)
+        barrier()
+    ms = max_over_ranks([statistics.mean(a.elapsed_time(b) for a, b in ev)], dev)[0]
+    value = nbytes * world / (ms * 1e-3) / 1e9
+
+    # the workload's attention kernel, for the fraction of attention time
+    plan = Plan(w, dev)
+    plan.step(q, k, v_h.to(dev))
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    a0.record(stream)
+    for _ in range(5):
+        plan.attention()
+    a1.record(stream)
+    barrier()
+    attn_ms = a0.elapsed_time(a1) / 5
+    del plan
+
+    e2e = None
+    if not args.no_e2e:
+        hq, hk = q_h.pin_memory(), k_h.pin_memory()
+        dq_, dk_ = torch.empty_like(q), torch.empty_like(k)
+        hs = torch.empty(scores.shape, dtype=scores.dtype).pin_memory()
+        hc = torch.empty(choice.shape, dtype=choice.dtype).pin_memory()
+        e_steps = max(3, args.steps // 2)
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e_steps):
+            dq_.copy_(hq, non_blocking=True)
+            dk_.copy_(hk, non_blocking=True)
+            scheme(dq_, dk_)
+            hs.copy_(scores, non_blocking=True)
+            hc.copy_(choice, non_blocking=True)
+        e1.record(stream)
+        barrier()
+        e_ms = max_over_ranks([e0.elapsed_time(e1) / e_steps], dev)[0]
+        e2e = {"value": nbytes * world / (e_ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": e_ms,
+               "h2d_bytes_per_step": 2 * q_h.numel() * q_h.element_size(),
+               "d2h_bytes_per_step": hs.numel() * 4 + hc.numel() * 4,
+               "note": "pinned host buffers; copies and the scheme serialised on one stream"}
+
+    peaks, peak_kind = load_peaks()
+    achieved = nbytes / (ms * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                "kernel": "sics_kernel<128> (one launch per tensor and menu shape)",
+                "peak_note": f"{peak_kind} HBM copy bandwidth"}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        val, sample = SicsOracleSample(w, q_h, k_h).run(args.cpu_budget)
+        cpu = {"value": val, "unit": "GB/s", "cores": cpu_cores(), "kind": "oracle",
+               "sample": sample}
+    if rank == 0:
+        line = {"metric": SICS_METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+                "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "f32", "data": "synthetic", "config": workload_config(w, "sics"),
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "clocks": sampler.summary(),
+                "gpu_launches": (2 * len(menu) + 1) * args.steps,
+                "attention_ms": attn_ms, "fraction_of_attention_time": ms / attn_ms,
+                "choice_histogram": torch.bincount(choice.flatten().long(),
+                                                   minlength=len(menu)).tolist()}
+        print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -446,8 +601,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--heads", type=int, default=0,
                     help="override the head count (smaller cases for profiler captures)")
-    ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "bwd"],
-                    help="fwd: the whole forward path (default); bwd: the attention backward")
+    ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "bwd", "sics"],
+                    help="fwd: the whole forward path (default); bwd: the attention "
+                         "backward; sics: SPADE scheme generation")
     args = ap.parse_args()
 
     from block_sparse_attention_tokens_b200 import configs
@@ -459,6 +615,8 @@ def main():
         return run_reference(args, w)
     if args.pass_ == "bwd":
         return run_backward(args, w)
+    if args.pass_ == "sics":
+        return run_sics(args, w)
 
     import torch
     import torch.distributed as dist

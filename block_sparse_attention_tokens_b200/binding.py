@@ -25,7 +25,8 @@ EXPORTS = [
     "bsa_tile_untile", "bsa_sta_mask", "bsa_radial_mask", "bsa_nabla_workspace_size",
     "bsa_nabla_mask", "bsa_mask_compact", "bsa_attn_workspace_size", "bsa_attn_fwd",
     "bsa_attn_fwd_noalloc", "bsa_read_status", "bsa_tile_permute_pool", "bsa_nabla_select",
-    "bsa_wait_selftest", "bsa_attn_bwd_workspace_size", "bsa_attn_bwd",
+    "bsa_wait_selftest", "bsa_attn_bwd_workspace_size", "bsa_attn_bwd", "bsa_sics_blocks",
+    "bsa_sics_workspace_size", "bsa_sics_scheme",
 ]
 
 
@@ -70,6 +71,10 @@ def load_library(path: str = _LIB_PATH) -> ctypes.CDLL:
         "bsa_attn_bwd_workspace_size": (c_size, [c_int] * 7),
         "bsa_attn_bwd": (c_int, [c_void] * 6 + [c_int] * 7 + [c_void, c_void, c_int, c_float]
                          + [c_void] * 4 + [c_size, c_void]),
+        "bsa_sics_blocks": (c_int, [c_void] + [c_int] * 9 + [c_void, c_void]),
+        "bsa_sics_workspace_size": (c_size, [c_int] * 5 + [c_void, c_int]),
+        "bsa_sics_scheme": (c_int, [c_void, c_void] + [c_int] * 6 + [c_void, c_int]
+                            + [c_void] * 3 + [c_size, c_void]),
         "bsa_read_status": (c_int, [c_void, ctypes.POINTER(c_int), c_void]),
         "bsa_wait_selftest": (c_int, [c_void, ctypes.c_ulonglong, c_void]),
         "bsa_tile_permute_pool": (c_int, [c_void, c_void] + [c_int] * 11 + [c_void, c_void]),
@@ -338,6 +343,54 @@ def bsa_attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Ten
                                        _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(), _stream()),
            "bsa_attn_bwd")
     return dq, dk, dv, ws
+
+
+def _n_tiles(grid, tile) -> int:
+    return (-(-grid[0] // tile[0])) * (-(-grid[1] // tile[1])) * (-(-grid[2] // tile[2]))
+
+
+def bsa_sics_blocks(x: torch.Tensor, grid, tile, out: Optional[torch.Tensor] = None):
+    """SICS of every tile of shape `tile` per head.  x: [B, T*H*W, heads, D] bf16 in
+    raster order.  Returns out [B, heads, n_tiles] float32."""
+    _cuda(x, "x")
+    B, _, Hh, D = x.shape
+    if out is None:
+        out = torch.empty((B, Hh, _n_tiles(grid, tile)), dtype=torch.float32, device=x.device)
+    _check(load_library().bsa_sics_blocks(_ptr(x), B, *grid, *tile, Hh, D, _ptr(out), _stream()),
+           "bsa_sics_blocks")
+    return out
+
+
+def _shape_array(shapes):
+    flat = [int(v) for s in shapes for v in s]
+    return (ctypes.c_int * len(flat))(*flat), len(shapes)
+
+
+def bsa_sics_workspace_size(batch, heads, grid, shapes) -> int:
+    arr, n = _shape_array(shapes)
+    return int(load_library().bsa_sics_workspace_size(batch, heads, *grid, arr, n))
+
+
+def bsa_sics_scheme(q: torch.Tensor, k: torch.Tensor, grid, shapes,
+                    scores: Optional[torch.Tensor] = None, choice: Optional[torch.Tensor] = None,
+                    ws: Optional[torch.Tensor] = None):
+    """Per-head slicing choice from a shape menu.  Returns (scores [B, H, n_shapes]
+    float32, choice [B, H] int32, ws)."""
+    _cuda(q, "q")
+    _cuda(k, "k")
+    B, _, Hh, D = q.shape
+    arr, n = _shape_array(shapes)
+    if scores is None:
+        scores = torch.empty((B, Hh, n), dtype=torch.float32, device=q.device)
+    if choice is None:
+        choice = torch.empty((B, Hh), dtype=torch.int32, device=q.device)
+    if ws is None:
+        ws = torch.empty(max(1, bsa_sics_workspace_size(B, Hh, grid, shapes)), dtype=torch.uint8,
+                         device=q.device)
+    _check(load_library().bsa_sics_scheme(_ptr(q), _ptr(k), B, *grid, Hh, D, arr, n,
+                                          _ptr(scores), _ptr(choice), _ptr(ws), ws.numel(),
+                                          _stream()), "bsa_sics_scheme")
+    return scores, choice, ws
 
 
 def bsa_read_status(ws: torch.Tensor) -> int:

@@ -103,3 +103,18 @@ def get(name_or_index) -> Workload:
     if isinstance(name_or_index, int):
         return WORKLOADS[name_or_index]
     return BY_NAME[name_or_index]
+
+
+# Slice-shape menus for SPADE scheme generation, one per block size: every shape
+# holds `block` tokens -- a cube, a wide flat slab (one or two frames), a mixed
+# slab and a tall thin column (many frames, a small spatial patch).
+SICS_MENUS = {
+    64: ((4, 4, 4), (1, 8, 8), (2, 4, 8), (16, 2, 2)),
+    128: ((2, 8, 8), (1, 8, 16), (4, 4, 8), (32, 2, 2)),
+    384: ((6, 8, 8), (1, 16, 24), (2, 12, 16), (24, 4, 4)),
+}
+
+
+def sics_menu(block: int):
+    return SICS_MENUS[block]
+

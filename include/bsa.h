@@ -283,6 +283,41 @@ int bsa_attn_fwd_noalloc(const void* q, const void* k, const void* v, int batch,
                          void* o, float* lse, int* device_status, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * (f) SPADE scheme generation: SICS and the per-head slicing choice.
+ * Source: SPADE summary (gist.science/ja/paper/2608.03335), solution part 1 (a
+ * menu of 3D slice shapes: wide and flat, tall and thin, mixed) and part 2
+ * (scheme generation by SICS, the sum of intra-block cosine similarities, from Q
+ * and K alone, per head).
+ *
+ * bsa_sics_blocks: for every tile of shape tT x tH x tW (tiles in raster order
+ *   over the tile grid, ragged at the far edges) and every head,
+ *     out[b][h][tile] = sum over ordered token pairs (i, j) of the tile of
+ *                       cos(x[b, i, h, :], x[b, j, h, :])   (i == j included;
+ *                       a zero vector contributes 0).
+ *   x : [batch, T*H*W, heads, head_dim] bf16, raster token order, 16-byte aligned
+ *   out : float32 [batch][heads][ceil(T/tT)*ceil(H/tH)*ceil(W/tW)], written
+ *   head_dim in {64, 128}; heads * head_dim <= 8192; tT*tH*tW <= 4096 tokens.
+ *
+ * bsa_sics_scheme: runs bsa_sics_blocks on q and k for every shape of the menu
+ *   shapes (HOST array of n_shapes x {tT, tH, tW}, 1 <= n_shapes <= 16) and writes
+ *     scores[b][h][s] = (sum_tiles SICS_q + sum_tiles SICS_k) / (2 * sum_tiles n^2)
+ *   (n = the tile's token count: the mean intra-block cosine similarity) and
+ *     choice[b][h] = the first s with the highest score (int32).
+ *   ws : device workspace of at least bsa_sics_workspace_size() bytes.
+ * A tile may be larger than the grid along an axis (one ragged tile there).
+ * Errors: BSA_ERR_INVALID_ARG (null / misaligned pointers, a non-positive
+ * extent), BSA_ERR_UNSUPPORTED (head_dim, heads * head_dim or tile volume out of
+ * range), BSA_ERR_WORKSPACE.
+ * ------------------------------------------------------------------------- */
+int bsa_sics_blocks(const void* x, int batch, int T, int H, int W, int tT, int tH, int tW,
+                    int heads, int head_dim, float* out, void* stream);
+size_t bsa_sics_workspace_size(int batch, int heads, int T, int H, int W, const int* shapes,
+                               int n_shapes);
+int bsa_sics_scheme(const void* q, const void* k, int batch, int T, int H, int W, int heads,
+                    int head_dim, const int* shapes, int n_shapes, float* scores, int* choice,
+                    void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Self-test of the bounded device-side waits (failure detection).
  * No counterpart in the pages.  Launches one thread that waits, through the
  * same bounded wait the attention pipeline uses, on a barrier phase that never
