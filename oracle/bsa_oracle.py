@@ -306,7 +306,8 @@ def nabla_select_row(probs: np.ndarray, p: float):
 
 def nabla_mask(qbar: np.ndarray, kbar: np.ndarray, p: float, scale: float,
                kb_begin: int = 0, kb_end: Optional[int] = None, force_outside: int = 0,
-               near_tol: float = 1e-5, tie_tol: float = 1e-5):
+               near_tol: float = 1e-5, tie_tol: float = 1e-5,
+               key_allowed: Optional[np.ndarray] = None):
     """Per-(batch, head) NABLA block mask from pooled queries and keys.
 
     Logits z[qb, kb] = qbar[qb] . kbar[kb] * scale (READING: the same 1/sqrt(D)
@@ -319,6 +320,10 @@ def nabla_mask(qbar: np.ndarray, kbar: np.ndarray, p: float, scale: float,
     the last kept and first dropped probabilities tie within ``tie_tol``
     (relative): on those rows a float32 evaluation may legitimately choose
     differently.
+    ``key_allowed`` ([B, KB] bool, optional): key blocks that may be chosen at all.
+    READING (Sparse Forcing summary, part 2: the cache keeps only the important
+    past): blocks evicted from a paged cache are not candidates -- they are left
+    out of the softmax and never selected.
     """
     Bn, H, QB, D = qbar.shape
     KB = kbar.shape[2]
@@ -331,14 +336,19 @@ def nabla_mask(qbar: np.ndarray, kbar: np.ndarray, p: float, scale: float,
     if kb_end <= kb_begin:
         return mask, near
     for b in range(Bn):
+        cand = np.arange(kb_begin, kb_end)
+        if key_allowed is not None:
+            cand = cand[key_allowed[b, kb_begin:kb_end]]
+        if cand.size == 0:
+            continue
         for h in range(H):
-            z = (qbar[b, h] @ kbar[b, h, kb_begin:kb_end].T) * scale        # [QB, nk]
+            z = (qbar[b, h] @ kbar[b, h, cand].T) * scale                    # [QB, n_cand]
             z = z - z.max(axis=1, keepdims=True)
             e = np.exp(z)
             probs = e / e.sum(axis=1, keepdims=True)
             for qb in range(QB):
                 kept, cum, k_star, order = nabla_select_row(probs[qb], p)
-                mask[b, h, qb, kb_begin + kept] = 1
+                mask[b, h, qb, cand[kept]] = 1
                 if p < 1.0:
                     c_last = cum[k_star - 1]
                     c_prev = cum[k_star - 2] if k_star >= 2 else 0.0
@@ -592,4 +602,103 @@ def sics_scheme(q: np.ndarray, k: np.ndarray, grid: Tuple[int, int, int],
                     best = si
             choice[b, h] = best
     return scores, choice
+
+
+# ---------------------------------------------------------------------------
+# Paged KV cache with persistent anchors (Sparse Forcing summary, part 2)
+# ---------------------------------------------------------------------------
+#
+# READING: the cache holds K and V in fixed-size pages of a physical pool, one
+# page table per batch maps each logical page (page_tokens consecutive tokens of
+# the key sequence) to a physical page or to -1 once evicted.  Anchor pages (those
+# touching the anchor frames) are persistent, the pages of the most recent frames
+# are kept, and of the pages in between only a fixed budget of the most important
+# survive, importance being the pooled attention mass the latest queries put on
+# the page -- the same pooled distribution NABLA selects from.
+
+
+def paged_view(pool: np.ndarray, page_table: np.ndarray, page_tokens: int, n_tokens: int):
+    """Logical [B, n_tokens, H, D] tensor of a paged cache and its residency.
+
+    pool: [P, page_tokens, H, D]; page_table: [B, n_pages] (physical page or -1).
+    Token j of batch b is row j % page_tokens of page page_table[b, j // page_tokens];
+    tokens of evicted pages read as 0 and are not resident.
+    """
+    Bn, n_pages = page_table.shape
+    _, _, H, D = pool.shape
+    out = np.zeros((Bn, n_tokens, H, D))
+    resident = np.zeros((Bn, n_tokens), dtype=bool)
+    for b in range(Bn):
+        for pg in range(n_pages):
+            lo, hi = pg * page_tokens, min((pg + 1) * page_tokens, n_tokens)
+            if lo >= hi or page_table[b, pg] < 0:
+                continue
+            out[b, lo:hi] = pool[page_table[b, pg], :hi - lo]
+            resident[b, lo:hi] = True
+    return out, resident
+
+
+def resident_blocks(page_table: np.ndarray, page_tokens: int, block: int, n_tokens: int) -> np.ndarray:
+    """[B, KB] bool: key block kb is resident iff the page holding it is (pages hold
+    whole blocks: page_tokens is a multiple of the block)."""
+    KB = ceil_div(n_tokens, block)
+    pages = (np.arange(KB) * block) // page_tokens
+    return page_table[:, pages] >= 0
+
+
+def paged_block_sparse_attention(q, k_pool, v_pool, page_table, page_tokens, nk, mask, block_q,
+                                 block_k, scale=None, rows=None):
+    """Block-sparse attention over a paged cache: the plain block-sparse attention
+    of the logical K/V with every block on an evicted page dropped from the mask.
+    mask: [Hm, QB, KB] with Hm == 1 or B * H.  Returns (O, LSE) like
+    block_sparse_attention."""
+    Bn, _, H, _ = q.shape
+    k, _ = paged_view(k_pool, page_table, page_tokens, nk)
+    v, _ = paged_view(v_pool, page_table, page_tokens, nk)
+    res = resident_blocks(page_table, page_tokens, block_k, nk)            # [B, KB]
+    full = np.broadcast_to(mask, (Bn * H,) + mask.shape[1:]) if mask.shape[0] == 1 else mask
+    m = np.array(full, dtype=np.uint8).reshape(Bn, H, mask.shape[1], mask.shape[2])
+    m = (m * res[:, None, None, :]).reshape(Bn * H, mask.shape[1], mask.shape[2])
+    return block_sparse_attention(q, k, v, m.astype(np.uint8), block_q, block_k, scale, rows)
+
+
+def kv_page_scores(qbar, kbar, scale, kb_begin, kb_end, block, page_tokens, n_pages,
+                   key_allowed=None):
+    """Importance of each logical page: the pooled attention probability (softmax of
+    qbar . kbar * scale over the candidate key blocks of [kb_begin, kb_end), as in
+    nabla_mask) summed over heads and query blocks and over the page's blocks.
+    Pages without candidate blocks score 0.  Returns [B, n_pages]."""
+    Bn, H, QB, _ = qbar.shape
+    out = np.zeros((Bn, n_pages))
+    for b in range(Bn):
+        cand = np.arange(kb_begin, kb_end)
+        if key_allowed is not None:
+            cand = cand[key_allowed[b, kb_begin:kb_end]]
+        if cand.size == 0:
+            continue
+        for h in range(H):
+            z = (qbar[b, h] @ kbar[b, h, cand].T) * scale
+            z = z - z.max(axis=1, keepdims=True)
+            e = np.exp(z)
+            probs = e / e.sum(axis=1, keepdims=True)
+            mass = probs.sum(axis=0)                                      # per candidate block
+            for i, kb in enumerate(cand):
+                out[b, (kb * block) // page_tokens] += mass[i]
+    return out
+
+
+def kv_keep_pages(scores, resident, anchor_pages, recent_begin, budget):
+    """Pages the cache keeps: every page below anchor_pages (persistent anchors) and
+    from recent_begin on (recent frames), and of the resident pages in between the
+    `budget` highest scores (ties: the lower page).  Returns keep [B, n_pages] bool."""
+    Bn, n_pages = scores.shape
+    keep = np.zeros((Bn, n_pages), dtype=bool)
+    keep[:, :anchor_pages] = True
+    keep[:, recent_begin:] = True
+    for b in range(Bn):
+        mid = [pg for pg in range(anchor_pages, recent_begin) if resident[b, pg]]
+        mid.sort(key=lambda pg: (-scores[b, pg], pg))
+        for pg in mid[:budget]:
+            keep[b, pg] = True
+    return keep
 
