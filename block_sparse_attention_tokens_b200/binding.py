@@ -26,7 +26,8 @@ EXPORTS = [
     "bsa_nabla_mask", "bsa_mask_compact", "bsa_attn_workspace_size", "bsa_attn_fwd",
     "bsa_attn_fwd_noalloc", "bsa_read_status", "bsa_tile_permute_pool", "bsa_nabla_select",
     "bsa_wait_selftest", "bsa_attn_bwd_workspace_size", "bsa_attn_bwd", "bsa_sics_blocks",
-    "bsa_sics_workspace_size", "bsa_sics_scheme",
+    "bsa_sics_workspace_size", "bsa_sics_scheme", "bsa_kv_write", "bsa_block_pool",
+    "bsa_kv_resident_blocks", "bsa_kv_page_scores", "bsa_kv_keep_pages", "bsa_attn_fwd_paged",
 ]
 
 
@@ -79,7 +80,17 @@ def load_library(path: str = _LIB_PATH) -> ctypes.CDLL:
         "bsa_wait_selftest": (c_int, [c_void, ctypes.c_ulonglong, c_void]),
         "bsa_tile_permute_pool": (c_int, [c_void, c_void] + [c_int] * 11 + [c_void, c_void]),
         "bsa_nabla_select": (c_int, [c_void, c_void] + [c_int] * 5 + [c_float, c_float]
-                             + [c_int] * 3 + [c_void, c_void, c_void, c_void]),
+                             + [c_int] * 3 + [c_void] * 5),
+        "bsa_kv_write": (c_int, [c_void] + [c_int] * 5 + [c_void, c_int, c_void, c_int, c_void,
+                                                           c_void]),
+        "bsa_block_pool": (c_int, [c_void, c_void] + [c_int] * 8 + [c_void, c_int, c_void]),
+        "bsa_kv_resident_blocks": (c_int, [c_void] + [c_int] * 4 + [c_void, c_void]),
+        "bsa_kv_page_scores": (c_int, [c_void, c_void] + [c_int] * 5 + [c_float, c_int, c_int]
+                               + [c_void, c_int, c_int, c_void, c_void]),
+        "bsa_kv_keep_pages": (c_int, [c_void] + [c_int] * 5 + [c_void, c_int] + [c_void] * 3),
+        "bsa_attn_fwd_paged": (c_int, [c_void] * 3 + [c_int, c_void] + [c_int] * 8
+                               + [c_void, c_void, c_int, c_float] + [c_void] * 3
+                               + [c_size, c_void]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -218,9 +229,11 @@ def bsa_nabla_select(qbar: torch.Tensor, kbar: torch.Tensor, p: float, scale: fl
                      kb_begin: int = 0, kb_end: Optional[int] = None, force_outside: int = 0,
                      base_mask: Optional[torch.Tensor] = None,
                      mask: Optional[torch.Tensor] = None,
-                     near_count: Optional[torch.Tensor] = None):
+                     near_count: Optional[torch.Tensor] = None,
+                     key_allowed: Optional[torch.Tensor] = None):
     """NABLA selection from pooled means qbar [B, H, QB, D], kbar [B, H, KB, D] (fp32),
-    optionally OR-ed with a head-shared base mask [QB, KB].  Returns (mask, near_count)."""
+    optionally OR-ed with a head-shared base mask [QB, KB] and restricted to the key
+    blocks with key_allowed [B, KB] != 0.  Returns (mask, near_count)."""
     _cuda(qbar, "qbar")
     _cuda(kbar, "kbar")
     B, H, QB, D = qbar.shape
@@ -232,8 +245,8 @@ def bsa_nabla_select(qbar: torch.Tensor, kbar: torch.Tensor, p: float, scale: fl
         near_count = torch.zeros(1, dtype=torch.int32, device=qbar.device)
     _check(load_library().bsa_nabla_select(_ptr(qbar), _ptr(kbar), B, H, QB, KB, D, float(p),
                                            float(scale), kb_begin, kb_end, int(force_outside),
-                                           _ptr(base_mask), _ptr(mask), _ptr(near_count),
-                                           _stream()), "bsa_nabla_select")
+                                           _ptr(base_mask), _ptr(key_allowed), _ptr(mask),
+                                           _ptr(near_count), _stream()), "bsa_nabla_select")
     return mask, near_count
 
 
@@ -391,6 +404,115 @@ def bsa_sics_scheme(q: torch.Tensor, k: torch.Tensor, grid, shapes,
                                           _ptr(scores), _ptr(choice), _ptr(ws), ws.numel(),
                                           _stream()), "bsa_sics_scheme")
     return scores, choice, ws
+
+
+# --------------------------------------------------------------------------- (g)
+# Paged KV cache: pages of KV_PAGE tokens, page tables [B, pages_per_batch] int32.
+
+KV_PAGE = 128
+
+
+def bsa_kv_write(src: torch.Tensor, first_token: int, page_table: torch.Tensor,
+                 pool: torch.Tensor, device_status: Optional[torch.Tensor] = None):
+    """Rows src [B, n_new, H, D] -> logical tokens first_token.. of each batch in the
+    pool [P, KV_PAGE, H, D] through page_table [B, pages_per_batch]."""
+    for t, n in ((src, "src"), (page_table, "page_table"), (pool, "pool")):
+        _cuda(t, n)
+    B, n_new, H, D = src.shape
+    _check(load_library().bsa_kv_write(_ptr(src), B, n_new, H, D, int(first_token),
+                                       _ptr(page_table), page_table.shape[1], _ptr(pool),
+                                       pool.shape[0], _ptr(device_status), _stream()),
+           "bsa_kv_write")
+
+
+def bsa_block_pool(x: torch.Tensor, n_tokens: int, block: int, first_block: int, n_blocks: int,
+                   out: torch.Tensor, page_table: Optional[torch.Tensor] = None, batch: int = 0):
+    """Block means of x ([B, n, H, D], or a paged pool [P, KV_PAGE, H, D] with its
+    page_table) into out [B, H, out_blocks, D] float32 at blocks first_block.."""
+    _cuda(x, "x")
+    _cuda(out, "out")
+    B = batch if page_table is not None else x.shape[0]
+    H, D = x.shape[2], x.shape[3]
+    ppb = page_table.shape[1] if page_table is not None else 0
+    _check(load_library().bsa_block_pool(_ptr(x), _ptr(page_table), ppb, B, int(n_tokens), H, D,
+                                         int(block), int(first_block), int(n_blocks), _ptr(out),
+                                         out.shape[2], _stream()), "bsa_block_pool")
+    return out
+
+
+def bsa_kv_resident_blocks(page_table: torch.Tensor, block: int, KB: int,
+                           allowed: Optional[torch.Tensor] = None):
+    _cuda(page_table, "page_table")
+    B, ppb = page_table.shape
+    if allowed is None:
+        allowed = torch.empty((B, KB), dtype=torch.uint8, device=page_table.device)
+    _check(load_library().bsa_kv_resident_blocks(_ptr(page_table), B, ppb, int(block), int(KB),
+                                                 _ptr(allowed), _stream()),
+           "bsa_kv_resident_blocks")
+    return allowed
+
+
+def bsa_kv_page_scores(qbar: torch.Tensor, kbar: torch.Tensor, kb_begin: int, kb_end: int,
+                       block: int, n_pages: int, scale: float = 0.0,
+                       key_allowed: Optional[torch.Tensor] = None,
+                       scores: Optional[torch.Tensor] = None):
+    """Page importance [B, n_pages] float32 from pooled means (see include/bsa.h)."""
+    _cuda(qbar, "qbar")
+    _cuda(kbar, "kbar")
+    B, H, QB, D = qbar.shape
+    KB = kbar.shape[2]
+    if scale <= 0:
+        scale = 1.0 / math.sqrt(D)
+    if scores is None:
+        scores = torch.empty((B, n_pages), dtype=torch.float32, device=qbar.device)
+    _check(load_library().bsa_kv_page_scores(_ptr(qbar), _ptr(kbar), B, H, QB, KB, D, float(scale),
+                                             int(kb_begin), int(kb_end), _ptr(key_allowed),
+                                             int(block), int(n_pages), _ptr(scores), _stream()),
+           "bsa_kv_page_scores")
+    return scores
+
+
+def bsa_kv_keep_pages(scores: torch.Tensor, anchor_pages: int, recent_begin: int, budget: int,
+                      page_table: torch.Tensor, freed: torch.Tensor, freed_count: torch.Tensor):
+    """Evicts middle pages beyond the budget in place (page_table entries -> -1); the
+    freed physical pages are appended to freed at atomic index freed_count."""
+    for t, n in ((scores, "scores"), (page_table, "page_table"), (freed, "freed"),
+                 (freed_count, "freed_count")):
+        _cuda(t, n)
+    B, n_pages = scores.shape
+    _check(load_library().bsa_kv_keep_pages(_ptr(scores), B, n_pages, int(anchor_pages),
+                                            int(recent_begin), int(budget), _ptr(page_table),
+                                            page_table.shape[1], _ptr(freed), _ptr(freed_count),
+                                            _stream()),
+           "bsa_kv_keep_pages")
+
+
+def bsa_attn_fwd_paged(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor,
+                       page_table: torch.Tensor, nk: int, row_ptr: torch.Tensor,
+                       col_idx: torch.Tensor, block_q: int, block_k: int, list_heads: int,
+                       nq: Optional[int] = None, scale: float = 0.0,
+                       o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                       ws: Optional[torch.Tensor] = None):
+    """Block-sparse attention with K/V in paged pools [P, KV_PAGE, H, D]."""
+    for t, n in ((q, "q"), (k_pool, "k_pool"), (v_pool, "v_pool"), (page_table, "page_table"),
+                 (row_ptr, "row_ptr"), (col_idx, "col_idx")):
+        _cuda(t, n)
+    B, _, H, D = q.shape
+    nq = q.shape[1] if nq is None else nq
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, nq), dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = torch.empty(bsa_attn_workspace_size(B, H, nq, nk, block_q, block_k, list_heads),
+                         dtype=torch.uint8, device=q.device)
+    _check(load_library().bsa_attn_fwd_paged(_ptr(q), _ptr(k_pool), _ptr(v_pool), k_pool.shape[0],
+                                             _ptr(page_table), page_table.shape[1], B, H, nq,
+                                             int(nk), D, block_q, block_k, _ptr(row_ptr),
+                                             _ptr(col_idx), list_heads, float(scale), _ptr(o),
+                                             _ptr(lse), _ptr(ws), ws.numel(), _stream()),
+           "bsa_attn_fwd_paged")
+    return o, lse, ws
 
 
 def bsa_read_status(ws: torch.Tensor) -> int:

@@ -32,7 +32,8 @@ constexpr int kListThreads = 256;
 __global__ void __launch_bounds__(kListThreads) build_lists_kernel(
     const int* __restrict__ row_ptr, const int* __restrict__ col_idx, int QB, int KB, int KT,
     int LR, int block_q, int block_k, int expand, long long nnz_cap, int* __restrict__ cnt,
-    uint32_t* __restrict__ entries, int* status) {
+    uint32_t* __restrict__ entries, int* status, const int* __restrict__ page_table,
+    int pages_per_batch, int heads) {
   extern __shared__ uint32_t quad[];
   __shared__ int warp_sums[kListThreads / 32];
   const int g = blockIdx.x;
@@ -64,6 +65,10 @@ __global__ void __launch_bounds__(kListThreads) build_lists_kernel(
   const int words = (KT + 7) / 8;
   for (int w = tid; w < words; w += kListThreads) quad[w] = 0u;
   __syncthreads();
+  // paged K/V: k-tiles on evicted pages (entry -1) are not listed; mask head mh
+  // belongs to batch mh / heads (a shared list implies a single batch)
+  const int* pt = page_table ? page_table + static_cast<long long>(mh / heads) * pages_per_batch
+                             : nullptr;
   for (int r = 0; r < nrows; ++r) {
     // q-half bits of this row: a block of >= 128 rows covers both halves
     const uint32_t qbits = block_q >= 128 ? 0x3u : (r == 0 ? 0x1u : 0x2u);
@@ -76,10 +81,12 @@ __global__ void __launch_bounds__(kListThreads) build_lists_kernel(
         // a last block that overhangs nk covers fewer than `expand` k-tiles
         for (int t = 0; t < expand && kb * expand + t < KT; ++t) {
           const int kt = kb * expand + t;
+          if (pt && (kt >= pages_per_batch || pt[kt] < 0)) continue;
           atomicOr(&quad[kt >> 3], bits << (4 * (kt & 7)));
         }
       } else {
         const int kt = kb >> 1, kh = kb & 1;
+        if (pt && (kt >= pages_per_batch || pt[kt] < 0)) continue;
         uint32_t bits = 0;
         if (qbits & 1u) bits |= 1u << kh;
         if (qbits & 2u) bits |= 1u << (2 + kh);
@@ -177,7 +184,8 @@ Geometry geometry(int batch, int heads, int nq, int nk, int block_q, int block_k
 // Launches the kept-list builder for a call's CSR (one CTA per list row).
 int launch_build_lists(const int* row_ptr, const int* col_idx, int list_heads, const Geometry& g,
                        int nk, int block_q, int block_k, int* cnt, uint32_t* entries, int* status,
-                       cudaStream_t st) {
+                       cudaStream_t st, const int* page_table = nullptr, int pages_per_batch = 0,
+                       int heads = 1) {
   const long long lists = static_cast<long long>(list_heads) * g.LR;
   const int KT = ceil_div(nk, kBN);
   const size_t list_smem = sizeof(uint32_t) * static_cast<size_t>((KT + 7) / 8);
@@ -190,7 +198,7 @@ int launch_build_lists(const int* row_ptr, const int* col_idx, int list_heads, c
   }
   build_lists_kernel<<<static_cast<int>(lists), kListThreads, list_smem, st>>>(
       row_ptr, col_idx, g.QB, g.KB, KT, g.LR, block_q, block_k, g.expand, g.nnz_cap, cnt,
-      entries, status);
+      entries, status, page_table, pages_per_batch, heads);
   return check_launch();
 }
 

@@ -94,6 +94,10 @@ struct AttnParams {
   int* status;
   int* unit_counter;  // next unit to hand out (zeroed before the launch)
   unsigned long long timeout_ns;
+  // paged K/V: logical 128-key tile kt of batch b is physical page
+  // page_table[b * pages_per_batch + kt] of a one-batch pool (nullptr: contiguous)
+  const int* page_table;
+  int pages_per_batch;
 };
 
 struct Item {
@@ -217,11 +221,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(EMPTY(st), ph ^ 1u, abort_flag, p.status, p.timeout_ns)) return false;
         BSA_TRACE_AT(tix + 1);
         const int kt = static_cast<int>(__ldg(itm.ent + step) & 0x0FFFFFFFu);
+        const int row = p.page_table
+                            ? __ldg(p.page_table + static_cast<long long>(itm.b) * p.pages_per_batch + kt) * kBN
+                            : kt * kBN;
+        const int bco = p.page_table ? 0 : itm.b;
         mbar_expect_tx(FULL(st), C::TILE_BYTES);
 #pragma unroll
         for (int c = 0; c < C::KCH; ++c)
           tma_load_4d(sRing + st * C::TILE_BYTES + c * C::CHUNK_BYTES, map, FULL(st), 64 * c,
-                      itm.h, kt * kBN, itm.b);
+                      itm.h, row, bco);
         filled |= 1u << st;
         fill_phase = (fill_phase & ~(1u << st)) | (ph << st);
         if (++st == C::NSTAGE) { st = 0; ph ^= 1u; }
@@ -727,11 +735,17 @@ extern "C" size_t bsa_attn_workspace_size(int batch, int heads, int nq, int nk, 
   return bsa::geometry(batch, heads, nq, nk, block_q, block_k, list_heads).total;
 }
 
-extern "C" int bsa_attn_fwd(const void* q, const void* k, const void* v, int batch, int heads,
-                            int nq, int nk, int head_dim, int block_q, int block_k,
-                            const int* row_ptr, const int* col_idx, int list_heads, float scale,
-                            void* o, float* lse, void* ws, size_t ws_bytes, void* stream) {
-  using namespace bsa;
+namespace bsa {
+namespace {
+
+// Shared body of bsa_attn_fwd and bsa_attn_fwd_paged.  page_table == nullptr: K/V
+// are [batch, nk, heads, head_dim]; else they are one-batch pools of n_pool_pages
+// 128-token pages addressed through page_table [batch][pages_per_batch].
+int attn_fwd_impl(const void* q, const void* k, const void* v, int batch, int heads, int nq,
+                  int nk, int head_dim, int block_q, int block_k, const int* row_ptr,
+                  const int* col_idx, int list_heads, float scale, void* o, float* lse, void* ws,
+                  size_t ws_bytes, const int* page_table, int pages_per_batch, int n_pool_pages,
+                  cudaStream_t st) {
   if (!q || !k || !v || !o || !lse || !row_ptr || !col_idx || !ws) return BSA_ERR_INVALID_ARG;
   if (batch < 1 || heads < 1 || nq < 1 || nk < 1) return BSA_ERR_INVALID_ARG;
   if (list_heads != 1 && list_heads != batch * heads) return BSA_ERR_INVALID_ARG;
@@ -739,18 +753,26 @@ extern "C" int bsa_attn_fwd(const void* q, const void* k, const void* v, int bat
     return BSA_ERR_INVALID_ARG;
   if (head_dim != 64 && head_dim != 128) return BSA_ERR_UNSUPPORTED;
   if (!block_ok(block_q) || !block_ok(block_k)) return BSA_ERR_UNSUPPORTED;
+  if (page_table) {
+    // pages hold whole key blocks; a shared list needs a single page table
+    if (block_k > kBN || (list_heads == 1 && batch > 1)) return BSA_ERR_UNSUPPORTED;
+    if (pages_per_batch < ceil_div(nk, kBN) || n_pool_pages < 1 ||
+        static_cast<long long>(n_pool_pages) * kBN > 0x7fffffffLL)
+      return BSA_ERR_INVALID_ARG;
+  }
   const Geometry g = geometry(batch, heads, nq, nk, block_q, block_k, list_heads);
   if (ws_bytes < g.total) return BSA_ERR_WORKSPACE;
   if (g.nnz_cap > 0x7fffffffLL || static_cast<long long>(ceil_div(nk, kBN)) >= (1LL << 28) ||
       static_cast<long long>(batch) * heads * g.QT > 0x3fffffffLL)
     return BSA_ERR_UNSUPPORTED;
   if (scale <= 0.0f) scale = 1.0f / sqrtf(static_cast<float>(head_dim));
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
 
   CUtensorMap mq, mk, mv;
+  const int kv_batch = page_table ? 1 : batch;
+  const int kv_rows = page_table ? n_pool_pages * kBN : nk;
   if (make_map(&mq, q, batch, nq, heads, head_dim) != BSA_OK ||
-      make_map(&mk, k, batch, nk, heads, head_dim) != BSA_OK ||
-      make_map(&mv, v, batch, nk, heads, head_dim) != BSA_OK)
+      make_map(&mk, k, kv_batch, kv_rows, heads, head_dim) != BSA_OK ||
+      make_map(&mv, v, kv_batch, kv_rows, heads, head_dim) != BSA_OK)
     return BSA_ERR_CUDA;
 
   char* wsb = static_cast<char*>(ws);
@@ -761,7 +783,7 @@ extern "C" int bsa_attn_fwd(const void* q, const void* k, const void* v, int bat
   if (e != cudaSuccess) return record_cuda_error(e);
 
   int rc = launch_build_lists(row_ptr, col_idx, list_heads, g, nk, block_q, block_k, cnt, entries,
-                              status, st);
+                              status, st, page_table, pages_per_batch, heads);
   if (rc != BSA_OK) return rc;
 
   AttnParams p;
@@ -787,7 +809,33 @@ extern "C" int bsa_attn_fwd(const void* q, const void* k, const void* v, int bat
   p.status = status;
   p.unit_counter = status + 1;
   p.timeout_ns = 2000000000ULL;
+  p.page_table = page_table;
+  p.pages_per_batch = pages_per_batch;
   return head_dim == 128 ? launch_attn<128>(mq, mk, mv, p, st) : launch_attn<64>(mq, mk, mv, p, st);
+}
+
+}  // namespace
+}  // namespace bsa
+
+extern "C" int bsa_attn_fwd(const void* q, const void* k, const void* v, int batch, int heads,
+                            int nq, int nk, int head_dim, int block_q, int block_k,
+                            const int* row_ptr, const int* col_idx, int list_heads, float scale,
+                            void* o, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  return bsa::attn_fwd_impl(q, k, v, batch, heads, nq, nk, head_dim, block_q, block_k, row_ptr,
+                            col_idx, list_heads, scale, o, lse, ws, ws_bytes, nullptr, 0, 0,
+                            static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int bsa_attn_fwd_paged(const void* q, const void* k_pool, const void* v_pool,
+                                  int n_pool_pages, const int* page_table, int pages_per_batch,
+                                  int batch, int heads, int nq, int nk, int head_dim, int block_q,
+                                  int block_k, const int* row_ptr, const int* col_idx,
+                                  int list_heads, float scale, void* o, float* lse, void* ws,
+                                  size_t ws_bytes, void* stream) {
+  if (!page_table) return BSA_ERR_INVALID_ARG;
+  return bsa::attn_fwd_impl(q, k_pool, v_pool, batch, heads, nq, nk, head_dim, block_q, block_k,
+                            row_ptr, col_idx, list_heads, scale, o, lse, ws, ws_bytes, page_table,
+                            pages_per_batch, n_pool_pages, static_cast<cudaStream_t>(stream));
 }
 
 // ---------------------------------------------------------------------------

@@ -103,8 +103,8 @@ template <int D>
 __global__ void __launch_bounds__(256) nabla_select_kernel(
     const float* __restrict__ qbar, const float* __restrict__ kbar, int heads, int qb_count,
     int kb_count, int kb_begin, int kb_end, float p, float scale, int force_outside,
-    const uint8_t* __restrict__ base_mask, uint8_t* __restrict__ mask,
-    int* __restrict__ near_count) {
+    const uint8_t* __restrict__ base_mask, const uint8_t* __restrict__ key_allowed,
+    uint8_t* __restrict__ mask, int* __restrict__ near_count) {
   extern __shared__ float smem[];
   const int nr = kb_end - kb_begin;
   float* qs = smem;
@@ -151,9 +151,21 @@ __global__ void __launch_bounds__(256) nabla_select_kernel(
 
   float* z = zs + warp * nr;
   float* e = es + warp * nr;
+  // key blocks that may not be chosen (evicted from a paged cache) leave the softmax
+  const uint8_t* arow = key_allowed ? key_allowed + static_cast<long long>(b) * kb_count + kb_begin
+                                    : nullptr;
+  if (arow) {
+    for (int c = lane; c < nr; c += 32)
+      if (!arow[c]) z[c] = -INFINITY;
+    __syncwarp();
+  }
   float m = -INFINITY;
   for (int c = lane; c < nr; c += 32) m = fmaxf(m, z[c]);
   m = warp_max(m);
+  if (m == -INFINITY) {  // no candidate: only the base mask
+    for (int c = lane; c < nr; c += 32) mrow[kb_begin + c] = (brow && brow[kb_begin + c] != 0) ? 1 : 0;
+    return;
+  }
   float tot = 0.f;
   for (int c = lane; c < nr; c += 32) {
     const float v = __expf(z[c] - m);
@@ -164,7 +176,8 @@ __global__ void __launch_bounds__(256) nabla_select_kernel(
   __syncwarp();
 
   if (p >= 1.0f) {
-    for (int c = lane; c < nr; c += 32) mrow[kb_begin + c] = 1;
+    for (int c = lane; c < nr; c += 32)
+      mrow[kb_begin + c] = (!arow || arow[c] || (brow && brow[kb_begin + c] != 0)) ? 1 : 0;
     return;
   }
   const float target = p * tot;
@@ -237,7 +250,8 @@ namespace {
 
 int launch_select(const float* qbar, const float* kbar, int batch, int heads, int qb, int kb,
                   int head_dim, float p, float scale, int kb_begin, int kb_end, int force_outside,
-                  const uint8_t* base_mask, uint8_t* mask, int* near_count, cudaStream_t st) {
+                  const uint8_t* base_mask, const uint8_t* key_allowed, uint8_t* mask,
+                  int* near_count, cudaStream_t st) {
   const int nr = kb_end - kb_begin;
   const size_t smem = sizeof(float) * (static_cast<size_t>(kSelRows) * head_dim +
                                        static_cast<size_t>(kSelTile) * (head_dim + 1) +
@@ -255,14 +269,14 @@ int launch_select(const float* qbar, const float* kbar, int batch, int heads, in
                              cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return record_cuda_error(e);
     nabla_select_kernel<128><<<sgrid, 256, smem, st>>>(qbar, kbar, heads, qb, kb, kb_begin, kb_end,
-                                                       p, scale, force_outside, base_mask, mask,
+                                                       p, scale, force_outside, base_mask, key_allowed, mask,
                                                        near_count);
   } else {
     e = cudaFuncSetAttribute(nabla_select_kernel<64>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return record_cuda_error(e);
     nabla_select_kernel<64><<<sgrid, 256, smem, st>>>(qbar, kbar, heads, qb, kb, kb_begin, kb_end,
-                                                      p, scale, force_outside, base_mask, mask,
+                                                      p, scale, force_outside, base_mask, key_allowed, mask,
                                                       near_count);
   }
   return check_launch();
@@ -274,14 +288,15 @@ int launch_select(const float* qbar, const float* kbar, int batch, int heads, in
 extern "C" int bsa_nabla_select(const float* qbar, const float* kbar, int batch, int heads,
                                 int QB, int KB, int head_dim, float p, float scale, int kb_begin,
                                 int kb_end, int force_outside, const uint8_t* base_mask,
-                                uint8_t* mask, int* near_count, void* stream) {
+                                const uint8_t* key_allowed, uint8_t* mask, int* near_count,
+                                void* stream) {
   using namespace bsa;
   if (!qbar || !kbar || !mask) return BSA_ERR_INVALID_ARG;
   if (batch < 1 || heads < 1 || QB < 1 || KB < 1 || !(p > 0.0f)) return BSA_ERR_INVALID_ARG;
   if (head_dim != 64 && head_dim != 128) return BSA_ERR_UNSUPPORTED;
   if (kb_begin < 0 || kb_end > KB || kb_begin > kb_end) return BSA_ERR_INVALID_ARG;
   return launch_select(qbar, kbar, batch, heads, QB, KB, head_dim, p, scale, kb_begin, kb_end,
-                       force_outside, base_mask, mask, near_count,
+                       force_outside, base_mask, key_allowed, mask, near_count,
                        static_cast<cudaStream_t>(stream));
 }
 
@@ -310,5 +325,5 @@ extern "C" int bsa_nabla_mask(const void* q, const void* k, int batch, int heads
   int rc = check_launch();
   if (rc != BSA_OK) return rc;
   return launch_select(qbar, kbar, batch, heads, qb, kb, head_dim, p, scale, kb_begin, kb_end,
-                       force_outside, nullptr, mask, near_count, st);
+                       force_outside, nullptr, nullptr, mask, near_count, st);
 }

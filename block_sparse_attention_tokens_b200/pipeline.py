@@ -162,3 +162,113 @@ def effective_flops(mask: torch.Tensor, nq: int, nk: int, block: int, head_dim: 
     if m.shape[0] == 1:
         pairs *= batch_heads
     return 4.0 * head_dim * pairs
+
+
+class PagedARCache:
+    """Paged K/V cache of an autoregressive run with persistent anchors.
+
+    The key sequence grows a chunk (``chunk_frames`` frames) at a time.  K and V
+    live in pools of 128-token pages with one page table per batch; the pools hold
+    only ``pool_pages_per_batch`` pages per batch -- anchors, the recent window,
+    ``budget`` middle pages and room for the next chunk -- not the whole sequence.
+    A chunk step is ``append`` (write the chunk's K/V to free pages), ``attend``
+    (mask = anchors + recent forced, NABLA over the resident middle blocks; paged
+    attention) and ``evict`` (page importance from the chunk's pooled queries, keep
+    the ``budget`` most important middle pages, free the rest).  Every step is a
+    libbsa kernel; the free list lives on the host (one small read-back per chunk).
+    """
+
+    def __init__(self, w: Workload, max_tokens: int, budget: int, device=torch.device("cuda")):
+        self.w, self.dev = w, device
+        Bt, Hh, D = w.batch, w.heads, w.head_dim
+        self.page = B.KV_PAGE
+        self.block = w.block
+        self.S = w.tokens_per_frame
+        self.budget = budget
+        self.max_pages = ceil_div(max_tokens, self.page)
+        self.anchor_tokens = w.anchor_frames * self.S
+        self.recent_tokens = w.recent_frames * self.S
+        chunk_tokens = (w.q_frames or 1) * self.S
+        per_batch = (ceil_div(self.anchor_tokens, self.page) + ceil_div(self.recent_tokens, self.page)
+                     + budget + ceil_div(chunk_tokens, self.page) + 3)
+        self.pool_pages_per_batch = min(per_batch, self.max_pages)
+        n_pool = Bt * self.pool_pages_per_batch
+        self.k_pool = torch.zeros((n_pool, self.page, Hh, D), dtype=torch.bfloat16, device=device)
+        self.v_pool = torch.zeros_like(self.k_pool)
+        self.table_host = torch.full((Bt, self.max_pages), -1, dtype=torch.int32)
+        self.table = self.table_host.to(device)
+        self.free = list(range(n_pool))
+        self.freed = torch.empty(Bt * self.max_pages, dtype=torch.int32, device=device)
+        self.freed_count = torch.zeros(1, dtype=torch.int32, device=device)
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        self.n_tokens = 0
+        self.attn_ws = None
+
+    def resident_bytes(self) -> int:
+        """Bytes of K and V the cache holds now (resident pages only)."""
+        pages = int((self.table_host >= 0).sum())
+        w = self.w
+        return 2 * pages * self.page * w.heads * w.head_dim * 2
+
+    def pool_bytes(self) -> int:
+        return 2 * self.k_pool.numel() * self.k_pool.element_size()
+
+    def append(self, k: torch.Tensor, v: torch.Tensor):
+        Bt, n_new = k.shape[0], k.shape[1]
+        first, last = self.n_tokens, self.n_tokens + n_new
+        if ceil_div(last, self.page) > self.max_pages:
+            raise ValueError("sequence longer than the cache was sized for")
+        for b in range(Bt):
+            for lp in range(first // self.page, ceil_div(last, self.page)):
+                if self.table_host[b, lp] < 0:
+                    if not self.free:
+                        raise RuntimeError("KV pool exhausted")
+                    self.table_host[b, lp] = self.free.pop()
+        self.table.copy_(self.table_host)
+        B.bsa_kv_write(k, first, self.table, self.k_pool, self.status)
+        B.bsa_kv_write(v, first, self.table, self.v_pool, self.status)
+        self.n_tokens = last
+
+    def attend(self, q: torch.Tensor, p: float, scale: float = 0.0):
+        """Attention of the chunk's queries q [B, nq, H, D] over the cache.  Returns
+        (O, LSE, mask); keeps the pooled means for ``evict``."""
+        w = self.w
+        Bt, nq, Hh, D = q.shape
+        nk, blk = self.n_tokens, self.block
+        QB, KB = ceil_div(nq, blk), ceil_div(nk, blk)
+        self.qbar = torch.empty((Bt, Hh, QB, D), dtype=torch.float32, device=self.dev)
+        self.kbar = torch.empty((Bt, Hh, KB, D), dtype=torch.float32, device=self.dev)
+        B.bsa_block_pool(q, nq, blk, 0, QB, self.qbar)
+        B.bsa_block_pool(self.k_pool, nk, blk, 0, KB, self.kbar, page_table=self.table, batch=Bt)
+        self.allowed = B.bsa_kv_resident_blocks(self.table, blk, KB)
+        self.kb_range = ar_block_ranges(nk, self.S, blk, w.anchor_frames, w.recent_frames)
+        a_end, r_begin = self.kb_range
+        mask, self.near = B.bsa_nabla_select(self.qbar, self.kbar, p, scale, a_end, r_begin, 1,
+                                             key_allowed=self.allowed)
+        row_ptr, col_idx = B.bsa_mask_compact(mask)
+        size = B.bsa_attn_workspace_size(Bt, Hh, nq, nk, blk, blk, Bt * Hh)
+        if self.attn_ws is None or self.attn_ws.numel() < size:
+            self.attn_ws = torch.empty(size, dtype=torch.uint8, device=self.dev)
+        o, lse, _ = B.bsa_attn_fwd_paged(q, self.k_pool, self.v_pool, self.table, nk, row_ptr,
+                                         col_idx, blk, blk, Bt * Hh, scale=scale, ws=self.attn_ws)
+        return o, lse, mask
+
+    def evict(self, scale: float = 0.0):
+        """Keeps the anchors, the recent window and the `budget` most important middle
+        pages (importance from the last ``attend``); frees the other pages."""
+        nk, blk = self.n_tokens, self.block
+        n_pages = ceil_div(nk, self.page)
+        a_end, r_begin = self.kb_range
+        scores = B.bsa_kv_page_scores(self.qbar, self.kbar, a_end, r_begin, blk, n_pages,
+                                      scale=scale, key_allowed=self.allowed)
+        anchor_pages = ceil_div(self.anchor_tokens, self.page)
+        recent_begin = max(anchor_pages, (nk - self.recent_tokens) // self.page)
+        self.freed_count.zero_()
+        B.bsa_kv_keep_pages(scores, anchor_pages, recent_begin, self.budget, self.table,
+                            self.freed, self.freed_count)
+        self.table_host.copy_(self.table.cpu())
+        n = int(self.freed_count.item())
+        self.free.extend(self.freed[:n].cpu().tolist())
+        self.last_scores = scores
+        self.last_pages = (anchor_pages, recent_begin)
+

@@ -172,12 +172,15 @@ int bsa_nabla_mask(const void* q, const void* k, int batch, int heads, int nq, i
  * Semantics of p, scale, kb_begin, kb_end, force_outside, mask and near_count
  * as for bsa_nabla_mask.  base_mask (may be NULL): [QB][KB] uint8 shared by all
  * batches and heads, OR-ed into every row of the result -- with a Sliding-Tile
- * mask this gives the NABLA-plus-window hybrid.  head_dim in {64, 128}.
+ * mask this gives the NABLA-plus-window hybrid.  key_allowed (may be NULL):
+ * [batch][KB] uint8; key blocks with 0 (e.g. evicted from a paged cache, see
+ * bsa_kv_resident_blocks) leave the softmax of [kb_begin, kb_end) and are never
+ * selected there.  head_dim in {64, 128}.
  * ------------------------------------------------------------------------- */
 int bsa_nabla_select(const float* qbar, const float* kbar, int batch, int heads, int QB, int KB,
                      int head_dim, float p, float scale, int kb_begin, int kb_end,
-                     int force_outside, const uint8_t* base_mask, uint8_t* mask,
-                     int* near_count, void* stream);
+                     int force_outside, const uint8_t* base_mask, const uint8_t* key_allowed,
+                     uint8_t* mask, int* near_count, void* stream);
 
 /* ---------------------------------------------------------------------------
  * (c) Mask compaction into per-row kept-block lists (CSR).
@@ -316,6 +319,66 @@ size_t bsa_sics_workspace_size(int batch, int heads, int T, int H, int W, const 
 int bsa_sics_scheme(const void* q, const void* k, int batch, int T, int H, int W, int heads,
                     int head_dim, const int* shapes, int n_shapes, float* scores, int* choice,
                     void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * (g) Paged KV cache with persistent anchors (autoregressive chunk decoding).
+ * Source: Sparse Forcing summary (gist.science/ja/paper/2604.21221), part 2
+ * (anchors kept as persistent memory, recent frames looked at closely, only the
+ * important points of the past stored) and part 4 (memory use down 42 %).
+ *
+ * Pages hold 128 consecutive tokens of the key sequence (one attention k-tile)
+ * with the [token][heads][head_dim] bf16 row layout.  A pool of n_pool_pages
+ * pages is shared by the batch; page_table [batch][pages_per_batch] int32 maps
+ * logical page lp (tokens 128*lp .. 128*lp+127) to a physical page, -1 when
+ * evicted.  The pool must be allocated initialised (e.g. zeros): rows past the
+ * end of the sequence in its last page are read and must be finite.
+ *
+ * bsa_kv_write: rows [batch, n_new, heads, head_dim] bf16 go to logical tokens
+ *   first_token .. first_token+n_new-1 of each batch; their pages must be
+ *   assigned.  A row whose page is -1 or out of range is skipped and
+ *   BSA_ERR_INVALID_ARG is written to *device_status (a device int, may be NULL).
+ * bsa_block_pool: out[b][h][first_block + i][:] = mean of tokens
+ *   [block*(first_block+i), min(block*(first_block+i+1), n_tokens)) of x, for
+ *   i < n_blocks; x is [batch, n_tokens, heads, head_dim] (page_table NULL) or a
+ *   paged pool; out is float32 [batch][heads][out_blocks][head_dim].
+ * bsa_kv_resident_blocks: allowed[b][kb] = 1 iff the page of key block kb
+ *   (block tokens, 128 % block == 0) is resident.
+ * bsa_kv_page_scores: scores[b][page] = sum over heads h and query blocks qb of
+ *   softmax_kb(qbar[b,h,qb] . kbar[b,h,kb] * scale) over the allowed kb in
+ *   [kb_begin, kb_end), summed over the blocks kb of that page (zeroed first).
+ * bsa_kv_keep_pages: scores [batch][n_pages]; page_table rows of
+ *   pages_per_batch >= n_pages entries.  Per batch, pages < anchor_pages and
+ *   >= recent_begin are kept; of the resident pages in between the `budget` highest scores are kept
+ *   (ties: the lower page) and every other one is evicted: its page_table entry
+ *   becomes -1 and its physical page is appended to freed[] (capacity: batch *
+ *   (recent_begin - anchor_pages) ints) at index atomicAdd(freed_count, 1).
+ *   recent_begin - anchor_pages <= 8192.
+ * bsa_attn_fwd_paged: bsa_attn_fwd with K and V read through the page table
+ *   from one-batch pools [n_pool_pages * 128, heads, head_dim]; key blocks on
+ *   evicted pages are dropped from the kept lists.  block_k in {64, 128};
+ *   pages_per_batch >= ceil(nk / 128); list_heads == batch * heads unless
+ *   batch == 1.
+ * ------------------------------------------------------------------------- */
+int bsa_kv_write(const void* src, int batch, int n_new, int heads, int head_dim, int first_token,
+                 const int* page_table, int pages_per_batch, void* pool, int n_pool_pages,
+                 int* device_status, void* stream);
+int bsa_block_pool(const void* x, const int* page_table, int pages_per_batch, int batch,
+                   int n_tokens, int heads, int head_dim, int block, int first_block,
+                   int n_blocks, float* out, int out_blocks, void* stream);
+int bsa_kv_resident_blocks(const int* page_table, int batch, int pages_per_batch, int block,
+                           int KB, uint8_t* allowed, void* stream);
+int bsa_kv_page_scores(const float* qbar, const float* kbar, int batch, int heads, int QB, int KB,
+                       int head_dim, float scale, int kb_begin, int kb_end,
+                       const uint8_t* key_allowed, int block, int n_pages, float* scores,
+                       void* stream);
+int bsa_kv_keep_pages(const float* scores, int batch, int n_pages, int anchor_pages,
+                      int recent_begin, int budget, int* page_table, int pages_per_batch,
+                      int* freed, int* freed_count, void* stream);
+int bsa_attn_fwd_paged(const void* q, const void* k_pool, const void* v_pool, int n_pool_pages,
+                       const int* page_table, int pages_per_batch, int batch, int heads, int nq,
+                       int nk, int head_dim, int block_q, int block_k, const int* row_ptr,
+                       const int* col_idx, int list_heads, float scale, void* o, float* lse,
+                       void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
  * Self-test of the bounded device-side waits (failure detection).
