@@ -14,6 +14,11 @@ tiles of 384 tokens, 3x3x5-tile window).  Metric: effective TFLOP/s =
 of the workload's slice-shape menu, per-head choice), metric: GB/s of Q and K read
 (one pass per shape), with its time as a fraction of the workload's attention.
 
+``--pass ar_paged`` runs the autoregressive workload's decode through the paged,
+persistent-anchor KV cache (one chunk of frames at a time: append, attend,
+evict) and times the last chunk's attention step over the cache; the line also
+reports the cache's memory against a plain cache of the whole sequence.
+
 ``--pass bwd`` times the block-sparse attention backward instead (dQ, dK, dV from
 Q, K, V, O, LSE and dO in the path's token order, over the kept lists of the
 workload's mask), metric: effective TFLOP/s = 10 * head_dim * kept pairs / time
@@ -240,6 +245,106 @@ class BackwardOracleSample(OracleSample):
 
 BWD_METRIC = "block-sparse attention backward effective TFLOP/s"
 SICS_METRIC = "SPADE SICS scheme generation GB/s (Q and K read once per menu shape)"
+AR_PAGED_METRIC = "paged AR chunk attention effective TFLOP/s (persistent-anchor KV cache)"
+AR_KEEP_FRACTION = 0.58   # pages kept at the end of the run: the Sparse Forcing summary's 42 % saving
+
+
+def ar_budget(w, keep_fraction=AR_KEEP_FRACTION):
+    """Middle pages the cache keeps so that anchors + recent + middle make up
+    keep_fraction of the pages of the whole sequence."""
+    page = 128
+    S = w.tokens_per_frame
+    n_pages = math.ceil(w.n_tokens / page)
+    anchor_pages = math.ceil(w.anchor_frames * S / page)
+    recent_begin = (w.n_tokens - w.recent_frames * S) // page
+    return max(0, round(keep_fraction * n_pages) - anchor_pages - (n_pages - recent_begin))
+
+
+def ar_all_queries(w):
+    """Q for every token of the AR workload (each chunk's queries), K and V."""
+    import numpy as np
+    from block_sparse_attention_tokens_b200 import synth
+    q, k, v, _ = synth.generate(w.batch, w.heads, w.head_dim, w.grid, w.seed, strength=w.strength,
+                                strength_range=w.strength_range, iid=w.iid,
+                                q_token_ids=np.arange(w.n_tokens))
+    return q, k, v
+
+
+class PagedAROracleSample:
+    """The oracle on the last chunk of the paged AR run: the cache's residency is
+    simulated with the oracle's own policy over every earlier chunk (untimed
+    setup); the timed part is the oracle's attention over the resident pages for
+    random query blocks of the last chunk (all heads)."""
+
+    def __init__(self, w, q, k, v):
+        import numpy as np
+        import oracle as O
+        self.w, self.O, self.np = w, O, np
+        t0 = time.perf_counter()
+        S, blk, page = w.tokens_per_frame, w.block, 128
+        chunk = w.q_frames * S
+        scale = 1.0 / math.sqrt(w.head_dim)
+        n_chunks = w.n_tokens // chunk
+        budget = ar_budget(w)
+        k64 = k.double().numpy()
+        KBmax = math.ceil(w.n_tokens / blk)
+        kpad = np.zeros((w.batch, KBmax * blk, w.heads, w.head_dim))
+        kpad[:, :w.n_tokens] = k64
+        kbar_all = O.nabla_pool(kpad, blk, w.n_tokens)     # every block's mean (causal per block)
+        resident = np.zeros((w.batch, math.ceil(w.n_tokens / page)), dtype=bool)
+        for c in range(n_chunks):
+            lo, hi = c * chunk, (c + 1) * chunk
+            resident[:, lo // page: math.ceil(hi / page)] = True
+            n_pages, KB = math.ceil(hi / page), math.ceil(hi / blk)
+            table = np.where(resident[:, :n_pages], 0, -1)
+            allowed = O.resident_blocks(table, page, blk, hi)
+            QB = math.ceil(chunk / blk)
+            qpad = np.zeros((w.batch, QB * blk, w.heads, w.head_dim))
+            qpad[:, :chunk] = q[:, lo:hi].double().numpy()
+            qbar = O.nabla_pool(qpad, blk, chunk)
+            kbar = kbar_all[:, :, :KB].copy()
+            if KB * blk > hi:                                # the last block is partial now
+                kbar[:, :, KB - 1] = k64[:, (KB - 1) * blk:hi].mean(axis=1)
+            a_end, r_begin = O.ar_block_ranges(hi, S, blk, w.anchor_frames, w.recent_frames)
+            if c == n_chunks - 1:
+                m, _ = O.nabla_mask(qbar, kbar, w.p, scale, a_end, r_begin, 1, key_allowed=allowed)
+                self.mask = (m * allowed[:, None, None, :]).reshape(-1, QB, KB).astype(np.uint8)
+                break
+            sc = O.kv_page_scores(qbar, kbar, scale, a_end, r_begin, blk, page, n_pages,
+                                  key_allowed=allowed)
+            anchor_pages = math.ceil(w.anchor_frames * S / page)
+            recent_begin = max(anchor_pages, (hi - w.recent_frames * S) // page)
+            resident[:, :n_pages] &= O.kv_keep_pages(sc, resident[:, :n_pages], anchor_pages,
+                                                     recent_begin, budget)
+        self.lo, self.hi, self.chunk = (n_chunks - 1) * chunk, n_chunks * chunk, chunk
+        self.heads64 = [(q[:, self.lo:self.hi, h:h + 1].double().numpy(),
+                         k64[:, :self.hi, h:h + 1], v[:, :self.hi, h:h + 1].double().numpy())
+                        for h in range(w.heads)]
+        self.setup_s = time.perf_counter() - t0
+        self.rng = np.random.default_rng(5)
+
+    def run(self, budget_s: float):
+        w, O, np = self.w, self.O, self.np
+        blk = w.block
+        QB = math.ceil(self.chunk / blk)
+        flops, done = 0.0, 0
+        t1 = time.perf_counter()
+        for qb in self.rng.permutation(QB):
+            rows = np.arange(qb * blk, min((qb + 1) * blk, self.chunk))
+            for h, (qh, kh, vh) in enumerate(self.heads64):
+                O.block_sparse_attention(qh, kh, vh, self.mask[h:h + 1], blk, blk, rows=rows)
+                kept = np.nonzero(self.mask[h, qb])[0]
+                nkeys = sum(min((kb + 1) * blk, self.hi) - kb * blk for kb in kept)
+                flops += 4.0 * w.head_dim * len(rows) * nkeys
+            done += 1
+            if time.perf_counter() - t1 > budget_s:
+                break
+        el = time.perf_counter() - t1
+        sample = (f"{done} random query blocks x {w.heads} heads of the last chunk of {w.name} "
+                  f"over the resident pages ({flops / 1e12:.4f} effective TFLOP), float64 oracle, "
+                  f"{el:.1f} s (+{self.setup_s:.1f} s untimed setup: the oracle's cache policy over "
+                  f"the earlier chunks)")
+        return flops / el / 1e12, sample
 
 
 class SicsOracleSample:
@@ -282,6 +387,8 @@ def run_reference(args, w):
     q, k, v, _ = synth.workload_inputs(w)
     if args.pass_ == "bwd":
         sampler = BackwardOracleSample(w, q, k, v, path_order_grad(w))
+    elif args.pass_ == "ar_paged":
+        sampler = PagedAROracleSample(w, *ar_all_queries(w))
     elif args.pass_ == "sics":
         sampler = SicsOracleSample(w, q, k)
     else:
@@ -295,7 +402,8 @@ def run_reference(args, w):
         if i >= args.warmup:
             vals.append(val)
     value = statistics.median(vals) if vals else val
-    metric = {"bwd": BWD_METRIC, "sics": SICS_METRIC}.get(args.pass_, FWD_METRIC)
+    metric = {"bwd": BWD_METRIC, "sics": SICS_METRIC,
+              "ar_paged": AR_PAGED_METRIC}.get(args.pass_, FWD_METRIC)
     unit = "GB/s" if args.pass_ == "sics" else "TFLOP/s"
     line = {"impl": "reference", "metric": metric,
             "value": value, "unit": unit, "n_gpus": args.gpus, "steps": args.steps,
@@ -337,6 +445,11 @@ def workload_config(w, pass_: str = "fwd"):
            "grid_thw": list(w.grid), "block": w.block, "mask": w.mask}
     if pass_ == "bwd":
         cfg["pass"] = "backward (dQ, dK, dV)"
+    if pass_ == "ar_paged":
+        cfg["pass"] = "paged persistent-anchor KV cache, last chunk of the decode"
+        cfg["kv_page_tokens"] = 128
+        cfg["kv_keep_fraction"] = AR_KEEP_FRACTION
+        cfg["kv_middle_budget_pages"] = ar_budget(w)
     if pass_ == "sics":
         from block_sparse_attention_tokens_b200 import configs
         cfg["pass"] = "SPADE scheme generation (SICS)"
@@ -588,6 +701,137 @@ def run_sics(args, w):
     return 0
 
 
+def run_ar_paged(args, w):
+    """The AR workload decoded chunk by chunk through PagedARCache; the timed step
+    is the last chunk's attention over the cache (block means, residency, NABLA
+    over the resident middle blocks, compaction, paged attention)."""
+    import torch
+    import torch.distributed as dist
+    from block_sparse_attention_tokens_b200.pipeline import PagedARCache, Plan, effective_flops
+
+    if w.mask != "ar":
+        raise ValueError("--pass ar_paged needs an autoregressive workload")
+    world, rank, dev = setup_ranks()
+    q_h, k_h, v_h = ar_all_queries(w)
+    S = w.tokens_per_frame
+    chunk = w.q_frames * S
+    n_chunks = w.n_tokens // chunk
+    budget = ar_budget(w)
+    cache = PagedARCache(w, w.n_tokens, budget, dev)
+    qd, kd, vd = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for c in range(n_chunks - 1):
+        lo, hi = c * chunk, (c + 1) * chunk
+        cache.append(kd[:, lo:hi], vd[:, lo:hi])
+        cache.attend(qd[:, lo:hi], w.p)
+        cache.evict()
+    lo, hi = (n_chunks - 1) * chunk, n_chunks * chunk
+    cache.append(kd[:, lo:hi], vd[:, lo:hi])
+    q_last = qd[:, lo:hi].contiguous()
+    for _ in range(max(3, args.warmup)):
+        o, lse, mask = cache.attend(q_last, w.p)
+    barrier()
+    if cache.status.item() != 0 or B_status(cache.attn_ws) != 0:
+        raise RuntimeError("paged cache kernels reported a device-side error")
+    flops = effective_flops(mask, chunk, hi, w.block, w.head_dim, w.batch * w.heads)
+    resident_before = cache.resident_bytes()
+
+    stream = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    sampler = ClockSampler(dev.index)
+    barrier()
+    with sampler:
+        time.sleep(0.5)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            cache.attend(q_last, w.p)
+            ev[i][1].record(stream)
+        barrier()
+    ms = max_over_ranks([statistics.mean(a.elapsed_time(b) for a, b in ev)], dev)[0]
+    value = weak_scaling_value(flops, world, ms)
+
+    # the same chunk through the plain (contiguous, never evicting) AR path
+    plan = Plan(w, dev)
+    plan.step(q_last, kd, vd)
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    a0.record(stream)
+    for _ in range(5):
+        plan.build_mask()
+        plan.compact()
+        plan.attention()
+    a1.record(stream)
+    barrier()
+    plain_ms = a0.elapsed_time(a1) / 5
+    del plan
+
+    e2e = None
+    if not args.no_e2e:
+        hq = q_h[:, lo:hi].contiguous().pin_memory()
+        ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        dq_ = torch.empty_like(q_last)
+        e_steps = max(3, args.steps // 2)
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e_steps):
+            dq_.copy_(hq, non_blocking=True)
+            o_, _, _ = cache.attend(dq_, w.p)
+            ho.copy_(o_, non_blocking=True)
+        e1.record(stream)
+        barrier()
+        e_ms = max_over_ranks([e0.elapsed_time(e1) / e_steps], dev)[0]
+        e2e = {"value": weak_scaling_value(flops, world, e_ms), "unit": "TFLOP/s",
+               "ms_per_step": e_ms, "h2d_bytes_per_step": hq.numel() * hq.element_size(),
+               "d2h_bytes_per_step": ho.numel() * ho.element_size(),
+               "note": "the chunk's queries from pinned host memory, O back; K/V stay in the "
+                       "device cache (that is the cache's job)"}
+
+    cache.evict()
+    barrier()
+    plain_bytes = 2 * w.batch * w.n_tokens * w.heads * w.head_dim * 2
+    kv = {"plain_cache_bytes": plain_bytes, "resident_bytes_before_evict": resident_before,
+          "resident_bytes_after_evict": cache.resident_bytes(), "pool_bytes": cache.pool_bytes(),
+          "saving_vs_plain": 1.0 - cache.resident_bytes() / plain_bytes,
+          "pool_saving_vs_plain": 1.0 - cache.pool_bytes() / plain_bytes}
+    peaks, peak_kind = load_peaks()
+    peak = peaks["bf16_tflops_sustained"]
+    roofline = {"bound": "tensor", "achieved": value / world, "peak": peak, "unit": "TFLOP/s",
+                "frac": value / world / peak, "traffic": None,
+                "kernel": "attn_fwd_kernel<128> through the page table, with the chunk's mask "
+                          "kernels (the whole attend step is timed)",
+                "peak_note": f"{peak_kind} sustained bf16"}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        val, sample = PagedAROracleSample(w, q_h, k_h, v_h).run(args.cpu_budget)
+        cpu = {"value": val, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+               "sample": sample}
+    if rank == 0:
+        line = {"metric": AR_PAGED_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+                "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic", "config": workload_config(w, "ar_paged"),
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "clocks": sampler.summary(), "gpu_launches": 6 * args.steps,
+                "kv_cache": kv, "plain_path_attend_ms": plain_ms,
+                "effective_tflop_per_step": flops / 1e12}
+        print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def B_status(ws):
+    from block_sparse_attention_tokens_b200 import binding as B
+    return B.bsa_read_status(ws)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -601,13 +845,17 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--heads", type=int, default=0,
                     help="override the head count (smaller cases for profiler captures)")
-    ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "bwd", "sics"],
+    ap.add_argument("--pass", dest="pass_", default="fwd",
+                    choices=["fwd", "bwd", "sics", "ar_paged"],
                     help="fwd: the whole forward path (default); bwd: the attention "
-                         "backward; sics: SPADE scheme generation")
+                         "backward; sics: SPADE scheme generation; ar_paged: the AR decode "
+                         "through the paged persistent-anchor KV cache")
     args = ap.parse_args()
 
     from block_sparse_attention_tokens_b200 import configs
     import dataclasses
+    if args.pass_ == "ar_paged" and args.workload == "sta_720p":
+        args.workload = "ar_decode"
     w = configs.get(args.workload)
     if args.heads > 0:
         w = dataclasses.replace(w, heads=args.heads)
@@ -617,6 +865,8 @@ def main():
         return run_backward(args, w)
     if args.pass_ == "sics":
         return run_sics(args, w)
+    if args.pass_ == "ar_paged":
+        return run_ar_paged(args, w)
 
     import torch
     import torch.distributed as dist
