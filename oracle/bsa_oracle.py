@@ -493,7 +493,7 @@ def block_sparse_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, mask: np
 # 8. Backward of the block-sparse attention (training)
 # ---------------------------------------------------------------------------
 
-def block_sparse_attention_backward(q, k, v, do, mask, block_q, block_k, scale=None):
+def block_sparse_attention_backward(q, k, v, do, mask, block_q, block_k, scale=None, rows=None):
     """Gradients of O = softmax(Q K^T * scale + M) V with respect to Q, K, V.
 
     The Radial explainer (section 4, training cost), the NABLA explainer
@@ -504,6 +504,9 @@ def block_sparse_attention_backward(q, k, v, do, mask, block_q, block_k, scale=N
         dS = P * (dP - rowsum(dO * O)),  dQ = dS K * scale,  dK = dS^T Q * scale,
     evaluated over each row's kept key blocks only (masked entries have P = 0).
     q: [B, Nq, H, D]; k, v: [B, Nk, H, D]; do: [B, Nq, H, D]; mask: [Hm, QB, KB].
+    ``rows`` (optional): evaluate only these query rows -- dq is exact on them (0
+    elsewhere) and dk, dv hold only their contributions (for sampled checks at
+    full size).
     Returns (dq, dk, dv) with the shapes of q, k, v.
     """
     Bn, nq, H, D = q.shape
@@ -516,23 +519,26 @@ def block_sparse_attention_backward(q, k, v, do, mask, block_q, block_k, scale=N
         for h in range(H):
             m = mask[0 if mask.shape[0] == 1 else b * H + h]
             for qb in range(m.shape[0]):
-                rows = np.arange(qb * block_q, min((qb + 1) * block_q, nq))
+                rows_b = np.arange(qb * block_q, min((qb + 1) * block_q, nq))
+                if rows is not None:
+                    rows_b = np.intersect1d(rows_b, np.asarray(rows))
                 kept = np.nonzero(m[qb])[0]
-                if kept.size == 0 or rows.size == 0:
+                if kept.size == 0 or rows_b.size == 0:
                     continue
+                rows_ = rows_b
                 cols = np.concatenate([np.arange(kb * block_k, min((kb + 1) * block_k, nk))
                                        for kb in kept])
-                s = (q[b, rows, h] @ k[b, cols, h].T) * scale
+                s = (q[b, rows_, h] @ k[b, cols, h].T) * scale
                 s = s - s.max(axis=1, keepdims=True)
                 p = np.exp(s)
                 p /= p.sum(axis=1, keepdims=True)
                 o = p @ v[b, cols, h]
-                g = do[b, rows, h]
+                g = do[b, rows_, h]
                 dv[b, cols, h] += p.T @ g
                 dp = g @ v[b, cols, h].T
                 ds = p * (dp - (g * o).sum(axis=1, keepdims=True))
-                dq[b, rows, h] += (ds @ k[b, cols, h]) * scale
-                dk[b, cols, h] += (ds.T @ q[b, rows, h]) * scale
+                dq[b, rows_, h] += (ds @ k[b, cols, h]) * scale
+                dk[b, cols, h] += (ds.T @ q[b, rows_, h]) * scale
     return dq, dk, dv
 
 

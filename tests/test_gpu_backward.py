@@ -37,9 +37,9 @@ pytestmark = pytest.mark.gpu
 U = 2.0 ** -9
 
 
-def envelopes(q, k, v, do, o_bf16, lse_ref, mask, bq, bk, scale):
+def envelopes(q, k, v, do, o_ref, lse_ref, mask, bq, bk, scale):
     """Per-entry error envelopes (see the module docstring); float64 numpy.
-    q, do, o_bf16: [B, nq, H, D]; k, v: [B, nk, H, D]; lse_ref: [B, H, nq]."""
+    q, do, o_ref: [B, nq, H, D]; k, v: [B, nk, H, D]; lse_ref: [B, H, nq]."""
     Bn, nq, H, D = q.shape
     nk = k.shape[1]
     env_q, env_k, env_v = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
@@ -55,7 +55,7 @@ def envelopes(q, k, v, do, o_bf16, lse_ref, mask, bq, bk, scale):
             g = do[b, :, h]
             dp = g @ v[b, :, h].T
             delta = (g * (p @ v[b, :, h])).sum(axis=1)
-            w = (np.abs(g) * (p @ np.abs(v[b, :, h]) + np.abs(o_bf16[b, :, h]))).sum(axis=1)
+            w = (np.abs(g) * (p @ np.abs(v[b, :, h]) + np.abs(o_ref[b, :, h]))).sum(axis=1)
             e = p * (np.abs(dp) + np.abs(delta)[:, None] + w[:, None])
             env_v[b, :, h] = p.T @ np.abs(g)
             env_q[b, :, h] = scale * (e @ np.abs(k[b, :, h]))
@@ -95,8 +95,8 @@ def run_bwd(Bn, H, nq, nk, D, bq, bk, mask, list_heads, seed, scale=0.0):
     sc = 1.0 / math.sqrt(D) if scale <= 0 else scale
     q64, k64, v64, do64 = to64(q), to64(k), to64(v), to64(do)
     rdq, rdk, rdv = O.block_sparse_attention_backward(q64, k64, v64, do64, mask, bq, bk, scale=sc)
-    _, rl = O.block_sparse_attention(q64, k64, v64, mask, bq, bk, scale=sc)
-    eq, ek, ev = envelopes(q64, k64, v64, do64, to64(o), rl, mask, bq, bk, sc)
+    ro, rl = O.block_sparse_attention(q64, k64, v64, mask, bq, bk, scale=sc)
+    eq, ek, ev = envelopes(q64, k64, v64, do64, ro, rl, mask, bq, bk, sc)
     return (assert_grad_close(to64(dq), rdq, eq, "dQ"), assert_grad_close(to64(dk), rdk, ek, "dK"),
             assert_grad_close(to64(dv), rdv, ev, "dV"))
 
@@ -138,3 +138,65 @@ def test_sta_mask_on_a_tiled_grid():
     tg, window = (1, 2, 2), (1, 3, 3)
     m = O.sta_tile_mask(tg, window)[None].astype(np.uint8)
     run_bwd(1, 2, 256, 256, 128, 64, 64, m, 1, seed=13)
+
+
+def test_full_size_sta_720p_sampled_rows_and_identities():
+    """The 720p Sliding-Tile workload at full size (24 heads, 115,200 tokens, the
+    benchmark's launch): dQ on sampled rows against the oracle within the per-entry
+    envelope, and two identities that hold at any size and involve every dK and dV
+    entry: sum_i q_i . dQ_i = sum_j k_j . dK_j (both equal scale * sum dS_ij q_i.k_j)
+    and sum_j dV_j = sum of dO_i over rows that keep a key (probability rows sum to
+    1).  The identities are coarse (1 % of the absolute sums) -- they catch a lost
+    quadrant, term or factor, not rounding."""
+    from block_sparse_attention_tokens_b200 import configs
+    from block_sparse_attention_tokens_b200.pipeline import Plan
+    w = configs.get("sta_720p")
+    q, k, v, _ = synth.workload_inputs(w)
+    plan = Plan(w)
+    plan.step(q.cuda(), k.cuda(), v.cuda())
+    do = synth.grad_output(w)
+    dq, dk, dv, ws = B.bsa_attn_bwd(plan.qp, plan.kp, plan.vp, plan.op, do.cuda(), plan.lse,
+                                    plan.row_ptr, plan.col_idx, w.block, w.block, plan.list_heads,
+                                    nq=plan.nq, nk=plan.nk)
+    torch.cuda.synchronize()
+    assert B.bsa_read_status(ws) == 0
+    perm = O.tile_order(w.grid, w.tile)
+    mask = O.sta_tile_mask(plan.tile_grid, w.window)[None]
+    sc = 1.0 / math.sqrt(w.head_dim)
+    rng = np.random.default_rng(3)
+    qbs = [0, plan.QB - 1] + list(rng.choice(plan.QB, 2, replace=False))
+    rows = np.unique(np.concatenate([qb * w.block + np.array([0, 191, w.block - 1]) for qb in qbs]))
+    dq_g = to64(dq[:, :w.nq])
+    for h in (0, 13):
+        qh = O.tile_permute(to64(q[:, :, h:h + 1]), perm, plan.n_pad)[:, :w.nq]
+        kh = O.tile_permute(to64(k[:, :, h:h + 1]), perm, plan.n_pad)[:, :w.nk]
+        vh = O.tile_permute(to64(v[:, :, h:h + 1]), perm, plan.n_pad)[:, :w.nk]
+        doh = to64(do[:, :, h:h + 1])
+        rdq, _, _ = O.block_sparse_attention_backward(qh, kh, vh, doh, mask, w.block, w.block,
+                                                      rows=rows)
+        ro, rl = O.block_sparse_attention(qh, kh, vh, mask, w.block, w.block, rows=rows)
+        for i in rows:
+            kept = np.nonzero(mask[0, i // w.block])[0]
+            cols = np.concatenate([np.arange(kb * w.block, min((kb + 1) * w.block, w.nk))
+                                   for kb in kept])
+            kk, vv, g = kh[0, cols, 0], vh[0, cols, 0], doh[0, i, 0]
+            p = np.exp((kk @ qh[0, i, 0]) * sc - rl[0, 0, i])
+            dp = vv @ g
+            delta = g @ ro[0, i, 0]
+            wi = np.sum(np.abs(g) * (p @ np.abs(vv) + np.abs(ro[0, i, 0])))
+            env = sc * ((p * (np.abs(dp) + abs(delta) + wi)) @ np.abs(kk))
+            err = np.abs(dq_g[0, i, h] - rdq[0, i, 0])
+            assert np.all(err <= 4 * U * env + 2 * U * np.abs(rdq[0, i, 0])), (h, i)
+    # identities over all heads and every entry of dK and dV
+    qp, kp, vpd = to64(plan.qp[:, :w.nq]), to64(plan.kp[:, :w.nk]), to64(dv[:, :w.nk])
+    dkg = to64(dk[:, :w.nk])
+    lhs = np.einsum("bnhd,bnhd->h", qp, dq_g)
+    rhs = np.einsum("bnhd,bnhd->h", kp, dkg)
+    scale_abs = (np.einsum("bnhd,bnhd->h", np.abs(qp), np.abs(dq_g))
+                 + np.einsum("bnhd,bnhd->h", np.abs(kp), np.abs(dkg)))
+    assert np.all(np.abs(lhs - rhs) <= 1e-2 * scale_abs)
+    do64 = to64(do)
+    dv_sum = vpd.sum(axis=1)
+    do_sum = do64.sum(axis=1)                       # every STA query row keeps keys
+    assert np.all(np.abs(dv_sum - do_sum) <= 1e-2 * np.abs(do64).sum(axis=1))
+

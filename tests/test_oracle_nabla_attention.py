@@ -234,3 +234,20 @@ def test_backward_matches_autograd_float64(bq, bk):
     o.backward(torch.from_numpy(do))
     for got, ref in ((dq, tq.grad), (dk, tk.grad), (dv, tv.grad)):
         assert np.max(np.abs(got - ref.numpy())) < 1e-12
+
+
+def test_backward_row_sampling_is_exact_on_dq_and_additive_on_dk_dv():
+    Bn, H, D, bq, bk = 1, 2, 16, 64, 64
+    nq, nk = 200, 300
+    q, k, v = _rand_qkv(Bn, nq, nk, H, D, 31)
+    do = np.random.default_rng(32).standard_normal((Bn, nq, H, D))
+    mask = (np.random.default_rng(33).random((Bn * H, 4, 5)) < 0.6).astype(np.uint8)
+    full = O.block_sparse_attention_backward(q, k, v, do, mask, bq, bk)
+    rows_a = np.arange(0, nq, 3)
+    rows_b = np.setdiff1d(np.arange(nq), rows_a)
+    ga = O.block_sparse_attention_backward(q, k, v, do, mask, bq, bk, rows=rows_a)
+    gb = O.block_sparse_attention_backward(q, k, v, do, mask, bq, bk, rows=rows_b)
+    assert np.allclose(ga[0][:, rows_a], full[0][:, rows_a], atol=1e-12)
+    assert np.all(ga[0][:, rows_b] == 0)
+    for i in (1, 2):                                    # dK, dV: the two halves add up
+        assert np.allclose(ga[i] + gb[i], full[i], atol=1e-12)
