@@ -582,7 +582,7 @@ def run_backward(args, w):
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16", "data": "synthetic", "config": workload_config(w, "bwd"),
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-                "clocks": sampler.summary(), "gpu_launches": 7 * args.steps,
+                "clocks": sampler.summary(), "gpu_launches": 6 * args.steps,
                 "effective_tflop_per_step": flops / 1e12}
         print(json.dumps(line))
     if world > 1:

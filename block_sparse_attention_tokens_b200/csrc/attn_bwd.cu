@@ -16,12 +16,14 @@
 //          dK += dS Q (TS MMAs, A operand from TMEM).
 //   kDQ  : one CTA per 128-row q-tile; iterates its kept list.  S = Q K^T and
 //          dP = dO V^T -> dS -> dQ += dS K.
-// TMEM: two (S | dP) half-step buffers of 64 + 64 columns, accA (dK or dQ) and
-// accB (dV) of 128 columns each; P and dS in bf16 over the S and dP columns they
-// came from.  Warps 0-7 compute (two per TMEM lane quarter, 32 columns each),
-// warp 8 feeds a ring of (half, half) pairs with TMA, warp 9 issues the MMAs.  Units are handed out from a
-// global counter through a shared-memory ring as in the forward kernel.  All waits
-// are bounded.
+// TMEM: S | dP (128 columns each, fp32), accA (dK or dQ) and accB (dV).  The
+// compute warps turn S and dP into P and dS (bf16, packed over the columns they
+// were read from) in two 64-column halves and publish each half on its own: the
+// MMA warp accumulates the first half while the second is computed, then issues
+// the next step's S and dP.  Warps 0-7 compute (two per TMEM lane quarter, 32
+// columns of each half), warp 8 feeds a ring of 128-row operand tiles with TMA,
+// warp 9 issues the MMAs.  Units are handed out from a global counter through a
+// shared-memory ring as in the forward kernel.  All waits are bounded.
 #include "bsa_common.cuh"
 #include "tmem_io.cuh"
 #include "attn_common.cuh"
@@ -29,16 +31,16 @@
 namespace bsa {
 namespace {
 
-// Optional per-half-step timeline of CTA 0 of the dK/dV pass (SM clock), compiled
-// only with -DBSA_TRACE and read back with bsa_btrace_dump().
+// Optional per-step timeline of CTA 0 of the dK/dV pass (SM clock), compiled only
+// with -DBSA_TRACE and read back with bsa_btrace_dump().
 #ifdef BSA_TRACE
 __device__ unsigned long long g_bsa_btrace[1 << 16];
-#define BSA_BTRACE_AT(half, slot)                                                      \
+#define BSA_BTRACE_AT(step, slot)                                                      \
   do {                                                                                 \
-    if (kDKV && blockIdx.x == 0 && (half) < (1 << 13)) g_bsa_btrace[(half) * 8 + (slot)] = clock64(); \
+    if (kDKV && blockIdx.x == 0 && (step) < (1 << 13)) g_bsa_btrace[(step) * 8 + (slot)] = clock64(); \
   } while (0)
 #else
-#define BSA_BTRACE_AT(half, slot) \
+#define BSA_BTRACE_AT(step, slot) \
   do {                            \
   } while (0)
 #endif
@@ -51,15 +53,13 @@ template <int D>
 struct BwdCfg {
   static constexpr int KCH = D / 64;
   static constexpr int CHUNK_BYTES = kBM * 128;          // 128 rows of one 64-column chunk
-  static constexpr int TILE_BYTES = KCH * CHUNK_BYTES;   // 128 rows x D bf16 (row operands)
-  static constexpr int HCHUNK_BYTES = 64 * 128;          // 64 rows of one chunk
-  static constexpr int HALF_BYTES = KCH * HCHUNK_BYTES;  // 64 rows x D bf16 (column halves)
-  // ring of (colA, colB) half pairs: as deep as shared memory allows, since a
-  // half-step load takes several half-steps of MMA time to arrive
-  static constexpr int NSTAGE = D == 128 ? 5 : 12;
+  static constexpr int TILE_BYTES = KCH * CHUNK_BYTES;   // 128 rows x D bf16
+  // ring of single operand tiles (colA, colB alternating): as deep as shared memory
+  // allows, a tile load takes several steps of MMA time to arrive
+  static constexpr int NSTAGE = D == 128 ? 5 : 10;
   static constexpr int OFF_ROW = 0;                      // the two row-operand tiles
   static constexpr int OFF_RING = 2 * TILE_BYTES;
-  static constexpr int OFF_BAR = OFF_RING + NSTAGE * 2 * HALF_BYTES;
+  static constexpr int OFF_BAR = OFF_RING + NSTAGE * TILE_BYTES;
   static constexpr int SMEM = OFF_BAR + 512 + 1024;
 };
 
@@ -73,8 +73,6 @@ struct BwdParams {
   const uint32_t* entries;   // forward per-q-tile lists
   const int* tcnt;
   const uint32_t* tentries;  // transposed per-k-tile lists, stride QT
-  const int* qhcnt;          // half-steps of each forward list (dQ pass)
-  const int* thcnt;          // half-steps of each transposed list (dK/dV pass)
   const float* lse2;         // [B*H][QT*128]: LSE * log2(e), +inf past nq / for empty rows
   const float* dvec;         // [B*H][QT*128]: rowsum(dO * O), 0 past nq
   __nv_bfloat16* outA;       // dK (kDKV) or dQ (kDQ)
@@ -86,7 +84,6 @@ struct BwdParams {
 
 struct BItem {
   int b, h, row_tile, n;     // n < 0: none
-  int nh;                    // half-steps (needed 64-column halves) of the list
   const uint32_t* ent;
 };
 
@@ -94,7 +91,6 @@ template <bool kDKV>
 __device__ __forceinline__ BItem get_bitem(const BwdParams& p, int it) {
   BItem r;
   r.n = -1;
-  r.nh = 0;
   r.ent = nullptr;
   r.b = r.h = r.row_tile = 0;
   if (it >= p.total_items) return r;
@@ -107,30 +103,19 @@ __device__ __forceinline__ BItem get_bitem(const BwdParams& p, int it) {
   if (kDKV) {
     const long long g = static_cast<long long>(mh) * p.KT + r.row_tile;
     r.n = p.tcnt[g];
-    r.nh = p.thcnt[g];
     r.ent = p.tentries + g * p.QT;
   } else {
     const int lr = p.block_q >= 128 ? (r.row_tile * kBM) / p.block_q : r.row_tile;
     const int first_qb = p.block_q >= 128 ? lr : 2 * lr;
     r.n = p.cnt[mh * p.LR + lr];
-    r.nh = p.qhcnt[mh * p.LR + lr];
     r.ent = p.entries + static_cast<long long>(p.row_ptr[mh * p.QB + first_qb]) * p.expand;
   }
   return r;
 }
 
-// Entry quadrant bits are (row_half * 2 + column_half): column half h of an entry
-// is needed when either row half keeps it.
-__device__ __forceinline__ bool half_needed(uint32_t bits, int h) {
-  return ((bits >> h) | (bits >> (2 + h))) & 1u;
-}
-
 // rowA / rowB: the item's fixed operands (kDKV: K, V; kDQ: Q, dO), 128-row tiles.
-// colA / colB: the per-step operands (kDKV: Q, dO; kDQ: K, V), loaded and consumed
-// as 64-row halves (one half-step = 64 columns of S and dP); halves that no row of
-// the tile keeps are neither loaded nor computed.  S and dP of a half-step go to one
-// of two TMEM buffers (S at 128*buf, dP at 128*buf + 64), so the tensor core works
-// on the next half-step while the compute warps turn this one into P and dS.
+// colA / colB: the per-step operands (kDKV: Q, dO; kDQ: K, V), 128-row tiles
+// streamed through the ring (colA then colB per kept entry).
 template <int D, bool kDKV>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tmRowA, const __grid_constant__ CUtensorMap tmRowB,
@@ -148,13 +133,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   auto EMPTY = [&](int i) { return bar0 + 8u * (C::NSTAGE + i); };
   const uint32_t ROWFULL = bar0 + 8u * (2 * C::NSTAGE + 0);
   const uint32_t ROWEMPTY = bar0 + 8u * (2 * C::NSTAGE + 1);
-  auto SFULL = [&](uint32_t b) { return bar0 + 8u * (2 * C::NSTAGE + 2 + b); };
-  auto PREADY = [&](uint32_t b) { return bar0 + 8u * (2 * C::NSTAGE + 4 + b); };
-  const uint32_t DONE = bar0 + 8u * (2 * C::NSTAGE + 6);
-  const uint32_t FINAL = bar0 + 8u * (2 * C::NSTAGE + 7);
-  auto UFULL = [&](int i) { return bar0 + 8u * (2 * C::NSTAGE + 8 + i); };
-  auto UEMPTY = [&](int i) { return bar0 + 8u * (2 * C::NSTAGE + 12 + i); };
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + 8 * (2 * C::NSTAGE + 16));
+  const uint32_t SFULL = bar0 + 8u * (2 * C::NSTAGE + 2);
+  auto PREADY = [&](int half) { return bar0 + 8u * (2 * C::NSTAGE + 3 + half); };
+  const uint32_t DONE = bar0 + 8u * (2 * C::NSTAGE + 5);
+  const uint32_t FINAL = bar0 + 8u * (2 * C::NSTAGE + 6);
+  auto UFULL = [&](int i) { return bar0 + 8u * (2 * C::NSTAGE + 7 + i); };
+  auto UEMPTY = [&](int i) { return bar0 + 8u * (2 * C::NSTAGE + 11 + i); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + 8 * (2 * C::NSTAGE + 15));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* unit_ring = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
@@ -166,10 +151,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     mbar_init(ROWFULL, 1);
     mbar_init(ROWEMPTY, 1);
-    for (uint32_t b = 0; b < 2; ++b) {
-      mbar_init(SFULL(b), 1);
-      mbar_init(PREADY(b), 8);
-    }
+    mbar_init(SFULL, 1);
+    mbar_init(PREADY(0), 8);
+    mbar_init(PREADY(1), 8);
     mbar_init(DONE, 1);
     mbar_init(FINAL, 1);
     for (int i = 0; i < 4; ++i) {
@@ -200,8 +184,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       uint32_t filled = 0, fill_phase = 0;
       int row_filled = -1;
       bool ok = true;
-      uint32_t hl = 0;  // half-steps loaded (trace index)
-      (void)hl;
+      uint32_t gl = 0;  // steps loaded (trace index)
+      (void)gl;
+      auto load_col = [&](const CUtensorMap* map, const BItem& it, int ct) -> bool {
+        if (!mbar_wait(EMPTY(st), ph ^ 1u, abort_flag, p.status, p.timeout_ns)) return false;
+        mbar_expect_tx(FULL(st), C::TILE_BYTES);
+        for (int c = 0; c < C::KCH; ++c)
+          tma_load_4d(sRing + st * C::TILE_BYTES + c * C::CHUNK_BYTES, map, FULL(st), 64 * c,
+                      it.h, ct * kBM, it.b);
+        filled |= 1u << st;
+        fill_phase = (fill_phase & ~(1u << st)) | (ph << st);
+        if (++st == C::NSTAGE) { st = 0; ph ^= 1u; }
+        return true;
+      };
       for (int uk = 0; ok; ++uk) {
         const int slot = uk & 3;
         if (!mbar_wait(UEMPTY(slot), ((uk >> 2) & 1) ^ 1u, abort_flag, p.status, p.timeout_ns)) {
@@ -237,27 +232,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           pf2 = pf3;
           pf3 = j + 4 < it.n ? __ldg(it.ent + j + 4) : 0u;
           const int ct = static_cast<int>(ent & 0x0FFFFFFFu);
-          const uint32_t bits = ent >> 28;
-          for (int h = 0; h < 2; ++h) {
-            if (!half_needed(bits, h)) continue;
-            if (!mbar_wait(EMPTY(st), ph ^ 1u, abort_flag, p.status, p.timeout_ns)) {
-              ok = false;
-              break;
-            }
-            BSA_BTRACE_AT(hl, 6);
-            ++hl;
-            mbar_expect_tx(FULL(st), 2 * C::HALF_BYTES);
-            const uint32_t dst = sRing + st * 2 * C::HALF_BYTES;
-            const int r0 = ct * kBM + 64 * h;
-            for (int c = 0; c < C::KCH; ++c) {
-              tma_load_4d(dst + c * C::HCHUNK_BYTES, &tmColA, FULL(st), 64 * c, it.h, r0, it.b);
-              tma_load_4d(dst + C::HALF_BYTES + c * C::HCHUNK_BYTES, &tmColB, FULL(st), 64 * c,
-                          it.h, r0, it.b);
-            }
-            filled |= 1u << st;
-            fill_phase = (fill_phase & ~(1u << st)) | (ph << st);
-            if (++st == C::NSTAGE) { st = 0; ph ^= 1u; }
-          }
+          ok = load_col(&tmColA, it, ct);
+          BSA_BTRACE_AT(gl, 7);
+          ++gl;
+          ok = ok && load_col(&tmColB, it, ct);
         }
       }
       for (int i = 0; i < C::NSTAGE; ++i)
@@ -269,61 +247,58 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else if (warp == kBwdMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_ss = idesc_bf16_f32(kBM, 64, 0, 0);
+      constexpr uint32_t idesc_ss = idesc_bf16_f32(kBM, kBN, 0, 0);
       constexpr uint32_t idesc_ts = idesc_bf16_f32(kBM, D, 0, 1);
       constexpr uint32_t kTileUnits = C::TILE_BYTES >> 4;
-      constexpr uint32_t kHalfUnits = C::HALF_BYTES >> 4;
       const uint64_t dRowK = smem_desc_sw128(sRow, 16, 1024);
       const uint64_t dColK = smem_desc_sw128(sRing, 16, 1024);
-      const uint64_t dColMN = smem_desc_sw128(sRing, C::HCHUNK_BYTES, 1024);
+      const uint64_t dColMN = smem_desc_sw128(sRing, C::CHUNK_BYTES, 1024);
       int st = 0;
-      uint32_t ph = 0, rph = 0;
-      uint32_t hc = 0;  // half-steps whose S / dP were issued (all items)
-      uint32_t ha = 0;  // half-steps whose accumulation was issued
-      int stage_b0 = 0, stage_b1 = 0;  // ring stage held by each TMEM buffer
+      uint32_t ph = 0, rph = 0, pph = 0;
       bool ok = true;
-      // S-like (rowA colA_half^T) and dP-like (rowB colB_half^T) into TMEM buffer `buf`
-      auto sd = [&](int stage, uint32_t buf) {
+      uint32_t gm = 0;  // steps issued (trace index)
+      (void)gm;
+      auto acquire = [&](int& stage) -> bool {
+        if (!mbar_wait(FULL(st), ph, abort_flag, p.status, p.timeout_ns)) return false;
+        stage = st;
+        if (++st == C::NSTAGE) { st = 0; ph ^= 1u; }
+        return true;
+      };
+      // S-like = rowA colA^T into TMEM [0,128), dP-like = rowB colB^T into [128,256)
+      auto sd = [&](int sa, int sb) {
         tc_fence_after();
-        const uint64_t dcol = dColK + static_cast<uint64_t>(stage * 2 * kHalfUnits);
-        const uint32_t tS = tmem + 128u * buf;
+        const uint64_t da = dColK + static_cast<uint64_t>(sa * kTileUnits);
+        const uint64_t db = dColK + static_cast<uint64_t>(sb * kTileUnits);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t offR =
+          const uint64_t off =
               static_cast<uint64_t>((((kk >> 2) * C::CHUNK_BYTES) + (kk & 3) * 32) >> 4);
-          const uint64_t offC =
-              static_cast<uint64_t>((((kk >> 2) * C::HCHUNK_BYTES) + (kk & 3) * 32) >> 4);
-          mma_ss(tS, dRowK + offR, dcol + offC, idesc_ss, kk > 0 ? 1u : 0u);
+          mma_ss(tmem, dRowK + off, da + off, idesc_ss, kk > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t offR =
+          const uint64_t off =
               static_cast<uint64_t>((((kk >> 2) * C::CHUNK_BYTES) + (kk & 3) * 32) >> 4);
-          const uint64_t offC =
-              static_cast<uint64_t>((((kk >> 2) * C::HCHUNK_BYTES) + (kk & 3) * 32) >> 4);
-          mma_ss(tS + 64, dRowK + kTileUnits + offR, dcol + kHalfUnits + offC, idesc_ss,
-                 kk > 0 ? 1u : 0u);
+          mma_ss(tmem + 128, dRowK + kTileUnits + off, db + off, idesc_ss, kk > 0 ? 1u : 0u);
         }
       };
-      // accA (+)= dS colA_half ; accB (+)= P colB_half (kDKV); A operands from TMEM
-      auto acc = [&](int stage, uint32_t buf, bool first) {
+      // one 64-column half of the accumulation: accA (+)= dS colA, accB (+)= P colB
+      // (kDKV); packed bf16 columns 16*kk .. of P / dS sit at TMEM column
+      // (kk / 2) * 32 + (kk % 2) * 8 of their half (each compute warp packs its 32
+      // columns into the first 16 of its own)
+      auto acc = [&](int sa, int sb, int half, bool first) {
         tc_fence_after();
-        const uint64_t dA = dColMN + static_cast<uint64_t>(stage * 2 * kHalfUnits);
-        const uint32_t tS = tmem + 128u * buf;
-        const uint32_t acc0 = first ? 0u : 1u;
-        // packed bf16 columns 16*kk .. 16*kk + 15 of P / dS sit at TMEM column
-        // (kk / 2) * 32 + (kk % 2) * 8 of the S / dP region (each compute warp packs
-        // its 32 columns into the first 16 of its own)
+        const uint64_t dA = dColMN + static_cast<uint64_t>(sa * kTileUnits);
+        const uint64_t dB = dColMN + static_cast<uint64_t>(sb * kTileUnits);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_ts(tmem + 256, tS + 64 + (kk >> 1) * 32 + (kk & 1) * 8,
-                 dA + static_cast<uint64_t>(kk * 128), idesc_ts, kk > 0 ? 1u : acc0);
-        if (kDKV) {
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_ts(tmem + 384, tS + (kk >> 1) * 32 + (kk & 1) * 8,
-                   dA + kHalfUnits + static_cast<uint64_t>(kk * 128), idesc_ts,
-                   kk > 0 ? 1u : acc0);
+        for (int k4 = 0; k4 < 4; ++k4) {
+          const int kk = half * 4 + k4;
+          const uint32_t col = half * 64 + (k4 >> 1) * 32 + (k4 & 1) * 8;
+          const uint32_t a0 = (first && k4 == 0) ? 0u : 1u;
+          mma_ts(tmem + 256, tmem + 128 + col, dA + static_cast<uint64_t>(kk * 128), idesc_ts, a0);
+          if (kDKV)
+            mma_ts(tmem + 256 + D, tmem + col, dB + static_cast<uint64_t>(kk * 128), idesc_ts,
+                   a0);
         }
       };
       for (int uk = 0; ok; ++uk) {
@@ -337,42 +312,40 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (u >= p.total_items) break;
         const BItem it = get_bitem<kDKV>(p, u);
         if (it.n <= 0) continue;
-        const int nh = it.nh;  // half-steps of this item
         if (!mbar_wait(ROWFULL, rph, abort_flag, p.status, p.timeout_ns)) {
           ok = false;
           break;
         }
         rph ^= 1u;
-        int issued = 0;
-        auto issue = [&]() -> bool {
-          if (!mbar_wait(FULL(st), ph, abort_flag, p.status, p.timeout_ns)) return false;
-          BSA_BTRACE_AT(hc, 4);
-          const uint32_t buf = hc & 1u;
-          if (buf) stage_b1 = st; else stage_b0 = st;
-          sd(st, buf);
-          mma_commit(SFULL(buf));
-          BSA_BTRACE_AT(hc, 5);
-          if (++st == C::NSTAGE) { st = 0; ph ^= 1u; }
-          ++hc;
-          if (++issued == nh) mma_commit(ROWEMPTY);
-          return true;
-        };
-        ok = issue() && (issued == nh || issue());
-        for (int done = 0; ok && done < nh; ++done) {
-          const uint32_t buf = ha & 1u;
-          if (!mbar_wait(PREADY(buf), (ha >> 1) & 1u, abort_flag, p.status, p.timeout_ns)) {
-            ok = false;
-            break;
+        int sa = 0, sb = 0;
+        if (!acquire(sa) || !acquire(sb)) { ok = false; break; }
+        sd(sa, sb);
+        mma_commit(SFULL);
+        if (it.n == 1) mma_commit(ROWEMPTY);
+        for (int j = 0; j < it.n && ok; ++j) {
+          for (int half = 0; half < 2; ++half) {
+            if (!mbar_wait(PREADY(half), pph, abort_flag, p.status, p.timeout_ns)) {
+              ok = false;
+              break;
+            }
+            BSA_BTRACE_AT(gm, 4 + half);
+            acc(sa, sb, half, j == 0 && half == 0);
           }
-          BSA_BTRACE_AT(ha, 3);
-          const int stage = buf ? stage_b1 : stage_b0;
-          acc(stage, buf, done == 0);
-          mma_commit(EMPTY(stage));
-          ++ha;
-          if (issued < nh) ok = issue();
+          if (!ok) break;
+          pph ^= 1u;
+          mma_commit(EMPTY(sa));
+          mma_commit(EMPTY(sb));
+          ++gm;
+          if (j == it.n - 1) {
+            mma_commit(DONE);
+          } else {
+            if (!acquire(sa) || !acquire(sb)) { ok = false; break; }
+            BSA_BTRACE_AT(gm, 6);
+            sd(sa, sb);
+            mma_commit(SFULL);
+            if (j + 1 == it.n - 1) mma_commit(ROWEMPTY);
+          }
         }
-        if (!ok) break;
-        mma_commit(DONE);
       }
       mma_commit(FINAL);
       mbar_wait_drain(FINAL, 0, p.status, p.timeout_ns);
@@ -380,15 +353,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else {
     // ------------------------------------------------------------ compute (8 warps)
     const int q4 = warp & 3;            // TMEM lane quarter
-    const int cg = warp >> 2;           // column group: columns 32*cg .. +31 of each half-step
+    const int cg = warp >> 2;           // column group: columns 32*cg .. +31 of each half
     const int row = q4 * 32 + lane;     // 0..127 = TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
     const uint32_t tA = tmem + lane_base + 256;
-    const uint32_t tB = tmem + lane_base + 384;
+    const uint32_t tB = tmem + lane_base + 256 + D;
     const int rh = q4 >> 1;  // which 64-row half of the row tile (warp-uniform)
     const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
-    uint32_t hc = 0, dph = 0;
+    uint32_t sph = 0, dph = 0;
     bool ok = true;
+    uint32_t gc = 0;  // steps computed (trace index)
+    (void)gc;
     for (int uk = 0; ok; ++uk) {
       const int slot = uk & 3;
       if (!mbar_wait(UFULL(slot), (uk >> 2) & 1, abort_flag, p.status, p.timeout_ns)) {
@@ -441,39 +416,37 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         // keys past nk in the dQ pass (ragged last key tile) are masked per column
         const int cvalid = kDKV ? kBN : p.nk - ct * kBN;
+        if (threadIdx.x == 0) BSA_BTRACE_AT(gc, 0);
+        ok = mbar_wait(SFULL, sph, abort_flag, p.status, p.timeout_ns);
+        if (!ok) break;
+        if (threadIdx.x == 0) BSA_BTRACE_AT(gc, 1);
+        sph ^= 1u;
+        tc_fence_after();
         for (int h = 0; h < 2; ++h) {
-          if (!half_needed(bits, h)) continue;
-          const uint32_t buf = hc & 1u;
-          if (threadIdx.x == 0) BSA_BTRACE_AT(hc, 0);
-          ok = mbar_wait(SFULL(buf), (hc >> 1) & 1u, abort_flag, p.status, p.timeout_ns);
-          if (!ok) break;
-          if (threadIdx.x == 0) BSA_BTRACE_AT(hc, 1);
-          ++hc;
-          tc_fence_after();
-          // this warp's 32 columns of S and dP; P and dS are packed into the first
-          // 16 columns of the same ranges
-          const uint32_t tS = tmem + lane_base + 128u * buf + 32u * cg;
+          // this warp's 32 columns of the half; P and dS are packed into the first 16
+          // columns of the same ranges of S and dP
+          const uint32_t tS = tmem + lane_base + 64u * h + 32u * cg;
           const bool row_ok = (bits >> (rh * 2 + h)) & 1u;
           if (!row_ok) {
             uint32_t z[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) z[i] = 0u;
             tmem_st32x32b_x16(tS, z);
-            tmem_st32x32b_x16(tS + 64, z);
+            tmem_st32x32b_x16(tS + 128, z);
           } else {
             uint32_t sr[32], dr[32];
             tmem_ld32x32b_x32_nowait(tS, sr);
-            tmem_ld32x32b_x32_nowait(tS + 64, dr);
+            tmem_ld32x32b_x32_nowait(tS + 128, dr);
             tmem_wait_ld_x32(sr);
             tmem_wait_ld_x32(dr);
             const int cbase = 64 * h + 32 * cg;
+            const float vl = h ? cl[1] : cl[0], vd = h ? cd[1] : cd[0];
             uint32_t ppk[16], dpk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const int c = cbase + 2 * i;
               float2 nl = nlse, dv = dd;
               if (kDKV) {
-                const float vl = h ? cl[1] : cl[0], vd = h ? cd[1] : cd[0];
                 nl = make_float2(__shfl_sync(0xffffffffu, vl, 2 * i),
                                  __shfl_sync(0xffffffffu, vl, 2 * i + 1));
                 dv = make_float2(__shfl_sync(0xffffffffu, vd, 2 * i),
@@ -495,14 +468,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               dpk[i] = *reinterpret_cast<uint32_t*>(&hd);
             }
             if (kDKV) tmem_st32x32b_x16(tS, ppk);
-            tmem_st32x32b_x16(tS + 64, dpk);
+            tmem_st32x32b_x16(tS + 128, dpk);
           }
           asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
           tc_fence_before();
           __syncwarp();
-          if (threadIdx.x == 0) BSA_BTRACE_AT(hc - 1, 2);
-          if (lane == 0) mbar_arrive(PREADY(buf));
+          if (threadIdx.x == 0) BSA_BTRACE_AT(gc, 2 + h);
+          if (lane == 0) mbar_arrive(PREADY(h));
         }
+        ++gc;
       }
       if (!ok) break;
       // epilogue: accA * scale -> outA, accB -> outB (rows past the tensor end
@@ -625,29 +599,19 @@ __global__ void tmap_kernel(const int* __restrict__ row_ptr, const int* __restri
 
 __global__ void __launch_bounds__(256) tcompact_kernel(const uint32_t* __restrict__ map, int QT,
                                                        int KT, int* __restrict__ tcnt,
-                                                       int* __restrict__ thcnt,
                                                        uint32_t* __restrict__ tentries) {
   __shared__ int warp_sums[8];
-  __shared__ int half_total;
-  if (threadIdx.x == 0) half_total = 0;
-  __syncthreads();
   const long long g = blockIdx.x;  // mask head * KT + k-tile
   const int words = (QT + 7) / 8;
   const uint32_t* row = map + g * words;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int per = (words + 255) / 256;
   const int w0 = min(words, tid * per), w1 = min(words, w0 + per);
-  int mine = 0, halves = 0;
+  int mine = 0;
   for (int w = w0; w < w1; ++w) {
     const uint32_t q = row[w];
-    for (int j = 0; j < 8; ++j) {
-      const uint32_t b = (q >> (4 * j)) & 0xFu;
-      mine += b != 0u;
-      halves += static_cast<int>(half_needed(b, 0)) + static_cast<int>(half_needed(b, 1));
-    }
+    for (int j = 0; j < 8; ++j) mine += ((q >> (4 * j)) & 0xFu) != 0u;
   }
-  for (int o = 16; o > 0; o >>= 1) halves += __shfl_xor_sync(0xffffffffu, halves, o);
-  if (lane == 0) atomicAdd(&half_total, halves);
   int incl = mine;
   for (int o = 1; o < 32; o <<= 1) {
     const int v = __shfl_up_sync(0xffffffffu, incl, o);
@@ -667,38 +631,12 @@ __global__ void __launch_bounds__(256) tcompact_kernel(const uint32_t* __restric
     }
   }
   if (tid == 255) tcnt[g] = pos;
-  __syncthreads();
-  if (tid == 0) thcnt[g] = half_total;
-}
-
-// Half-steps of each forward list (one CTA per list row), for the dQ pass.
-__global__ void __launch_bounds__(128) qhcount_kernel(const int* __restrict__ row_ptr,
-                                                      const int* __restrict__ cnt,
-                                                      const uint32_t* __restrict__ entries, int LR,
-                                                      int QB, int block_q, int expand,
-                                                      int* __restrict__ qhcnt) {
-  __shared__ int total;
-  const int g = blockIdx.x;  // mask head * LR + list row
-  const int mh = g / LR, lr = g - mh * LR;
-  const int first_qb = block_q >= 128 ? lr : 2 * lr;
-  const uint32_t* ent = entries + static_cast<long long>(row_ptr[mh * QB + first_qb]) * expand;
-  if (threadIdx.x == 0) total = 0;
-  __syncthreads();
-  int halves = 0;
-  for (int j = threadIdx.x; j < cnt[g]; j += blockDim.x) {
-    const uint32_t b = ent[j] >> 28;
-    halves += static_cast<int>(half_needed(b, 0)) + static_cast<int>(half_needed(b, 1));
-  }
-  for (int o = 16; o > 0; o >>= 1) halves += __shfl_xor_sync(0xffffffffu, halves, o);
-  if ((threadIdx.x & 31) == 0) atomicAdd(&total, halves);
-  __syncthreads();
-  if (threadIdx.x == 0) qhcnt[g] = total;
 }
 
 struct BwdGeometry {
   Geometry fwd;
   int KT;
-  size_t tcnt_off, thcnt_off, qhcnt_off, tent_off, map_off, lse_off, dvec_off, total;
+  size_t tcnt_off, tent_off, map_off, lse_off, dvec_off, total;
 };
 
 BwdGeometry bwd_geometry(int batch, int heads, int nq, int nk, int block_q, int block_k,
@@ -709,9 +647,7 @@ BwdGeometry bwd_geometry(int batch, int heads, int nq, int nk, int block_q, int 
   auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
   const size_t mhk = static_cast<size_t>(list_heads) * g.KT;
   g.tcnt_off = up(g.fwd.total);
-  g.thcnt_off = up(g.tcnt_off + sizeof(int) * mhk);
-  g.qhcnt_off = up(g.thcnt_off + sizeof(int) * mhk);
-  g.tent_off = up(g.qhcnt_off + sizeof(int) * static_cast<size_t>(list_heads) * g.fwd.LR);
+  g.tent_off = up(g.tcnt_off + sizeof(int) * mhk);
   g.map_off = up(g.tent_off + sizeof(uint32_t) * mhk * g.fwd.QT);
   g.lse_off = up(g.map_off + sizeof(uint32_t) * mhk * ((g.fwd.QT + 7) / 8));
   const size_t vec = sizeof(float) * static_cast<size_t>(batch) * heads * g.fwd.QT * kBM;
@@ -769,16 +705,11 @@ extern "C" int bsa_attn_bwd(const void* q, const void* k, const void* v, const v
   if (scale <= 0.0f) scale = 1.0f / sqrtf(static_cast<float>(head_dim));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-  // 128-row boxes for the row operands, 64-row boxes for the column halves
-  CUtensorMap mq, mk, mv, mdo, hq, hk, hv, hdo;
+  CUtensorMap mq, mk, mv, mdo;
   if (make_map(&mq, q, batch, nq, heads, head_dim) != BSA_OK ||
       make_map(&mk, k, batch, nk, heads, head_dim) != BSA_OK ||
       make_map(&mv, v, batch, nk, heads, head_dim) != BSA_OK ||
-      make_map(&mdo, dout, batch, nq, heads, head_dim) != BSA_OK ||
-      make_map(&hq, q, batch, nq, heads, head_dim, 64) != BSA_OK ||
-      make_map(&hk, k, batch, nk, heads, head_dim, 64) != BSA_OK ||
-      make_map(&hv, v, batch, nk, heads, head_dim, 64) != BSA_OK ||
-      make_map(&hdo, dout, batch, nq, heads, head_dim, 64) != BSA_OK)
+      make_map(&mdo, dout, batch, nq, heads, head_dim) != BSA_OK)
     return BSA_ERR_CUDA;
 
   char* wsb = static_cast<char*>(ws);
@@ -786,8 +717,6 @@ extern "C" int bsa_attn_bwd(const void* q, const void* k, const void* v, const v
   int* cnt = reinterpret_cast<int*>(wsb + g.fwd.cnt_off);
   uint32_t* entries = reinterpret_cast<uint32_t*>(wsb + g.fwd.ent_off);
   int* tcnt = reinterpret_cast<int*>(wsb + g.tcnt_off);
-  int* thcnt = reinterpret_cast<int*>(wsb + g.thcnt_off);
-  int* qhcnt = reinterpret_cast<int*>(wsb + g.qhcnt_off);
   uint32_t* tentries = reinterpret_cast<uint32_t*>(wsb + g.tent_off);
   uint32_t* map = reinterpret_cast<uint32_t*>(wsb + g.map_off);
   float* lse2 = reinterpret_cast<float*>(wsb + g.lse_off);
@@ -810,10 +739,7 @@ extern "C" int bsa_attn_bwd(const void* q, const void* k, const void* v, const v
                                                      g.fwd.LR, g.fwd.QB, block_q, g.fwd.expand,
                                                      list_heads, map);
   if ((rc = check_launch()) != BSA_OK) return rc;
-  tcompact_kernel<<<list_heads * g.KT, 256, 0, st>>>(map, g.fwd.QT, g.KT, tcnt, thcnt, tentries);
-  if ((rc = check_launch()) != BSA_OK) return rc;
-  qhcount_kernel<<<list_heads * g.fwd.LR, 128, 0, st>>>(row_ptr, cnt, entries, g.fwd.LR, g.fwd.QB,
-                                                        block_q, g.fwd.expand, qhcnt);
+  tcompact_kernel<<<list_heads * g.KT, 256, 0, st>>>(map, g.fwd.QT, g.KT, tcnt, tentries);
   if ((rc = check_launch()) != BSA_OK) return rc;
 
   BwdParams p;
@@ -834,8 +760,6 @@ extern "C" int bsa_attn_bwd(const void* q, const void* k, const void* v, const v
   p.cnt = cnt;
   p.entries = entries;
   p.tcnt = tcnt;
-  p.thcnt = thcnt;
-  p.qhcnt = qhcnt;
   p.tentries = tentries;
   p.lse2 = lse2;
   p.dvec = dvec;
@@ -846,16 +770,16 @@ extern "C" int bsa_attn_bwd(const void* q, const void* k, const void* v, const v
   p.outA = static_cast<__nv_bfloat16*>(dk);
   p.outB = static_cast<__nv_bfloat16*>(dv);
   p.unit_counter = status + 1;
-  rc = head_dim == 128 ? launch_bwd<128, true>(mk, mv, hq, hdo, p, st)
-                       : launch_bwd<64, true>(mk, mv, hq, hdo, p, st);
+  rc = head_dim == 128 ? launch_bwd<128, true>(mk, mv, mq, mdo, p, st)
+                       : launch_bwd<64, true>(mk, mv, mq, mdo, p, st);
   if (rc != BSA_OK) return rc;
   // pass 2: dQ (rows = q-tiles, columns = key tiles)
   p.total_items = batch * heads * g.fwd.QT;
   p.outA = static_cast<__nv_bfloat16*>(dq);
   p.outB = nullptr;
   p.unit_counter = status + 2;
-  return head_dim == 128 ? launch_bwd<128, false>(mq, mdo, hk, hv, p, st)
-                         : launch_bwd<64, false>(mq, mdo, hk, hv, p, st);
+  return head_dim == 128 ? launch_bwd<128, false>(mq, mdo, mk, mv, p, st)
+                         : launch_bwd<64, false>(mq, mdo, mk, mv, p, st);
 }
 
 #ifdef BSA_TRACE
