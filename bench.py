@@ -60,6 +60,7 @@ def load_peaks():
 KERNEL_SOURCES = {
     "attn_fwd": ("attn_fwd.cu", "attn_common.cuh", "bsa_common.cuh", "tmem_io.cuh"),
     "attn_bwd": ("attn_bwd.cu", "attn_common.cuh", "bsa_common.cuh", "tmem_io.cuh"),
+    "sics": ("sics.cu", "bsa_common.cuh"),
 }
 
 
@@ -676,7 +677,7 @@ def run_sics(args, w):
     peaks, peak_kind = load_peaks()
     achieved = nbytes / (ms * 1e-3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                "frac": achieved / peaks["hbm_gbs"], "traffic": profiled_traffic(w.name, "sics"),
                 "kernel": "sics_kernel<128> (one launch per tensor and menu shape)",
                 "peak_note": f"{peak_kind} HBM copy bandwidth"}
     cpu = None
