@@ -134,7 +134,8 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, i
   }
 }
 
-// ---- TMA (bulk tensor copy global -> shared, completion on an mbarrier, no multicast)
+// ---- TMA (bulk tensor copy global -> shared, completion on an mbarrier; every CTA
+// loads its own tiles)
 __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
                                             int c0, int c1, int c2, int c3) {
   asm volatile(
