@@ -737,7 +737,7 @@ def run_ar_paged(args, w):
     for _ in range(max(3, args.warmup)):
         o, lse, mask = cache.attend(q_last, w.p)
     barrier()
-    if cache.status.item() != 0 or B_status(cache.attn_ws) != 0:
+    if cache.status.item() != 0 or device_status(cache.attn_ws) != 0:
         raise RuntimeError("paged cache kernels reported a device-side error")
     flops = effective_flops(mask, chunk, hi, w.block, w.head_dim, w.batch * w.heads)
     resident_before = cache.resident_bytes()
@@ -828,7 +828,8 @@ def run_ar_paged(args, w):
     return 0
 
 
-def B_status(ws):
+def device_status(ws):
+    """The device-side status word of a libbsa workspace (0 = no error)."""
     from block_sparse_attention_tokens_b200 import binding as B
     return B.bsa_read_status(ws)
 
