@@ -1,0 +1,46 @@
+"""The benchmark's JSON line contract, exercised on the CPU through the reference
+arm (the float64 oracle on a bounded sample), and the AR cache budget."""
+import json
+import math
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def run_bench(*args):
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *args],
+                         capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, out.stdout
+    return json.loads(lines[0])
+
+
+@pytest.mark.parametrize("pass_", ["fwd", "bwd"])
+def test_reference_arm_prints_one_contract_line(pass_):
+    d = run_bench("--impl", "reference", "--workload", "sta_tiny", "--steps", "1", "--warmup",
+                  "0", "--pass", pass_)
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup",
+                "higher_is_better", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == "TFLOP/s"
+    assert d["config"]["workload"] == "sta_tiny"
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_ar_budget_keeps_the_target_fraction():
+    sys.path.insert(0, ROOT)
+    import bench
+    from block_sparse_attention_tokens_b200 import configs
+    w = configs.get("ar_decode")
+    budget = bench.ar_budget(w)
+    n_pages = math.ceil(w.n_tokens / 128)
+    anchor = math.ceil(w.anchor_frames * w.tokens_per_frame / 128)
+    recent = n_pages - (w.n_tokens - w.recent_frames * w.tokens_per_frame) // 128
+    kept = (anchor + recent + budget) / n_pages
+    assert abs(kept - bench.AR_KEEP_FRACTION) < 1.0 / n_pages
