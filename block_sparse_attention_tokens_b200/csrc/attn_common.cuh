@@ -124,6 +124,116 @@ __global__ void __launch_bounds__(kListThreads) build_lists_kernel(
   if (tid == kListThreads - 1) cnt[g] = pos;
 }
 
+// Kept lists with gathered key tiles (64-token key blocks): each 128-key tile is
+// any two kept key blocks of the list row, so a tile carries an empty 64-key half
+// only when the row keeps an odd number of blocks.  Entry: bits 0-13 the first
+// block, bits 14-27 the second block + 1 (0: none), bits 28-31 the quadrant bits
+// (q_half * 2 + k_half).  Blocks both q-halves keep are paired first, ascending,
+// then the blocks one q-half keeps.  One CTA per list row; dynamic shared memory
+// 4 * ceil(KB / 16) bytes (2 bits per key block: which q-halves keep it).
+constexpr int kGatherMaxBlocks = 16382;
+
+__global__ void __launch_bounds__(kListThreads) build_gather_lists_kernel(
+    const int* __restrict__ row_ptr, const int* __restrict__ col_idx, int QB, int KB, int LR,
+    int block_q, long long nnz_cap, int* __restrict__ cnt, uint32_t* __restrict__ entries,
+    int* status, const int* __restrict__ page_table, int pages_per_batch, int heads) {
+  extern __shared__ uint32_t qm[];
+  __shared__ int sums_a[kListThreads / 32], sums_b[kListThreads / 32];
+  const int g = blockIdx.x;
+  const int mh = g / LR, lr = g - mh * LR;
+  const int nrows = block_q >= 128 ? 1 : ((2 * lr + 1 < QB) ? 2 : 1);
+  const int first_qb = block_q >= 128 ? lr : 2 * lr;
+  const int* rp = row_ptr + static_cast<long long>(mh) * QB + first_qb;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  bool bad = false;
+  for (int r = 0; r < nrows; ++r) {
+    const int b0 = rp[r], b1 = rp[r + 1];
+    if (b0 < 0 || b0 > b1 || b1 > nnz_cap) {
+      bad = true;
+      break;
+    }
+    for (int i = b0 + tid; i < b1; i += kListThreads) {
+      const int c = col_idx[i];
+      if (c < 0 || c >= KB || (i > b0 && c <= col_idx[i - 1])) bad = true;
+    }
+  }
+  if (__syncthreads_or(bad)) {
+    if (tid == 0) {
+      set_status(status, BSA_ERR_INVALID_ARG);
+      cnt[g] = 0;
+    }
+    return;
+  }
+  const int words = (KB + 15) / 16;
+  for (int w = tid; w < words; w += kListThreads) qm[w] = 0u;
+  __syncthreads();
+  // paged K/V: blocks on evicted pages (128-token pages hold two blocks) are dropped
+  const int* pt = page_table ? page_table + static_cast<long long>(mh / heads) * pages_per_batch
+                             : nullptr;
+  for (int r = 0; r < nrows; ++r) {
+    const uint32_t qbits = block_q >= 128 ? 0x3u : (r == 0 ? 0x1u : 0x2u);
+    for (int i = rp[r] + tid; i < rp[r + 1]; i += kListThreads) {
+      const int kb = col_idx[i];
+      if (pt && ((kb >> 1) >= pages_per_batch || pt[kb >> 1] < 0)) continue;
+      atomicOr(&qm[kb >> 4], qbits << (2 * (kb & 15)));
+    }
+  }
+  __syncthreads();
+  // thread t owns words [t*per, (t+1)*per); class A = kept by both q-halves
+  const int per = (words + kListThreads - 1) / kListThreads;
+  const int w0 = min(words, tid * per), w1 = min(words, w0 + per);
+  int na = 0, nb = 0;
+  for (int w = w0; w < w1; ++w) {
+    const uint32_t q = qm[w];
+    for (int j = 0; j < 16; ++j) {
+      const uint32_t m = (q >> (2 * j)) & 3u;
+      na += m == 3u;
+      nb += m == 1u || m == 2u;
+    }
+  }
+  int ia = na, ib = nb;
+  for (int o = 1; o < 32; o <<= 1) {
+    const int va = __shfl_up_sync(0xffffffffu, ia, o);
+    const int vb = __shfl_up_sync(0xffffffffu, ib, o);
+    if (lane >= o) {
+      ia += va;
+      ib += vb;
+    }
+  }
+  if (lane == 31) {
+    sums_a[warp] = ia;
+    sums_b[warp] = ib;
+  }
+  __syncthreads();
+  int base_a = 0, base_b = 0, tot_a = 0, tot_b = 0;
+  for (int w = 0; w < kListThreads / 32; ++w) {
+    if (w < warp) {
+      base_a += sums_a[w];
+      base_b += sums_b[w];
+    }
+    tot_a += sums_a[w];
+    tot_b += sums_b[w];
+  }
+  const int n_entries = (tot_a + tot_b + 1) / 2;
+  uint32_t* out = entries + rp[0];
+  for (int e = tid; e < n_entries; e += kListThreads) out[e] = 0u;
+  __syncthreads();
+  int pa = base_a + ia - na, pb = tot_a + base_b + ib - nb;
+  for (int w = w0; w < w1; ++w) {
+    const uint32_t q = qm[w];
+    for (int j = 0; j < 16; ++j) {
+      const uint32_t m = (q >> (2 * j)) & 3u;
+      if (m == 0u) continue;
+      const int pos = m == 3u ? pa++ : pb++;
+      const int kb = w * 16 + j, h = pos & 1;
+      const uint32_t field = h == 0 ? static_cast<uint32_t>(kb) : static_cast<uint32_t>(kb + 1) << 14;
+      const uint32_t bits = ((m & 1u) << h) | (((m >> 1) & 1u) << (2 + h));
+      atomicOr(&out[pos >> 1], field | (bits << 28));
+    }
+  }
+  if (tid == 0) cnt[g] = n_entries;
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -185,8 +295,16 @@ Geometry geometry(int batch, int heads, int nq, int nk, int block_q, int block_k
 int launch_build_lists(const int* row_ptr, const int* col_idx, int list_heads, const Geometry& g,
                        int nk, int block_q, int block_k, int* cnt, uint32_t* entries, int* status,
                        cudaStream_t st, const int* page_table = nullptr, int pages_per_batch = 0,
-                       int heads = 1) {
+                       int heads = 1, bool gather_k = false) {
   const long long lists = static_cast<long long>(list_heads) * g.LR;
+  if (gather_k) {
+    const size_t gsmem = sizeof(uint32_t) * static_cast<size_t>((g.KB + 15) / 16);
+    if (block_k != 64 || g.KB > kGatherMaxBlocks || lists > 0x7fffffffLL) return BSA_ERR_UNSUPPORTED;
+    build_gather_lists_kernel<<<static_cast<int>(lists), kListThreads, gsmem, st>>>(
+        row_ptr, col_idx, g.QB, g.KB, g.LR, block_q, g.nnz_cap, cnt, entries, status, page_table,
+        pages_per_batch, heads);
+    return check_launch();
+  }
   const int KT = ceil_div(nk, kBN);
   const size_t list_smem = sizeof(uint32_t) * static_cast<size_t>((KT + 7) / 8);
   if (list_smem > 200 * 1024 || lists > 0x7fffffffLL) return BSA_ERR_UNSUPPORTED;

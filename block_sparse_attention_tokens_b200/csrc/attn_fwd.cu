@@ -98,7 +98,18 @@ struct AttnParams {
   // page_table[b * pages_per_batch + kt] of a one-batch pool (nullptr: contiguous)
   const int* page_table;
   int pages_per_batch;
+  // 64-token key blocks: list entries name two arbitrary key blocks per tile
+  // (block, block + 1 or 0, quadrant bits) instead of one 128-key tile
+  int gather_k;
 };
+
+// Key row (in the K/V tensor or pool) of 64-token key block kb of batch b.
+__device__ __forceinline__ int key_block_row(const AttnParams& p, int b, int kb) {
+  if (p.page_table)
+    return __ldg(p.page_table + static_cast<long long>(b) * p.pages_per_batch + (kb >> 1)) * kBN +
+           (kb & 1) * 64;
+  return kb * 64;
+}
 
 struct Item {
   int b, h, qt, n;  // n < 0: no item; n == 0: empty kept list
@@ -134,7 +145,9 @@ __device__ __forceinline__ bool shares_kv(const Item& a, const Item& b) {
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+                    const __grid_constant__ CUtensorMap tmV,
+                    const __grid_constant__ CUtensorMap tmK64,
+                    const __grid_constant__ CUtensorMap tmV64, const AttnParams p) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -215,21 +228,38 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       int gld = 0;
       (void)gld;
-      auto load_tile = [&](const CUtensorMap* map, const Item& itm, int step) -> bool {
+      auto load_tile = [&](const CUtensorMap* map, const CUtensorMap* map64, const Item& itm,
+                           int step) -> bool {
         const int tix = 32768 + min(gld++, 8191) * 2;
         BSA_TRACE_AT(tix + 0);
         if (!mbar_wait(EMPTY(st), ph ^ 1u, abort_flag, p.status, p.timeout_ns)) return false;
         BSA_TRACE_AT(tix + 1);
-        const int kt = static_cast<int>(__ldg(itm.ent + step) & 0x0FFFFFFFu);
-        const int row = p.page_table
-                            ? __ldg(p.page_table + static_cast<long long>(itm.b) * p.pages_per_batch + kt) * kBN
-                            : kt * kBN;
+        const uint32_t ent = __ldg(itm.ent + step);
         const int bco = p.page_table ? 0 : itm.b;
         mbar_expect_tx(FULL(st), C::TILE_BYTES);
+        if (p.gather_k) {
+          // two 64-row boxes; a missing second block repeats the first (its columns
+          // are masked, the rows only need to be finite)
+          const int kb0 = static_cast<int>(ent & 0x3FFFu);
+          const int kb1p = static_cast<int>((ent >> 14) & 0x3FFFu);
+          const int r0 = key_block_row(p, itm.b, kb0);
+          const int r1 = key_block_row(p, itm.b, kb1p ? kb1p - 1 : kb0);
 #pragma unroll
-        for (int c = 0; c < C::KCH; ++c)
-          tma_load_4d(sRing + st * C::TILE_BYTES + c * C::CHUNK_BYTES, map, FULL(st), 64 * c,
-                      itm.h, row, bco);
+          for (int c = 0; c < C::KCH; ++c) {
+            const uint32_t dst = sRing + st * C::TILE_BYTES + c * C::CHUNK_BYTES;
+            tma_load_4d(dst, map64, FULL(st), 64 * c, itm.h, r0, bco);
+            tma_load_4d(dst + C::CHUNK_BYTES / 2, map64, FULL(st), 64 * c, itm.h, r1, bco);
+          }
+        } else {
+          const int kt = static_cast<int>(ent & 0x0FFFFFFFu);
+          const int row = p.page_table
+                              ? __ldg(p.page_table + static_cast<long long>(itm.b) * p.pages_per_batch + kt) * kBN
+                              : kt * kBN;
+#pragma unroll
+          for (int c = 0; c < C::KCH; ++c)
+            tma_load_4d(sRing + st * C::TILE_BYTES + c * C::CHUNK_BYTES, map, FULL(st), 64 * c,
+                        itm.h, row, bco);
+        }
         filled |= 1u << st;
         fill_phase = (fill_phase & ~(1u << st)) | (ph << st);
         if (++st == C::NSTAGE) { st = 0; ph ^= 1u; }
@@ -260,21 +290,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (shares_kv(it[0], it[1])) {  // one K/V stream read by both slots
           const int n = it[0].n;
-          ok = ok && load_tile(&tmK, it[0], 0);
+          ok = ok && load_tile(&tmK, &tmK64, it[0], 0);
           for (int r = 0; r < n && ok; ++r) {
-            ok = load_tile(&tmV, it[0], r);
-            if (ok && r + 1 < n) ok = load_tile(&tmK, it[0], r + 1);
+            ok = load_tile(&tmV, &tmV64, it[0], r);
+            if (ok && r + 1 < n) ok = load_tile(&tmK, &tmK64, it[0], r + 1);
           }
           continue;
         }
         for (int s = 0; s < 2 && ok; ++s)
-          if (it[s].n > 0) ok = load_tile(&tmK, it[s], 0);
+          if (it[s].n > 0) ok = load_tile(&tmK, &tmK64, it[s], 0);
         const int R = max(it[0].n, it[1].n);
         for (int r = 0; r < R && ok; ++r) {
           for (int s = 0; s < 2 && ok; ++s) {
             if (r >= it[s].n) continue;
-            ok = load_tile(&tmV, it[s], r);
-            if (ok && r + 1 < it[s].n) ok = load_tile(&tmK, it[s], r + 1);
+            ok = load_tile(&tmV, &tmV64, it[s], r);
+            if (ok && r + 1 < it[s].n) ok = load_tile(&tmK, &tmK64, it[s], r + 1);
           }
         }
       }
@@ -463,10 +493,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         sph ^= 1u;
         tc_fence_after();
-        const int kt = static_cast<int>(ent & 0x0FFFFFFFu);
         const uint32_t bits = ent >> 28;
-        const int kvalid = p.nk - kt * kBN;  // keys of this tile that exist
-        const bool ragged = kvalid < kBN;
+        // keys that exist in each 64-column half of the tile
+        int v0, v1;
+        if (p.gather_k) {
+          const int kb0 = static_cast<int>(ent & 0x3FFFu);
+          const int kb1p = static_cast<int>((ent >> 14) & 0x3FFFu);
+          v0 = min(64, p.nk - kb0 * 64);
+          v1 = kb1p ? min(64, p.nk - (kb1p - 1) * 64) : 64;  // an empty half is masked by bits
+        } else {
+          const int kvalid = p.nk - static_cast<int>(ent & 0x0FFFFFFFu) * kBN;
+          v0 = max(0, min(64, kvalid));
+          v1 = max(0, min(64, kvalid - 64));
+        }
+        const bool ragged = v0 < 64 || v1 < 64;
         // Quadrant mask of 64-token blocks: each warp's 32 rows lie in one q-half, so
         // whether a 64-column half is kept is uniform across the warp.
         const bool lo_ok = (bits >> (qh * 2)) & 1u, hi_ok = (bits >> (qh * 2 + 1)) & 1u;
@@ -568,7 +608,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else {
 #pragma unroll
               for (int i = 0; i < 64; ++i)
-                if (c0 + i < kvalid) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(sr[i]));
+                if (i < (c0 < 64 ? v0 : v1)) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(sr[i]));
             }
           }
           const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
@@ -607,10 +647,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               } else {
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                  const int c = c0 + 2 * i;
+                  const int c = (c0 & 63) + 2 * i;       // column within its half
+                  const int hv = c0 < 64 ? v0 : v1;
                   const float p0 =
-                      c < kvalid ? fast_exp2(fmaf(__uint_as_float(sr[2 * i]), sl2, -msub)) : 0.f;
-                  const float p1 = c + 1 < kvalid
+                      c < hv ? fast_exp2(fmaf(__uint_as_float(sr[2 * i]), sl2, -msub)) : 0.f;
+                  const float p1 = c + 1 < hv
                                        ? fast_exp2(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -msub))
                                        : 0.f;
                   lp[(2 * i) & 3] += p0;
@@ -699,6 +740,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------------------
 template <int D>
 int launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                const CUtensorMap& mk64, const CUtensorMap& mv64,
                 const AttnParams& p, cudaStream_t st) {
   using C = Cfg<D>;
   static bool attr_done[64] = {false};
@@ -712,7 +754,7 @@ int launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap&
   }
   int grid = device_sm_count();
   if (grid > p.total_units) grid = p.total_units;
-  attn_fwd_kernel<D><<<grid, kThreads, C::SMEM, st>>>(mq, mk, mv, p);
+  attn_fwd_kernel<D><<<grid, kThreads, C::SMEM, st>>>(mq, mk, mv, mk64, mv64, p);
   return check_launch();
 }
 
@@ -767,12 +809,16 @@ int attn_fwd_impl(const void* q, const void* k, const void* v, int batch, int he
     return BSA_ERR_UNSUPPORTED;
   if (scale <= 0.0f) scale = 1.0f / sqrtf(static_cast<float>(head_dim));
 
-  CUtensorMap mq, mk, mv;
+  // 64-token key blocks: tiles are gathered from two arbitrary blocks (64-row boxes)
+  const bool gather_k = block_k == 64 && g.KB <= kGatherMaxBlocks;
+  CUtensorMap mq, mk, mv, mk64, mv64;
   const int kv_batch = page_table ? 1 : batch;
   const int kv_rows = page_table ? n_pool_pages * kBN : nk;
   if (make_map(&mq, q, batch, nq, heads, head_dim) != BSA_OK ||
       make_map(&mk, k, kv_batch, kv_rows, heads, head_dim) != BSA_OK ||
-      make_map(&mv, v, kv_batch, kv_rows, heads, head_dim) != BSA_OK)
+      make_map(&mv, v, kv_batch, kv_rows, heads, head_dim) != BSA_OK ||
+      make_map(&mk64, k, kv_batch, kv_rows, heads, head_dim, 64) != BSA_OK ||
+      make_map(&mv64, v, kv_batch, kv_rows, heads, head_dim, 64) != BSA_OK)
     return BSA_ERR_CUDA;
 
   char* wsb = static_cast<char*>(ws);
@@ -783,7 +829,7 @@ int attn_fwd_impl(const void* q, const void* k, const void* v, int batch, int he
   if (e != cudaSuccess) return record_cuda_error(e);
 
   int rc = launch_build_lists(row_ptr, col_idx, list_heads, g, nk, block_q, block_k, cnt, entries,
-                              status, st, page_table, pages_per_batch, heads);
+                              status, st, page_table, pages_per_batch, heads, gather_k);
   if (rc != BSA_OK) return rc;
 
   AttnParams p;
@@ -811,7 +857,9 @@ int attn_fwd_impl(const void* q, const void* k, const void* v, int batch, int he
   p.timeout_ns = 2000000000ULL;
   p.page_table = page_table;
   p.pages_per_batch = pages_per_batch;
-  return head_dim == 128 ? launch_attn<128>(mq, mk, mv, p, st) : launch_attn<64>(mq, mk, mv, p, st);
+  p.gather_k = gather_k ? 1 : 0;
+  return head_dim == 128 ? launch_attn<128>(mq, mk, mv, mk64, mv64, p, st)
+                         : launch_attn<64>(mq, mk, mv, mk64, mv64, p, st);
 }
 
 }  // namespace
