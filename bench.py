@@ -997,7 +997,7 @@ def main():
     traffic = profiled_traffic(w.name)
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": traffic,
-                "kernel": "attn_fwd_kernel<128>", "attn_ms": attn_ms,
+                "kernel": "attn_fwd_kernel<128, adjacent key tiles>", "attn_ms": attn_ms,
                 "peak_note": f"{peak_kind} sustained bf16 (kernel timed inside back-to-back steps)",
                 "frac_of_burst": achieved / peaks["bf16_tflops"]}
 

@@ -142,7 +142,7 @@ __device__ __forceinline__ bool shares_kv(const Item& a, const Item& b) {
 // ---------------------------------------------------------------------------
 // The attention kernel.
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, bool kGather>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV,
@@ -237,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ent = __ldg(itm.ent + step);
         const int bco = p.page_table ? 0 : itm.b;
         mbar_expect_tx(FULL(st), C::TILE_BYTES);
-        if (p.gather_k) {
+        if constexpr (kGather) {
           // two 64-row boxes; a missing second block repeats the first (its columns
           // are masked, the rows only need to be finite)
           const int kb0 = static_cast<int>(ent & 0x3FFFu);
@@ -494,19 +494,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         sph ^= 1u;
         tc_fence_after();
         const uint32_t bits = ent >> 28;
-        // keys that exist in each 64-column half of the tile
-        int v0, v1;
-        if (p.gather_k) {
+        // keys that exist: in the tile (adjacent blocks) or in each 64-column half
+        // (gathered blocks)
+        int kvalid = 0, v0 = 64, v1 = 64;
+        if constexpr (kGather) {
           const int kb0 = static_cast<int>(ent & 0x3FFFu);
           const int kb1p = static_cast<int>((ent >> 14) & 0x3FFFu);
           v0 = min(64, p.nk - kb0 * 64);
           v1 = kb1p ? min(64, p.nk - (kb1p - 1) * 64) : 64;  // an empty half is masked by bits
         } else {
-          const int kvalid = p.nk - static_cast<int>(ent & 0x0FFFFFFFu) * kBN;
-          v0 = max(0, min(64, kvalid));
-          v1 = max(0, min(64, kvalid - 64));
+          kvalid = p.nk - static_cast<int>(ent & 0x0FFFFFFFu) * kBN;
         }
-        const bool ragged = v0 < 64 || v1 < 64;
+        const bool ragged = kGather ? (v0 < 64 || v1 < 64) : kvalid < kBN;
         // Quadrant mask of 64-token blocks: each warp's 32 rows lie in one q-half, so
         // whether a 64-column half is kept is uniform across the warp.
         const bool lo_ok = (bits >> (qh * 2)) & 1u, hi_ok = (bits >> (qh * 2 + 1)) & 1u;
@@ -608,7 +607,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else {
 #pragma unroll
               for (int i = 0; i < 64; ++i)
-                if (i < (c0 < 64 ? v0 : v1)) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(sr[i]));
+                if (kGather ? i < (c0 < 64 ? v0 : v1) : c0 + i < kvalid)
+                  mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(sr[i]));
             }
           }
           const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
@@ -647,8 +647,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               } else {
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                  const int c = (c0 & 63) + 2 * i;       // column within its half
-                  const int hv = c0 < 64 ? v0 : v1;
+                  // gathered: column within its half against that half's keys
+                  const int c = kGather ? (c0 & 63) + 2 * i : c0 + 2 * i;
+                  const int hv = kGather ? (c0 < 64 ? v0 : v1) : kvalid;
                   const float p0 =
                       c < hv ? fast_exp2(fmaf(__uint_as_float(sr[2 * i]), sl2, -msub)) : 0.f;
                   const float p1 = c + 1 < hv
@@ -747,14 +748,20 @@ int launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap&
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64 || !attr_done[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D>,
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(attn_fwd_kernel<D, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return record_cuda_error(e);
     if (dev >= 0 && dev < 64) attr_done[dev] = true;
   }
   int grid = device_sm_count();
   if (grid > p.total_units) grid = p.total_units;
-  attn_fwd_kernel<D><<<grid, kThreads, C::SMEM, st>>>(mq, mk, mv, mk64, mv64, p);
+  if (p.gather_k)
+    attn_fwd_kernel<D, true><<<grid, kThreads, C::SMEM, st>>>(mq, mk, mv, mk64, mv64, p);
+  else
+    attn_fwd_kernel<D, false><<<grid, kThreads, C::SMEM, st>>>(mq, mk, mv, mk64, mv64, p);
   return check_launch();
 }
 
