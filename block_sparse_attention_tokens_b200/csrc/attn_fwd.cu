@@ -28,6 +28,10 @@
 // Lazy rescaling: the running max used for the exponentials only moves when a
 // row's new max exceeds it by more than 8 (log2 units), so O in TMEM is rarely
 // touched by the softmax warps.
+// Key tiles: with 128-token (or larger) key blocks a tile is 128 consecutive
+// keys; with 64-token key blocks (template parameter kGather) a tile is any two
+// kept key blocks of the list row, loaded as two 64-row TMA boxes into one tile.
+// Paged K/V: the key rows of a tile come through a page table into a pool.
 // All mbarrier waits are bounded; on expiry BSA_ERR_TIMEOUT is recorded in the
 // workspace status word and every role leaves its loop.
 #include <cudaTypedefs.h>
@@ -47,8 +51,9 @@ constexpr int kMmaWarp = 9;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // The fast path keeps the running max while a tile's P sum stays <= 2^12.
 constexpr float kFastSumLimit = 4096.0f;
-// Software 2^x (FMA pipe) for a quarter of the fast-path exponentials, relieving
-// the MUFU, which carries one exponential per 512 tensor FLOPs at head_dim 128.
+// Optional software 2^x (FMA pipe) for a quarter of the fast-path exponentials, to
+// relieve the MUFU (one exponential per 512 tensor FLOPs at head_dim 128); off by
+// default: it measured slower on the attention workloads.
 #ifndef BSA_POLY_EXP2
 #define BSA_POLY_EXP2 0
 #endif
