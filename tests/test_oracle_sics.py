@@ -91,3 +91,12 @@ def test_scheme_ties_take_the_first_menu_entry():
     x = np.ones((1, 256, 1, 8))
     scores, choice = O.sics_scheme(x, x, grid, MENU[:3])
     assert np.allclose(scores, 1.0) and choice[0, 0] == 0
+
+
+def test_every_menu_shape_holds_its_block_size():
+    from block_sparse_attention_tokens_b200 import configs
+    for block, menu in configs.SICS_MENUS.items():
+        assert len(menu) >= 3
+        for shape in menu:
+            assert shape[0] * shape[1] * shape[2] == block, (block, shape)
+        assert len(set(menu)) == len(menu)
