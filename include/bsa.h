@@ -184,6 +184,10 @@ int bsa_nabla_select(const float* qbar, const float* kbar, int batch, int heads,
 
 /* ---------------------------------------------------------------------------
  * (c) Mask compaction into per-row kept-block lists (CSR).
+ * Source: the NABLA explainer (aibr.jp/archives/124678), section 3, and the STA
+ * explainer, section 3: the binary block mask decides which block pairs are
+ * computed; listing the kept blocks per row is this library's step (no
+ * counterpart in the pages).
  *   mask    : [rows][KB] uint8
  *   row_ptr : [rows + 1] int32, written; row_ptr[rows] = number of kept blocks
  *   col_idx : int32 with room for rows*KB entries (worst case), written with the
@@ -391,7 +395,8 @@ int bsa_attn_fwd_paged(const void* q, const void* k_pool, const void* v_pool, in
 int bsa_wait_selftest(int* device_status, unsigned long long timeout_ns, void* stream);
 
 /* ---------------------------------------------------------------------------
- * Device status word of a workspace (attention or NABLA): synchronises `stream`,
+ * Device status word of a workspace (attention or NABLA; no counterpart in the
+ * pages): synchronises `stream`,
  * copies the word to *status (a bsa_status value) and clears it.
  * ------------------------------------------------------------------------- */
 int bsa_read_status(void* ws, int* status, void* stream);
