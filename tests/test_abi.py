@@ -93,3 +93,34 @@ def test_binding_argument_counts_match_the_header(lib):
         f = getattr(lib, name)
         assert f.argtypes is not None, name
         assert len(f.argtypes) == len(params), (name, len(f.argtypes), len(params))
+
+
+def test_header_compiles_as_c_and_links(tmp_path, lib):
+    """A plain C program includes bsa.h, links libbsa.so and calls entry points whose
+    argument checks run before any CUDA call (no GPU needed)."""
+    import shutil
+    import subprocess
+    from block_sparse_attention_tokens_b200 import binding
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_bsa.c"
+    src.write_text(r"""
+#include <stdio.h>
+#include "bsa.h"
+int main(void) {
+  if (bsa_version() < 100) return 1;
+  if (bsa_sta_mask(1, 1, 1, 1, 1, 1, 0, NULL, NULL) != BSA_ERR_INVALID_ARG) return 2;
+  if (bsa_attn_workspace_size(1, 1, 1, 1, 96, 128, 1) != 0) return 3;
+  printf("%s\n", bsa_status_string(BSA_ERR_TIMEOUT));
+  return 0;
+}
+""")
+    exe = tmp_path / "use_bsa"
+    lib_dir = os.path.dirname(binding._LIB_PATH)
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-L", lib_dir, "-lbsa", f"-Wl,-rpath,{lib_dir}", "-o", str(exe)],
+                   check=True, capture_output=True, text=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0, (out.returncode, out.stderr)
+    assert out.stdout.strip() == "BSA_ERR_TIMEOUT"
