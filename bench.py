@@ -692,7 +692,7 @@ def run_sics(args, w):
                 "dtype": "f32", "data": "synthetic", "config": workload_config(w, "sics"),
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "clocks": sampler.summary(),
-                "gpu_launches": (2 * len(menu) + 1) * args.steps,
+                "gpu_launches": 2 * args.steps,   # one SICS launch for every shape + the choice
                 "attention_ms": attn_ms, "fraction_of_attention_time": ms / attn_ms,
                 "choice_histogram": torch.bincount(choice.flatten().long(),
                                                    minlength=len(menu)).tolist()}
@@ -819,7 +819,9 @@ def run_ar_paged(args, w):
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16", "data": "synthetic", "config": workload_config(w, "ar_paged"),
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-                "clocks": sampler.summary(), "gpu_launches": 6 * args.steps,
+                # per attend step: 2 block means, residency, selection, 3 compaction,
+                # kept-list build, attention
+                "clocks": sampler.summary(), "gpu_launches": 9 * args.steps,
                 "kv_cache": kv, "plain_path_attend_ms": plain_ms,
                 "effective_tflop_per_step": flops / 1e12}
         print(json.dumps(line))
