@@ -138,8 +138,10 @@ def test_radial_token_rule_golden():
 
 
 @pytest.mark.parametrize("frames,S,B,n", [(12, 16, 4, None), (20, 8, 8, None), (9, 6, 8, 50),
-                                          (17, 16, 8, 16 * 17 - 5), (33, 4, 8, None)])
+                                          (17, 16, 8, 16 * 17 - 5), (33, 4, 8, None),
+                                          (11, 5, 8, None)])
 def test_radial_block_mask_equals_token_enumeration(frames, S, B, n):
+    # (11, 5, 8): block 3 = tokens 24..31 touches frames 4, 5 and 6
     n = frames * S if n is None else n
     nb = math.ceil(n / B)
     brute = np.zeros((nb, nb), dtype=np.uint8)

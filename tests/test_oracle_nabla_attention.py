@@ -71,6 +71,17 @@ def test_select_small_p_is_argmax_and_p_one_keeps_all():
     assert k_star == 4
 
 
+def test_select_reaching_p_exactly_covers_it():
+    # dyadic probabilities are exact in binary floating point: a prefix whose mass
+    # equals p reaches it (READING: the kept set is the smallest one whose mass is
+    # at least p), and of two equal entries the lower index comes first
+    probs = np.array([0.25, 0.5, 0.125, 0.125])
+    kept, cum, k_star, _ = O.nabla_select_row(probs, 0.75)
+    assert cum[1] == 0.75 and k_star == 2 and sorted(kept.tolist()) == [0, 1]
+    kept, _, k_star, _ = O.nabla_select_row(probs, 0.875)
+    assert k_star == 3 and sorted(kept.tolist()) == [0, 1, 2]
+
+
 def test_nabla_mask_dominant_block_and_constant_queries():
     rng = np.random.default_rng(7)
     Bn, H, QB, KB, D = 1, 2, 3, 16, 8
@@ -103,6 +114,23 @@ def test_nabla_mask_range_and_forced_outside():
         kept = np.nonzero(mask[0, 0, qb, 3:15])[0]
         assert probs[qb, kept].sum() >= 0.8
         assert np.sort(probs[qb])[::-1][:len(kept) - 1].sum() < 0.8
+
+
+def test_ar_mask_forces_anchors_and_recent_and_selects_the_middle():
+    # 10 frames of 8 tokens, 4-token blocks: 2 anchor frames are blocks 0..3, the
+    # last 3 frames touch blocks 14..19; NABLA picks among blocks 4..13 with the
+    # softmax renormalised over them
+    rng = np.random.default_rng(13)
+    qbar = rng.normal(size=(1, 2, 5, 8))
+    kbar = rng.normal(size=(1, 2, 20, 8))
+    mask, _ = O.ar_mask(qbar, kbar, 0.7, 0.5, 80, 8, 4, 2, 3)
+    assert np.all(mask[..., :4] == 1) and np.all(mask[..., 14:] == 1)
+    for h in range(2):
+        probs = scipy.special.softmax((qbar[0, h] @ kbar[0, h, 4:14].T) * 0.5, axis=1)
+        for qb in range(5):
+            kept = np.nonzero(mask[0, h, qb, 4:14])[0]
+            assert probs[qb, kept].sum() >= 0.7
+            assert np.sort(probs[qb])[::-1][:len(kept) - 1].sum() < 0.7
 
 
 def test_nabla_sta_union_contains_both_masks():
@@ -184,6 +212,24 @@ def test_block_mask_equals_token_level_definition(bq, bk):
         assert np.allclose(lse[0, h][fin], rl[fin], atol=1e-12)
     rows = np.arange(bq, 2 * bq)
     assert np.all(o[0, rows, 1] == 0) and np.all(np.isneginf(lse[0, 1, rows]))
+
+
+def test_per_batch_head_masks_index_b_times_h_plus_h():
+    # a mask per (batch, head) is row b * H + h of the mask stack
+    Bn, H, D, blk = 2, 3, 8, 64
+    nq, nk = 150, 190
+    q, k, v = _rand_qkv(Bn, nq, nk, H, D, 8)
+    QB, KB = math.ceil(nq / blk), math.ceil(nk / blk)
+    mask = (np.random.default_rng(9).random((Bn * H, QB, KB)) < 0.5).astype(np.uint8)
+    mask[:, :, 0] = 1
+    o, lse = O.block_sparse_attention(q, k, v, mask, blk, blk)
+    for b in range(Bn):
+        for h in range(H):
+            allowed = O.token_mask_from_blocks(mask[b * H + h], nq, nk, blk, blk)
+            ro, rl = O.dense_masked_attention(q[b, :, h], k[b, :, h], v[b, :, h], allowed,
+                                              1 / math.sqrt(D))
+            assert np.allclose(o[b, :, h], ro, atol=1e-12, rtol=0)
+            assert np.allclose(lse[b, h], rl, atol=1e-12, rtol=0)
 
 
 def test_single_kept_block_is_softmax_over_that_block_and_lse_normalises():

@@ -86,6 +86,22 @@ def test_scheme_picks_the_slicing_the_field_is_constant_along():
     assert 0.2 < scores[0, 0, 3] < 0.35
 
 
+def test_scheme_scores_queries_and_keys_alike():
+    # one 8x8 frame, D = 64: Q = 64 orthonormal vectors (SICS = n, the diagonal
+    # alone), K = one vector repeated (SICS = n^2).  Shape 1x8x8 is one block of 64
+    # tokens, shape 1x4x16 two ragged 4x8 blocks of 32, so the score
+    # (SICS_Q + SICS_K) / (2 sum n_b^2) is (64 + 4096) / 8192 and (64 + 2048) / 4096
+    grid = (1, 8, 8)
+    q = np.eye(64)[None, :, None, :]
+    k = np.ones((1, 64, 1, 64))
+    scores, choice = O.sics_scheme(q, k, grid, [(1, 8, 8), (1, 4, 16)])
+    assert abs(scores[0, 0, 0] - 4160 / 8192) < 1e-12
+    assert abs(scores[0, 0, 1] - 2112 / 4096) < 1e-12
+    assert choice[0, 0] == 1
+    swapped, _ = O.sics_scheme(k, q, grid, [(1, 8, 8), (1, 4, 16)])
+    assert np.allclose(swapped, scores, atol=1e-12, rtol=0)
+
+
 def test_scheme_ties_take_the_first_menu_entry():
     grid = (4, 8, 8)
     x = np.ones((1, 256, 1, 8))
