@@ -46,6 +46,14 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# B200 datasheet figures (dense bf16 tensor, HBM3e on HGX boards), for the
+# fraction of nominal reported beside the fraction of the measured peak.
+NOMINAL_PEAKS = {"TFLOP/s": 2250.0, "GB/s": 7700.0}
+
+
+def with_nominal(roofline: dict) -> dict:
+    roofline["frac_of_nominal"] = roofline["achieved"] / NOMINAL_PEAKS[roofline["unit"]]
+    return roofline
 
 
 def load_peaks():
@@ -582,7 +590,7 @@ def run_backward(args, w):
                 "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16", "data": "synthetic", "config": workload_config(w, "bwd"),
-                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "roofline": with_nominal(roofline), "cpu_baseline": cpu, "e2e": e2e,
                 "clocks": sampler.summary(), "gpu_launches": 6 * args.steps,
                 "effective_tflop_per_step": flops / 1e12}
         print(json.dumps(line))
@@ -690,7 +698,7 @@ def run_sics(args, w):
                 "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "f32", "data": "synthetic", "config": workload_config(w, "sics"),
-                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "roofline": with_nominal(roofline), "cpu_baseline": cpu, "e2e": e2e,
                 "clocks": sampler.summary(),
                 "gpu_launches": 2 * args.steps,   # one SICS launch for every shape + the choice
                 "attention_ms": attn_ms, "fraction_of_attention_time": ms / attn_ms,
@@ -818,7 +826,7 @@ def run_ar_paged(args, w):
                 "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16", "data": "synthetic", "config": workload_config(w, "ar_paged"),
-                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "roofline": with_nominal(roofline), "cpu_baseline": cpu, "e2e": e2e,
                 # per attend step: 2 block means, residency, selection, 3 compaction,
                 # kept-list build, attention
                 "clocks": sampler.summary(), "gpu_launches": 9 * args.steps,
@@ -1015,7 +1023,7 @@ def main():
                 "warmup": max(3, args.warmup), "ms_per_step": ms_per_step,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16", "data": "synthetic", "config": workload_config(w),
-                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "roofline": with_nominal(roofline), "cpu_baseline": cpu, "e2e": e2e,
                 "clocks": sampler.summary(),
                 "gpu_launches": plan.kernel_launches_per_step() * args.steps,
                 "effective_tflop_per_step": flops / 1e12}

@@ -44,3 +44,11 @@ def test_ar_budget_keeps_the_target_fraction():
     recent = n_pages - (w.n_tokens - w.recent_frames * w.tokens_per_frame) // 128
     kept = (anchor + recent + budget) / n_pages
     assert abs(kept - bench.AR_KEEP_FRACTION) < 1.0 / n_pages
+
+
+def test_roofline_reports_the_fraction_of_nominal_for_both_bounds():
+    sys.path.insert(0, ROOT)
+    import bench
+    t = bench.with_nominal({"bound": "tensor", "achieved": 1125.0, "unit": "TFLOP/s"})
+    h = bench.with_nominal({"bound": "hbm", "achieved": 3850.0, "unit": "GB/s"})
+    assert t["frac_of_nominal"] == 0.5 and h["frac_of_nominal"] == 0.5
