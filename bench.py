@@ -449,6 +449,19 @@ def path_order_grad(w):
     return synth.grad_output(w)
 
 
+def mask_stats(flops: float, w, nq: int, nk: int, attn_times_ms, near=None) -> dict:
+    """Kept share of the (query, key) token pairs, spread of the attention call times
+    over the timed steps, and the NABLA rows whose cut lies within 1e-5 of p (or on
+    a tie), counted by the selection kernel of the last step."""
+    t = sorted(attn_times_ms)
+    pct = lambda f: t[min(len(t) - 1, int(round(f * (len(t) - 1))))]
+    out = {"kept_pair_fraction": flops / (4.0 * w.head_dim * nq * nk * w.batch * w.heads),
+           "attn_ms_p10": pct(0.1), "attn_ms_median": pct(0.5), "attn_ms_p90": pct(0.9)}
+    if near is not None:
+        out["near_threshold_rows"] = int(near)
+    return out
+
+
 def workload_config(w, pass_: str = "fwd"):
     cfg = {"workload": w.name, "batch": w.batch, "heads": w.heads, "head_dim": w.head_dim,
            "grid_thw": list(w.grid), "block": w.block, "mask": w.mask}
@@ -930,7 +943,8 @@ def main():
         end.record(stream)
         barrier()
     ms_total = start.elapsed_time(end)
-    attn_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_a)
+    attn_times = [a.elapsed_time(b) for a, b in ev_a]
+    attn_ms = statistics.mean(attn_times)
     ms_total, attn_ms = max_over_ranks([ms_total, attn_ms], dev)
     ms_per_step = ms_total / args.steps
     value = weak_scaling_value(flops, world, ms_per_step)
@@ -1026,7 +1040,9 @@ def main():
                 "roofline": with_nominal(roofline), "cpu_baseline": cpu, "e2e": e2e,
                 "clocks": sampler.summary(),
                 "gpu_launches": plan.kernel_launches_per_step() * args.steps,
-                "effective_tflop_per_step": flops / 1e12}
+                "effective_tflop_per_step": flops / 1e12,
+                "mask_stats": mask_stats(flops, w, plan.nq, plan.nk, attn_times,
+                                         plan.near.item() if hasattr(plan, "near") else None)}
         print(json.dumps(line))
     if world > 1:
         dist.destroy_process_group()

@@ -52,3 +52,17 @@ def test_roofline_reports_the_fraction_of_nominal_for_both_bounds():
     t = bench.with_nominal({"bound": "tensor", "achieved": 1125.0, "unit": "TFLOP/s"})
     h = bench.with_nominal({"bound": "hbm", "achieved": 3850.0, "unit": "GB/s"})
     assert t["frac_of_nominal"] == 0.5 and h["frac_of_nominal"] == 0.5
+
+
+def test_mask_stats_of_the_forward_line():
+    sys.path.insert(0, ROOT)
+    import bench
+    from block_sparse_attention_tokens_b200 import configs
+    w = configs.get("sta_720p")
+    # the 720p window keeps 9,152 of 90,000 tile pairs, all tiles full
+    flops = 4.0 * w.head_dim * 9152 * 384 * 384 * w.batch * w.heads
+    st = bench.mask_stats(flops, w, w.nq, w.nk, [3.0, 1.0, 2.0, 5.0, 4.0], near=None)
+    assert abs(st["kept_pair_fraction"] - 9152 / 90000) < 1e-12
+    assert (st["attn_ms_p10"], st["attn_ms_median"], st["attn_ms_p90"]) == (1.0, 3.0, 5.0)
+    assert "near_threshold_rows" not in st
+    assert bench.mask_stats(flops, w, w.nq, w.nk, [1.0], near=7)["near_threshold_rows"] == 7
