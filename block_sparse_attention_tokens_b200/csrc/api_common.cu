@@ -3,6 +3,7 @@
 #include <cstring>
 
 #include "bsa_common.cuh"
+#include "nvtx_range.cuh"
 
 namespace bsa {
 
@@ -50,6 +51,7 @@ extern "C" const char* bsa_last_error_message(void) { return bsa::g_last_error; 
 extern "C" int bsa_version(void) { return 100; }
 
 extern "C" int bsa_read_status(void* ws, int* status, void* stream) {
+  BSA_NVTX_RANGE("bsa_read_status");
   if (!ws || !status) return BSA_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int value = 0;

@@ -27,6 +27,7 @@
 #include "bsa_common.cuh"
 #include "tmem_io.cuh"
 #include "attn_common.cuh"
+#include "nvtx_range.cuh"
 
 namespace bsa {
 namespace {
@@ -686,6 +687,7 @@ extern "C" int bsa_attn_bwd(const void* q, const void* k, const void* v, const v
                             int nk, int head_dim, int block_q, int block_k, const int* row_ptr,
                             const int* col_idx, int list_heads, float scale, void* dq, void* dk,
                             void* dv, void* ws, size_t ws_bytes, void* stream) {
+  BSA_NVTX_RANGE("bsa_attn_bwd");
   using namespace bsa;
   if (!q || !k || !v || !o || !dout || !lse || !row_ptr || !col_idx || !dq || !dk || !dv || !ws)
     return BSA_ERR_INVALID_ARG;

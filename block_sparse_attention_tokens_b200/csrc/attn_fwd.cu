@@ -41,6 +41,7 @@
 #include "bsa_common.cuh"
 #include "tmem_io.cuh"
 #include "attn_common.cuh"
+#include "nvtx_range.cuh"
 
 namespace bsa {
 namespace {
@@ -881,6 +882,7 @@ extern "C" int bsa_attn_fwd(const void* q, const void* k, const void* v, int bat
                             int nq, int nk, int head_dim, int block_q, int block_k,
                             const int* row_ptr, const int* col_idx, int list_heads, float scale,
                             void* o, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  BSA_NVTX_RANGE("bsa_attn_fwd");
   return bsa::attn_fwd_impl(q, k, v, batch, heads, nq, nk, head_dim, block_q, block_k, row_ptr,
                             col_idx, list_heads, scale, o, lse, ws, ws_bytes, nullptr, 0, 0,
                             static_cast<cudaStream_t>(stream));
@@ -892,6 +894,7 @@ extern "C" int bsa_attn_fwd_paged(const void* q, const void* k_pool, const void*
                                   int block_k, const int* row_ptr, const int* col_idx,
                                   int list_heads, float scale, void* o, float* lse, void* ws,
                                   size_t ws_bytes, void* stream) {
+  BSA_NVTX_RANGE("bsa_attn_fwd_paged");
   if (!page_table) return BSA_ERR_INVALID_ARG;
   return bsa::attn_fwd_impl(q, k_pool, v_pool, batch, heads, nq, nk, head_dim, block_q, block_k,
                             row_ptr, col_idx, list_heads, scale, o, lse, ws, ws_bytes, page_table,
@@ -943,6 +946,7 @@ extern "C" int bsa_attn_fwd_noalloc(const void* q, const void* k, const void* v,
                                     int block_k, const int* row_ptr, const int* col_idx,
                                     int list_heads, float scale, void* o, float* lse,
                                     int* device_status, void* stream) {
+  BSA_NVTX_RANGE("bsa_attn_fwd_noalloc");
   using namespace bsa;
   const size_t need =
       bsa_attn_workspace_size(batch, heads, nq, nk, block_q, block_k, list_heads);

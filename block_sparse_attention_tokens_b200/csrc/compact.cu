@@ -6,6 +6,7 @@
 // rows are 16-byte aligned), one exclusive scan over the rows (one CTA), and the
 // ordered write of the kept indices (warp ballots, 32 columns per step).
 #include "bsa_common.cuh"
+#include "nvtx_range.cuh"
 
 namespace bsa {
 namespace {
@@ -87,6 +88,7 @@ __global__ void __launch_bounds__(256) compact_fill_kernel(const uint8_t* __rest
 
 extern "C" int bsa_mask_compact(const uint8_t* mask, int rows, int KB, int* row_ptr,
                                 int* col_idx, void* stream) {
+  BSA_NVTX_RANGE("bsa_mask_compact");
   if (!mask || !row_ptr || !col_idx || rows < 1 || KB < 1) return BSA_ERR_INVALID_ARG;
   if (static_cast<long long>(rows) * KB > 0x7fffffffLL) return BSA_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

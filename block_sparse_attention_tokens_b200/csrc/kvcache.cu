@@ -13,6 +13,7 @@
 // query blocks); the cache keeps the anchor pages, the recent pages and a fixed
 // budget of the most important pages in between, and frees the rest.
 #include "bsa_common.cuh"
+#include "nvtx_range.cuh"
 
 #include <cuda_bf16.h>
 
@@ -219,6 +220,7 @@ __global__ void __launch_bounds__(1024) keep_pages_kernel(
 extern "C" int bsa_kv_write(const void* src, int batch, int n_new, int heads, int head_dim,
                             int first_token, const int* page_table, int pages_per_batch,
                             void* pool, int n_pool_pages, int* device_status, void* stream) {
+  BSA_NVTX_RANGE("bsa_kv_write");
   using namespace bsa;
   if (!src || !page_table || !pool || !aligned16(src) || !aligned16(pool)) return BSA_ERR_INVALID_ARG;
   if (batch < 1 || n_new < 1 || heads < 1 || first_token < 0 || pages_per_batch < 1 ||
@@ -238,6 +240,7 @@ extern "C" int bsa_kv_write(const void* src, int batch, int n_new, int heads, in
 extern "C" int bsa_block_pool(const void* x, const int* page_table, int pages_per_batch, int batch,
                               int n_tokens, int heads, int head_dim, int block, int first_block,
                               int n_blocks, float* out, int out_blocks, void* stream) {
+  BSA_NVTX_RANGE("bsa_block_pool");
   using namespace bsa;
   if (!x || !out || !aligned16(x)) return BSA_ERR_INVALID_ARG;
   if (batch < 1 || n_tokens < 1 || heads < 1 || block < 1 || first_block < 0 || n_blocks < 1 ||
@@ -256,6 +259,7 @@ extern "C" int bsa_block_pool(const void* x, const int* page_table, int pages_pe
 
 extern "C" int bsa_kv_resident_blocks(const int* page_table, int batch, int pages_per_batch,
                                       int block, int KB, uint8_t* allowed, void* stream) {
+  BSA_NVTX_RANGE("bsa_kv_resident_blocks");
   using namespace bsa;
   if (!page_table || !allowed || batch < 1 || pages_per_batch < 1 || block < 1 || KB < 1)
     return BSA_ERR_INVALID_ARG;
@@ -271,6 +275,7 @@ extern "C" int bsa_kv_page_scores(const float* qbar, const float* kbar, int batc
                                   int QB, int KB, int head_dim, float scale, int kb_begin,
                                   int kb_end, const uint8_t* key_allowed, int block, int n_pages,
                                   float* scores, void* stream) {
+  BSA_NVTX_RANGE("bsa_kv_page_scores");
   using namespace bsa;
   if (!qbar || !kbar || !scores || batch < 1 || heads < 1 || QB < 1 || KB < 1 || n_pages < 1)
     return BSA_ERR_INVALID_ARG;
@@ -308,6 +313,7 @@ extern "C" int bsa_kv_page_scores(const float* qbar, const float* kbar, int batc
 extern "C" int bsa_kv_keep_pages(const float* scores, int batch, int n_pages, int anchor_pages,
                                  int recent_begin, int budget, int* page_table,
                                  int pages_per_batch, int* freed, int* freed_count, void* stream) {
+  BSA_NVTX_RANGE("bsa_kv_keep_pages");
   using namespace bsa;
   if (!scores || !page_table || !freed || !freed_count || batch < 1 || n_pages < 1 ||
       budget < 0 || anchor_pages < 0 || recent_begin > n_pages || anchor_pages > recent_begin ||

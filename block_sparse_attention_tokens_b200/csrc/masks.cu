@@ -10,6 +10,7 @@
 // Both masks are pure functions of the block indices: one thread per mask byte,
 // consecutive threads write consecutive bytes of a row (coalesced).
 #include "bsa_common.cuh"
+#include "nvtx_range.cuh"
 
 namespace bsa {
 namespace {
@@ -114,6 +115,7 @@ int grid_for(long long total, int threads) {
 
 extern "C" int bsa_sta_mask(int nT, int nH, int nW, int wT, int wH, int wW, int shift,
                             uint8_t* mask, void* stream) {
+  BSA_NVTX_RANGE("bsa_sta_mask");
   if (!mask || nT < 1 || nH < 1 || nW < 1 || wT < 1 || wH < 1 || wW < 1) return BSA_ERR_INVALID_ARG;
   const long long n = static_cast<long long>(nT) * nH * nW;
   if (n > (1LL << 20)) return BSA_ERR_UNSUPPORTED;
@@ -125,6 +127,7 @@ extern "C" int bsa_sta_mask(int nT, int nH, int nW, int wT, int wH, int wW, int 
 
 extern "C" int bsa_radial_mask(int n_tokens, int tokens_per_frame, int block, uint8_t* mask,
                                void* stream) {
+  BSA_NVTX_RANGE("bsa_radial_mask");
   if (!mask || n_tokens < 1 || tokens_per_frame < 1 || block < 1) return BSA_ERR_INVALID_ARG;
   const long long nb = bsa::ceil_div<long long>(n_tokens, block);
   if (nb > (1LL << 20)) return BSA_ERR_UNSUPPORTED;

@@ -19,6 +19,7 @@
 //            image of the fp32 logits for the cut, ties resolved to the lower
 //            block index, and the row of mask bytes.
 #include "bsa_common.cuh"
+#include "nvtx_range.cuh"
 
 namespace bsa {
 namespace {
@@ -290,6 +291,7 @@ extern "C" int bsa_nabla_select(const float* qbar, const float* kbar, int batch,
                                 int kb_end, int force_outside, const uint8_t* base_mask,
                                 const uint8_t* key_allowed, uint8_t* mask, int* near_count,
                                 void* stream) {
+  BSA_NVTX_RANGE("bsa_nabla_select");
   using namespace bsa;
   if (!qbar || !kbar || !mask) return BSA_ERR_INVALID_ARG;
   if (batch < 1 || heads < 1 || QB < 1 || KB < 1 || !(p > 0.0f)) return BSA_ERR_INVALID_ARG;
@@ -304,6 +306,7 @@ extern "C" int bsa_nabla_mask(const void* q, const void* k, int batch, int heads
                               int head_dim, int block, float p, float scale, int kb_begin,
                               int kb_end, int force_outside, uint8_t* mask, int* near_count,
                               void* ws, size_t ws_bytes, void* stream) {
+  BSA_NVTX_RANGE("bsa_nabla_mask");
   using namespace bsa;
   if (!q || !k || !mask || !ws) return BSA_ERR_INVALID_ARG;
   if (batch < 1 || heads < 1 || nq < 1 || nk < 1 || block < 16 || block > 1024 ||

@@ -13,6 +13,7 @@
 // pure HBM stream: one warp per token row, 16-byte vector loads and stores,
 // four vectors in flight per lane.
 #include "bsa_common.cuh"
+#include "nvtx_range.cuh"
 
 namespace bsa {
 namespace {
@@ -200,6 +201,7 @@ int permute_common(bool forward, const void* src, void* dst, int batch, int T, i
 extern "C" int bsa_tile_permute_pool(const void* x, void* y, int batch, int T, int H, int W,
                                      int tT, int tH, int tW, int heads, int head_dim, int n_pad,
                                      int block, float* pooled, void* stream) {
+  BSA_NVTX_RANGE("bsa_tile_permute_pool");
   using namespace bsa;
   if (!x || !y || !pooled) return BSA_ERR_INVALID_ARG;
   if (batch < 1 || T < 1 || H < 1 || W < 1 || tT < 1 || tH < 1 || tW < 1 || heads < 1 ||
@@ -224,10 +226,12 @@ extern "C" int bsa_tile_permute_pool(const void* x, void* y, int batch, int T, i
 
 extern "C" int bsa_tile_permute(const void* x, void* y, int batch, int T, int H, int W, int tT,
                                 int tH, int tW, int row_bytes, int n_pad, void* stream) {
+  BSA_NVTX_RANGE("bsa_tile_permute");
   return bsa::permute_common(true, x, y, batch, T, H, W, tT, tH, tW, row_bytes, n_pad, stream);
 }
 
 extern "C" int bsa_tile_untile(const void* y, void* x, int batch, int T, int H, int W, int tT,
                                int tH, int tW, int row_bytes, int n_pad, void* stream) {
+  BSA_NVTX_RANGE("bsa_tile_untile");
   return bsa::permute_common(false, y, x, batch, T, H, W, tT, tH, tW, row_bytes, n_pad, stream);
 }

@@ -3,6 +3,7 @@
 // pipeline uses, and must give up after `timeout_ns`, record BSA_ERR_TIMEOUT in
 // the status word and return -- the context stays usable.
 #include "bsa_common.cuh"
+#include "nvtx_range.cuh"
 
 namespace bsa {
 namespace {
@@ -24,6 +25,7 @@ __global__ void wait_selftest_kernel(int* status, unsigned long long timeout_ns)
 }  // namespace bsa
 
 extern "C" int bsa_wait_selftest(int* device_status, unsigned long long timeout_ns, void* stream) {
+  BSA_NVTX_RANGE("bsa_wait_selftest");
   using namespace bsa;
   if (!device_status || timeout_ns == 0 || timeout_ns > 10000000000ULL) return BSA_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

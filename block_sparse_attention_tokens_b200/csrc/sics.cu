@@ -14,6 +14,7 @@
 // kernel is HBM-bound: each token row (heads x head_dim bf16) is read once per
 // slicing.
 #include "bsa_common.cuh"
+#include "nvtx_range.cuh"
 
 #include <cuda_bf16.h>
 
@@ -202,6 +203,7 @@ double pairs_of(int T, int H, int W, int tT, int tH, int tW) {
 
 extern "C" int bsa_sics_blocks(const void* x, int batch, int T, int H, int W, int tT, int tH,
                                int tW, int heads, int head_dim, float* out, void* stream) {
+  BSA_NVTX_RANGE("bsa_sics_blocks");
   using namespace bsa;
   if (!x || !out || !aligned16(x)) return BSA_ERR_INVALID_ARG;
   int rc = check_sics_args(batch, T, H, W, heads, head_dim);
@@ -234,6 +236,7 @@ extern "C" int bsa_sics_scheme(const void* q, const void* k, int batch, int T, i
                                int heads, int head_dim, const int* shapes, int n_shapes,
                                float* scores, int* choice, void* ws, size_t ws_bytes,
                                void* stream) {
+  BSA_NVTX_RANGE("bsa_sics_scheme");
   using namespace bsa;
   if (!q || !k || !shapes || !scores || !choice || !ws || !aligned16(q) || !aligned16(k))
     return BSA_ERR_INVALID_ARG;
