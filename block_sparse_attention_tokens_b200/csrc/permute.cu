@@ -213,7 +213,8 @@ extern "C" int bsa_tile_permute_pool(const void* x, void* y, int batch, int T, i
   const long long row_bytes = static_cast<long long>(heads) * head_dim * 2;
   const char* s0 = static_cast<const char*>(x);
   const char* d0 = static_cast<const char*>(y);
-  if (s0 < d0 + batch * n_pad * row_bytes && d0 < s0 + batch * n * row_bytes)
+  if (s0 < d0 + static_cast<long long>(batch) * n_pad * row_bytes &&
+      d0 < s0 + static_cast<long long>(batch) * n * row_bytes)
     return BSA_ERR_INVALID_ARG;
   PermGeo g{T, H, W, tT, tH, tW};
   const int vpr = static_cast<int>(row_bytes / 16);

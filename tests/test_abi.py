@@ -14,6 +14,16 @@ HEADER = os.path.join(ROOT, "include", "bsa.h")
 
 
 @pytest.fixture(scope="module")
+def no_gpu():
+    """The argument-check cases pass stand-in pointers (small integers): a case
+    that got past the checks would reach CUDA with them.  Without a GPU that can
+    only fail with an error code, so these cases run only where no GPU is visible."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("argument-check cases use stand-in pointers; they run where no GPU is visible")
+
+
+@pytest.fixture(scope="module")
 def lib():
     from block_sparse_attention_tokens_b200 import build, binding
     if not os.path.exists(binding._LIB_PATH):
@@ -47,7 +57,7 @@ def test_status_strings_and_version(lib):
     assert lib.bsa_version() >= 100
 
 
-def test_host_argument_validation_without_gpu(lib):
+def test_host_argument_validation_without_gpu(lib, no_gpu):
     # null pointers and bad shapes are rejected before anything touches CUDA
     assert lib.bsa_tile_permute(None, None, 1, 2, 2, 2, 1, 1, 1, 256, 8, None) == 1
     assert lib.bsa_sta_mask(1, 1, 1, 1, 1, 1, 0, None, None) == 1
@@ -67,6 +77,123 @@ def test_host_argument_validation_without_gpu(lib):
     # list_heads must be 1 or batch*heads
     args[12] = 3
     assert lib.bsa_attn_fwd(*args) == 1
+
+
+def test_every_entry_rejects_bad_arguments_before_touching_cuda(lib, no_gpu):
+    """Each case below is refused by the host-side checks, which run before any
+    CUDA call: null pointers, unaligned pointers, unsupported head sizes and block
+    sizes, inconsistent ranges, too small a workspace, overlapping buffers."""
+    A = ctypes.c_void_p(16)          # 16-byte aligned stand-in; never dereferenced here
+    U = ctypes.c_void_p(8)           # not 16-byte aligned
+    INV, UNS, WS = 1, 2, 3
+    # backward: q k v o dO lse B H nq nk d bq bk row_ptr col_idx list_heads scale dq dk dv ws ws_bytes
+    bwd = [A, A, A, A, A, A, 1, 2, 256, 256, 128, 128, 128, A, A, 1, 0.0, A, A, A, A, 1 << 30, None]
+    assert lib.bsa_attn_bwd(*([None] * 6 + bwd[6:13] + [None, None] + bwd[15:17] + [None] * 4
+                               + bwd[21:])) == INV
+    for i, val, rc in ((10, 96, UNS), (11, 192, UNS), (21, 16, WS), (15, 3, INV), (0, U, INV),
+                       (20, U, INV)):
+        args = list(bwd)
+        args[i] = val
+        assert lib.bsa_attn_bwd(*args) == rc, (i, val)
+    # paged forward: q kp vp n_pool table ppb B H nq nk d bq bk row_ptr col_idx list_heads scale o lse ws ws_bytes
+    paged = [A, A, A, 8, A, 4, 1, 2, 200, 500, 128, 128, 128, A, A, 2, 0.0, A, A, A, 1 << 30, None]
+    args = list(paged)
+    args[4] = None
+    assert lib.bsa_attn_fwd_paged(*args) == INV                  # no page table
+    args = list(paged)
+    args[12] = 384
+    assert lib.bsa_attn_fwd_paged(*args) == UNS                  # key block larger than a page
+    args = list(paged)
+    args[5] = 3
+    assert lib.bsa_attn_fwd_paged(*args) == INV                  # 500 keys need 4 pages
+    args = list(paged)
+    args[6], args[15] = 2, 1
+    assert lib.bsa_attn_fwd_paged(*args) == UNS                  # one shared list, two page tables
+    # allocation-free forward: q k v B H nq nk d bq bk row_ptr col_idx list_heads scale o lse status
+    na = [A, A, A, 1, 40, 453600, 453600, 128, 96, 128, A, A, 40, 0.0, A, A, A, None]
+    assert lib.bsa_attn_fwd_noalloc(*na) == INV                  # block 96: no workspace size
+    na[8] = 128
+    assert lib.bsa_attn_fwd_noalloc(*na) == WS                   # needs more than the fixed 8 MiB
+    # NABLA: select (qbar kbar B H QB KB d p scale kb_begin kb_end force base allowed mask near)
+    sel = [A, A, 1, 2, 8, 8, 128, 0.9, 0.0, 0, 8, 0, None, None, A, None, None]
+    for i, val, rc in ((7, 0.0, INV), (6, 96, UNS), (10, 9, INV), (9, 5, INV), (0, None, INV)):
+        args = list(sel)
+        args[i] = val
+        if i == 9:
+            args[10] = 4                                         # kb_begin > kb_end
+        assert lib.bsa_nabla_select(*args) == rc, (i, val)
+    # NABLA mask (q k B H nq nk d block p scale kb_begin kb_end force mask near ws ws_bytes)
+    nm = [A, A, 1, 2, 1000, 1000, 128, 64, 0.9, 0.0, 0, 16, 0, A, None, A, 1 << 30, None]
+    for i, val, rc in ((7, 8, INV), (7, 72, INV), (16, 64, WS), (0, U, INV), (11, 17, INV),
+                       (6, 32, UNS)):
+        args = list(nm)
+        args[i] = val
+        assert lib.bsa_nabla_mask(*args) == rc, (i, val)
+    # permutes: x y B T H W tT tH tW row_bytes n_pad
+    for f in (lib.bsa_tile_permute, lib.bsa_tile_untile):
+        base = [A, ctypes.c_void_p(1 << 40), 1, 4, 8, 8, 4, 4, 4, 256, 256, None]
+        for i, val in ((9, 8), (9, 24), (10, 255), (1, A), (0, U), (6, 0)):
+            args = list(base)
+            args[i] = val
+            assert f(*args) == INV, (f, i, val)
+    # fused permute + pooling: x y B T H W tT tH tW heads d n_pad block pooled
+    pp = [A, ctypes.c_void_p(1 << 40), 1, 4, 8, 8, 4, 4, 4, 2, 128, 256, 64, A, None]
+    for i, val in ((11, 250), (12, 96), (12, 2048), (10, 12), (1, A), (13, U)):
+        args = list(pp)
+        args[i] = val
+        assert lib.bsa_tile_permute_pool(*args) == INV, (i, val)
+    # SICS: blocks (x B T H W tT tH tW heads d out) and scheme
+    sb = [A, 1, 4, 8, 8, 4, 4, 4, 2, 128, A, None]
+    for i, val, rc in ((9, 96, UNS), (5, 300, UNS), (8, 200, UNS), (0, U, INV), (2, 0, INV)):
+        args = list(sb)
+        args[i] = val
+        assert lib.bsa_sics_blocks(*args) == rc, (i, val)
+    shapes = (ctypes.c_int * 6)(4, 4, 4, 1, 8, 8)
+    need = lib.bsa_sics_workspace_size(1, 2, 4, 8, 8, shapes, 2)
+    assert need == 4 * 2 * 1 * 2 * (4 + 4)
+    sch = [A, A, 1, 4, 8, 8, 2, 128, shapes, 2, A, A, A, need, None]
+    for i, val, rc in ((9, 0, INV), (9, 17, INV), (13, need - 4, WS), (1, U, INV)):
+        args = list(sch)
+        args[i] = val
+        assert lib.bsa_sics_scheme(*args) == rc, (i, val)
+    # paged cache: write (src B n_new H d first table ppb pool n_pool status)
+    kw = [A, 1, 100, 2, 128, 0, A, 1, A, 4, None, None]
+    for i, val, rc in ((0, None, INV), (4, 4, UNS), (5, 40, INV), (2, 0, INV), (8, U, INV)):
+        args = list(kw)
+        args[i] = val
+        assert lib.bsa_kv_write(*args) == rc, (i, val)
+    # block means (x table ppb B n_tokens H d block first n out out_blocks)
+    bp = [A, A, 4, 1, 500, 2, 128, 64, 0, 8, A, 8, None]
+    for i, val, rc in ((9, 9, INV), (6, 96, UNS), (2, 3, INV), (8, -1, INV), (10, None, INV)):
+        args = list(bp)
+        args[i] = val
+        assert lib.bsa_block_pool(*args) == rc, (i, val)
+    assert lib.bsa_kv_resident_blocks(None, 1, 4, 64, 8, A, None) == INV
+    assert lib.bsa_kv_resident_blocks(A, 1, 4, 96, 8, A, None) == UNS
+    # page scores (qbar kbar B H QB KB d scale kb_begin kb_end allowed block n_pages scores)
+    ps = [A, A, 1, 2, 4, 16, 128, 0.1, 2, 12, None, 64, 8, A, None]
+    for i, val, rc in ((6, 96, UNS), (9, 17, INV), (8, 13, INV), (11, 96, INV), (13, None, INV)):
+        args = list(ps)
+        args[i] = val
+        assert lib.bsa_kv_page_scores(*args) == rc, (i, val)
+    # keep/evict (scores B n_pages anchors recent_begin budget table ppb freed freed_count)
+    kp = [A, 1, 40, 4, 32, 10, A, 40, A, A, None]
+    for i, val, rc in ((3, 33, INV), (4, 41, INV), (7, 39, INV), (5, -1, INV), (8, None, INV)):
+        args = list(kp)
+        args[i] = val
+        assert lib.bsa_kv_keep_pages(*args) == rc, (i, val)
+    args = list(kp)
+    args[2], args[3], args[4], args[7] = 9000, 0, 8193, 9000
+    assert lib.bsa_kv_keep_pages(*args) == UNS                   # one CTA ranks <= 8192 pages
+    args = list(kp)
+    args[3] = args[4] = 10
+    assert lib.bsa_kv_keep_pages(*args) == 0                     # no middle pages: nothing to do
+    # status read-back and the bounded-wait self-test
+    status = ctypes.c_int(0)
+    assert lib.bsa_read_status(None, ctypes.byref(status), None) == INV
+    assert lib.bsa_wait_selftest(None, 1000, None) == INV
+    assert lib.bsa_wait_selftest(A, 0, None) == INV
+    assert lib.bsa_wait_selftest(A, 20_000_000_000, None) == INV
 
 
 def test_workspace_sizes(lib):
@@ -95,7 +222,7 @@ def test_binding_argument_counts_match_the_header(lib):
         assert len(f.argtypes) == len(params), (name, len(f.argtypes), len(params))
 
 
-def test_header_compiles_as_c_and_links(tmp_path, lib):
+def test_header_compiles_as_c_and_links(tmp_path, lib, no_gpu):
     """A plain C program includes bsa.h, links libbsa.so and calls entry points whose
     argument checks run before any CUDA call (no GPU needed)."""
     import shutil
