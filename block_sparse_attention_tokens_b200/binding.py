@@ -121,6 +121,47 @@ def _cuda(t: torch.Tensor, name: str):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _token_problem(shape, dtype, batch: int, n: int, heads: int, head_dim: int):
+    """Why a tensor of this shape and dtype cannot serve as n token rows of the C ABI's
+    [batch, n, heads, head_dim] bf16 layout (None if it can).  The library derives
+    the batch stride from n, so with batch > 1 the tensor must hold exactly n rows;
+    with batch == 1 extra rows (e.g. a zero-padded tail) are allowed and ignored."""
+    if dtype != torch.bfloat16:
+        return f"must be bfloat16, got {dtype}"
+    if len(shape) != 4 or shape[0] != batch or tuple(shape[2:]) != (heads, head_dim):
+        return f"must be [{batch}, n, {heads}, {head_dim}], got {tuple(shape)}"
+    if shape[1] < n:
+        return f"has {shape[1]} rows for {n} tokens"
+    if batch > 1 and shape[1] != n:
+        return f"has {shape[1]} rows per batch for {n} tokens (batch > 1 needs exactly {n})"
+    return None
+
+
+def _tokens(t: torch.Tensor, name: str, batch: int, n: int, heads: int, head_dim: int):
+    _cuda(t, name)
+    problem = _token_problem(tuple(t.shape), t.dtype, batch, n, heads, head_dim)
+    if problem:
+        raise ValueError(f"{name} {problem}")
+
+
+def _buffer(t: torch.Tensor, name: str, dtype, numel: int):
+    _cuda(t, name)
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.numel() < numel:
+        raise ValueError(f"{name} holds {t.numel()} elements, {numel} needed")
+
+
+def _lists(row_ptr: torch.Tensor, col_idx: torch.Tensor, list_heads: int, nq: int, block_q: int):
+    """Kept lists: row_ptr has one entry per (list head, query block) plus one."""
+    _buffer(row_ptr, "row_ptr", torch.int32, list_heads * (-(-nq // block_q)) + 1)
+    _buffer(col_idx, "col_idx", torch.int32, 1)
+
+
+def _nbytes(t: torch.Tensor) -> int:
+    return t.numel() * t.element_size()
+
+
 # --------------------------------------------------------------------------- (a)
 
 def bsa_tile_permute(x: torch.Tensor, grid: Tuple[int, int, int], tile: Tuple[int, int, int],
@@ -280,21 +321,27 @@ def bsa_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, row_ptr: tor
                  o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
                  ws: Optional[torch.Tensor] = None):
     """Block-sparse attention forward.  Returns (o [B, nq_rows, H, D] bf16, lse [B, H, nq])."""
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (row_ptr, "row_ptr"), (col_idx, "col_idx")):
-        _cuda(t, n)
+    _cuda(q, "q")
     B, _, H, D = q.shape
     nq = q.shape[1] if nq is None else nq
     nk = k.shape[1] if nk is None else nk
+    _tokens(q, "q", B, nq, H, D)
+    _tokens(k, "k", B, nk, H, D)
+    _tokens(v, "v", B, nk, H, D)
+    _lists(row_ptr, col_idx, list_heads, nq, block_q)
     if o is None:
         o = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, nq), dtype=torch.float32, device=q.device)
+    _tokens(o, "o", B, nq, H, D)
+    _buffer(lse, "lse", torch.float32, B * H * nq)
     if ws is None:
         ws = torch.empty(bsa_attn_workspace_size(B, H, nq, nk, block_q, block_k, list_heads),
                          dtype=torch.uint8, device=q.device)
+    _cuda(ws, "ws")
     _check(load_library().bsa_attn_fwd(_ptr(q), _ptr(k), _ptr(v), B, H, nq, nk, D, block_q,
                                        block_k, _ptr(row_ptr), _ptr(col_idx), list_heads,
-                                       float(scale), _ptr(o), _ptr(lse), _ptr(ws), ws.numel(),
+                                       float(scale), _ptr(o), _ptr(lse), _ptr(ws), _nbytes(ws),
                                        _stream()), "bsa_attn_fwd")
     return o, lse, ws
 
@@ -309,15 +356,22 @@ def bsa_attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     scratch array is used instead (for callers that may not allocate device
     memory; see include/bsa.h).  Outputs are passed in or created here by the
     caller-side wrapper.  Returns (o, lse)."""
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (row_ptr, "row_ptr"), (col_idx, "col_idx")):
-        _cuda(t, n)
+    _cuda(q, "q")
     B, _, H, D = q.shape
     nq = q.shape[1] if nq is None else nq
     nk = k.shape[1] if nk is None else nk
+    _tokens(q, "q", B, nq, H, D)
+    _tokens(k, "k", B, nk, H, D)
+    _tokens(v, "v", B, nk, H, D)
+    _lists(row_ptr, col_idx, list_heads, nq, block_q)
     if o is None:
         o = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, nq), dtype=torch.float32, device=q.device)
+    _tokens(o, "o", B, nq, H, D)
+    _buffer(lse, "lse", torch.float32, B * H * nq)
+    if device_status is not None:
+        _buffer(device_status, "device_status", torch.int32, 1)
     _check(load_library().bsa_attn_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), B, H, nq, nk, D,
                                                block_q, block_k, _ptr(row_ptr), _ptr(col_idx),
                                                list_heads, float(scale), _ptr(o), _ptr(lse),
@@ -338,22 +392,28 @@ def bsa_attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Ten
                  dq: Optional[torch.Tensor] = None, dk: Optional[torch.Tensor] = None,
                  dv: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None):
     """Block-sparse attention backward.  Returns (dq, dk, dv, ws)."""
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout"), (lse, "lse"),
-                 (row_ptr, "row_ptr"), (col_idx, "col_idx")):
-        _cuda(t, n)
+    _cuda(q, "q")
     B, _, H, D = q.shape
     nq = q.shape[1] if nq is None else nq
     nk = k.shape[1] if nk is None else nk
+    for t, n, rows in ((q, "q", nq), (k, "k", nk), (v, "v", nk), (o, "o", nq),
+                       (dout, "dout", nq)):
+        _tokens(t, n, B, rows, H, D)
+    _buffer(lse, "lse", torch.float32, B * H * nq)
+    _lists(row_ptr, col_idx, list_heads, nq, block_q)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
+    for t, n, rows in ((dq, "dq", nq), (dk, "dk", nk), (dv, "dv", nk)):
+        _tokens(t, n, B, rows, H, D)
     if ws is None:
         ws = torch.empty(bsa_attn_bwd_workspace_size(B, H, nq, nk, block_q, block_k, list_heads),
                          dtype=torch.uint8, device=q.device)
+    _cuda(ws, "ws")
     _check(load_library().bsa_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
                                        B, H, nq, nk, D, block_q, block_k, _ptr(row_ptr),
                                        _ptr(col_idx), list_heads, float(scale), _ptr(dq),
-                                       _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(), _stream()),
+                                       _ptr(dk), _ptr(dv), _ptr(ws), _nbytes(ws), _stream()),
            "bsa_attn_bwd")
     return dq, dk, dv, ws
 
@@ -494,23 +554,37 @@ def bsa_attn_fwd_paged(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tens
                        o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
                        ws: Optional[torch.Tensor] = None):
     """Block-sparse attention with K/V in paged pools [P, KV_PAGE, H, D]."""
-    for t, n in ((q, "q"), (k_pool, "k_pool"), (v_pool, "v_pool"), (page_table, "page_table"),
-                 (row_ptr, "row_ptr"), (col_idx, "col_idx")):
-        _cuda(t, n)
+    _cuda(q, "q")
     B, _, H, D = q.shape
     nq = q.shape[1] if nq is None else nq
+    _tokens(q, "q", B, nq, H, D)
+    for t, n in ((k_pool, "k_pool"), (v_pool, "v_pool")):
+        _cuda(t, n)
+        if t.dtype != torch.bfloat16 or t.dim() != 4 or tuple(t.shape[1:]) != (KV_PAGE, H, D):
+            raise ValueError(f"{n} must be bfloat16 [pages, {KV_PAGE}, {H}, {D}], "
+                             f"got {t.dtype} {tuple(t.shape)}")
+    if v_pool.shape[0] != k_pool.shape[0]:
+        raise ValueError("k_pool and v_pool must hold the same number of pages")
+    _cuda(page_table, "page_table")
+    if page_table.dtype != torch.int32 or page_table.dim() != 2 or page_table.shape[0] < B:
+        raise ValueError(f"page_table must be int32 [{B}, pages], got {page_table.dtype} "
+                         f"{tuple(page_table.shape)}")
+    _lists(row_ptr, col_idx, list_heads, nq, block_q)
     if o is None:
         o = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, nq), dtype=torch.float32, device=q.device)
+    _tokens(o, "o", B, nq, H, D)
+    _buffer(lse, "lse", torch.float32, B * H * nq)
     if ws is None:
         ws = torch.empty(bsa_attn_workspace_size(B, H, nq, nk, block_q, block_k, list_heads),
                          dtype=torch.uint8, device=q.device)
+    _cuda(ws, "ws")
     _check(load_library().bsa_attn_fwd_paged(_ptr(q), _ptr(k_pool), _ptr(v_pool), k_pool.shape[0],
                                              _ptr(page_table), page_table.shape[1], B, H, nq,
                                              int(nk), D, block_q, block_k, _ptr(row_ptr),
                                              _ptr(col_idx), list_heads, float(scale), _ptr(o),
-                                             _ptr(lse), _ptr(ws), ws.numel(), _stream()),
+                                             _ptr(lse), _ptr(ws), _nbytes(ws), _stream()),
            "bsa_attn_fwd_paged")
     return o, lse, ws
 
