@@ -246,22 +246,26 @@ def bsa_nabla_mask(q: torch.Tensor, k: torch.Tensor, block: int, p: float, scale
     Returns (mask, near_count tensor).
     """
     _cuda(q, "q")
-    _cuda(k, "k")
     B, _, H, D = q.shape
     nq = q.shape[1] if nq is None else nq
     nk = k.shape[1] if nk is None else nk
+    _tokens(q, "q", B, nq, H, D)
+    _tokens(k, "k", B, nk, H, D)
     QB, KB = -(-nq // block), -(-nk // block)
     kb_end = KB if kb_end is None else kb_end
     if mask is None:
         mask = torch.empty((B, H, QB, KB), dtype=torch.uint8, device=q.device)
+    _buffer(mask, "mask", torch.uint8, B * H * QB * KB)
     if near_count is None:
         near_count = torch.zeros(1, dtype=torch.int32, device=q.device)
+    _buffer(near_count, "near_count", torch.int32, 1)
     if ws is None:
         ws = torch.empty(bsa_nabla_workspace_size(B, H, nq, nk, D, block), dtype=torch.uint8,
                          device=q.device)
+    _cuda(ws, "ws")
     _check(load_library().bsa_nabla_mask(_ptr(q), _ptr(k), B, H, nq, nk, D, block, float(p),
                                          float(scale), kb_begin, kb_end, int(force_outside),
-                                         _ptr(mask), _ptr(near_count), _ptr(ws), ws.numel(),
+                                         _ptr(mask), _ptr(near_count), _ptr(ws), _nbytes(ws),
                                          _stream()), "bsa_nabla_mask")
     return mask, near_count
 
