@@ -158,8 +158,63 @@ def _lists(row_ptr: torch.Tensor, col_idx: torch.Tensor, list_heads: int, nq: in
     _buffer(col_idx, "col_idx", torch.int32, 1)
 
 
+def _means(t: torch.Tensor, name: str, batch: int, heads: int, head_dim: int):
+    """Pooled block means [batch, heads, blocks, head_dim] float32."""
+    _cuda(t, name)
+    if t.dtype != torch.float32 or t.dim() != 4 or tuple(t.shape[:2]) != (batch, heads) \
+            or t.shape[3] != head_dim:
+        raise ValueError(f"{name} must be float32 [{batch}, {heads}, blocks, {head_dim}], "
+                         f"got {t.dtype} {tuple(t.shape)}")
+
+
+def _pool(t: torch.Tensor, name: str, heads: int, head_dim: int):
+    """A paged K or V pool [pages, KV_PAGE, heads, head_dim] bf16."""
+    _cuda(t, name)
+    if t.dtype != torch.bfloat16 or t.dim() != 4 or tuple(t.shape[1:]) != (KV_PAGE, heads, head_dim):
+        raise ValueError(f"{name} must be bfloat16 [pages, {KV_PAGE}, {heads}, {head_dim}], "
+                         f"got {t.dtype} {tuple(t.shape)}")
+
+
+def _table(t: torch.Tensor, name: str, batch: int, pages: int = 0):
+    """A page table [>= batch, >= pages] int32 (physical page or -1)."""
+    _cuda(t, name)
+    if t.dtype != torch.int32 or t.dim() != 2 or t.shape[0] < batch or t.shape[1] < pages:
+        raise ValueError(f"{name} must be int32 [{batch}, >= {pages} pages], "
+                         f"got {t.dtype} {tuple(t.shape)}")
+
+
 def _nbytes(t: torch.Tensor) -> int:
     return t.numel() * t.element_size()
+
+
+def _row_problem(shape, elem_bytes: int, batch: int, n: int, row_bytes: int):
+    """Why a tensor cannot serve as n rows of row_bytes each per batch ([batch, n, ...]
+    with the batch stride n rows; extra rows allowed only for one batch)."""
+    if len(shape) < 2 or shape[0] != batch:
+        return f"must be [{batch}, rows, ...], got {tuple(shape)}"
+    if math.prod(shape[2:]) * elem_bytes != row_bytes:
+        return f"rows of {math.prod(shape[2:]) * elem_bytes} bytes, {row_bytes} expected"
+    if shape[1] < n:
+        return f"has {shape[1]} rows for {n}"
+    if batch > 1 and shape[1] != n:
+        return f"has {shape[1]} rows per batch for {n} (batch > 1 needs exactly {n})"
+    return None
+
+
+def _rows(t: torch.Tensor, name: str, batch: int, n: int, row_bytes: int):
+    _cuda(t, name)
+    problem = _row_problem(tuple(t.shape), t.element_size(), batch, n, row_bytes)
+    if problem:
+        raise ValueError(f"{name} {problem}")
+
+
+def _bytes(t: torch.Tensor, name: str, numel: int):
+    """A byte mask / flag buffer (uint8 or bool) of at least numel entries."""
+    _cuda(t, name)
+    if t.dtype not in (torch.uint8, torch.bool):
+        raise ValueError(f"{name} must be uint8 (or bool), got {t.dtype}")
+    if t.numel() < numel:
+        raise ValueError(f"{name} holds {t.numel()} entries, {numel} needed")
 
 
 # --------------------------------------------------------------------------- (a)
@@ -168,10 +223,13 @@ def bsa_tile_permute(x: torch.Tensor, grid: Tuple[int, int, int], tile: Tuple[in
                      n_pad: int, y: Optional[torch.Tensor] = None) -> torch.Tensor:
     """x [B, N, ...] raster order -> y [B, n_pad, ...] tile order with a zero tail."""
     _cuda(x, "x")
-    B, N = x.shape[0], x.shape[1]
-    row_bytes = x[0, 0].numel() * x.element_size()
+    B = x.shape[0]
+    N = grid[0] * grid[1] * grid[2]
+    row_bytes = math.prod(x.shape[2:]) * x.element_size()
+    _rows(x, "x", B, N, row_bytes)
     if y is None:
         y = torch.empty((B, n_pad) + tuple(x.shape[2:]), dtype=x.dtype, device=x.device)
+    _rows(y, "y", B, n_pad, row_bytes)
     _check(load_library().bsa_tile_permute(_ptr(x), _ptr(y), B, *grid, *tile, row_bytes, n_pad,
                                            _stream()), "bsa_tile_permute")
     return y
@@ -183,9 +241,10 @@ def bsa_tile_untile(y: torch.Tensor, grid: Tuple[int, int, int], tile: Tuple[int
     _cuda(y, "y")
     B, n_pad = y.shape[0], y.shape[1]
     N = grid[0] * grid[1] * grid[2]
-    row_bytes = y[0, 0].numel() * y.element_size()
+    row_bytes = math.prod(y.shape[2:]) * y.element_size()
     if x is None:
         x = torch.empty((B, N) + tuple(y.shape[2:]), dtype=y.dtype, device=y.device)
+    _rows(x, "x", B, N, row_bytes)
     _check(load_library().bsa_tile_untile(_ptr(y), _ptr(x), B, *grid, *tile, row_bytes, n_pad,
                                           _stream()), "bsa_tile_untile")
     return x
@@ -198,11 +257,14 @@ def bsa_tile_permute_pool(x: torch.Tensor, grid: Tuple[int, int, int],
     """x [B, N, H, D] bf16 raster -> (y [B, n_pad, H, D] tile order,
     pooled [B, H, n_pad / block, D] fp32 block means)."""
     _cuda(x, "x")
-    B, N, H, D = x.shape
+    B, _, H, D = x.shape
+    _tokens(x, "x", B, grid[0] * grid[1] * grid[2], H, D)
     if y is None:
         y = torch.empty((B, n_pad, H, D), dtype=x.dtype, device=x.device)
+    _tokens(y, "y", B, n_pad, H, D)
     if pooled is None:
         pooled = torch.empty((B, H, n_pad // block, D), dtype=torch.float32, device=x.device)
+    _buffer(pooled, "pooled", torch.float32, B * H * (n_pad // max(block, 1)) * D)
     _check(load_library().bsa_tile_permute_pool(_ptr(x), _ptr(y), B, *grid, *tile, H, D, n_pad,
                                                 block, _ptr(pooled), _stream()),
            "bsa_tile_permute_pool")
@@ -216,6 +278,7 @@ def bsa_sta_mask(tile_grid: Tuple[int, int, int], window: Tuple[int, int, int], 
     n = tile_grid[0] * tile_grid[1] * tile_grid[2]
     if mask is None:
         mask = torch.empty((n, n), dtype=torch.uint8, device=device)
+    _bytes(mask, "mask", n * n)
     _check(load_library().bsa_sta_mask(*tile_grid, *window, int(shift), _ptr(mask), _stream()),
            "bsa_sta_mask")
     return mask
@@ -226,6 +289,7 @@ def bsa_radial_mask(n_tokens: int, tokens_per_frame: int, block: int,
     nb = -(-n_tokens // block)
     if mask is None:
         mask = torch.empty((nb, nb), dtype=torch.uint8, device=device)
+    _bytes(mask, "mask", nb * nb)
     _check(load_library().bsa_radial_mask(n_tokens, tokens_per_frame, block, _ptr(mask),
                                           _stream()), "bsa_radial_mask")
     return mask
@@ -283,11 +347,19 @@ def bsa_nabla_select(qbar: torch.Tensor, kbar: torch.Tensor, p: float, scale: fl
     _cuda(kbar, "kbar")
     B, H, QB, D = qbar.shape
     KB = kbar.shape[2]
+    _means(qbar, "qbar", B, H, D)
+    _means(kbar, "kbar", B, H, D)
     kb_end = KB if kb_end is None else kb_end
     if mask is None:
         mask = torch.empty((B, H, QB, KB), dtype=torch.uint8, device=qbar.device)
+    _bytes(mask, "mask", B * H * QB * KB)
+    if base_mask is not None:
+        _bytes(base_mask, "base_mask", QB * KB)
+    if key_allowed is not None:
+        _bytes(key_allowed, "key_allowed", B * KB)
     if near_count is None:
         near_count = torch.zeros(1, dtype=torch.int32, device=qbar.device)
+    _buffer(near_count, "near_count", torch.int32, 1)
     _check(load_library().bsa_nabla_select(_ptr(qbar), _ptr(kbar), B, H, QB, KB, D, float(p),
                                            float(scale), kb_begin, kb_end, int(force_outside),
                                            _ptr(base_mask), _ptr(key_allowed), _ptr(mask),
@@ -303,10 +375,13 @@ def bsa_mask_compact(mask: torch.Tensor, row_ptr: Optional[torch.Tensor] = None,
     _cuda(mask, "mask")
     KB = mask.shape[-1]
     rows = mask.numel() // KB
+    _bytes(mask, "mask", rows * KB)
     if row_ptr is None:
         row_ptr = torch.empty(rows + 1, dtype=torch.int32, device=mask.device)
     if col_idx is None:
         col_idx = torch.empty(rows * KB, dtype=torch.int32, device=mask.device)
+    _buffer(row_ptr, "row_ptr", torch.int32, rows + 1)
+    _buffer(col_idx, "col_idx", torch.int32, rows * KB)
     _check(load_library().bsa_mask_compact(_ptr(mask), rows, KB, _ptr(row_ptr), _ptr(col_idx),
                                            _stream()), "bsa_mask_compact")
     return row_ptr, col_idx
@@ -431,8 +506,10 @@ def bsa_sics_blocks(x: torch.Tensor, grid, tile, out: Optional[torch.Tensor] = N
     raster order.  Returns out [B, heads, n_tiles] float32."""
     _cuda(x, "x")
     B, _, Hh, D = x.shape
+    _tokens(x, "x", B, grid[0] * grid[1] * grid[2], Hh, D)
     if out is None:
         out = torch.empty((B, Hh, _n_tiles(grid, tile)), dtype=torch.float32, device=x.device)
+    _buffer(out, "out", torch.float32, B * Hh * _n_tiles(grid, tile))
     _check(load_library().bsa_sics_blocks(_ptr(x), B, *grid, *tile, Hh, D, _ptr(out), _stream()),
            "bsa_sics_blocks")
     return out
@@ -454,18 +531,23 @@ def bsa_sics_scheme(q: torch.Tensor, k: torch.Tensor, grid, shapes,
     """Per-head slicing choice from a shape menu.  Returns (scores [B, H, n_shapes]
     float32, choice [B, H] int32, ws)."""
     _cuda(q, "q")
-    _cuda(k, "k")
     B, _, Hh, D = q.shape
+    N = grid[0] * grid[1] * grid[2]
+    _tokens(q, "q", B, N, Hh, D)
+    _tokens(k, "k", B, N, Hh, D)
     arr, n = _shape_array(shapes)
     if scores is None:
         scores = torch.empty((B, Hh, n), dtype=torch.float32, device=q.device)
     if choice is None:
         choice = torch.empty((B, Hh), dtype=torch.int32, device=q.device)
+    _buffer(scores, "scores", torch.float32, B * Hh * n)
+    _buffer(choice, "choice", torch.int32, B * Hh)
     if ws is None:
         ws = torch.empty(max(1, bsa_sics_workspace_size(B, Hh, grid, shapes)), dtype=torch.uint8,
                          device=q.device)
+    _cuda(ws, "ws")
     _check(load_library().bsa_sics_scheme(_ptr(q), _ptr(k), B, *grid, Hh, D, arr, n,
-                                          _ptr(scores), _ptr(choice), _ptr(ws), ws.numel(),
+                                          _ptr(scores), _ptr(choice), _ptr(ws), _nbytes(ws),
                                           _stream()), "bsa_sics_scheme")
     return scores, choice, ws
 
@@ -480,9 +562,13 @@ def bsa_kv_write(src: torch.Tensor, first_token: int, page_table: torch.Tensor,
                  pool: torch.Tensor, device_status: Optional[torch.Tensor] = None):
     """Rows src [B, n_new, H, D] -> logical tokens first_token.. of each batch in the
     pool [P, KV_PAGE, H, D] through page_table [B, pages_per_batch]."""
-    for t, n in ((src, "src"), (page_table, "page_table"), (pool, "pool")):
-        _cuda(t, n)
+    _cuda(src, "src")
     B, n_new, H, D = src.shape
+    _tokens(src, "src", B, n_new, H, D)
+    _table(page_table, "page_table", B)
+    _pool(pool, "pool", H, D)
+    if device_status is not None:
+        _buffer(device_status, "device_status", torch.int32, 1)
     _check(load_library().bsa_kv_write(_ptr(src), B, n_new, H, D, int(first_token),
                                        _ptr(page_table), page_table.shape[1], _ptr(pool),
                                        pool.shape[0], _ptr(device_status), _stream()),
@@ -494,9 +580,18 @@ def bsa_block_pool(x: torch.Tensor, n_tokens: int, block: int, first_block: int,
     """Block means of x ([B, n, H, D], or a paged pool [P, KV_PAGE, H, D] with its
     page_table) into out [B, H, out_blocks, D] float32 at blocks first_block.."""
     _cuda(x, "x")
-    _cuda(out, "out")
     B = batch if page_table is not None else x.shape[0]
     H, D = x.shape[2], x.shape[3]
+    if page_table is not None:
+        _pool(x, "x", H, D)
+        _table(page_table, "page_table", B)
+    else:
+        _tokens(x, "x", B, int(n_tokens), H, D)
+    _cuda(out, "out")
+    if out.dtype != torch.float32 or out.dim() != 4 or out.shape[0] < B or out.shape[1] != H \
+            or out.shape[3] != D:
+        raise ValueError(f"out must be float32 [{B}, {H}, blocks, {D}], got {out.dtype} "
+                         f"{tuple(out.shape)}")
     ppb = page_table.shape[1] if page_table is not None else 0
     _check(load_library().bsa_block_pool(_ptr(x), _ptr(page_table), ppb, B, int(n_tokens), H, D,
                                          int(block), int(first_block), int(n_blocks), _ptr(out),
@@ -506,10 +601,11 @@ def bsa_block_pool(x: torch.Tensor, n_tokens: int, block: int, first_block: int,
 
 def bsa_kv_resident_blocks(page_table: torch.Tensor, block: int, KB: int,
                            allowed: Optional[torch.Tensor] = None):
-    _cuda(page_table, "page_table")
+    _table(page_table, "page_table", 1)
     B, ppb = page_table.shape
     if allowed is None:
         allowed = torch.empty((B, KB), dtype=torch.uint8, device=page_table.device)
+    _bytes(allowed, "allowed", B * KB)
     _check(load_library().bsa_kv_resident_blocks(_ptr(page_table), B, ppb, int(block), int(KB),
                                                  _ptr(allowed), _stream()),
            "bsa_kv_resident_blocks")
@@ -522,13 +618,17 @@ def bsa_kv_page_scores(qbar: torch.Tensor, kbar: torch.Tensor, kb_begin: int, kb
                        scores: Optional[torch.Tensor] = None):
     """Page importance [B, n_pages] float32 from pooled means (see include/bsa.h)."""
     _cuda(qbar, "qbar")
-    _cuda(kbar, "kbar")
     B, H, QB, D = qbar.shape
+    _means(qbar, "qbar", B, H, D)
+    _means(kbar, "kbar", B, H, D)
     KB = kbar.shape[2]
+    if key_allowed is not None:
+        _bytes(key_allowed, "key_allowed", B * KB)
     if scale <= 0:
         scale = 1.0 / math.sqrt(D)
     if scores is None:
         scores = torch.empty((B, n_pages), dtype=torch.float32, device=qbar.device)
+    _buffer(scores, "scores", torch.float32, B * n_pages)
     _check(load_library().bsa_kv_page_scores(_ptr(qbar), _ptr(kbar), B, H, QB, KB, D, float(scale),
                                              int(kb_begin), int(kb_end), _ptr(key_allowed),
                                              int(block), int(n_pages), _ptr(scores), _stream()),
@@ -540,10 +640,15 @@ def bsa_kv_keep_pages(scores: torch.Tensor, anchor_pages: int, recent_begin: int
                       page_table: torch.Tensor, freed: torch.Tensor, freed_count: torch.Tensor):
     """Evicts middle pages beyond the budget in place (page_table entries -> -1); the
     freed physical pages are appended to freed at atomic index freed_count."""
-    for t, n in ((scores, "scores"), (page_table, "page_table"), (freed, "freed"),
-                 (freed_count, "freed_count")):
-        _cuda(t, n)
+    _cuda(scores, "scores")
+    if scores.dtype != torch.float32 or scores.dim() != 2:
+        raise ValueError(f"scores must be float32 [batch, pages], got {scores.dtype} "
+                         f"{tuple(scores.shape)}")
     B, n_pages = scores.shape
+    _table(page_table, "page_table", B, n_pages)
+    # at most (middle pages - budget) pages per batch are evicted and appended
+    _buffer(freed, "freed", torch.int32, B * max(0, recent_begin - anchor_pages - max(budget, 0)))
+    _buffer(freed_count, "freed_count", torch.int32, 1)
     _check(load_library().bsa_kv_keep_pages(_ptr(scores), B, n_pages, int(anchor_pages),
                                             int(recent_begin), int(budget), _ptr(page_table),
                                             page_table.shape[1], _ptr(freed), _ptr(freed_count),
@@ -562,17 +667,11 @@ def bsa_attn_fwd_paged(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tens
     B, _, H, D = q.shape
     nq = q.shape[1] if nq is None else nq
     _tokens(q, "q", B, nq, H, D)
-    for t, n in ((k_pool, "k_pool"), (v_pool, "v_pool")):
-        _cuda(t, n)
-        if t.dtype != torch.bfloat16 or t.dim() != 4 or tuple(t.shape[1:]) != (KV_PAGE, H, D):
-            raise ValueError(f"{n} must be bfloat16 [pages, {KV_PAGE}, {H}, {D}], "
-                             f"got {t.dtype} {tuple(t.shape)}")
+    _pool(k_pool, "k_pool", H, D)
+    _pool(v_pool, "v_pool", H, D)
     if v_pool.shape[0] != k_pool.shape[0]:
         raise ValueError("k_pool and v_pool must hold the same number of pages")
-    _cuda(page_table, "page_table")
-    if page_table.dtype != torch.int32 or page_table.dim() != 2 or page_table.shape[0] < B:
-        raise ValueError(f"page_table must be int32 [{B}, pages], got {page_table.dtype} "
-                         f"{tuple(page_table.shape)}")
+    _table(page_table, "page_table", B)
     _lists(row_ptr, col_idx, list_heads, nq, block_q)
     if o is None:
         o = torch.empty_like(q)

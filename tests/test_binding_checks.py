@@ -24,3 +24,13 @@ def test_too_few_rows_wrong_dtype_or_head_layout_are_refused():
     assert "must be" in B._token_problem((1, 256, 64, 2), BF, 1, 256, 2, 64)
     assert "must be" in B._token_problem((2, 256, 2, 64), BF, 1, 256, 2, 64)
     assert "must be" in B._token_problem((256, 2, 64), BF, 1, 256, 2, 64)
+
+
+def test_row_rule_of_the_permutes():
+    # 3 x 256-byte rows per token (heads x head_dim bf16), 105 tokens
+    assert B._row_problem((2, 105, 2, 64), 2, 2, 105, 256) is None
+    assert B._row_problem((1, 128, 2, 64), 2, 1, 105, 256) is None        # padded, one batch
+    assert "exactly" in B._row_problem((2, 128, 2, 64), 2, 2, 105, 256)
+    assert "rows for" in B._row_problem((1, 100, 2, 64), 2, 1, 105, 256)
+    assert "bytes" in B._row_problem((1, 105, 2, 32), 2, 1, 105, 256)
+    assert "must be" in B._row_problem((3, 105, 2, 64), 2, 2, 105, 256)
