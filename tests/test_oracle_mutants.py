@@ -147,6 +147,13 @@ MUTANTS = [
     Mutant("nabla_mask/range-offset-forgotten", "nabla_mask",
            "mask[b, h, qb, cand[kept]] = 1", "mask[b, h, qb, kept] = 1",
            [pin(TN.test_nabla_mask_range_and_forced_outside)]),
+    Mutant("nabla_mask/near-flag-ignores-the-previous-prefix", "nabla_mask",
+           "flag = abs(c_last - p) < near_tol or abs(c_prev - p) < near_tol",
+           "flag = abs(c_last - p) < near_tol",
+           [pin(TN.test_near_threshold_flag)]),
+    Mutant("nabla_mask/near-flag-ignores-ties", "nabla_mask",
+           "flag = flag or abs(a - bb) <= tie_tol * max(a, bb)", "flag = flag",
+           [pin(TN.test_near_threshold_flag)]),
     Mutant("nabla_mask/allowed-blocks-ignored", "nabla_mask",
            "cand = cand[key_allowed[b, kb_begin:kb_end]]", "cand = cand",
            [pin(TP.test_nabla_with_allowed_blocks_equals_nabla_on_the_allowed_subset)]),

@@ -164,6 +164,13 @@ def test_near_threshold_flag():
     assert near[0, 0, 0]
     _, near = O.nabla_mask(qbar, kbar, 0.8, 1.0)
     assert not near[0, 0, 0]
+    # the prefix before the cut (0.5) lies 1e-7 below p: a float32 sum may reach p there
+    _, near = O.nabla_mask(qbar, kbar, 0.5 + 1e-7, 1.0)
+    assert near[0, 0, 0]
+    # last kept and first dropped probabilities tie (0.3, 0.3): either may be kept
+    kbar[0, 0, :, 0] = np.log(np.array([0.4, 0.3, 0.3]))
+    mask, near = O.nabla_mask(qbar, kbar, 0.6, 1.0)
+    assert mask[0, 0, 0].tolist() == [1, 1, 0] and near[0, 0, 0]
 
 
 # ----------------------------------------------------------------- attention
