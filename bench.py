@@ -882,6 +882,9 @@ def main():
     if args.pass_ == "ar_paged" and args.workload == "sta_720p":
         args.workload = "ar_decode"
     w = configs.get(args.workload)
+    if args.pass_ == "ar_paged" and w.mask != "ar":
+        ap.error(f"--pass ar_paged decodes an autoregressive workload (mask 'ar'); "
+                 f"{w.name} has mask '{w.mask}'")
     if args.heads > 0:
         w = dataclasses.replace(w, heads=args.heads)
     if args.impl == "reference":

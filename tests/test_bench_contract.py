@@ -20,14 +20,15 @@ def run_bench(*args):
     return json.loads(lines[0])
 
 
-@pytest.mark.parametrize("pass_", ["fwd", "bwd"])
+@pytest.mark.parametrize("pass_", ["fwd", "bwd", "sics"])
 def test_reference_arm_prints_one_contract_line(pass_):
     d = run_bench("--impl", "reference", "--workload", "sta_tiny", "--steps", "1", "--warmup",
                   "0", "--pass", pass_)
     for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup",
                 "higher_is_better", "dtype", "data", "config", "cpu_baseline", "e2e"):
         assert key in d, key
-    assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == "TFLOP/s"
+    assert d["impl"] == "reference" and d["value"] > 0
+    assert d["unit"] == ("GB/s" if pass_ == "sics" else "TFLOP/s")
     assert d["config"]["workload"] == "sta_tiny"
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
@@ -66,3 +67,10 @@ def test_mask_stats_of_the_forward_line():
     assert (st["attn_ms_p10"], st["attn_ms_median"], st["attn_ms_p90"]) == (1.0, 3.0, 5.0)
     assert "near_threshold_rows" not in st
     assert bench.mask_stats(flops, w, w.nq, w.nk, [1.0], near=7)["near_threshold_rows"] == 7
+
+
+def test_paged_pass_refuses_a_workload_without_ar_decoding():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--pass", "ar_paged", "--workload", "sta_tiny", "--steps", "1"],
+                         capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 2 and "autoregressive" in out.stderr
