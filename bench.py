@@ -926,6 +926,8 @@ def main():
     stream = torch.cuda.current_stream()
     ev_a = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
             for _ in range(args.steps)]
+    # stage boundaries: step start, after the permute, after the mask, step end
+    ev_s = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(dev.index)
     barrier()
@@ -933,21 +935,32 @@ def main():
         time.sleep(0.5)          # let nvidia-smi start sampling before the timed region
         start.record(stream)
         for i in range(args.steps):
+            ev_s[i][0].record(stream)
             plan._q, plan._k, plan._v = q, k, v
             if plan.permuted:
                 plan.permute_inputs(q, k, v)
+            ev_s[i][1].record(stream)
             plan.build_mask()
+            ev_s[i][2].record(stream)
             plan.compact()
             ev_a[i][0].record(stream)
             plan.attention()
             ev_a[i][1].record(stream)
             if plan.permuted:
                 plan.untile()
+            ev_s[i][3].record(stream)
         end.record(stream)
         barrier()
     ms_total = start.elapsed_time(end)
     attn_times = [a.elapsed_time(b) for a, b in ev_a]
     attn_ms = statistics.mean(attn_times)
+    stage_ms = {
+        "permute": statistics.mean(e[0].elapsed_time(e[1]) for e in ev_s),
+        "mask": statistics.mean(e[1].elapsed_time(e[2]) for e in ev_s),
+        "compact": statistics.mean(e[2].elapsed_time(a[0]) for e, a in zip(ev_s, ev_a)),
+        "attention": attn_ms,
+        "untile": statistics.mean(a[1].elapsed_time(e[3]) for e, a in zip(ev_s, ev_a)),
+    }
     ms_total, attn_ms = max_over_ranks([ms_total, attn_ms], dev)
     ms_per_step = ms_total / args.steps
     value = weak_scaling_value(flops, world, ms_per_step)
@@ -1045,7 +1058,9 @@ def main():
                 "gpu_launches": plan.kernel_launches_per_step() * args.steps,
                 "effective_tflop_per_step": flops / 1e12,
                 "mask_stats": mask_stats(flops, w, plan.nq, plan.nk, attn_times,
-                                         plan.near.item() if hasattr(plan, "near") else None)}
+                                         plan.near.item() if hasattr(plan, "near") else None),
+                # mean device time of each stage of a timed step (this rank, CUDA events)
+                "stage_ms": stage_ms}
         print(json.dumps(line))
     if world > 1:
         dist.destroy_process_group()
