@@ -85,6 +85,9 @@ MUTANTS = [
            "start = min(max(a - lo_off, 0), max(n - w, 0))", "start = max(a - lo_off, 0)",
            [pin(TM.test_sta_kept_count_closed_form_720p, shift=True),
             pin(TM.test_sta_matches_token_level_enumeration, shift=True)]),
+    Mutant("sta/shifted-window-one-too-wide", "sta_axis_keep",
+           "lo, hi = start, min(start + w, n) - 1", "lo, hi = start, min(start + w, n)",
+           [pin(TM.test_sta_kept_count_closed_form_720p, shift=True)]),
     Mutant("sta/window-axes-reversed", "sta_tile_mask",
            "zip(tile_grid, window)", "zip(tile_grid, window[::-1])",
            [pin(TM.test_sta_kept_count_closed_form_720p, shift=False)]),
@@ -188,6 +191,10 @@ MUTANTS = [
     Mutant("token_mask/query-blocks-of-key-size", "token_mask_from_blocks",
            "qi = np.arange(nq) // block_q", "qi = np.arange(nq) // block_k",
            [pin(TN.test_block_mask_equals_token_level_definition, bq=64, bk=128)]),
+    Mutant("dense/empty-rows-divide-by-zero", "dense_masked_attention",
+           "o = np.where(empty[:, None], 0.0, (e @ v) / np.where(empty, 1.0, l)[:, None])",
+           "o = (e @ v) / np.where(empty, 1.0, l)[:, None] + np.where(empty, np.nan, 0.0)[:, None]",
+           [pin(TN.test_block_mask_equals_token_level_definition, bq=64, bk=64)]),
     Mutant("attn/scale-1-over-d", "block_sparse_attention",
            "scale = 1.0 / math.sqrt(D) if scale is None else scale",
            "scale = 1.0 / D if scale is None else scale",
@@ -222,6 +229,10 @@ MUTANTS = [
            "dq[b, rows_, h] += (ds @ k[b, cols, h]) * scale",
            "dq[b, rows_, h] += (ds @ v[b, cols, h]) * scale",
            [pin(TN.test_backward_matches_autograd_float64, bq=64, bk=64)]),
+    Mutant("bwd/default-scale-1-over-d", "block_sparse_attention_backward",
+           "scale = 1.0 / math.sqrt(D) if scale is None else scale",
+           "scale = 1.0 / D if scale is None else scale",
+           [pin(TN.test_backward_matches_autograd_float64, bq=64, bk=64)]),
     Mutant("bwd/row-sample-ignored", "block_sparse_attention_backward",
            "rows_b = np.intersect1d(rows_b, np.asarray(rows))", "rows_b = rows_b",
            [pin(TN.test_backward_row_sampling_is_exact_on_dq_and_additive_on_dk_dv)]),
@@ -236,6 +247,10 @@ MUTANTS = [
             pin(TS.test_scale_invariance)]),
     Mutant("sics/diagonal-excluded", "sics_blocks",
            "out[b, h, t] = (u @ u.T).sum()", "out[b, h, t] = (u @ u.T).sum() - len(idx)",
+           [pin(TS.test_identical_orthogonal_and_opposite_vectors)]),
+    Mutant("sics/zero-vector-normalised", "sics_blocks",
+           "u = np.where(norm[:, None] > 0, v / np.where(norm > 0, norm, 1.0)[:, None], 0.0)",
+           "u = v / np.where(norm > 0, norm, 0.0)[:, None]",
            [pin(TS.test_identical_orthogonal_and_opposite_vectors)]),
     Mutant("scheme/ties-to-later-entry", "sics_scheme",
            "if scores[b, h, si] > scores[b, h, best]:", "if scores[b, h, si] >= scores[b, h, best]:",
@@ -273,6 +288,12 @@ MUTANTS = [
     Mutant("keep_pages/evicted-pages-revived", "kv_keep_pages",
            "mid = [pg for pg in range(anchor_pages, recent_begin) if resident[b, pg]]",
            "mid = list(range(anchor_pages, recent_begin))",
+           [pin(TP.test_keep_pages_anchors_recent_and_budget)]),
+    Mutant("keep_pages/last-anchor-page-dropped", "kv_keep_pages",
+           "keep[:, :anchor_pages] = True", "keep[:, :anchor_pages - 1] = True",
+           [pin(TP.test_keep_pages_anchors_recent_and_budget)]),
+    Mutant("keep_pages/first-recent-page-dropped", "kv_keep_pages",
+           "keep[:, recent_begin:] = True", "keep[:, recent_begin + 1:] = True",
            [pin(TP.test_keep_pages_anchors_recent_and_budget)]),
     Mutant("keep_pages/tie-to-higher-page", "kv_keep_pages",
            "mid.sort(key=lambda pg: (-scores[b, pg], pg))", "mid.sort(key=lambda pg: (-scores[b, pg], -pg))",
