@@ -251,3 +251,28 @@ int main(void) {
     out = subprocess.run([str(exe)], capture_output=True, text=True)
     assert out.returncode == 0, (out.returncode, out.stderr)
     assert out.stdout.strip() == "BSA_ERR_TIMEOUT"
+
+
+def test_binding_fails_loudly_without_the_library(tmp_path):
+    """A copy of the package with no libbsa.so: the first binding call raises
+    ImportError; nothing falls back to another implementation."""
+    import shutil
+    import subprocess
+    import sys
+    pkg = os.path.join(ROOT, "block_sparse_attention_tokens_b200")
+    dst = tmp_path / "block_sparse_attention_tokens_b200"
+    shutil.copytree(pkg, dst, ignore=shutil.ignore_patterns("*.so", "csrc", "__pycache__"))
+    code = ("from block_sparse_attention_tokens_b200 import binding, configs\n"
+            "from block_sparse_attention_tokens_b200.pipeline import Plan\n"
+            "for call in (lambda: binding.bsa_attn_workspace_size(1, 1, 128, 128, 128, 128, 1),\n"
+            "             lambda: Plan(configs.get('sta_tiny'), 'cpu')):\n"
+            "    try:\n"
+            "        call()\n"
+            "    except ImportError as e:\n"
+            "        assert 'libbsa.so not found' in str(e)\n"
+            "    else:\n"
+            "        raise SystemExit('no error without the library')\n"
+            "print('refused')\n")
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True,
+                         cwd=str(tmp_path), env={**os.environ, "PYTHONPATH": str(tmp_path)})
+    assert out.returncode == 0 and out.stdout.strip() == "refused", out.stderr[-2000:]
