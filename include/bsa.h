@@ -7,9 +7,15 @@
  *   (a) a 3D tile permute of a T x H x W token grid (and its inverse),
  *   (b) block masks: the static Sliding-Tile window, the static radial
  *       (energy-decay) mask, and the dynamic per-head NABLA top-p mask,
- *   (c) compaction of a block mask into per-row kept-block lists, and
+ *   (c) compaction of a block mask into per-row kept-block lists,
  *   (d) the attention forward that visits only kept (query block, key block)
- *       pairs, with an online softmax, producing O and the log-sum-exp.
+ *       pairs, with an online softmax, producing O and the log-sum-exp,
+ *   (e) its backward (dQ, dK, dV) over the same kept pairs,
+ *   (f) SPADE scheme generation (SICS per block for a menu of 3D slice shapes
+ *       and the per-head choice), and
+ *   (g) a paged key/value cache with persistent anchors for autoregressive
+ *       chunk decoding (page writes, block means, page importance, keep/evict,
+ *       attention through the page table).
  *
  * Conventions for every entry point
  *   - All tensor pointers are DEVICE pointers owned by the caller; the library
@@ -354,8 +360,10 @@ int bsa_sics_scheme(const void* q, const void* k, int batch, int T, int H, int W
  *   pages_per_batch >= n_pages entries.  Per batch, pages < anchor_pages and
  *   >= recent_begin are kept; of the resident pages in between the `budget` highest scores are kept
  *   (ties: the lower page) and every other one is evicted: its page_table entry
- *   becomes -1 and its physical page is appended to freed[] (capacity: batch *
- *   (recent_begin - anchor_pages) ints) at index atomicAdd(freed_count, 1).
+ *   becomes -1 and its physical page is appended to freed[] at index
+ *   atomicAdd(freed_count, 1).  *freed_count is not cleared by the call, so
+ *   freed[] needs room for batch * (recent_begin - anchor_pages - budget) ints
+ *   past its current value (zero it first to start at freed[0]).
  *   recent_begin - anchor_pages <= 8192.
  * bsa_attn_fwd_paged: bsa_attn_fwd with K and V read through the page table
  *   from one-batch pools [n_pool_pages * 128, heads, head_dim]; key blocks on
