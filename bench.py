@@ -462,6 +462,24 @@ def mask_stats(flops: float, w, nq: int, nk: int, attn_times_ms, near=None) -> d
     return out
 
 
+def permute_bandwidth(w, plan, stage_ms: dict, hbm_peak: float):
+    """Algorithmic GB/s of the tile permute (Q, K, V: N rows read, n_pad rows
+    written, the zero tail included) and of the untile (O: N rows read and
+    written), with the fraction of the HBM peak; None without a tile order."""
+    if not plan.permuted:
+        return None
+    row = w.heads * w.head_dim * 2
+    n, n_pad = w.n_tokens, plan.n_pad
+    out = {}
+    for name, nbytes in (("permute", 3 * w.batch * (n + n_pad) * row),
+                         ("untile", 2 * w.batch * n * row)):
+        ms = stage_ms[name]
+        gbs = nbytes / (ms * 1e-3) / 1e9 if ms > 0 else None
+        out[name] = {"bytes": nbytes, "gb_s": gbs,
+                     "frac_of_hbm": gbs / hbm_peak if gbs else None}
+    return out
+
+
 def workload_config(w, pass_: str = "fwd"):
     cfg = {"workload": w.name, "batch": w.batch, "heads": w.heads, "head_dim": w.head_dim,
            "grid_thw": list(w.grid), "block": w.block, "mask": w.mask}
@@ -1060,7 +1078,8 @@ def main():
                 "mask_stats": mask_stats(flops, w, plan.nq, plan.nk, attn_times,
                                          plan.near.item() if hasattr(plan, "near") else None),
                 # mean device time of each stage of a timed step (this rank, CUDA events)
-                "stage_ms": stage_ms}
+                "stage_ms": stage_ms,
+                "stage_gbs": permute_bandwidth(w, plan, stage_ms, peaks["hbm_gbs"])}
         print(json.dumps(line))
     if world > 1:
         dist.destroy_process_group()

@@ -74,3 +74,19 @@ def test_paged_pass_refuses_a_workload_without_ar_decoding():
                           "--pass", "ar_paged", "--workload", "sta_tiny", "--steps", "1"],
                          capture_output=True, text=True, timeout=600, cwd=ROOT)
     assert out.returncode == 2 and "autoregressive" in out.stderr
+
+
+def test_permute_bandwidth_counts_the_algorithmic_bytes():
+    from types import SimpleNamespace
+    sys.path.insert(0, ROOT)
+    import bench
+    from block_sparse_attention_tokens_b200 import configs
+    w = configs.get("sta_720p")
+    plan = SimpleNamespace(permuted=True, n_pad=115200)
+    row = 24 * 128 * 2
+    got = bench.permute_bandwidth(w, plan, {"permute": 0.714, "untile": 0.235}, 6543.4)
+    assert got["permute"]["bytes"] == 3 * 2 * 115200 * row       # Q, K, V read + written
+    assert got["untile"]["bytes"] == 2 * 115200 * row             # O read + written
+    assert abs(got["permute"]["gb_s"] - 3 * 2 * 115200 * row / 0.714e-3 / 1e9) < 1e-6
+    assert 0.9 < got["permute"]["frac_of_hbm"] < 0.92
+    assert bench.permute_bandwidth(w, SimpleNamespace(permuted=False), {}, 6543.4) is None
