@@ -493,7 +493,8 @@ def block_sparse_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, mask: np
 # 8. Backward of the block-sparse attention (training)
 # ---------------------------------------------------------------------------
 
-def block_sparse_attention_backward(q, k, v, do, mask, block_q, block_k, scale=None, rows=None):
+def block_sparse_attention_backward(q, k, v, do, mask, block_q, block_k, scale=None, rows=None,
+                                    cols=None):
     """Gradients of O = softmax(Q K^T * scale + M) V with respect to Q, K, V.
 
     The Radial explainer (section 4, training cost), the NABLA explainer
@@ -507,6 +508,11 @@ def block_sparse_attention_backward(q, k, v, do, mask, block_q, block_k, scale=N
     ``rows`` (optional): evaluate only these query rows -- dq is exact on them (0
     elsewhere) and dk, dv hold only their contributions (for sampled checks at
     full size).
+    ``cols`` (optional): key rows whose dk and dv are wanted -- only query blocks
+    that keep a block holding one of them are evaluated (each over its whole kept
+    row, since P and rowsum(dO * O) need every kept key), so dk and dv are exact
+    on these keys; dq, and dk / dv at other keys, hold only the evaluated rows'
+    contributions.
     Returns (dq, dk, dv) with the shapes of q, k, v.
     """
     Bn, nq, H, D = q.shape
@@ -515,6 +521,7 @@ def block_sparse_attention_backward(q, k, v, do, mask, block_q, block_k, scale=N
     dq = np.zeros_like(q)
     dk = np.zeros_like(k)
     dv = np.zeros_like(v)
+    want_kb = None if cols is None else np.unique(np.asarray(cols, dtype=np.int64) // block_k)
     for b in range(Bn):
         for h in range(H):
             m = mask[0 if mask.shape[0] == 1 else b * H + h]
@@ -525,20 +532,22 @@ def block_sparse_attention_backward(q, k, v, do, mask, block_q, block_k, scale=N
                 kept = np.nonzero(m[qb])[0]
                 if kept.size == 0 or rows_b.size == 0:
                     continue
+                if want_kb is not None and np.intersect1d(kept, want_kb).size == 0:
+                    continue
                 rows_ = rows_b
-                cols = np.concatenate([np.arange(kb * block_k, min((kb + 1) * block_k, nk))
+                keys = np.concatenate([np.arange(kb * block_k, min((kb + 1) * block_k, nk))
                                        for kb in kept])
-                s = (q[b, rows_, h] @ k[b, cols, h].T) * scale
+                s = (q[b, rows_, h] @ k[b, keys, h].T) * scale
                 s = s - s.max(axis=1, keepdims=True)
                 p = np.exp(s)
                 p /= p.sum(axis=1, keepdims=True)
-                o = p @ v[b, cols, h]
+                o = p @ v[b, keys, h]
                 g = do[b, rows_, h]
-                dv[b, cols, h] += p.T @ g
-                dp = g @ v[b, cols, h].T
+                dv[b, keys, h] += p.T @ g
+                dp = g @ v[b, keys, h].T
                 ds = p * (dp - (g * o).sum(axis=1, keepdims=True))
-                dq[b, rows_, h] += (ds @ k[b, cols, h]) * scale
-                dk[b, cols, h] += (ds.T @ q[b, rows_, h]) * scale
+                dq[b, rows_, h] += (ds @ k[b, keys, h]) * scale
+                dk[b, keys, h] += (ds.T @ q[b, rows_, h]) * scale
     return dq, dk, dv
 
 

@@ -140,14 +140,50 @@ def test_sta_mask_on_a_tiled_grid():
     run_bwd(1, 2, 256, 256, 128, 64, 64, m, 1, seed=13)
 
 
-def test_full_size_sta_720p_sampled_rows_and_identities():
+def key_envelopes(qh, kh, vh, doh, mask, block, keys, sc):
+    """Envelopes of dK and dV (module docstring) on the given key rows of one head:
+    every query block that keeps one of their blocks is evaluated over its whole
+    kept row (P, dP, Delta and W need all of the row's keys).  Arrays [1, n, 1, D]."""
+    nq, nk = qh.shape[1], kh.shape[1]
+    want = np.unique(keys // block)
+    env_k = np.zeros((len(keys), qh.shape[-1]))
+    env_v = np.zeros_like(env_k)
+    for qb in range(mask.shape[1]):
+        kept = np.nonzero(mask[0, qb])[0]
+        if not np.isin(want, kept).any():
+            continue
+        rows = np.arange(qb * block, min((qb + 1) * block, nq))
+        cols = np.concatenate([np.arange(kb * block, min((kb + 1) * block, nk)) for kb in kept])
+        qq, kk, vv, g = qh[0, rows, 0], kh[0, cols, 0], vh[0, cols, 0], doh[0, rows, 0]
+        s = (qq @ kk.T) * sc
+        p = np.exp(s - s.max(axis=1, keepdims=True))
+        p /= p.sum(axis=1, keepdims=True)
+        o = p @ vv
+        dp = g @ vv.T
+        delta = (g * o).sum(axis=1)
+        w = (np.abs(g) * (p @ np.abs(vv) + np.abs(o))).sum(axis=1)
+        e = p * (np.abs(dp) + np.abs(delta)[:, None] + w[:, None])
+        idx = np.minimum(np.searchsorted(cols, keys), cols.size - 1)   # cols ascending
+        hit = cols[idx] == keys
+        env_v[hit] += p[:, idx[hit]].T @ np.abs(g)
+        env_k[hit] += sc * (e[:, idx[hit]].T @ np.abs(qq))
+    return env_k, env_v
+
+
+def test_full_size_sta_720p_sampled_rows_keys_and_identities():
     """The 720p Sliding-Tile workload at full size (24 heads, 115,200 tokens, the
-    benchmark's launch): dQ on sampled rows against the oracle within the per-entry
-    envelope, and two identities that hold at any size and involve every dK and dV
-    entry: sum_i q_i . dQ_i = sum_j k_j . dK_j (both equal scale * sum dS_ij q_i.k_j)
-    and sum_j dV_j = sum of dO_i over rows that keep a key (probability rows sum to
-    1).  The identities are coarse (1 % of the absolute sums) -- they catch a lost
-    quadrant, term or factor, not rounding."""
+    benchmark's launch), element by element within the per-entry envelope:
+    dQ on sampled query rows and dK, dV on every key of sampled 128-key tiles,
+    against the oracle (its key sampling evaluates every query block that keeps a
+    sampled key).  Both kernel passes are persistent (one CTA per SM takes work
+    items in (head, tile) order from a global counter), so every item past the
+    first SM-count ones -- all of head 13's, and head 0's tiles beyond the first
+    148 -- is a CTA's second or later item: barrier phases, TMEM reuse and the
+    transposed lists at scale are compared, not only summed.  Two identities that
+    involve every dK and dV entry follow: sum_i q_i . dQ_i = sum_j k_j . dK_j (both
+    equal scale * sum dS_ij q_i.k_j) and sum_j dV_j = sum of dO_i over rows that
+    keep a key; they are coarse (1 % of the absolute sums) and catch a lost
+    quadrant, term or factor anywhere."""
     from block_sparse_attention_tokens_b200 import configs
     from block_sparse_attention_tokens_b200.pipeline import Plan
     w = configs.get("sta_720p")
@@ -166,7 +202,14 @@ def test_full_size_sta_720p_sampled_rows_and_identities():
     rng = np.random.default_rng(3)
     qbs = [0, plan.QB - 1] + list(rng.choice(plan.QB, 2, replace=False))
     rows = np.unique(np.concatenate([qb * w.block + np.array([0, 191, w.block - 1]) for qb in qbs]))
+    # 8 key tiles of 128 keys: the first and last, and two of the three tiles of
+    # three random 384-key blocks
+    KT = math.ceil(w.nk / 128)
+    kbs = rng.choice(np.arange(1, plan.QB - 1), 3, replace=False)
+    tiles = [0, KT - 1] + [int(kb) * 3 + t for kb in kbs for t in (0, 2)]
+    keys = np.unique(np.concatenate([np.arange(t * 128, min((t + 1) * 128, w.nk)) for t in tiles]))
     dq_g = to64(dq[:, :w.nq])
+    dk_g, dv_g = to64(dk[:, :w.nk]), to64(dv[:, :w.nk])
     for h in (0, 13):
         qh = O.tile_permute(to64(q[:, :, h:h + 1]), perm, plan.n_pad)[:, :w.nq]
         kh = O.tile_permute(to64(k[:, :, h:h + 1]), perm, plan.n_pad)[:, :w.nk]
@@ -187,16 +230,20 @@ def test_full_size_sta_720p_sampled_rows_and_identities():
             env = sc * ((p * (np.abs(dp) + abs(delta) + wi)) @ np.abs(kk))
             err = np.abs(dq_g[0, i, h] - rdq[0, i, 0])
             assert np.all(err <= 4 * U * env + 2 * U * np.abs(rdq[0, i, 0])), (h, i)
+        # dK and dV of the sampled key tiles
+        _, rdk, rdv = O.block_sparse_attention_backward(qh, kh, vh, doh, mask, w.block, w.block,
+                                                        cols=keys)
+        env_k, env_v = key_envelopes(qh, kh, vh, doh, mask, w.block, keys, sc)
+        assert_grad_close(dk_g[0, keys, h], rdk[0, keys, 0], env_k, f"dK head {h}")
+        assert_grad_close(dv_g[0, keys, h], rdv[0, keys, 0], env_v, f"dV head {h}")
     # identities over all heads and every entry of dK and dV
-    qp, kp, vpd = to64(plan.qp[:, :w.nq]), to64(plan.kp[:, :w.nk]), to64(dv[:, :w.nk])
-    dkg = to64(dk[:, :w.nk])
+    qp, kp, vpd = to64(plan.qp[:, :w.nq]), to64(plan.kp[:, :w.nk]), dv_g
     lhs = np.einsum("bnhd,bnhd->h", qp, dq_g)
-    rhs = np.einsum("bnhd,bnhd->h", kp, dkg)
+    rhs = np.einsum("bnhd,bnhd->h", kp, dk_g)
     scale_abs = (np.einsum("bnhd,bnhd->h", np.abs(qp), np.abs(dq_g))
-                 + np.einsum("bnhd,bnhd->h", np.abs(kp), np.abs(dkg)))
+                 + np.einsum("bnhd,bnhd->h", np.abs(kp), np.abs(dk_g)))
     assert np.all(np.abs(lhs - rhs) <= 1e-2 * scale_abs)
     do64 = to64(do)
     dv_sum = vpd.sum(axis=1)
     do_sum = do64.sum(axis=1)                       # every STA query row keeps keys
     assert np.all(np.abs(dv_sum - do_sum) <= 1e-2 * np.abs(do64).sum(axis=1))
-

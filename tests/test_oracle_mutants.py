@@ -220,15 +220,15 @@ MUTANTS = [
            "ds = p * (dp - (g * o).sum(axis=1, keepdims=True))", "ds = p * dp",
            [pin(TN.test_backward_matches_autograd_float64, bq=64, bk=64)]),
     Mutant("bwd/dk-scale-dropped", "block_sparse_attention_backward",
-           "dk[b, cols, h] += (ds.T @ q[b, rows_, h]) * scale",
-           "dk[b, cols, h] += (ds.T @ q[b, rows_, h])",
+           "dk[b, keys, h] += (ds.T @ q[b, rows_, h]) * scale",
+           "dk[b, keys, h] += (ds.T @ q[b, rows_, h])",
            [pin(TN.test_backward_matches_autograd_float64, bq=64, bk=64)]),
     Mutant("bwd/dv-from-output", "block_sparse_attention_backward",
-           "dv[b, cols, h] += p.T @ g", "dv[b, cols, h] += p.T @ o",
+           "dv[b, keys, h] += p.T @ g", "dv[b, keys, h] += p.T @ o",
            [pin(TN.test_backward_matches_autograd_float64, bq=64, bk=64)]),
     Mutant("bwd/dq-with-v", "block_sparse_attention_backward",
-           "dq[b, rows_, h] += (ds @ k[b, cols, h]) * scale",
-           "dq[b, rows_, h] += (ds @ v[b, cols, h]) * scale",
+           "dq[b, rows_, h] += (ds @ k[b, keys, h]) * scale",
+           "dq[b, rows_, h] += (ds @ v[b, keys, h]) * scale",
            [pin(TN.test_backward_matches_autograd_float64, bq=64, bk=64)]),
     Mutant("bwd/default-scale-1-over-d", "block_sparse_attention_backward",
            "scale = 1.0 / math.sqrt(D) if scale is None else scale",
@@ -237,6 +237,13 @@ MUTANTS = [
     Mutant("bwd/row-sample-ignored", "block_sparse_attention_backward",
            "rows_b = np.intersect1d(rows_b, np.asarray(rows))", "rows_b = rows_b",
            [pin(TN.test_backward_row_sampling_is_exact_on_dq_and_additive_on_dk_dv)]),
+    Mutant("bwd/col-sample-in-query-blocks", "block_sparse_attention_backward",
+           "np.asarray(cols, dtype=np.int64) // block_k", "np.asarray(cols, dtype=np.int64) // block_q",
+           [pin(TN.test_backward_column_sampling_is_exact_on_dk_dv)]),
+    Mutant("bwd/col-sample-softmax-over-wanted-blocks-only", "block_sparse_attention_backward",
+           "                                       for kb in kept])\n                s = (q",
+           "                                       for kb in (kept if want_kb is None else np.intersect1d(kept, want_kb))])\n                s = (q",
+           [pin(TN.test_backward_column_sampling_is_exact_on_dk_dv)]),
 
     # ------------------------------------------------------------ SICS
     Mutant("tile_tokens/ragged-edge-overrun", "tile_tokens",

@@ -304,3 +304,32 @@ def test_backward_row_sampling_is_exact_on_dq_and_additive_on_dk_dv():
     assert np.all(ga[0][:, rows_b] == 0)
     for i in (1, 2):                                    # dK, dV: the two halves add up
         assert np.allclose(ga[i] + gb[i], full[i], atol=1e-12)
+
+
+def test_backward_column_sampling_is_exact_on_dk_dv():
+    # key sampling evaluates every query block that keeps a wanted key's block, each
+    # over its whole kept row: dk and dv on the wanted keys equal the full evaluation
+    Bn, H, D, bq, bk = 1, 2, 16, 128, 64
+    nq, nk = 300, 330
+    q, k, v = _rand_qkv(Bn, nq, nk, H, D, 41)
+    do = np.random.default_rng(42).standard_normal((Bn, nq, H, D))
+    QB, KB = math.ceil(nq / bq), math.ceil(nk / bk)
+    mask = (np.random.default_rng(43).random((Bn * H, QB, KB)) < 0.6).astype(np.uint8)
+    mask[:, :, 2] = 0
+    mask[:, 0, 2] = 1                                   # block 2: only query block 0
+    mask[:, :, 4:] = 1
+    mask[:, 0, 4:] = 0                                  # blocks 4, 5: query blocks 1, 2
+    mask[1, :, 4] = 0                                   # head 1: block 4 kept by nobody
+    full = O.block_sparse_attention_backward(q, k, v, do, mask, bq, bk)
+    cols = np.array([4 * bk, 4 * bk + 37, 5 * bk + 3, nk - 1])
+    part = O.block_sparse_attention_backward(q, k, v, do, mask, bq, bk, cols=cols)
+    for i in (1, 2):
+        assert np.allclose(part[i][:, cols], full[i][:, cols], atol=1e-12, rtol=0)
+        assert np.any(part[i][:, cols] != 0)
+    assert np.all(part[1][0, 4 * bk, 1] == 0) and np.all(part[2][0, 4 * bk, 1] == 0)
+    # rows of query blocks that keep none of the wanted blocks are not evaluated
+    wanted = np.unique(cols // bk)
+    for h in range(H):
+        for qb in range(QB):
+            if not mask[h, qb, wanted].any():
+                assert np.all(part[0][0, qb * bq:(qb + 1) * bq, h] == 0)
