@@ -152,10 +152,15 @@ def _buffer(t: torch.Tensor, name: str, dtype, numel: int):
         raise ValueError(f"{name} holds {t.numel()} elements, {numel} needed")
 
 
-def _lists(row_ptr: torch.Tensor, col_idx: torch.Tensor, list_heads: int, nq: int, block_q: int):
-    """Kept lists: row_ptr has one entry per (list head, query block) plus one."""
-    _buffer(row_ptr, "row_ptr", torch.int32, list_heads * (-(-nq // block_q)) + 1)
-    _buffer(col_idx, "col_idx", torch.int32, 1)
+def _lists(row_ptr: torch.Tensor, col_idx: torch.Tensor, list_heads: int, nq: int, block_q: int,
+           nk: int, block_k: int):
+    """Kept lists: row_ptr has one entry per (list head, query block) plus one;
+    col_idx has room for every (list head, query block, key block), the worst case
+    bsa_mask_compact writes, because the library trusts row_ptr up to that bound
+    (checking the actual count would need a device synchronisation)."""
+    QB, KB = -(-nq // block_q), -(-nk // block_k)
+    _buffer(row_ptr, "row_ptr", torch.int32, list_heads * QB + 1)
+    _buffer(col_idx, "col_idx", torch.int32, list_heads * QB * KB)
 
 
 def _means(t: torch.Tensor, name: str, batch: int, heads: int, head_dim: int):
@@ -407,7 +412,7 @@ def bsa_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, row_ptr: tor
     _tokens(q, "q", B, nq, H, D)
     _tokens(k, "k", B, nk, H, D)
     _tokens(v, "v", B, nk, H, D)
-    _lists(row_ptr, col_idx, list_heads, nq, block_q)
+    _lists(row_ptr, col_idx, list_heads, nq, block_q, nk, block_k)
     if o is None:
         o = torch.empty_like(q)
     if lse is None:
@@ -442,7 +447,7 @@ def bsa_attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     _tokens(q, "q", B, nq, H, D)
     _tokens(k, "k", B, nk, H, D)
     _tokens(v, "v", B, nk, H, D)
-    _lists(row_ptr, col_idx, list_heads, nq, block_q)
+    _lists(row_ptr, col_idx, list_heads, nq, block_q, nk, block_k)
     if o is None:
         o = torch.empty_like(q)
     if lse is None:
@@ -479,7 +484,7 @@ def bsa_attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Ten
                        (dout, "dout", nq)):
         _tokens(t, n, B, rows, H, D)
     _buffer(lse, "lse", torch.float32, B * H * nq)
-    _lists(row_ptr, col_idx, list_heads, nq, block_q)
+    _lists(row_ptr, col_idx, list_heads, nq, block_q, nk, block_k)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
@@ -672,7 +677,7 @@ def bsa_attn_fwd_paged(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tens
     if v_pool.shape[0] != k_pool.shape[0]:
         raise ValueError("k_pool and v_pool must hold the same number of pages")
     _table(page_table, "page_table", B)
-    _lists(row_ptr, col_idx, list_heads, nq, block_q)
+    _lists(row_ptr, col_idx, list_heads, nq, block_q, nk, block_k)
     if o is None:
         o = torch.empty_like(q)
     if lse is None:

@@ -796,18 +796,31 @@ namespace {
 // Shared body of bsa_attn_fwd and bsa_attn_fwd_paged.  page_table == nullptr: K/V
 // are [batch, nk, heads, head_dim]; else they are one-batch pools of n_pool_pages
 // 128-token pages addressed through page_table [batch][pages_per_batch].
+// Argument checks of the forward that need no workspace, in the order every
+// forward entry point applies them: pointers, sizes, list heads, alignment
+// (BSA_ERR_INVALID_ARG), then head_dim and block sizes (BSA_ERR_UNSUPPORTED).
+int check_fwd_args(const void* q, const void* k, const void* v, int batch, int heads, int nq,
+                   int nk, int head_dim, int block_q, int block_k, const int* row_ptr,
+                   const int* col_idx, int list_heads, const void* o, const float* lse) {
+  if (!q || !k || !v || !o || !lse || !row_ptr || !col_idx) return BSA_ERR_INVALID_ARG;
+  if (batch < 1 || heads < 1 || nq < 1 || nk < 1) return BSA_ERR_INVALID_ARG;
+  if (list_heads != 1 && list_heads != batch * heads) return BSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return BSA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return BSA_ERR_UNSUPPORTED;
+  if (!block_ok(block_q) || !block_ok(block_k)) return BSA_ERR_UNSUPPORTED;
+  return BSA_OK;
+}
+
 int attn_fwd_impl(const void* q, const void* k, const void* v, int batch, int heads, int nq,
                   int nk, int head_dim, int block_q, int block_k, const int* row_ptr,
                   const int* col_idx, int list_heads, float scale, void* o, float* lse, void* ws,
                   size_t ws_bytes, const int* page_table, int pages_per_batch, int n_pool_pages,
                   cudaStream_t st) {
-  if (!q || !k || !v || !o || !lse || !row_ptr || !col_idx || !ws) return BSA_ERR_INVALID_ARG;
-  if (batch < 1 || heads < 1 || nq < 1 || nk < 1) return BSA_ERR_INVALID_ARG;
-  if (list_heads != 1 && list_heads != batch * heads) return BSA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(ws))
-    return BSA_ERR_INVALID_ARG;
-  if (head_dim != 64 && head_dim != 128) return BSA_ERR_UNSUPPORTED;
-  if (!block_ok(block_q) || !block_ok(block_k)) return BSA_ERR_UNSUPPORTED;
+  if (!ws) return BSA_ERR_INVALID_ARG;
+  int rc0 = check_fwd_args(q, k, v, batch, heads, nq, nk, head_dim, block_q, block_k, row_ptr,
+                           col_idx, list_heads, o, lse);
+  if (rc0 != BSA_OK) return rc0;
+  if (!aligned16(ws)) return BSA_ERR_INVALID_ARG;
   if (page_table) {
     // pages hold whole key blocks; a shared list needs a single page table
     if (block_k > kBN || (list_heads == 1 && batch > 1)) return BSA_ERR_UNSUPPORTED;
@@ -917,22 +930,54 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB per device
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-// Device address of g_noalloc_scratch for the current device, resolved on the
-// first call made with that device current (the host-side name of a __device__
-// array is only a stand-in, never a device address).
+// Device address of g_noalloc_scratch in the current device's context, looked up
+// with cudaGetSymbolAddress (the host-side name of a __device__ array is only a
+// stand-in, never a device address) on the first call made with that device
+// current, and again whenever the calling thread's current context is not the one
+// the cached address was taken in: after a cudaDeviceReset the module is loaded
+// anew and the array may move.  Contexts are told apart by their process-unique
+// ids (cuCtxGetId), which a re-created context never repeats.
 int noalloc_scratch(void** out) {
   static std::mutex mu;
   static void* addr[64] = {nullptr};
+  static unsigned long long ctx_id_of[64] = {0};
+  static PFN_cuCtxGetCurrent_v4000 get_ctx = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_ctx = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(fn);
+    fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(fn);
+  });
+  if (!get_ctx || !get_id) return BSA_ERR_CUDA;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return record_cuda_error(e);
   if (dev < 0 || dev >= 64) return BSA_ERR_UNSUPPORTED;
+  // id of the calling thread's current context; 0 when the runtime has not bound
+  // one to this thread yet (the symbol lookup below does)
+  auto current_id = [&]() -> unsigned long long {
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (get_ctx(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+  };
+  unsigned long long id = current_id();
   std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
+  if (!addr[dev] || id == 0 || ctx_id_of[dev] != id) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return record_cuda_error(e);
+    id = current_id();
+    if (id == 0) return BSA_ERR_CUDA;
     addr[dev] = p;
+    ctx_id_of[dev] = id;
   }
   *out = addr[dev];
   return BSA_OK;
@@ -948,6 +993,10 @@ extern "C" int bsa_attn_fwd_noalloc(const void* q, const void* k, const void* v,
                                     int* device_status, void* stream) {
   BSA_NVTX_RANGE("bsa_attn_fwd_noalloc");
   using namespace bsa;
+  // the same argument checks, in the same order, as bsa_attn_fwd before the size check
+  int rc = check_fwd_args(q, k, v, batch, heads, nq, nk, head_dim, block_q, block_k, row_ptr,
+                          col_idx, list_heads, o, lse);
+  if (rc != BSA_OK) return rc;
   const size_t need =
       bsa_attn_workspace_size(batch, heads, nq, nk, block_q, block_k, list_heads);
   if (need == 0) return BSA_ERR_INVALID_ARG;
@@ -957,7 +1006,7 @@ extern "C" int bsa_attn_fwd_noalloc(const void* q, const void* k, const void* v,
     return BSA_ERR_WORKSPACE;
   }
   void* scratch = nullptr;
-  int rc = noalloc_scratch(&scratch);
+  rc = noalloc_scratch(&scratch);
   if (rc != BSA_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   rc = bsa_attn_fwd(q, k, v, batch, heads, nq, nk, head_dim, block_q, block_k, row_ptr, col_idx,

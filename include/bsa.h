@@ -280,9 +280,14 @@ int bsa_attn_bwd(const void* q, const void* k, const void* v, const void* o, con
  * the process exits.
  *   - Shapes whose bsa_attn_workspace_size() exceeds 8 MiB are rejected with
  *     BSA_ERR_WORKSPACE (see bsa_last_error_message()) before any work.
+ *   - Arguments are checked as bsa_attn_fwd checks them, in the same order and
+ *     with the same codes, before the size check.
  *   - The first call made with a given device current looks up that device's
  *     array address (cudaGetSymbolAddress); make that first call before any
- *     stream capture.
+ *     stream capture.  The address is looked up again when the calling
+ *     thread's current context differs from the one it was taken in (e.g.
+ *     after cudaDeviceReset), so the first call after such a reset also belongs
+ *     before any capture.
  *   - All calls share the one array per device: calls that can overlap on the
  *     GPU (different streams without ordering) race and must be serialised by
  *     the caller.  Everything the call needs zeroed is cleared by the call.

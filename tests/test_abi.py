@@ -110,10 +110,15 @@ def test_every_entry_rejects_bad_arguments_before_touching_cuda(lib, no_gpu):
     args[6], args[15] = 2, 1
     assert lib.bsa_attn_fwd_paged(*args) == UNS                  # one shared list, two page tables
     # allocation-free forward: q k v B H nq nk d bq bk row_ptr col_idx list_heads scale o lse status
+    # (the same checks, order and codes as bsa_attn_fwd come before the size check)
     na = [A, A, A, 1, 40, 453600, 453600, 128, 96, 128, A, A, 40, 0.0, A, A, A, None]
-    assert lib.bsa_attn_fwd_noalloc(*na) == INV                  # block 96: no workspace size
+    assert lib.bsa_attn_fwd_noalloc(*na) == UNS                  # block 96, as bsa_attn_fwd
     na[8] = 128
     assert lib.bsa_attn_fwd_noalloc(*na) == WS                   # needs more than the fixed 8 MiB
+    for i, val, rc in ((0, U, INV), (14, None, INV), (7, 96, UNS), (12, 3, INV), (10, None, INV)):
+        args = list(na)
+        args[i] = val
+        assert lib.bsa_attn_fwd_noalloc(*args) == rc, (i, val)   # refused before the size
     # NABLA: select (qbar kbar B H QB KB d p scale kb_begin kb_end force base allowed mask near)
     sel = [A, A, 1, 2, 8, 8, 128, 0.9, 0.0, 0, 8, 0, None, None, A, None, None]
     for i, val, rc in ((7, 0.0, INV), (6, 96, UNS), (10, 9, INV), (9, 5, INV), (0, None, INV)):

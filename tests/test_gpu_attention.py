@@ -94,7 +94,7 @@ def test_all_masked_everywhere():
 def test_invalid_kept_list_is_reported_not_faulted():
     q = torch.randn(1, 256, 1, 128).to(torch.bfloat16).cuda()
     rp = torch.tensor([0, 2, 3], dtype=torch.int32).cuda()
-    ci = torch.tensor([1, 0, 7], dtype=torch.int32).cuda()   # descending row, out-of-range block
+    ci = torch.tensor([1, 0, 7, 0], dtype=torch.int32).cuda()  # descending row, out-of-range block
     o, lse, ws = B.bsa_attn_fwd(q, q, q, rp, ci, 128, 128, 1)
     torch.cuda.synchronize()
     assert B.bsa_read_status(ws) == 1
