@@ -6,8 +6,11 @@
 One step = one pass of the whole path over one batch of synthetic input already
 resident in HBM: tile permute of Q, K, V -> block mask -> CSR compaction ->
 block-sparse attention forward -> inverse permute of O.  The default workload is
-the Sliding-Tile 720p DiT shape (1 x 24 heads x 128, 30x48x80 tokens, 6x8x8
-tiles of 384 tokens, 3x3x5-tile window).  Metric: effective TFLOP/s =
+the largest single-GPU one: the radial (energy-decay) mask at 500 frames of
+720p video (1 x 12 heads x 128, 126x45x80 = 453,600 tokens in raster order,
+128-token blocks); ``--workload sta_720p`` is the Sliding-Tile 720p DiT shape
+(1 x 24 heads x 128, 30x48x80 tokens, 6x8x8 tiles of 384 tokens, 3x3x5-tile
+window), ``nabla_480p`` and ``ar_decode`` the dynamic-mask ones.  Metric: effective TFLOP/s =
 4 * head_dim * (query, key) pairs inside kept blocks / time.
 
 ``--pass sics`` times SPADE scheme generation (SICS of Q and K under every shape
@@ -54,6 +57,38 @@ NOMINAL_PEAKS = {"TFLOP/s": 2250.0, "GB/s": 7700.0}
 def with_nominal(roofline: dict) -> dict:
     roofline["frac_of_nominal"] = roofline["achieved"] / NOMINAL_PEAKS[roofline["unit"]]
     return roofline
+
+
+def choose_tensor_peak(peaks: dict, clocks: dict, timed_s: float):
+    """The bf16 peak a kernel timed in this run is held to: the burst figure
+    (a GEMM timed alone, at the maximum clock) when the timed region was short
+    (under 3 s) or the median SM clock stayed within 3 % of the maximum, else the
+    sustained figure (a seconds-long GEMM loop under the power cap)."""
+    mhz, mx = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+    at_max = bool(mhz and mx and mhz >= 0.97 * mx)
+    if timed_s < 3.0 or at_max:
+        why = "timed region under 3 s" if timed_s < 3.0 else "median SM clock at its maximum"
+        return peaks["bf16_tflops"], "burst", why
+    return peaks["bf16_tflops_sustained"], "sustained", \
+        f"{timed_s:.1f} s timed region, median SM clock {mhz} of {mx} MHz"
+
+
+def tensor_roofline(achieved: float, kernel_ms: float, peaks: dict, peak_kind: str,
+                    clocks: dict, timed_s: float, **extra) -> dict:
+    """Roofline object of a tensor-bound kernel: frac against the peak that
+    choose_tensor_peak picks, the fractions of both measured figures, and the
+    kernel's mean time times the median SM clock (ms x MHz = thousands of SM
+    cycles), which compares runs taken at different clocks."""
+    peak, kind, why = choose_tensor_peak(peaks, clocks, timed_s)
+    mhz = clocks.get("sm_mhz")
+    r = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+         "frac": achieved / peak,
+         "peak_note": f"{peak_kind} {kind} bf16 ({why})",
+         "frac_of_burst": achieved / peaks["bf16_tflops"],
+         "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
+         "kernel_ms_x_sm_mhz": kernel_ms * mhz if mhz else None}
+    r.update(extra)
+    return with_nominal(r)
 
 
 def load_peaks():
@@ -153,12 +188,61 @@ def cpu_cores() -> int:
         return os.cpu_count() or 1
 
 
+def oracle_workload_mask(w, q, k):
+    """The oracle's own block mask of the workload, [Hm, QB, KB] uint8 (Hm = 1 for
+    the static masks, batch * heads otherwise), from the raster-order bf16 inputs:
+    the Sliding-Tile window, the radial rule, NABLA (per-head pooled means of the
+    tile-ordered Q and K), NABLA united with the window, or the autoregressive
+    composition."""
+    import numpy as np
+    import oracle as O
+    QB, KB = math.ceil(w.nq / w.block), math.ceil(w.nk / w.block)
+    if w.tile is not None:
+        perm = O.tile_order(w.grid, w.tile)
+        n_pad = QB * w.block
+        tg = tuple(math.ceil(g / t) for g, t in zip(w.grid, w.tile))
+    if w.mask == "sta":
+        return O.sta_tile_mask(tg, w.window)[None]
+    if w.mask == "radial":
+        return O.radial_block_mask_fast(w.nk, w.tokens_per_frame, w.block)[None]
+    D = w.head_dim
+    scale = 1.0 / math.sqrt(D)
+    qbar = np.zeros((w.batch, w.heads, QB, D))
+    kbar = np.zeros((w.batch, w.heads, KB, D))
+    for h in range(w.heads):
+        qh = q[:, :, h:h + 1].double().numpy()
+        kh = k[:, :, h:h + 1].double().numpy()
+        if w.tile is not None:
+            qh, kh = O.tile_permute(qh, perm, n_pad), O.tile_permute(kh, perm, n_pad)
+        else:
+            qh = np.concatenate([qh, np.zeros((w.batch, QB * w.block - w.nq, 1, D))], axis=1)
+            kh = np.concatenate([kh, np.zeros((w.batch, KB * w.block - w.nk, 1, D))], axis=1)
+        qbar[:, h] = O.nabla_pool(qh, w.block, w.nq)[:, 0]
+        kbar[:, h] = O.nabla_pool(kh, w.block, w.nk)[:, 0]
+    if w.mask == "nabla":
+        m, _ = O.nabla_mask(qbar, kbar, w.p, scale)
+    elif w.mask == "nabla_sta":
+        m, _ = O.nabla_sta_mask(qbar, kbar, w.p, scale, O.sta_tile_mask(tg, w.window))
+    elif w.mask == "ar":
+        m, _ = O.ar_mask(qbar, kbar, w.p, scale, w.nk, w.tokens_per_frame, w.block,
+                         w.anchor_frames, w.recent_frames)
+    else:
+        raise ValueError(w.mask)
+    return m.reshape(-1, QB, KB).astype(np.uint8)
+
+
 class OracleSample:
     """The CPU oracle on whole query blocks of the workload (all heads).
 
-    Setup (untimed): the oracle's own mask and float64, tile-ordered copies of
-    Q, K, V per head.  ``run(budget_s)`` evaluates random query blocks until about
-    budget_s seconds of oracle work and returns (effective TFLOP/s, sample text).
+    Setup (untimed): the oracle's own mask of the workload (for NABLA and the
+    autoregressive mask this runs the oracle's pooling and top-p selection) and,
+    for tiled workloads, the oracle's tile order.  ``run(budget_s)`` evaluates
+    random query blocks until about budget_s seconds of oracle work: per block and
+    head, the block's query rows and the keys of its kept blocks are gathered from
+    the bf16 inputs in the path's token order and upcast to float64 (untimed), and
+    the oracle's attention is timed on them -- the same rows over the same kept
+    keys as a call on the whole sequence, without holding float64 copies of it.
+    Returns (effective TFLOP/s, sample text).
     """
 
     def __init__(self, w, q, k, v):
@@ -166,90 +250,88 @@ class OracleSample:
         import oracle as O
         self.w, self.O, self.np = w, O, np
         t0 = time.perf_counter()
-        if w.tile is not None:
-            perm = O.tile_order(w.grid, w.tile)
-            n_pad = math.ceil(w.n_tokens / w.block) * w.block
-            tg = tuple(math.ceil(g / t) for g, t in zip(w.grid, w.tile))
-        if w.mask == "sta":
-            self.mask = O.sta_tile_mask(tg, w.window)[None]
-        elif w.mask == "radial":
-            self.mask = O.radial_block_mask_fast(w.nk, w.tokens_per_frame, w.block)[None]
-        else:
-            raise ValueError("cpu baseline implemented for static-mask workloads")
-        self.heads64 = []
-        for h in range(w.heads):
-            qh = q[:, :, h:h + 1].double().numpy()
-            kh = k[:, :, h:h + 1].double().numpy()
-            vh = v[:, :, h:h + 1].double().numpy()
-            if w.tile is not None:
-                qh = O.tile_permute(qh, perm, n_pad)[:, :w.nq]
-                kh = O.tile_permute(kh, perm, n_pad)[:, :w.nk]
-                vh = O.tile_permute(vh, perm, n_pad)[:, :w.nk]
-            self.heads64.append((qh, kh, vh))
+        self.q, self.k, self.v = q, k, v
+        self.perm = O.tile_order(w.grid, w.tile) if w.tile is not None else None
+        self.mask = oracle_workload_mask(w, q, k)
         self.setup_s = time.perf_counter() - t0
         self.rng = np.random.default_rng(7)
 
+    def path_rows(self, t, rows, h):
+        """float64 [B, len(rows), 1, D] of tensor t at path-order rows, head h."""
+        idx = rows if self.perm is None else self.perm[rows]
+        return t[:, self.np.asarray(idx), h:h + 1].double().numpy()
+
+    def gather(self, qb, h):
+        """(rows, keys, kept blocks) of query block qb under head h's mask row."""
+        w, np = self.w, self.np
+        hm = 0 if self.mask.shape[0] == 1 else h
+        rows = np.arange(qb * w.block, min((qb + 1) * w.block, w.nq))
+        kept = np.nonzero(self.mask[hm, qb])[0]
+        keys = np.concatenate([np.arange(kb * w.block, min((kb + 1) * w.block, w.nk))
+                               for kb in kept]) if kept.size else np.zeros(0, np.int64)
+        return rows, keys, kept
+
     def run(self, budget_s: float):
         w, O, np = self.w, self.O, self.np
         QB = math.ceil(w.nq / w.block)
-        flops, done = 0.0, 0
-        t1 = time.perf_counter()
+        flops, done, timed = 0.0, 0, 0.0
         for qb in self.rng.permutation(QB):
-            rows = np.arange(qb * w.block, min((qb + 1) * w.block, w.nq))
-            for qh, kh, vh in self.heads64:
-                O.block_sparse_attention(qh, kh, vh, self.mask, w.block, w.block, rows=rows)
-            kept = np.nonzero(self.mask[0, qb])[0]
-            nkeys = sum(min((kb + 1) * w.block, w.nk) - kb * w.block for kb in kept)
-            flops += 4.0 * w.head_dim * len(rows) * nkeys * w.heads
+            for h in range(w.heads):
+                rows, keys, kept = self.gather(qb, h)
+                if keys.size == 0:
+                    continue
+                qh, kh, vh = (self.path_rows(t, r, h) for t, r in
+                              ((self.q, rows), (self.k, keys), (self.v, keys)))
+                ones = np.ones((1, 1, kept.size), np.uint8)   # the gathered kept blocks
+                t1 = time.perf_counter()
+                O.block_sparse_attention(qh, kh, vh, ones, w.block, w.block)
+                timed += time.perf_counter() - t1
+                flops += 4.0 * w.head_dim * rows.size * keys.size
             done += 1
-            if time.perf_counter() - t1 > budget_s:
+            if timed > budget_s:
                 break
-        el = time.perf_counter() - t1
         sample = (f"{done} random query blocks x {w.heads} heads of {w.name} "
-                  f"({flops / 1e12:.4f} effective TFLOP), float64 oracle, {el:.1f} s "
-                  f"(+{self.setup_s:.1f} s untimed setup: oracle mask, tile permute, upcast)")
-        return flops / el / 1e12, sample
+                  f"({flops / 1e12:.4f} effective TFLOP), float64 oracle, {timed:.1f} s "
+                  f"(+{self.setup_s:.1f} s untimed setup: the oracle's own mask; rows and kept "
+                  f"keys gathered and upcast outside the timing)")
+        return flops / timed / 1e12, sample
 
 
 class BackwardOracleSample(OracleSample):
-    """The CPU oracle's backward on whole query blocks of the workload (all heads).
-
-    Each sampled query block runs the oracle's block-sparse backward with the
-    mask restricted to that block's row (the other rows keep nothing), which is
-    the backward work of those queries: 10 * head_dim flops per kept pair."""
+    """The CPU oracle's backward on whole query blocks of the workload (all heads):
+    each sampled block and head runs the oracle's block-sparse backward on the
+    block's query rows and its kept keys (dO of those rows), which is the backward
+    work of those queries: 10 * head_dim flops per kept pair."""
 
     def __init__(self, w, q, k, v, do):
         super().__init__(w, q, k, v)
-        O = self.O
-        t0 = time.perf_counter()
-        self.do64 = []
-        for h in range(w.heads):
-            dh = do[:, :, h:h + 1].double().numpy()   # already in the path's token order
-            self.do64.append(dh)
-        self.setup_s += time.perf_counter() - t0
+        self.do = do                     # already in the path's token order
 
     def run(self, budget_s: float):
         w, O, np = self.w, self.O, self.np
         QB = math.ceil(w.nq / w.block)
-        flops, done = 0.0, 0
-        t1 = time.perf_counter()
+        flops, done, timed = 0.0, 0, 0.0
         for qb in self.rng.permutation(QB):
-            m = np.zeros_like(self.mask)
-            m[0, qb] = self.mask[0, qb]
-            for (qh, kh, vh), dh in zip(self.heads64, self.do64):
-                O.block_sparse_attention_backward(qh, kh, vh, dh, m, w.block, w.block)
-            rows = min((qb + 1) * w.block, w.nq) - qb * w.block
-            kept = np.nonzero(self.mask[0, qb])[0]
-            nkeys = sum(min((kb + 1) * w.block, w.nk) - kb * w.block for kb in kept)
-            flops += 10.0 * w.head_dim * rows * nkeys * w.heads
+            for h in range(w.heads):
+                rows, keys, kept = self.gather(qb, h)
+                if keys.size == 0:
+                    continue
+                qh, kh, vh = (self.path_rows(t, r, h) for t, r in
+                              ((self.q, rows), (self.k, keys), (self.v, keys)))
+                dh = self.do[:, rows, h:h + 1].double().numpy()
+                ones = np.ones((1, 1, kept.size), np.uint8)
+                t1 = time.perf_counter()
+                O.block_sparse_attention_backward(qh, kh, vh, dh, ones, w.block, w.block)
+                timed += time.perf_counter() - t1
+                flops += 10.0 * w.head_dim * rows.size * keys.size
             done += 1
-            if time.perf_counter() - t1 > budget_s:
+            if timed > budget_s:
                 break
-        el = time.perf_counter() - t1
         sample = (f"{done} random query blocks x {w.heads} heads of {w.name} "
-                  f"({flops / 1e12:.4f} effective TFLOP), float64 oracle backward, {el:.1f} s "
-                  f"(+{self.setup_s:.1f} s untimed setup: oracle mask, tile permute, upcast)")
-        return flops / el / 1e12, sample
+                  f"({flops / 1e12:.4f} effective TFLOP), float64 oracle backward, {timed:.1f} s "
+                  f"(+{self.setup_s:.1f} s untimed setup: the oracle's own mask; rows and kept "
+                  f"keys gathered and upcast outside the timing)")
+        return flops / timed / 1e12, sample
 
 
 BWD_METRIC = "block-sparse attention backward effective TFLOP/s"
@@ -403,7 +485,7 @@ def run_reference(args, w):
     else:
         sampler = OracleSample(w, q, k, v)
     n = max(1, args.steps + args.warmup)
-    budget = max(0.5, min(10.0, 90.0 / n))
+    budget = max(0.5, min(10.0, 90.0 / n, args.cpu_budget))
     vals = []
     sample = ""
     for i in range(n):
@@ -604,13 +686,11 @@ def run_backward(args, w):
 
     peaks, peak_kind = load_peaks()
     achieved = flops / (ms * 1e-3) / 1e12
-    peak = peaks["bf16_tflops_sustained"]
-    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": profiled_traffic(w.name, "attn_bwd"),
-                "kernel": "attn_bwd_kernel<128> (dK/dV pass + dQ pass) and list preparation",
-                "bwd_ms": ms,
-                "peak_note": f"{peak_kind} sustained bf16 (calls timed back to back)",
-                "frac_of_burst": achieved / peaks["bf16_tflops"]}
+    clocks = sampler.summary()
+    roofline = tensor_roofline(
+        achieved, ms, peaks, peak_kind, clocks, ms_total * 1e-3,
+        traffic=profiled_traffic(w.name, "attn_bwd"),
+        kernel="attn_bwd_kernel<128> (dK/dV pass + dQ pass) and list preparation", bwd_ms=ms)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         val, sample = BackwardOracleSample(w, q_h, k_h, v_h, do_h).run(args.cpu_budget)
@@ -621,8 +701,8 @@ def run_backward(args, w):
                 "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16", "data": "synthetic", "config": workload_config(w, "bwd"),
-                "roofline": with_nominal(roofline), "cpu_baseline": cpu, "e2e": e2e,
-                "clocks": sampler.summary(), "gpu_launches": 6 * args.steps,
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "clocks": clocks, "gpu_launches": 6 * args.steps,
                 "effective_tflop_per_step": flops / 1e12}
         print(json.dumps(line))
     if world > 1:
@@ -841,12 +921,11 @@ def run_ar_paged(args, w):
           "saving_vs_plain": 1.0 - cache.resident_bytes() / plain_bytes,
           "pool_saving_vs_plain": 1.0 - cache.pool_bytes() / plain_bytes}
     peaks, peak_kind = load_peaks()
-    peak = peaks["bf16_tflops_sustained"]
-    roofline = {"bound": "tensor", "achieved": value / world, "peak": peak, "unit": "TFLOP/s",
-                "frac": value / world / peak, "traffic": None,
-                "kernel": "attn_fwd_kernel<128> through the page table, with the chunk's mask "
-                          "kernels (the whole attend step is timed)",
-                "peak_note": f"{peak_kind} sustained bf16"}
+    clocks = sampler.summary()
+    roofline = tensor_roofline(
+        value / world, ms, peaks, peak_kind, clocks, ms * args.steps * 1e-3, traffic=None,
+        kernel="attn_fwd_kernel<128> through the page table, with the chunk's mask kernels "
+               "(the whole attend step is timed)")
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         val, sample = PagedAROracleSample(w, q_h, k_h, v_h).run(args.cpu_budget)
@@ -857,10 +936,10 @@ def run_ar_paged(args, w):
                 "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16", "data": "synthetic", "config": workload_config(w, "ar_paged"),
-                "roofline": with_nominal(roofline), "cpu_baseline": cpu, "e2e": e2e,
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 # per attend step: 2 block means, residency, selection, 3 compaction,
                 # kept-list build, attention
-                "clocks": sampler.summary(), "gpu_launches": 9 * args.steps,
+                "clocks": clocks, "gpu_launches": 9 * args.steps,
                 "kv_cache": kv, "plain_path_attend_ms": plain_ms,
                 "effective_tflop_per_step": flops / 1e12}
         print(json.dumps(line))
@@ -880,7 +959,8 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="sta_720p")
+    ap.add_argument("--workload", default="radial_long",
+                    help="workload name (default: the largest, 453,600-token radial one)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle work for the cpu_baseline field")
@@ -897,7 +977,7 @@ def main():
 
     from block_sparse_attention_tokens_b200 import configs
     import dataclasses
-    if args.pass_ == "ar_paged" and args.workload == "sta_720p":
+    if args.pass_ == "ar_paged" and args.workload == "radial_long":
         args.workload = "ar_decode"
     w = configs.get(args.workload)
     if args.pass_ == "ar_paged" and w.mask != "ar":
@@ -1051,13 +1131,13 @@ def main():
 
     peaks, peak_kind = load_peaks()
     achieved = flops / (attn_ms * 1e-3) / 1e12
-    peak = peaks["bf16_tflops_sustained"]
-    traffic = profiled_traffic(w.name)
-    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": traffic,
-                "kernel": "attn_fwd_kernel<128, adjacent key tiles>", "attn_ms": attn_ms,
-                "peak_note": f"{peak_kind} sustained bf16 (kernel timed inside back-to-back steps)",
-                "frac_of_burst": achieved / peaks["bf16_tflops"]}
+    clocks = sampler.summary()
+    gathered = w.block == 64
+    roofline = tensor_roofline(
+        achieved, attn_ms, peaks, peak_kind, clocks, ms_total * 1e-3,
+        traffic=profiled_traffic(w.name),
+        kernel=f"attn_fwd_kernel<{w.head_dim}, {'gathered' if gathered else 'adjacent'} key tiles>",
+        attn_ms=attn_ms)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -1071,8 +1151,8 @@ def main():
                 "warmup": max(3, args.warmup), "ms_per_step": ms_per_step,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16", "data": "synthetic", "config": workload_config(w),
-                "roofline": with_nominal(roofline), "cpu_baseline": cpu, "e2e": e2e,
-                "clocks": sampler.summary(),
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "clocks": clocks,
                 "gpu_launches": plan.kernel_launches_per_step() * args.steps,
                 "effective_tflop_per_step": flops / 1e12,
                 "mask_stats": mask_stats(flops, w, plan.nq, plan.nk, attn_times,

@@ -34,6 +34,30 @@ def test_reference_arm_prints_one_contract_line(pass_):
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
 
 
+@pytest.mark.parametrize("workload", ["nabla_480p", "ar_decode"])
+def test_reference_arm_on_dynamic_masks(workload):
+    # the oracle builds its own NABLA / autoregressive mask (untimed) and is timed
+    # on sampled query blocks (two heads keep the CPU run short)
+    d = run_bench("--impl", "reference", "--workload", workload, "--heads", "2", "--steps", "1",
+                  "--warmup", "0", "--cpu-budget", "1")
+    assert d["config"]["workload"] == workload and d["value"] > 0
+    assert "oracle's own mask" in d["cpu_baseline"]["sample"]
+
+
+def test_peak_choice_follows_the_run():
+    sys.path.insert(0, ROOT)
+    import bench
+    peaks = {"bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6500.0}
+    at_max = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0}
+    capped = {"sm_mhz": 1500.0, "sm_max_mhz": 1965.0}
+    assert bench.choose_tensor_peak(peaks, at_max, 10.0)[:2] == (1600.0, "burst")
+    assert bench.choose_tensor_peak(peaks, capped, 1.0)[:2] == (1600.0, "burst")
+    assert bench.choose_tensor_peak(peaks, capped, 10.0)[:2] == (1400.0, "sustained")
+    r = bench.tensor_roofline(700.0, 20.0, peaks, "measured", capped, 10.0, attn_ms=20.0)
+    assert r["frac"] == 0.5 and r["frac_of_burst"] == 700.0 / 1600.0
+    assert r["kernel_ms_x_sm_mhz"] == 20.0 * 1500.0 and r["attn_ms"] == 20.0
+
+
 def test_ar_budget_keeps_the_target_fraction():
     sys.path.insert(0, ROOT)
     import bench
