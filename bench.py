@@ -28,9 +28,12 @@ workload's mask), metric: effective TFLOP/s = 10 * head_dim * kept pairs / time
 (five matrix products of 2 * head_dim flops per pair: the recomputed scores, dP,
 dV, dQ and dK).
 
-Under torchrun (N > 1) every rank runs its own batch of the same shape (the path
-shards by batch/head with no collective): weak scaling, value = all ranks' work
-divided by the slowest rank's time.
+Under torchrun (N > 1) the forward path splits the workload's heads over the
+ranks (each rank holds and computes its own range of heads; masks are per head,
+so nothing is exchanged): strong scaling, value = the whole workload's work
+divided by the slowest rank's time; ``--pass bwd`` splits the heads the same
+way.  The SICS and paged passes run one copy of the workload per rank (weak
+scaling).
 """
 from __future__ import annotations
 
@@ -519,6 +522,24 @@ def max_over_ranks(values, device=None):
     return t.tolist()
 
 
+def sum_over_ranks(values, device=None):
+    """Element-wise sum of a float (or list of floats) over all ranks (identity
+    when not distributed).  Every rank must call it at the same point."""
+    import torch
+    import torch.distributed as dist
+    scalar = not isinstance(values, (list, tuple))
+    t = torch.tensor([values] if scalar else list(values), dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return t.item() if scalar else t.tolist()
+
+
+def job_value(flops_all_ranks, ms_per_step):
+    """Whole-job throughput (TFLOP/s): the work of all ranks in the slowest rank's
+    step time."""
+    return flops_all_ranks / (ms_per_step * 1e-3) / 1e12
+
+
 def weak_scaling_value(flops_per_rank, world, ms_per_step):
     """Whole-job throughput (TFLOP/s): every rank processes its own batch of the
     same shape, the slowest rank's time bounds the step."""
@@ -607,18 +628,21 @@ def run_backward(args, w):
     import torch.distributed as dist
     from block_sparse_attention_tokens_b200 import binding as B
     from block_sparse_attention_tokens_b200 import synth
-    from block_sparse_attention_tokens_b200.pipeline import Plan, effective_flops
+    from block_sparse_attention_tokens_b200.pipeline import Plan, effective_flops, head_range
 
     world, rank, dev = setup_ranks()
     q_h, k_h, v_h, _ = synth.workload_inputs(w)
     do_h = path_order_grad(w)
-    plan = Plan(w, dev)
+    # with N ranks each rank takes its range of heads, as in the forward
+    h0, h1 = head_range(rank, world, w.heads)
+    q_h, k_h, v_h, do_h = (t_[:, :, h0:h1].contiguous() for t_ in (q_h, k_h, v_h, do_h))
+    plan = Plan(w, dev, heads=(h0, h1))
     plan.step(q_h.to(dev), k_h.to(dev), v_h.to(dev))
     qq, kk, vv = (plan.qp, plan.kp, plan.vp) if plan.permuted else (plan._q, plan._k, plan._v)
     oo = plan.op if plan.permuted else plan.o
     do = do_h.to(dev)
     dq, dk, dv = torch.empty_like(qq), torch.empty_like(kk), torch.empty_like(vv)
-    ws = torch.empty(B.bsa_attn_bwd_workspace_size(w.batch, w.heads, plan.nq, plan.nk, w.block,
+    ws = torch.empty(B.bsa_attn_bwd_workspace_size(w.batch, plan.heads, plan.nq, plan.nk, w.block,
                                                    w.block, plan.list_heads),
                      dtype=torch.uint8, device=dev)
 
@@ -638,7 +662,8 @@ def run_backward(args, w):
     if B.bsa_read_status(ws) != 0:
         raise RuntimeError("backward kernel reported a device-side error")
     flops = 2.5 * effective_flops(plan.mask, plan.nq, plan.nk, w.block, w.head_dim,
-                                  w.batch * w.heads)
+                                  w.batch * plan.heads)
+    flops_all = sum_over_ranks(flops, dev)
 
     stream = torch.cuda.current_stream()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -655,7 +680,7 @@ def run_backward(args, w):
     ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
     ms_total = sum(a.elapsed_time(b) for a, b in ev)
     ms, ms_total = max_over_ranks([ms, ms_total], dev)
-    value = weak_scaling_value(flops, world, ms)
+    value = job_value(flops_all, ms)
 
     # end to end through the public API: every step copies its inputs from pinned
     # host memory (Q, K, V, O, dO in the path's token order, LSE, the kept lists),
@@ -678,14 +703,15 @@ def run_backward(args, w):
         e1.record(stream)
         barrier()
         e_ms = max_over_ranks([e0.elapsed_time(e1) / e_steps], dev)[0]
-        e2e = {"value": weak_scaling_value(flops, world, e_ms), "unit": "TFLOP/s",
-               "ms_per_step": e_ms,
-               "h2d_bytes_per_step": sum(t_.numel() * t_.element_size() for t_ in host_in),
-               "d2h_bytes_per_step": sum(t_.numel() * t_.element_size() for t_ in host_out),
+        h2d, d2h = sum_over_ranks(
+            [sum(t_.numel() * t_.element_size() for t_ in host_in),
+             sum(t_.numel() * t_.element_size() for t_ in host_out)], dev)
+        e2e = {"value": job_value(flops_all, e_ms), "unit": "TFLOP/s",
+               "ms_per_step": e_ms, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "note": "pinned host buffers; copies and the backward serialised on one stream"}
 
     peaks, peak_kind = load_peaks()
-    achieved = flops / (ms * 1e-3) / 1e12
+    achieved = flops_all / world / (ms * 1e-3) / 1e12
     clocks = sampler.summary()
     roofline = tensor_roofline(
         achieved, ms, peaks, peak_kind, clocks, ms_total * 1e-3,
@@ -697,13 +723,15 @@ def run_backward(args, w):
         cpu = {"value": val, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
                "sample": sample}
     if rank == 0:
+        cfg = workload_config(w, "bwd")
+        cfg["parallelism"] = f"heads split over {world} GPU(s), no data-path collective"
         line = {"metric": BWD_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
                 "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms,
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-                "dtype": "bf16", "data": "synthetic", "config": workload_config(w, "bwd"),
+                "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic", "config": cfg,
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "clocks": clocks, "gpu_launches": 6 * args.steps,
-                "effective_tflop_per_step": flops / 1e12}
+                "effective_tflop_per_step": flops_all / 1e12}
         print(json.dumps(line))
     if world > 1:
         dist.destroy_process_group()
@@ -998,14 +1026,19 @@ def main():
     import torch.distributed as dist
     from block_sparse_attention_tokens_b200 import binding as B
     from block_sparse_attention_tokens_b200 import synth
-    from block_sparse_attention_tokens_b200.pipeline import Plan, effective_flops
+    from block_sparse_attention_tokens_b200.pipeline import Plan, effective_flops, head_range
 
     world, rank, dev = setup_ranks()
 
-    # inputs (the same seeded batch on every rank: each rank owns one batch of work)
-    q_h, k_h, v_h, _ = synth.workload_inputs(w)
+    # inputs: the workload's seeded Q, K, V; with N ranks each rank takes its range
+    # of heads (masks are per head and every head is independent, so nothing is
+    # exchanged) and holds only those heads, as after a head-parallel projection
+    q_all, k_all, v_all, _ = synth.workload_inputs(w)
+    h0, h1 = head_range(rank, world, w.heads)
+    q_h, k_h, v_h = (t_[:, :, h0:h1].contiguous() for t_ in (q_all, k_all, v_all))
+    del q_all, k_all, v_all
     q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
-    plan = Plan(w, dev)
+    plan = Plan(w, dev, heads=(h0, h1))
 
     def barrier():
         if world > 1:
@@ -1016,7 +1049,8 @@ def main():
         plan.step(q, k, v)
     barrier()
     flops = effective_flops(plan.mask, plan.nq, plan.nk, w.block, w.head_dim,
-                            w.batch * w.heads)
+                            w.batch * plan.heads)
+    flops_all = sum_over_ranks(flops, dev)
     if B.bsa_read_status(plan.attn_ws) != 0:
         raise RuntimeError("attention kernel reported a device-side error")
 
@@ -1061,7 +1095,7 @@ def main():
     }
     ms_total, attn_ms = max_over_ranks([ms_total, attn_ms], dev)
     ms_per_step = ms_total / args.steps
-    value = weak_scaling_value(flops, world, ms_per_step)
+    value = job_value(flops_all, ms_per_step)
 
     # ---- end to end through the public API: pinned host inputs in, O back to host.
     # Steps are pipelined the way a serving loop would run them: the host->device
@@ -1124,13 +1158,16 @@ def main():
                             dtype=torch.float64)
         h2d_bytes = sum(t_.numel() * t_.element_size() for t_ in (q_h, k_h, v_h))
         d2h_bytes = o_host.numel() * o_host.element_size()
-        e2e = {"value": weak_scaling_value(flops, world, e_ms.item()), "unit": "TFLOP/s",
+        h2d_bytes, d2h_bytes = (int(x) for x in sum_over_ranks([h2d_bytes, d2h_bytes], dev))
+        e2e = {"value": job_value(flops_all, e_ms.item()), "unit": "TFLOP/s",
                "ms_per_step": e_ms.item(), "h2d_bytes_per_step": h2d_bytes,
                "d2h_bytes_per_step": d2h_bytes,
-               "note": "pinned host buffers; copies of neighbouring steps overlap compute"}
+               "note": "pinned host buffers (each rank its heads); copies of neighbouring steps "
+                       "overlap compute"}
 
     peaks, peak_kind = load_peaks()
-    achieved = flops / (attn_ms * 1e-3) / 1e12
+    # the slowest rank's attention time, for that rank's share of the work
+    achieved = flops_all / world / (attn_ms * 1e-3) / 1e12
     clocks = sampler.summary()
     gathered = w.block == 64
     roofline = tensor_roofline(
@@ -1146,15 +1183,17 @@ def main():
                "sample": sample}
 
     if rank == 0:
+        cfg = workload_config(w)
+        cfg["parallelism"] = f"heads split over {world} GPU(s), no data-path collective"
         line = {"metric": FWD_METRIC,
                 "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
                 "warmup": max(3, args.warmup), "ms_per_step": ms_per_step,
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-                "dtype": "bf16", "data": "synthetic", "config": workload_config(w),
+                "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic", "config": cfg,
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "clocks": clocks,
                 "gpu_launches": plan.kernel_launches_per_step() * args.steps,
-                "effective_tflop_per_step": flops / 1e12,
+                "effective_tflop_per_step": flops_all / 1e12,
                 "mask_stats": mask_stats(flops, w, plan.nq, plan.nk, attn_times,
                                          plan.near.item() if hasattr(plan, "near") else None),
                 # mean device time of each stage of a timed step (this rank, CUDA events)

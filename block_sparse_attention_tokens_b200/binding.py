@@ -54,23 +54,23 @@ def load_library(path: str = _LIB_PATH) -> ctypes.CDLL:
         "bsa_status_string": (ctypes.c_char_p, [c_int]),
         "bsa_last_error_message": (ctypes.c_char_p, []),
         "bsa_version": (c_int, []),
-        "bsa_tile_permute": (c_int, [c_void, c_void] + [c_int] * 9 + [c_void]),
-        "bsa_tile_untile": (c_int, [c_void, c_void] + [c_int] * 9 + [c_void]),
+        "bsa_tile_permute": (c_int, [c_void, c_void] + [c_int] * 11 + [c_void]),
+        "bsa_tile_untile": (c_int, [c_void, c_void] + [c_int] * 11 + [c_void]),
         "bsa_sta_mask": (c_int, [c_int] * 7 + [c_void, c_void]),
         "bsa_radial_mask": (c_int, [c_int] * 3 + [c_void, c_void]),
         "bsa_nabla_workspace_size": (c_size, [c_int] * 6),
-        "bsa_nabla_mask": (c_int, [c_void, c_void] + [c_int] * 6 + [c_float, c_float] + [c_int] * 3
+        "bsa_nabla_mask": (c_int, [c_void, c_void] + [c_int] * 7 + [c_float, c_float] + [c_int] * 3
                            + [c_void, c_void, c_void, c_size, c_void]),
         "bsa_mask_compact": (c_int, [c_void, c_int, c_int, c_void, c_void, c_void]),
         "bsa_attn_workspace_size": (c_size, [c_int] * 7),
-        "bsa_attn_fwd": (c_int, [c_void, c_void, c_void] + [c_int] * 7 + [c_void, c_void, c_int,
+        "bsa_attn_fwd": (c_int, [c_void, c_void, c_void] + [c_int] * 9 + [c_void, c_void, c_int,
                                                                            c_float, c_void, c_void,
                                                                            c_void, c_size, c_void]),
         "bsa_attn_fwd_noalloc": (c_int, [c_void, c_void, c_void] + [c_int] * 7
                                  + [c_void, c_void, c_int, c_float, c_void, c_void, c_void,
                                     c_void]),
         "bsa_attn_bwd_workspace_size": (c_size, [c_int] * 7),
-        "bsa_attn_bwd": (c_int, [c_void] * 6 + [c_int] * 7 + [c_void, c_void, c_int, c_float]
+        "bsa_attn_bwd": (c_int, [c_void] * 6 + [c_int] * 9 + [c_void, c_void, c_int, c_float]
                          + [c_void] * 4 + [c_size, c_void]),
         "bsa_sics_blocks": (c_int, [c_void] + [c_int] * 9 + [c_void, c_void]),
         "bsa_sics_workspace_size": (c_size, [c_int] * 5 + [c_void, c_int]),
@@ -78,7 +78,8 @@ def load_library(path: str = _LIB_PATH) -> ctypes.CDLL:
                             + [c_void] * 3 + [c_size, c_void]),
         "bsa_read_status": (c_int, [c_void, ctypes.POINTER(c_int), c_void]),
         "bsa_wait_selftest": (c_int, [c_void, ctypes.c_ulonglong, c_void]),
-        "bsa_tile_permute_pool": (c_int, [c_void, c_void] + [c_int] * 11 + [c_void, c_void]),
+        "bsa_tile_permute_pool": (c_int, [c_void, c_void] + [c_int] * 11 + [c_void, c_int, c_int,
+                                                                             c_void]),
         "bsa_nabla_select": (c_int, [c_void, c_void] + [c_int] * 5 + [c_float, c_float]
                              + [c_int] * 3 + [c_void] * 5),
         "bsa_kv_write": (c_int, [c_void] + [c_int] * 5 + [c_void, c_int, c_void, c_int, c_void,
@@ -142,6 +143,51 @@ def _tokens(t: torch.Tensor, name: str, batch: int, n: int, heads: int, head_dim
     problem = _token_problem(tuple(t.shape), t.dtype, batch, n, heads, head_dim)
     if problem:
         raise ValueError(f"{name} {problem}")
+
+
+def _stride_problem(shape, strides, n: int, dense_row: int, align_elems: int):
+    """Why token rows of this shape and strides (elements) cannot be described by
+    one row stride: every row contiguous, rows row_stride = strides[1] apart (at
+    least a whole row, a multiple of align_elems), batches n rows apart (None if
+    they can)."""
+    inner = 1
+    for size, st in zip(reversed(shape[2:]), reversed(strides[2:])):
+        if size > 1 and st != inner:
+            return "rows must be contiguous (only the token-row stride may differ)"
+        inner *= size
+    rs = strides[1] if shape[1] > 1 else dense_row
+    if rs < dense_row or rs % align_elems:
+        return f"row stride {rs} must be >= {dense_row} and a multiple of {align_elems}"
+    if shape[0] > 1 and strides[0] != n * rs:
+        return f"batch stride {strides[0]} must be {n} rows of {rs}"
+    return None
+
+
+def _strided_tokens(t: torch.Tensor, name: str, batch: int, n: int, heads: int,
+                    head_dim: int) -> int:
+    """Checks a [batch, >= n, heads, head_dim] bf16 CUDA tensor whose token rows may
+    be a slice of wider rows (a range of heads, or Q / K / V of a fused projection)
+    and returns its row stride in elements."""
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    problem = _token_problem(tuple(t.shape), t.dtype, batch, n, heads, head_dim)
+    if problem and "rows per batch" not in problem:
+        raise ValueError(f"{name} {problem}")
+    problem = _stride_problem(tuple(t.shape), tuple(t.stride()), n, heads * head_dim, 8)
+    if problem:
+        raise ValueError(f"{name}: {problem}")
+    if t.data_ptr() % 16:
+        raise ValueError(f"{name} must start on a 16-byte boundary")
+    return t.stride(1) if t.shape[1] > 1 else heads * head_dim
+
+
+def _shared_stride(pairs) -> int:
+    """The one row stride of several token tensors [(tensor, name, stride)]."""
+    strides = {st for _, _, st in pairs}
+    if len(strides) != 1:
+        raise ValueError(", ".join(n for _, n, _ in pairs) + " must share one token-row stride, got "
+                         + str(sorted(strides)))
+    return strides.pop()
 
 
 def _buffer(t: torch.Tensor, name: str, dtype, numel: int):
@@ -213,6 +259,25 @@ def _rows(t: torch.Tensor, name: str, batch: int, n: int, row_bytes: int):
         raise ValueError(f"{name} {problem}")
 
 
+def _strided_rows(t: torch.Tensor, name: str, batch: int, n: int) -> Tuple[int, int]:
+    """A [batch, >= n, ...] CUDA tensor whose rows (the trailing dims) are contiguous
+    but may lie further apart than their size: returns (row bytes, row stride in
+    bytes)."""
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    es = t.element_size()
+    row_bytes = math.prod(t.shape[2:]) * es
+    if t.dim() < 2 or t.shape[0] != batch or t.shape[1] < n:
+        raise ValueError(f"{name} must be [{batch}, >= {n}, ...], got {tuple(t.shape)}")
+    problem = _stride_problem(tuple(t.shape), tuple(t.stride()), n, row_bytes // es,
+                              max(1, 16 // es))
+    if problem:
+        raise ValueError(f"{name}: {problem}")
+    if t.data_ptr() % 16:
+        raise ValueError(f"{name} must start on a 16-byte boundary")
+    return row_bytes, (t.stride(1) if t.shape[1] > 1 else row_bytes // es) * es
+
+
 def _bytes(t: torch.Tensor, name: str, numel: int):
     """A byte mask / flag buffer (uint8 or bool) of at least numel entries."""
     _cuda(t, name)
@@ -226,32 +291,36 @@ def _bytes(t: torch.Tensor, name: str, numel: int):
 
 def bsa_tile_permute(x: torch.Tensor, grid: Tuple[int, int, int], tile: Tuple[int, int, int],
                      n_pad: int, y: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """x [B, N, ...] raster order -> y [B, n_pad, ...] tile order with a zero tail."""
-    _cuda(x, "x")
+    """x [B, N, ...] raster order -> y [B, n_pad, ...] tile order with a zero tail.
+    x and y may be slices of wider rows (e.g. x[:, :, h0:h1] of a [B, N, H, D]
+    tensor): only the row stride may differ from a dense layout."""
     B = x.shape[0]
     N = grid[0] * grid[1] * grid[2]
-    row_bytes = math.prod(x.shape[2:]) * x.element_size()
-    _rows(x, "x", B, N, row_bytes)
+    row_bytes, xs = _strided_rows(x, "x", B, N)
     if y is None:
         y = torch.empty((B, n_pad) + tuple(x.shape[2:]), dtype=x.dtype, device=x.device)
-    _rows(y, "y", B, n_pad, row_bytes)
+    y_bytes, ys = _strided_rows(y, "y", B, n_pad)
+    if y_bytes != row_bytes:
+        raise ValueError(f"y rows of {y_bytes} bytes, {row_bytes} expected")
     _check(load_library().bsa_tile_permute(_ptr(x), _ptr(y), B, *grid, *tile, row_bytes, n_pad,
-                                           _stream()), "bsa_tile_permute")
+                                           xs, ys, _stream()), "bsa_tile_permute")
     return y
 
 
 def bsa_tile_untile(y: torch.Tensor, grid: Tuple[int, int, int], tile: Tuple[int, int, int],
                     x: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """y [B, n_pad, ...] tile order -> x [B, N, ...] raster order."""
-    _cuda(y, "y")
+    """y [B, n_pad, ...] tile order -> x [B, N, ...] raster order (either may be a
+    slice of wider rows)."""
     B, n_pad = y.shape[0], y.shape[1]
     N = grid[0] * grid[1] * grid[2]
-    row_bytes = math.prod(y.shape[2:]) * y.element_size()
+    row_bytes, ys = _strided_rows(y, "y", B, n_pad)
     if x is None:
         x = torch.empty((B, N) + tuple(y.shape[2:]), dtype=y.dtype, device=y.device)
-    _rows(x, "x", B, N, row_bytes)
+    x_bytes, xs = _strided_rows(x, "x", B, N)
+    if x_bytes != row_bytes:
+        raise ValueError(f"x rows of {x_bytes} bytes, {row_bytes} expected")
     _check(load_library().bsa_tile_untile(_ptr(y), _ptr(x), B, *grid, *tile, row_bytes, n_pad,
-                                          _stream()), "bsa_tile_untile")
+                                          ys, xs, _stream()), "bsa_tile_untile")
     return x
 
 
@@ -260,18 +329,18 @@ def bsa_tile_permute_pool(x: torch.Tensor, grid: Tuple[int, int, int],
                           y: Optional[torch.Tensor] = None,
                           pooled: Optional[torch.Tensor] = None):
     """x [B, N, H, D] bf16 raster -> (y [B, n_pad, H, D] tile order,
-    pooled [B, H, n_pad / block, D] fp32 block means)."""
-    _cuda(x, "x")
+    pooled [B, H, n_pad / block, D] fp32 block means).  x and y may be head
+    slices of wider tensors."""
     B, _, H, D = x.shape
-    _tokens(x, "x", B, grid[0] * grid[1] * grid[2], H, D)
+    xs = _strided_tokens(x, "x", B, grid[0] * grid[1] * grid[2], H, D)
     if y is None:
         y = torch.empty((B, n_pad, H, D), dtype=x.dtype, device=x.device)
-    _tokens(y, "y", B, n_pad, H, D)
+    ys = _strided_tokens(y, "y", B, n_pad, H, D)
     if pooled is None:
         pooled = torch.empty((B, H, n_pad // block, D), dtype=torch.float32, device=x.device)
     _buffer(pooled, "pooled", torch.float32, B * H * (n_pad // max(block, 1)) * D)
     _check(load_library().bsa_tile_permute_pool(_ptr(x), _ptr(y), B, *grid, *tile, H, D, n_pad,
-                                                block, _ptr(pooled), _stream()),
+                                                block, _ptr(pooled), xs, ys, _stream()),
            "bsa_tile_permute_pool")
     return y, pooled
 
@@ -314,12 +383,11 @@ def bsa_nabla_mask(q: torch.Tensor, k: torch.Tensor, block: int, p: float, scale
     nq / nk: number of valid tokens (default: the tensors' lengths).
     Returns (mask, near_count tensor).
     """
-    _cuda(q, "q")
     B, _, H, D = q.shape
     nq = q.shape[1] if nq is None else nq
     nk = k.shape[1] if nk is None else nk
-    _tokens(q, "q", B, nq, H, D)
-    _tokens(k, "k", B, nk, H, D)
+    rs = _shared_stride([(q, "q", _strided_tokens(q, "q", B, nq, H, D)),
+                         (k, "k", _strided_tokens(k, "k", B, nk, H, D))])
     QB, KB = -(-nq // block), -(-nk // block)
     kb_end = KB if kb_end is None else kb_end
     if mask is None:
@@ -332,7 +400,7 @@ def bsa_nabla_mask(q: torch.Tensor, k: torch.Tensor, block: int, p: float, scale
         ws = torch.empty(bsa_nabla_workspace_size(B, H, nq, nk, D, block), dtype=torch.uint8,
                          device=q.device)
     _cuda(ws, "ws")
-    _check(load_library().bsa_nabla_mask(_ptr(q), _ptr(k), B, H, nq, nk, D, block, float(p),
+    _check(load_library().bsa_nabla_mask(_ptr(q), _ptr(k), B, H, nq, nk, D, rs, block, float(p),
                                          float(scale), kb_begin, kb_end, int(force_outside),
                                          _ptr(mask), _ptr(near_count), _ptr(ws), _nbytes(ws),
                                          _stream()), "bsa_nabla_mask")
@@ -404,27 +472,30 @@ def bsa_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, row_ptr: tor
                  nq: Optional[int] = None, nk: Optional[int] = None, scale: float = 0.0,
                  o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
                  ws: Optional[torch.Tensor] = None):
-    """Block-sparse attention forward.  Returns (o [B, nq_rows, H, D] bf16, lse [B, H, nq])."""
-    _cuda(q, "q")
+    """Block-sparse attention forward.  Returns (o [B, nq_rows, H, D] bf16, lse [B, H, nq], ws).
+
+    q, k, v (and o) may be head slices of wider [B, N, H_total, D] tensors or the Q,
+    K, V views of a fused projection: q, k and v must share one token-row stride,
+    o may have its own."""
     B, _, H, D = q.shape
     nq = q.shape[1] if nq is None else nq
     nk = k.shape[1] if nk is None else nk
-    _tokens(q, "q", B, nq, H, D)
-    _tokens(k, "k", B, nk, H, D)
-    _tokens(v, "v", B, nk, H, D)
+    qkv_rs = _shared_stride([(q, "q", _strided_tokens(q, "q", B, nq, H, D)),
+                             (k, "k", _strided_tokens(k, "k", B, nk, H, D)),
+                             (v, "v", _strided_tokens(v, "v", B, nk, H, D))])
     _lists(row_ptr, col_idx, list_heads, nq, block_q, nk, block_k)
     if o is None:
-        o = torch.empty_like(q)
+        o = torch.empty((B, q.shape[1], H, D), dtype=q.dtype, device=q.device)
     if lse is None:
         lse = torch.empty((B, H, nq), dtype=torch.float32, device=q.device)
-    _tokens(o, "o", B, nq, H, D)
+    o_rs = _strided_tokens(o, "o", B, nq, H, D)
     _buffer(lse, "lse", torch.float32, B * H * nq)
     if ws is None:
         ws = torch.empty(bsa_attn_workspace_size(B, H, nq, nk, block_q, block_k, list_heads),
                          dtype=torch.uint8, device=q.device)
     _cuda(ws, "ws")
-    _check(load_library().bsa_attn_fwd(_ptr(q), _ptr(k), _ptr(v), B, H, nq, nk, D, block_q,
-                                       block_k, _ptr(row_ptr), _ptr(col_idx), list_heads,
+    _check(load_library().bsa_attn_fwd(_ptr(q), _ptr(k), _ptr(v), B, H, nq, nk, D, qkv_rs, o_rs,
+                                       block_q, block_k, _ptr(row_ptr), _ptr(col_idx), list_heads,
                                        float(scale), _ptr(o), _ptr(lse), _ptr(ws), _nbytes(ws),
                                        _stream()), "bsa_attn_fwd")
     return o, lse, ws
@@ -475,27 +546,29 @@ def bsa_attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Ten
                  nq: Optional[int] = None, nk: Optional[int] = None, scale: float = 0.0,
                  dq: Optional[torch.Tensor] = None, dk: Optional[torch.Tensor] = None,
                  dv: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None):
-    """Block-sparse attention backward.  Returns (dq, dk, dv, ws)."""
-    _cuda(q, "q")
+    """Block-sparse attention backward.  Returns (dq, dk, dv, ws).
+
+    q, k, v, dq, dk, dv share one token-row stride, o and dout another (each may be
+    a head slice of a wider tensor; see bsa_attn_fwd)."""
     B, _, H, D = q.shape
     nq = q.shape[1] if nq is None else nq
     nk = k.shape[1] if nk is None else nk
-    for t, n, rows in ((q, "q", nq), (k, "k", nk), (v, "v", nk), (o, "o", nq),
-                       (dout, "dout", nq)):
-        _tokens(t, n, B, rows, H, D)
     _buffer(lse, "lse", torch.float32, B * H * nq)
     _lists(row_ptr, col_idx, list_heads, nq, block_q, nk, block_k)
-    dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(k) if dk is None else dk
-    dv = torch.empty_like(v) if dv is None else dv
-    for t, n, rows in ((dq, "dq", nq), (dk, "dk", nk), (dv, "dv", nk)):
-        _tokens(t, n, B, rows, H, D)
+    dq = torch.empty((B, q.shape[1], H, D), dtype=q.dtype, device=q.device) if dq is None else dq
+    dk = torch.empty((B, k.shape[1], H, D), dtype=k.dtype, device=k.device) if dk is None else dk
+    dv = torch.empty((B, v.shape[1], H, D), dtype=v.dtype, device=v.device) if dv is None else dv
+    qkv_rs = _shared_stride([(t, n, _strided_tokens(t, n, B, rows, H, D)) for t, n, rows in
+                             ((q, "q", nq), (k, "k", nk), (v, "v", nk), (dq, "dq", nq),
+                              (dk, "dk", nk), (dv, "dv", nk))])
+    o_rs = _shared_stride([(t, n, _strided_tokens(t, n, B, nq, H, D)) for t, n in
+                           ((o, "o"), (dout, "dout"))])
     if ws is None:
         ws = torch.empty(bsa_attn_bwd_workspace_size(B, H, nq, nk, block_q, block_k, list_heads),
                          dtype=torch.uint8, device=q.device)
     _cuda(ws, "ws")
     _check(load_library().bsa_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
-                                       B, H, nq, nk, D, block_q, block_k, _ptr(row_ptr),
+                                       B, H, nq, nk, D, qkv_rs, o_rs, block_q, block_k, _ptr(row_ptr),
                                        _ptr(col_idx), list_heads, float(scale), _ptr(dq),
                                        _ptr(dk), _ptr(dv), _ptr(ws), _nbytes(ws), _stream()),
            "bsa_attn_bwd")

@@ -78,6 +78,7 @@ struct BwdParams {
   const float* dvec;         // [B*H][QT*128]: rowsum(dO * O), 0 past nq
   __nv_bfloat16* outA;       // dK (kDKV) or dQ (kDQ)
   __nv_bfloat16* outB;       // dV (kDKV)
+  long long out_stride;      // elements between consecutive token rows of outA / outB
   int* status;
   int* unit_counter;
   unsigned long long timeout_ns;
@@ -483,9 +484,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // epilogue: accA * scale -> outA, accB -> outB (rows past the tensor end
       // skipped); the two warps of a lane quarter take half of the D columns each
       const int nrows = kDKV ? p.nk : p.nq;
-      __nv_bfloat16* rowA = p.outA + ((static_cast<long long>(it.b) * nrows + grow) * p.H + it.h) * D;
-      __nv_bfloat16* rowB =
-          kDKV ? p.outB + ((static_cast<long long>(it.b) * nrows + grow) * p.H + it.h) * D : nullptr;
+      const long long orow_off =
+          (static_cast<long long>(it.b) * nrows + grow) * p.out_stride + static_cast<long long>(it.h) * D;
+      __nv_bfloat16* rowA = p.outA + orow_off;
+      __nv_bfloat16* rowB = kDKV ? p.outB + orow_off : nullptr;
       if (it.n > 0) {
         ok = mbar_wait(DONE, dph, abort_flag, p.status, p.timeout_ns);
         if (!ok) break;
@@ -542,7 +544,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ o,
                                 const __nv_bfloat16* __restrict__ dout,
                                 const float* __restrict__ lse, int B, int H, int nq, int D,
-                                int rows_pad, float* __restrict__ lse2, float* __restrict__ dvec) {
+                                long long o_stride, int rows_pad, float* __restrict__ lse2,
+                                float* __restrict__ dvec) {
   const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const long long total = static_cast<long long>(B) * H * rows_pad;
   if (idx >= total) return;
@@ -556,8 +559,9 @@ __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ o,
   }
   const float l = lse[bh * nq + i];
   lse2[idx] = l == -INFINITY ? INFINITY : l * 1.4426950408889634f;
-  const uint4* po = reinterpret_cast<const uint4*>(o + ((static_cast<long long>(b) * nq + i) * H + h) * D);
-  const uint4* pd = reinterpret_cast<const uint4*>(dout + ((static_cast<long long>(b) * nq + i) * H + h) * D);
+  const long long off = (static_cast<long long>(b) * nq + i) * o_stride + static_cast<long long>(h) * D;
+  const uint4* po = reinterpret_cast<const uint4*>(o + off);
+  const uint4* pd = reinterpret_cast<const uint4*>(dout + off);
   float acc = 0.f;
   for (int c = 0; c < D / 8; ++c) {
     const uint4 a = __ldg(po + c), g = __ldg(pd + c);
@@ -684,9 +688,10 @@ extern "C" size_t bsa_attn_bwd_workspace_size(int batch, int heads, int nq, int 
 
 extern "C" int bsa_attn_bwd(const void* q, const void* k, const void* v, const void* o,
                             const void* dout, const float* lse, int batch, int heads, int nq,
-                            int nk, int head_dim, int block_q, int block_k, const int* row_ptr,
-                            const int* col_idx, int list_heads, float scale, void* dq, void* dk,
-                            void* dv, void* ws, size_t ws_bytes, void* stream) {
+                            int nk, int head_dim, int qkv_row_stride, int o_row_stride,
+                            int block_q, int block_k, const int* row_ptr, const int* col_idx,
+                            int list_heads, float scale, void* dq, void* dk, void* dv, void* ws,
+                            size_t ws_bytes, void* stream) {
   BSA_NVTX_RANGE("bsa_attn_bwd");
   using namespace bsa;
   if (!q || !k || !v || !o || !dout || !lse || !row_ptr || !col_idx || !dq || !dk || !dv || !ws)
@@ -698,6 +703,9 @@ extern "C" int bsa_attn_bwd(const void* q, const void* k, const void* v, const v
                           static_cast<const void*>(ws)})
     if (!aligned16(ptr)) return BSA_ERR_INVALID_ARG;
   if (head_dim != 64 && head_dim != 128) return BSA_ERR_UNSUPPORTED;
+  const long long qkv_rs = token_row_stride(qkv_row_stride, heads, head_dim);
+  const long long o_rs = token_row_stride(o_row_stride, heads, head_dim);
+  if (qkv_rs < 0 || o_rs < 0) return BSA_ERR_INVALID_ARG;
   if (!block_ok(block_q) || !block_ok(block_k)) return BSA_ERR_UNSUPPORTED;
   const BwdGeometry g = bwd_geometry(batch, heads, nq, nk, block_q, block_k, list_heads);
   if (ws_bytes < g.total) return BSA_ERR_WORKSPACE;
@@ -708,10 +716,10 @@ extern "C" int bsa_attn_bwd(const void* q, const void* k, const void* v, const v
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
   CUtensorMap mq, mk, mv, mdo;
-  if (make_map(&mq, q, batch, nq, heads, head_dim) != BSA_OK ||
-      make_map(&mk, k, batch, nk, heads, head_dim) != BSA_OK ||
-      make_map(&mv, v, batch, nk, heads, head_dim) != BSA_OK ||
-      make_map(&mdo, dout, batch, nq, heads, head_dim) != BSA_OK)
+  if (make_map(&mq, q, batch, nq, heads, head_dim, qkv_rs) != BSA_OK ||
+      make_map(&mk, k, batch, nk, heads, head_dim, qkv_rs) != BSA_OK ||
+      make_map(&mv, v, batch, nk, heads, head_dim, qkv_rs) != BSA_OK ||
+      make_map(&mdo, dout, batch, nq, heads, head_dim, o_rs) != BSA_OK)
     return BSA_ERR_CUDA;
 
   char* wsb = static_cast<char*>(ws);
@@ -735,7 +743,7 @@ extern "C" int bsa_attn_bwd(const void* q, const void* k, const void* v, const v
   const long long prep_total = static_cast<long long>(batch) * heads * rows_pad;
   bwd_prep_kernel<<<static_cast<int>(ceil_div<long long>(prep_total, 256)), 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, batch,
-      heads, nq, head_dim, rows_pad, lse2, dvec);
+      heads, nq, head_dim, o_rs, rows_pad, lse2, dvec);
   if ((rc = check_launch()) != BSA_OK) return rc;
   tmap_kernel<<<list_heads * g.fwd.QT, 128, 0, st>>>(row_ptr, cnt, entries, g.fwd.QT, g.KT,
                                                      g.fwd.LR, g.fwd.QB, block_q, g.fwd.expand,
@@ -765,6 +773,7 @@ extern "C" int bsa_attn_bwd(const void* q, const void* k, const void* v, const v
   p.tentries = tentries;
   p.lse2 = lse2;
   p.dvec = dvec;
+  p.out_stride = qkv_rs;
   p.status = status;
   p.timeout_ns = 2000000000ULL;
   // pass 1: dK, dV (rows = key tiles, columns = q-tiles)

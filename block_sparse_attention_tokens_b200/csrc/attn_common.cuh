@@ -249,15 +249,20 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
 }
 
 // 4D map over [B, N, H, D] bf16 (D contiguous), dimensions listed innermost first as
-// (D, H, N, B); box 64 x 1 x box_rows x 1 = box_rows token rows of 128 bytes,
-// 128-byte swizzle.
-int make_map(CUtensorMap* map, const void* base, int B, int N, int H, int D, int box_rows = kBM) {
+// (D, H, N, B); consecutive token rows lie row_stride elements apart (heads * D
+// for a dense tensor, more for a head slice of a wider tensor or a fused QKV
+// buffer) and batches N * row_stride apart.  Box 64 x 1 x box_rows x 1 =
+// box_rows token rows of 128 bytes, 128-byte swizzle.  The map covers only the
+// caller's own buffer (no peer memory), and every load through it is a plain
+// per-CTA TMA load.
+int make_map(CUtensorMap* map, const void* base, int B, int N, int H, int D, long long row_stride,
+             int box_rows = kBM) {
   auto fn = get_encode_fn();
   if (!fn) return BSA_ERR_CUDA;
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
                         static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(B)};
-  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2,
-                           static_cast<cuuint64_t>(N) * H * D * 2};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(row_stride) * 2,
+                           static_cast<cuuint64_t>(N) * row_stride * 2};
   cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
@@ -267,6 +272,16 @@ int make_map(CUtensorMap* map, const void* base, int B, int N, int H, int D, int
 }
 
 bool block_ok(int blk) { return blk == 64 || (blk >= 128 && blk % 128 == 0); }
+
+// Row stride (elements) of a token tensor: 0 selects the dense heads * head_dim;
+// otherwise it must hold a whole row and keep every row 16-byte aligned (the TMA
+// maps need strides in multiples of 16 bytes).  Returns -1 if invalid.
+long long token_row_stride(int row_stride, int heads, int head_dim) {
+  const long long dense = static_cast<long long>(heads) * head_dim;
+  if (row_stride == 0) return dense;
+  if (row_stride < dense || (row_stride % 8) != 0) return -1;
+  return row_stride;
+}
 
 struct Geometry {
   int QB, KB, QT, LR, expand;

@@ -96,6 +96,7 @@ struct AttnParams {
   const int* cnt;
   const uint32_t* entries;
   __nv_bfloat16* o;
+  long long o_stride;  // elements between consecutive token rows of o
   float* lse;
   int* status;
   int* unit_counter;  // next unit to hand out (zeroed before the launch)
@@ -691,7 +692,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         BSA_TRACE_AT(tix + 3);
       }
       if (!ok) break;
-      __nv_bfloat16* orow = p.o + ((static_cast<long long>(me.b) * p.nq + qrow) * p.H + me.h) * D;
+      __nv_bfloat16* orow =
+          p.o + (static_cast<long long>(me.b) * p.nq + qrow) * p.o_stride + static_cast<long long>(me.h) * D;
       float* lrow = p.lse + (static_cast<long long>(me.b) * p.H + me.h) * p.nq + qrow;
       if (me.n == 0) {
         if (qrow < p.nq) {
@@ -800,26 +802,34 @@ namespace {
 // forward entry point applies them: pointers, sizes, list heads, alignment
 // (BSA_ERR_INVALID_ARG), then head_dim and block sizes (BSA_ERR_UNSUPPORTED).
 int check_fwd_args(const void* q, const void* k, const void* v, int batch, int heads, int nq,
-                   int nk, int head_dim, int block_q, int block_k, const int* row_ptr,
-                   const int* col_idx, int list_heads, const void* o, const float* lse) {
+                   int nk, int head_dim, int qkv_row_stride, int o_row_stride, int block_q,
+                   int block_k, const int* row_ptr, const int* col_idx, int list_heads,
+                   const void* o, const float* lse) {
   if (!q || !k || !v || !o || !lse || !row_ptr || !col_idx) return BSA_ERR_INVALID_ARG;
   if (batch < 1 || heads < 1 || nq < 1 || nk < 1) return BSA_ERR_INVALID_ARG;
   if (list_heads != 1 && list_heads != batch * heads) return BSA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return BSA_ERR_INVALID_ARG;
   if (head_dim != 64 && head_dim != 128) return BSA_ERR_UNSUPPORTED;
+  if (token_row_stride(qkv_row_stride, heads, head_dim) < 0 ||
+      token_row_stride(o_row_stride, heads, head_dim) < 0)
+    return BSA_ERR_INVALID_ARG;
   if (!block_ok(block_q) || !block_ok(block_k)) return BSA_ERR_UNSUPPORTED;
   return BSA_OK;
 }
 
 int attn_fwd_impl(const void* q, const void* k, const void* v, int batch, int heads, int nq,
-                  int nk, int head_dim, int block_q, int block_k, const int* row_ptr,
-                  const int* col_idx, int list_heads, float scale, void* o, float* lse, void* ws,
-                  size_t ws_bytes, const int* page_table, int pages_per_batch, int n_pool_pages,
-                  cudaStream_t st) {
+                  int nk, int head_dim, int qkv_row_stride, int o_row_stride, int block_q,
+                  int block_k, const int* row_ptr, const int* col_idx, int list_heads, float scale,
+                  void* o, float* lse, void* ws, size_t ws_bytes, const int* page_table,
+                  int pages_per_batch, int n_pool_pages, cudaStream_t st) {
   if (!ws) return BSA_ERR_INVALID_ARG;
-  int rc0 = check_fwd_args(q, k, v, batch, heads, nq, nk, head_dim, block_q, block_k, row_ptr,
-                           col_idx, list_heads, o, lse);
+  int rc0 = check_fwd_args(q, k, v, batch, heads, nq, nk, head_dim, qkv_row_stride, o_row_stride,
+                           block_q, block_k, row_ptr, col_idx, list_heads, o, lse);
   if (rc0 != BSA_OK) return rc0;
+  const long long qkv_rs = token_row_stride(qkv_row_stride, heads, head_dim);
+  const long long o_rs = token_row_stride(o_row_stride, heads, head_dim);
+  // pools of the paged cache are dense [pages * 128, heads, head_dim]
+  const long long kv_rs = page_table ? static_cast<long long>(heads) * head_dim : qkv_rs;
   if (!aligned16(ws)) return BSA_ERR_INVALID_ARG;
   if (page_table) {
     // pages hold whole key blocks; a shared list needs a single page table
@@ -840,11 +850,11 @@ int attn_fwd_impl(const void* q, const void* k, const void* v, int batch, int he
   CUtensorMap mq, mk, mv, mk64, mv64;
   const int kv_batch = page_table ? 1 : batch;
   const int kv_rows = page_table ? n_pool_pages * kBN : nk;
-  if (make_map(&mq, q, batch, nq, heads, head_dim) != BSA_OK ||
-      make_map(&mk, k, kv_batch, kv_rows, heads, head_dim) != BSA_OK ||
-      make_map(&mv, v, kv_batch, kv_rows, heads, head_dim) != BSA_OK ||
-      make_map(&mk64, k, kv_batch, kv_rows, heads, head_dim, 64) != BSA_OK ||
-      make_map(&mv64, v, kv_batch, kv_rows, heads, head_dim, 64) != BSA_OK)
+  if (make_map(&mq, q, batch, nq, heads, head_dim, qkv_rs) != BSA_OK ||
+      make_map(&mk, k, kv_batch, kv_rows, heads, head_dim, kv_rs) != BSA_OK ||
+      make_map(&mv, v, kv_batch, kv_rows, heads, head_dim, kv_rs) != BSA_OK ||
+      make_map(&mk64, k, kv_batch, kv_rows, heads, head_dim, kv_rs, 64) != BSA_OK ||
+      make_map(&mv64, v, kv_batch, kv_rows, heads, head_dim, kv_rs, 64) != BSA_OK)
     return BSA_ERR_CUDA;
 
   char* wsb = static_cast<char*>(ws);
@@ -877,6 +887,7 @@ int attn_fwd_impl(const void* q, const void* k, const void* v, int batch, int he
   p.cnt = cnt;
   p.entries = entries;
   p.o = static_cast<__nv_bfloat16*>(o);
+  p.o_stride = o_rs;
   p.lse = lse;
   p.status = status;
   p.unit_counter = status + 1;
@@ -892,13 +903,14 @@ int attn_fwd_impl(const void* q, const void* k, const void* v, int batch, int he
 }  // namespace bsa
 
 extern "C" int bsa_attn_fwd(const void* q, const void* k, const void* v, int batch, int heads,
-                            int nq, int nk, int head_dim, int block_q, int block_k,
-                            const int* row_ptr, const int* col_idx, int list_heads, float scale,
-                            void* o, float* lse, void* ws, size_t ws_bytes, void* stream) {
+                            int nq, int nk, int head_dim, int qkv_row_stride, int o_row_stride,
+                            int block_q, int block_k, const int* row_ptr, const int* col_idx,
+                            int list_heads, float scale, void* o, float* lse, void* ws,
+                            size_t ws_bytes, void* stream) {
   BSA_NVTX_RANGE("bsa_attn_fwd");
-  return bsa::attn_fwd_impl(q, k, v, batch, heads, nq, nk, head_dim, block_q, block_k, row_ptr,
-                            col_idx, list_heads, scale, o, lse, ws, ws_bytes, nullptr, 0, 0,
-                            static_cast<cudaStream_t>(stream));
+  return bsa::attn_fwd_impl(q, k, v, batch, heads, nq, nk, head_dim, qkv_row_stride, o_row_stride,
+                            block_q, block_k, row_ptr, col_idx, list_heads, scale, o, lse, ws,
+                            ws_bytes, nullptr, 0, 0, static_cast<cudaStream_t>(stream));
 }
 
 extern "C" int bsa_attn_fwd_paged(const void* q, const void* k_pool, const void* v_pool,
@@ -909,9 +921,10 @@ extern "C" int bsa_attn_fwd_paged(const void* q, const void* k_pool, const void*
                                   size_t ws_bytes, void* stream) {
   BSA_NVTX_RANGE("bsa_attn_fwd_paged");
   if (!page_table) return BSA_ERR_INVALID_ARG;
-  return bsa::attn_fwd_impl(q, k_pool, v_pool, batch, heads, nq, nk, head_dim, block_q, block_k,
-                            row_ptr, col_idx, list_heads, scale, o, lse, ws, ws_bytes, page_table,
-                            pages_per_batch, n_pool_pages, static_cast<cudaStream_t>(stream));
+  return bsa::attn_fwd_impl(q, k_pool, v_pool, batch, heads, nq, nk, head_dim, 0, 0, block_q,
+                            block_k, row_ptr, col_idx, list_heads, scale, o, lse, ws, ws_bytes,
+                            page_table, pages_per_batch, n_pool_pages,
+                            static_cast<cudaStream_t>(stream));
 }
 
 // ---------------------------------------------------------------------------
@@ -994,8 +1007,8 @@ extern "C" int bsa_attn_fwd_noalloc(const void* q, const void* k, const void* v,
   BSA_NVTX_RANGE("bsa_attn_fwd_noalloc");
   using namespace bsa;
   // the same argument checks, in the same order, as bsa_attn_fwd before the size check
-  int rc = check_fwd_args(q, k, v, batch, heads, nq, nk, head_dim, block_q, block_k, row_ptr,
-                          col_idx, list_heads, o, lse);
+  int rc = check_fwd_args(q, k, v, batch, heads, nq, nk, head_dim, 0, 0, block_q, block_k,
+                          row_ptr, col_idx, list_heads, o, lse);
   if (rc != BSA_OK) return rc;
   const size_t need =
       bsa_attn_workspace_size(batch, heads, nq, nk, block_q, block_k, list_heads);
@@ -1009,8 +1022,8 @@ extern "C" int bsa_attn_fwd_noalloc(const void* q, const void* k, const void* v,
   rc = noalloc_scratch(&scratch);
   if (rc != BSA_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  rc = bsa_attn_fwd(q, k, v, batch, heads, nq, nk, head_dim, block_q, block_k, row_ptr, col_idx,
-                    list_heads, scale, o, lse, scratch, kNoAllocScratchBytes, stream);
+  rc = bsa_attn_fwd(q, k, v, batch, heads, nq, nk, head_dim, 0, 0, block_q, block_k, row_ptr,
+                    col_idx, list_heads, scale, o, lse, scratch, kNoAllocScratchBytes, stream);
   if (rc != BSA_OK || device_status == nullptr) return rc;
   cudaError_t e = cudaMemcpyAsync(device_status, scratch, sizeof(int), cudaMemcpyDeviceToDevice, st);
   return e == cudaSuccess ? BSA_OK : record_cuda_error(e);

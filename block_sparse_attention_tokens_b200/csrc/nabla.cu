@@ -42,7 +42,7 @@ __device__ __forceinline__ void add_bf16x8(float* acc, const uint4& v) {
 // grid: x = block index, y = column chunk, z = batch * 2 + tensor (0 = q, 1 = k)
 __global__ void __launch_bounds__(kPoolThreads) nabla_pool_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k, int heads,
-    int head_dim, int nq, int nk, int block, int qb_count, int kb_count,
+    int head_dim, long long row_stride, int nq, int nk, int block, int qb_count, int kb_count,
     float* __restrict__ qbar, float* __restrict__ kbar) {
   const int which = blockIdx.z & 1;
   const int b = blockIdx.z >> 1;
@@ -58,8 +58,8 @@ __global__ void __launch_bounds__(kPoolThreads) nabla_pool_kernel(
   const int r0 = blk * block;
   const int r1 = min(r0 + block, n);
   const uint4* base =
-      reinterpret_cast<const uint4*>(src + (static_cast<long long>(b) * n + r0) * C + col);
-  const long long stride = C / 8;  // uint4 per token row
+      reinterpret_cast<const uint4*>(src + (static_cast<long long>(b) * n + r0) * row_stride + col);
+  const long long stride = row_stride / 8;  // uint4 per token row
   float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   int r = r0;
   for (; r + 4 <= r1; r += 4) {
@@ -303,9 +303,9 @@ extern "C" int bsa_nabla_select(const float* qbar, const float* kbar, int batch,
 }
 
 extern "C" int bsa_nabla_mask(const void* q, const void* k, int batch, int heads, int nq, int nk,
-                              int head_dim, int block, float p, float scale, int kb_begin,
-                              int kb_end, int force_outside, uint8_t* mask, int* near_count,
-                              void* ws, size_t ws_bytes, void* stream) {
+                              int head_dim, int row_stride, int block, float p, float scale,
+                              int kb_begin, int kb_end, int force_outside, uint8_t* mask,
+                              int* near_count, void* ws, size_t ws_bytes, void* stream) {
   BSA_NVTX_RANGE("bsa_nabla_mask");
   using namespace bsa;
   if (!q || !k || !mask || !ws) return BSA_ERR_INVALID_ARG;
@@ -314,6 +314,9 @@ extern "C" int bsa_nabla_mask(const void* q, const void* k, int batch, int heads
     return BSA_ERR_INVALID_ARG;
   if (head_dim != 64 && head_dim != 128) return BSA_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(ws)) return BSA_ERR_INVALID_ARG;
+  const long long dense = static_cast<long long>(heads) * head_dim;
+  const long long rs = row_stride == 0 ? dense : row_stride;
+  if (rs < dense || (rs % 8) != 0) return BSA_ERR_INVALID_ARG;
   const int qb = ceil_div(nq, block), kb = ceil_div(nk, block);
   if (kb_begin < 0 || kb_end > kb || kb_begin > kb_end) return BSA_ERR_INVALID_ARG;
   if (ws_bytes < nabla_ws_bytes(batch, heads, nq, nk, head_dim, block)) return BSA_ERR_WORKSPACE;
@@ -324,7 +327,7 @@ extern "C" int bsa_nabla_mask(const void* q, const void* k, int batch, int heads
   dim3 pgrid(qb > kb ? qb : kb, ceil_div(C, kPoolCols), batch * 2);
   nabla_pool_kernel<<<pgrid, kPoolThreads, 0, st>>>(
       static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), heads,
-      head_dim, nq, nk, block, qb, kb, qbar, kbar);
+      head_dim, rs, nq, nk, block, qb, kb, qbar, kbar);
   int rc = check_launch();
   if (rc != BSA_OK) return rc;
   return launch_select(qbar, kbar, batch, heads, qb, kb, head_dim, p, scale, kb_begin, kb_end,

@@ -53,10 +53,13 @@ __device__ __forceinline__ void copy_row(const uint4* __restrict__ in, uint4* __
 
 // kForward: x (raster, n rows) -> y (tile order, n_pad rows, zero tail)
 // !kForward: y -> x
+// vpr: 16-byte vectors copied per row; svpr / dvpr: row strides of src / dst in
+// 16-byte vectors (>= vpr: a row may be a slice of a wider row, e.g. some heads).
 template <bool kForward>
 __global__ void __launch_bounds__(256) permute_rows_kernel(const uint4* __restrict__ src,
                                                            uint4* __restrict__ dst, int n,
-                                                           int n_pad, int vpr, PermGeo g,
+                                                           int n_pad, int vpr, long long svpr,
+                                                           long long dvpr, PermGeo g,
                                                            long long total_rows) {
   const int lane = threadIdx.x & 31;
   const long long warp0 = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -67,15 +70,15 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(const uint4* __restri
     const int tok = static_cast<int>(r - b * rows_per_batch);
     if (kForward) {
       if (tok >= n) {  // zero tail of the padded sequence
-        uint4* out = dst + (b * n_pad + tok) * vpr;
+        uint4* out = dst + (b * n_pad + tok) * dvpr;
         for (int c = lane; c < vpr; c += 32) out[c] = make_uint4(0, 0, 0, 0);
         continue;
       }
       const long long pos = tile_position(tok, g);
-      copy_row(src + (b * n + tok) * vpr, dst + (b * n_pad + pos) * vpr, vpr, lane);
+      copy_row(src + (b * n + tok) * svpr, dst + (b * n_pad + pos) * dvpr, vpr, lane);
     } else {
       const long long pos = tile_position(tok, g);
-      copy_row(src + (b * n_pad + pos) * vpr, dst + (b * n + tok) * vpr, vpr, lane);
+      copy_row(src + (b * n_pad + pos) * svpr, dst + (b * n + tok) * dvpr, vpr, lane);
     }
   }
 }
@@ -105,10 +108,12 @@ __device__ __forceinline__ int tile_token(long long p, const PermGeo& g) {
 // slice, batch).  Each thread owns 8 adjacent bf16 columns, gathers its column
 // slice of every row of the block (8 rows in flight), stores it in tile order and
 // sums it in fp32.  Rows past N are the zero tail and are not averaged.
-// pooled: [B, heads, NB, head_dim] fp32.
+// pooled: [B, heads, NB, head_dim] fp32.  svpr / dvpr: row strides of src / dst in
+// 16-byte vectors (>= vpr, the vectors of the heads moved).
 __global__ void __launch_bounds__(128) permute_pool_kernel(
     const uint4* __restrict__ src, uint4* __restrict__ dst, int n, int n_pad, int vpr,
-    int head_dim, int heads, int block, PermGeo g, float* __restrict__ pooled) {
+    long long svpr, long long dvpr, int head_dim, int heads, int block, PermGeo g,
+    float* __restrict__ pooled) {
   const int blk = blockIdx.x, b = blockIdx.z;
   const int nb = n_pad / block;
   const long long p0 = static_cast<long long>(blk) * block;
@@ -118,8 +123,8 @@ __global__ void __launch_bounds__(128) permute_pool_kernel(
   for (int r = threadIdx.x; r < block; r += blockDim.x)
     src_row[r] = (p0 + r < n) ? tile_token(p0 + r, g) : -1;
   __syncthreads();
-  const uint4* sb = src + static_cast<long long>(b) * n * vpr;
-  uint4* db = dst + (static_cast<long long>(b) * n_pad + p0) * vpr;
+  const uint4* sb = src + static_cast<long long>(b) * n * svpr;
+  uint4* db = dst + (static_cast<long long>(b) * n_pad + p0) * dvpr;
   for (int v = blockIdx.y * blockDim.x + threadIdx.x; v < vpr && v < (blockIdx.y + 1) * blockDim.x;
        v += blockDim.x) {
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
@@ -127,10 +132,10 @@ __global__ void __launch_bounds__(128) permute_pool_kernel(
     for (; r + 8 <= rows_valid; r += 8) {
       uint4 x[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) x[u] = __ldg(sb + static_cast<long long>(src_row[r + u]) * vpr + v);
+      for (int u = 0; u < 8; ++u) x[u] = __ldg(sb + static_cast<long long>(src_row[r + u]) * svpr + v);
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        db[static_cast<long long>(r + u) * vpr + v] = x[u];
+        db[static_cast<long long>(r + u) * dvpr + v] = x[u];
         const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&x[u]);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -141,8 +146,8 @@ __global__ void __launch_bounds__(128) permute_pool_kernel(
       }
     }
     for (; r < rows_valid; ++r) {
-      const uint4 x = __ldg(sb + static_cast<long long>(src_row[r]) * vpr + v);
-      db[static_cast<long long>(r) * vpr + v] = x;
+      const uint4 x = __ldg(sb + static_cast<long long>(src_row[r]) * svpr + v);
+      db[static_cast<long long>(r) * dvpr + v] = x;
       const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&x);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -151,7 +156,7 @@ __global__ void __launch_bounds__(128) permute_pool_kernel(
         acc[2 * e + 1] += f.y;
       }
     }
-    for (; r < block; ++r) db[static_cast<long long>(r) * vpr + v] = make_uint4(0, 0, 0, 0);
+    for (; r < block; ++r) db[static_cast<long long>(r) * dvpr + v] = make_uint4(0, 0, 0, 0);
     const float inv = rows_valid > 0 ? 1.0f / static_cast<float>(rows_valid) : 0.f;
     const int col = v * 8, h = col / head_dim, j = col - h * head_dim;
     float4* out = reinterpret_cast<float4*>(
@@ -161,8 +166,28 @@ __global__ void __launch_bounds__(128) permute_pool_kernel(
   }
 }
 
+// Row stride in bytes: 0 selects row_bytes (dense rows); otherwise at least
+// row_bytes and a multiple of 16.  Returns -1 if invalid.
+long long row_stride_bytes(long long stride, long long row_bytes) {
+  if (stride == 0) return row_bytes;
+  if (stride < row_bytes || (stride % 16) != 0) return -1;
+  return stride;
+}
+
+// Buffers [batch][rows] of rows `row_bytes` long every `stride` bytes (the last
+// row ends after row_bytes) overlap?
+bool spans_overlap(const void* a, long long a_rows, long long a_stride, const void* b,
+                   long long b_rows, long long b_stride, long long row_bytes) {
+  const char* a0 = static_cast<const char*>(a);
+  const char* b0 = static_cast<const char*>(b);
+  const char* a1 = a0 + (a_rows - 1) * a_stride + row_bytes;
+  const char* b1 = b0 + (b_rows - 1) * b_stride + row_bytes;
+  return a0 < b1 && b0 < a1;
+}
+
 int permute_common(bool forward, const void* src, void* dst, int batch, int T, int H, int W,
-                   int tT, int tH, int tW, int row_bytes, int n_pad, void* stream) {
+                   int tT, int tH, int tW, int row_bytes, int n_pad, int src_stride_bytes,
+                   int dst_stride_bytes, void* stream) {
   if (!src || !dst) return BSA_ERR_INVALID_ARG;
   if (batch < 1 || T < 1 || H < 1 || W < 1 || tT < 1 || tH < 1 || tW < 1 || row_bytes < 16 ||
       (row_bytes % 16) != 0)
@@ -170,13 +195,13 @@ int permute_common(bool forward, const void* src, void* dst, int batch, int T, i
   const long long n = static_cast<long long>(T) * H * W;
   if (n > 0x7fffffffLL || n_pad < n) return BSA_ERR_INVALID_ARG;
   if (!aligned16(src) || !aligned16(dst)) return BSA_ERR_INVALID_ARG;
+  const long long ss = row_stride_bytes(src_stride_bytes, row_bytes);
+  const long long ds = row_stride_bytes(dst_stride_bytes, row_bytes);
+  if (ss < 0 || ds < 0) return BSA_ERR_INVALID_ARG;
   const long long vpr = row_bytes / 16;
-  const char* s0 = static_cast<const char*>(src);
-  const char* d0 = static_cast<const char*>(dst);
   const long long src_rows = forward ? n : n_pad, dst_rows = forward ? n_pad : n;
-  const long long sb = static_cast<long long>(batch) * src_rows * row_bytes;
-  const long long db = static_cast<long long>(batch) * dst_rows * row_bytes;
-  if (s0 < d0 + db && d0 < s0 + sb) return BSA_ERR_INVALID_ARG;  // overlapping buffers
+  if (spans_overlap(src, batch * src_rows, ss, dst, batch * dst_rows, ds, row_bytes))
+    return BSA_ERR_INVALID_ARG;  // overlapping buffers
   PermGeo g{T, H, W, tT, tH, tW};
   const long long total_rows = static_cast<long long>(batch) * (forward ? n_pad : n);
   const int threads = 256;
@@ -187,11 +212,11 @@ int permute_common(bool forward, const void* src, void* dst, int batch, int T, i
   if (forward)
     permute_rows_kernel<true><<<static_cast<int>(blocks), threads, 0, st>>>(
         static_cast<const uint4*>(src), static_cast<uint4*>(dst), static_cast<int>(n), n_pad,
-        static_cast<int>(vpr), g, total_rows);
+        static_cast<int>(vpr), ss / 16, ds / 16, g, total_rows);
   else
     permute_rows_kernel<false><<<static_cast<int>(blocks), threads, 0, st>>>(
         static_cast<const uint4*>(src), static_cast<uint4*>(dst), static_cast<int>(n), n_pad,
-        static_cast<int>(vpr), g, total_rows);
+        static_cast<int>(vpr), ss / 16, ds / 16, g, total_rows);
   return check_launch();
 }
 
@@ -200,7 +225,8 @@ int permute_common(bool forward, const void* src, void* dst, int batch, int T, i
 
 extern "C" int bsa_tile_permute_pool(const void* x, void* y, int batch, int T, int H, int W,
                                      int tT, int tH, int tW, int heads, int head_dim, int n_pad,
-                                     int block, float* pooled, void* stream) {
+                                     int block, float* pooled, int x_row_stride, int y_row_stride,
+                                     void* stream) {
   BSA_NVTX_RANGE("bsa_tile_permute_pool");
   using namespace bsa;
   if (!x || !y || !pooled) return BSA_ERR_INVALID_ARG;
@@ -211,28 +237,32 @@ extern "C" int bsa_tile_permute_pool(const void* x, void* y, int batch, int T, i
   if (n > 0x7fffffffLL || n_pad < n || (n_pad % block) != 0) return BSA_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(y) || !aligned16(pooled)) return BSA_ERR_INVALID_ARG;
   const long long row_bytes = static_cast<long long>(heads) * head_dim * 2;
-  const char* s0 = static_cast<const char*>(x);
-  const char* d0 = static_cast<const char*>(y);
-  if (s0 < d0 + static_cast<long long>(batch) * n_pad * row_bytes &&
-      d0 < s0 + static_cast<long long>(batch) * n * row_bytes)
+  const long long xs = row_stride_bytes(2LL * x_row_stride, row_bytes);
+  const long long ys = row_stride_bytes(2LL * y_row_stride, row_bytes);
+  if (x_row_stride < 0 || y_row_stride < 0 || xs < 0 || ys < 0) return BSA_ERR_INVALID_ARG;
+  if (spans_overlap(x, batch * n, xs, y, batch * static_cast<long long>(n_pad), ys, row_bytes))
     return BSA_ERR_INVALID_ARG;
   PermGeo g{T, H, W, tT, tH, tW};
   const int vpr = static_cast<int>(row_bytes / 16);
   dim3 grid(n_pad / block, ceil_div(vpr, 128), batch);
   permute_pool_kernel<<<grid, 128, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<const uint4*>(x), static_cast<uint4*>(y), static_cast<int>(n), n_pad, vpr,
-      head_dim, heads, block, g, pooled);
+      xs / 16, ys / 16, head_dim, heads, block, g, pooled);
   return check_launch();
 }
 
 extern "C" int bsa_tile_permute(const void* x, void* y, int batch, int T, int H, int W, int tT,
-                                int tH, int tW, int row_bytes, int n_pad, void* stream) {
+                                int tH, int tW, int row_bytes, int n_pad, int x_row_stride_bytes,
+                                int y_row_stride_bytes, void* stream) {
   BSA_NVTX_RANGE("bsa_tile_permute");
-  return bsa::permute_common(true, x, y, batch, T, H, W, tT, tH, tW, row_bytes, n_pad, stream);
+  return bsa::permute_common(true, x, y, batch, T, H, W, tT, tH, tW, row_bytes, n_pad,
+                             x_row_stride_bytes, y_row_stride_bytes, stream);
 }
 
 extern "C" int bsa_tile_untile(const void* y, void* x, int batch, int T, int H, int W, int tT,
-                               int tH, int tW, int row_bytes, int n_pad, void* stream) {
+                               int tH, int tW, int row_bytes, int n_pad, int y_row_stride_bytes,
+                               int x_row_stride_bytes, void* stream) {
   BSA_NVTX_RANGE("bsa_tile_untile");
-  return bsa::permute_common(false, y, x, batch, T, H, W, tT, tH, tW, row_bytes, n_pad, stream);
+  return bsa::permute_common(false, y, x, batch, T, H, W, tT, tH, tW, row_bytes, n_pad,
+                             y_row_stride_bytes, x_row_stride_bytes, stream);
 }

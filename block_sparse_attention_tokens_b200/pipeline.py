@@ -32,13 +32,33 @@ def ar_block_ranges(n_tokens_k: int, tokens_per_frame: int, block: int, anchor_f
     return a_end, max(r_begin, a_end)
 
 
-class Plan:
-    """Buffers and call sequence for one workload on one device."""
+def head_range(rank: int, world: int, heads: int) -> Tuple[int, int]:
+    """Heads [h0, h1) of rank `rank` when `world` ranks share `heads` heads: every
+    (batch, head) row of the attention is independent given Q, K, V and the masks
+    are per head, so the heads split with no exchange between ranks.  The ranges
+    are contiguous, cover every head once and differ in size by at most one."""
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError(f"rank {rank} of {world}")
+    return rank * heads // world, (rank + 1) * heads // world
 
-    def __init__(self, w: Workload, device: torch.device = torch.device("cuda")):
+
+class Plan:
+    """Buffers and call sequence for one workload on one device.
+
+    ``heads=(h0, h1)`` restricts the plan to that range of the workload's heads (a
+    rank's share when the heads are split over GPUs).  ``step`` then takes either
+    the whole-head tensors [B, N, H, D] -- the range is read in place through the
+    library's token-row stride -- or tensors holding only the range's heads."""
+
+    def __init__(self, w: Workload, device: torch.device = torch.device("cuda"),
+                 heads: Optional[Tuple[int, int]] = None):
         self.w = w
         self.dev = device
-        Hh, D, Bt = w.heads, w.head_dim, w.batch
+        self.h0, self.h1 = (0, w.heads) if heads is None else heads
+        if not 0 <= self.h0 < self.h1 <= w.heads:
+            raise ValueError(f"head range {heads} of {w.heads} heads")
+        Hh, D, Bt = self.h1 - self.h0, w.head_dim, w.batch
+        self.heads = Hh
         self.nq, self.nk = w.nq, w.nk
         self.permuted = w.tile is not None
         if self.permuted:
@@ -71,6 +91,7 @@ class Plan:
             dtype=torch.uint8, device=device)
         self.lse = torch.empty((Bt, Hh, self.nq), dtype=torch.float32, device=device)
         self.o = torch.empty((Bt, self.nq, Hh, D), dtype=torch.bfloat16, device=device)
+        self.out = self.o
         if w.tile is not None:
             g, t = w.grid, w.tile
             self.tile_grid = (ceil_div(g[0], t[0]), ceil_div(g[1], t[1]), ceil_div(g[2], t[2]))
@@ -81,8 +102,19 @@ class Plan:
                                             w.recent_frames)
 
     # --- individual stages (each one or a few libbsa launches) ---
+    def _mine(self, t: torch.Tensor) -> torch.Tensor:
+        """This plan's heads of a token tensor: a strided view of a whole-head
+        tensor, or the tensor itself when it holds only the plan's heads."""
+        if t.shape[2] == self.heads:
+            return t
+        if t.shape[2] == self.w.heads:
+            return t[:, :, self.h0:self.h1]
+        raise ValueError(f"tensor with {t.shape[2]} heads for a plan of heads "
+                         f"[{self.h0}, {self.h1}) of {self.w.heads}")
+
     def permute_inputs(self, q, k, v):
         w = self.w
+        q, k, v = self._mine(q), self._mine(k), self._mine(v)
         if w.mask in ("nabla", "nabla_sta"):
             # NABLA pools Q and K per block while they are permuted
             B.bsa_tile_permute_pool(q, w.grid, w.tile, self.n_pad, w.block, y=self.qp,
@@ -108,8 +140,9 @@ class Plan:
                                mask=self.mask, near_count=self.near)
         elif w.mask == "ar":
             a_end, r_begin = self.kb_range
-            B.bsa_nabla_mask(self._q, self._k, w.block, w.p, 0.0, a_end, r_begin, 1, nq=self.nq,
-                             nk=self.nk, mask=self.mask, near_count=self.near, ws=self.nabla_ws)
+            B.bsa_nabla_mask(self._mine(self._q), self._mine(self._k), w.block, w.p, 0.0, a_end,
+                             r_begin, 1, nq=self.nq, nk=self.nk, mask=self.mask,
+                             near_count=self.near, ws=self.nabla_ws)
         else:
             raise ValueError(w.mask)
 
@@ -118,16 +151,23 @@ class Plan:
 
     def attention(self):
         w = self.w
-        q, k, v = (self.qp, self.kp, self.vp) if self.permuted else (self._q, self._k, self._v)
-        out = self.op if self.permuted else self.o
+        if self.permuted:
+            q, k, v, out = self.qp, self.kp, self.vp, self.op
+        else:
+            q, k, v = self._mine(self._q), self._mine(self._k), self._mine(self._v)
+            out = self._mine(self.out)
         B.bsa_attn_fwd(q, k, v, self.row_ptr, self.col_idx, w.block, w.block, self.list_heads,
                        nq=self.nq, nk=self.nk, o=out, lse=self.lse, ws=self.attn_ws)
 
     def untile(self):
-        B.bsa_tile_untile(self.op, self.w.grid, self.w.tile, x=self.o)
+        B.bsa_tile_untile(self.op, self.w.grid, self.w.tile, x=self._mine(self.out))
 
-    def step(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor):
-        """One pass of the whole path.  Returns (O raster order, LSE in the path's token order)."""
+    def step(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+             out: Optional[torch.Tensor] = None):
+        """One pass of the whole path.  Returns (O raster order, LSE in the path's token
+        order).  ``out`` (optional): a whole-head [B, nq, H, D] tensor whose heads of
+        this plan receive O (in place); by default the plan's own O buffer."""
+        self.set_output(out)
         self._q, self._k, self._v = q, k, v
         if self.permuted:
             self.permute_inputs(q, k, v)
@@ -136,7 +176,13 @@ class Plan:
         self.attention()
         if self.permuted:
             self.untile()
-        return self.o, self.lse
+        return self.out, self.lse
+
+    def set_output(self, out: Optional[torch.Tensor] = None):
+        """Where the next steps write O: a whole-head tensor (this plan's heads of
+        it), or the plan's own buffer (None)."""
+        self.out = self.o if out is None else out
+        self._mine(self.out)
 
     def kernel_launches_per_step(self) -> int:
         """libbsa kernels one step launches (for the benchmark's launch count)."""

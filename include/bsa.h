@@ -28,7 +28,14 @@
  *     fallback path of any kind.
  *   - Token tensors are bfloat16, layout [B, N, heads, head_dim] with
  *     head_dim contiguous (one token row = heads * head_dim elements), 16-byte
- *     aligned base addresses.
+ *     aligned base addresses.  Calls that take a row stride also accept token
+ *     rows that are a slice of wider rows: consecutive rows lie row_stride
+ *     elements apart (0 = the dense heads * head_dim; otherwise at least that
+ *     and a multiple of 8) and batches N * row_stride apart.  That runs a range
+ *     of heads of a [B, N, H_total, head_dim] tensor in place (pass the pointer
+ *     to the first head of the range, heads = the range's size, row_stride =
+ *     H_total * head_dim), or Q, K and V straight out of a fused
+ *     [B, N, 3, H, head_dim] projection (row_stride = 3 * H * head_dim).
  *   - Masks are uint8, one byte per (query block, key block), 0 = dropped,
  *     nonzero = kept, row-major [rows][KB].
  *   - Errors never abort the process.  Errors detected on the device (a
@@ -75,17 +82,23 @@ int bsa_version(void);
  * (ragged); they are not padded.  Positions N .. n_pad-1 (N = T*H*W) of the
  * output are written with zeros so the sequence fills whole blocks.
  *
- *   x    : [batch, N, row_bytes] input rows in raster order (any element type)
- *   y    : [batch, n_pad, row_bytes] output rows in tile order
- *   row_bytes : bytes per token row (heads * head_dim * 2 for bf16), multiple of 16
+ *   x    : [batch, N] input rows in raster order (any element type)
+ *   y    : [batch, n_pad] output rows in tile order
+ *   row_bytes : bytes moved per token row (heads * head_dim * 2 for bf16),
+ *               multiple of 16
+ *   x_row_stride_bytes, y_row_stride_bytes : bytes from one row of x / y to the
+ *               next (0 = row_bytes; else >= row_bytes, multiple of 16), so a
+ *               row may be a slice (e.g. a range of heads) of a wider row
  *   n_pad >= N.  x and y must not overlap.
  * bsa_tile_untile is the inverse: reads y (tile order, n_pad rows), writes the
  * N raster-order rows of x; the zero tail of y is not read.
  * ------------------------------------------------------------------------- */
 int bsa_tile_permute(const void* x, void* y, int batch, int T, int H, int W,
-                     int tT, int tH, int tW, int row_bytes, int n_pad, void* stream);
+                     int tT, int tH, int tW, int row_bytes, int n_pad, int x_row_stride_bytes,
+                     int y_row_stride_bytes, void* stream);
 int bsa_tile_untile(const void* y, void* x, int batch, int T, int H, int W,
-                    int tT, int tH, int tW, int row_bytes, int n_pad, void* stream);
+                    int tT, int tH, int tW, int row_bytes, int n_pad, int y_row_stride_bytes,
+                    int x_row_stride_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
  * (a') Tile permute fused with per-block mean pooling.
@@ -98,10 +111,12 @@ int bsa_tile_untile(const void* y, void* x, int batch, int T, int H, int W,
  * the rows that hold tokens (the zero tail is excluded), so the NABLA mask needs
  * no second pass over Q and K.
  *   pooled : [batch, heads, n_pad / block, head_dim] float32, written completely.
+ *   x_row_stride, y_row_stride : token row strides of x and y in elements (0 =
+ *            heads * head_dim; else >= that and a multiple of 8).
  * ------------------------------------------------------------------------- */
 int bsa_tile_permute_pool(const void* x, void* y, int batch, int T, int H, int W, int tT,
                           int tH, int tW, int heads, int head_dim, int n_pad, int block,
-                          float* pooled, void* stream);
+                          float* pooled, int x_row_stride, int y_row_stride, void* stream);
 
 /* ---------------------------------------------------------------------------
  * (b1) Sliding Tile Attention mask.
@@ -145,7 +160,8 @@ int bsa_radial_mask(int n_tokens, int tokens_per_frame, int block, uint8_t* mask
  * part 2 -- persistent anchor frames and recent frames kept, sparse selection
  * elsewhere.
  *
- *   q : [batch, nq, heads, head_dim] bf16 (tile order); k : [batch, nk, ...]
+ *   q : [batch, nq, heads, head_dim] bf16 (tile order); k : [batch, nk, ...];
+ *   row_stride : token row stride of q and k in elements (0 = heads * head_dim)
  *   Blocks of `block` tokens; the last block of q / k may be partial and is
  *   averaged over its valid tokens only.  QB = ceil(nq/block), KB = ceil(nk/block).
  *   Row (b, h, qb): logits z_c = mean_q . mean_k[c] * scale (scale <= 0 means
@@ -162,8 +178,8 @@ int bsa_radial_mask(int n_tokens, int tokens_per_frame, int block, uint8_t* mask
  * ------------------------------------------------------------------------- */
 size_t bsa_nabla_workspace_size(int batch, int heads, int nq, int nk, int head_dim, int block);
 int bsa_nabla_mask(const void* q, const void* k, int batch, int heads, int nq, int nk,
-                   int head_dim, int block, float p, float scale, int kb_begin, int kb_end,
-                   int force_outside, uint8_t* mask, int* near_count, void* ws,
+                   int head_dim, int row_stride, int block, float p, float scale, int kb_begin,
+                   int kb_end, int force_outside, uint8_t* mask, int* near_count, void* ws,
                    size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
@@ -216,7 +232,9 @@ int bsa_mask_compact(const uint8_t* mask, int rows, int KB, int* row_ptr, int* c
  *
  *   q : [batch, nq, heads, head_dim] bf16; k, v : [batch, nk, heads, head_dim]
  *   o : [batch, nq, heads, head_dim] bf16 (rows >= nq are never written)
- *   lse : [batch, heads, nq] float32
+ *   qkv_row_stride : token row stride of q, k and v in elements; o_row_stride :
+ *       that of o (each 0 = heads * head_dim; see the conventions above)
+ *   lse : [batch, heads, nq] float32 (dense, for the heads of this call)
  *   row_ptr, col_idx : CSR over rows m * QB + qb (QB = ceil(nq/block_q)),
  *                      col_idx ascending within a row, values < KB = ceil(nk/block_k)
  *                      (as written by bsa_mask_compact).  Malformed lists set
@@ -230,9 +248,9 @@ int bsa_mask_compact(const uint8_t* mask, int rows, int KB, int* row_ptr, int* c
 size_t bsa_attn_workspace_size(int batch, int heads, int nq, int nk, int block_q, int block_k,
                                int list_heads);
 int bsa_attn_fwd(const void* q, const void* k, const void* v, int batch, int heads, int nq,
-                 int nk, int head_dim, int block_q, int block_k, const int* row_ptr,
-                 const int* col_idx, int list_heads, float scale, void* o, float* lse,
-                 void* ws, size_t ws_bytes, void* stream);
+                 int nk, int head_dim, int qkv_row_stride, int o_row_stride, int block_q,
+                 int block_k, const int* row_ptr, const int* col_idx, int list_heads,
+                 float scale, void* o, float* lse, void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
  * (e) Block-sparse attention backward.
@@ -251,6 +269,8 @@ int bsa_attn_fwd(const void* q, const void* k, const void* v, int batch, int hea
  *   o, lse : that call's outputs; dout : dL/dO, same layout as o (bf16)
  *   dq : [batch, nq, heads, head_dim] bf16, written (rows with no kept key: 0)
  *   dk, dv : [batch, nk, heads, head_dim] bf16, written (keys no row keeps: 0)
+ *   qkv_row_stride : token row stride (elements) of q, k, v, dq, dk and dv;
+ *   o_row_stride : that of o and dout (each 0 = heads * head_dim)
  *   head_dim in {64, 128}; block_q, block_k each 64 or a multiple of 128.
  *   ws : device workspace of at least bsa_attn_bwd_workspace_size() bytes (its
  *        status word, read with bsa_read_status, is cleared by every call).
@@ -262,9 +282,9 @@ size_t bsa_attn_bwd_workspace_size(int batch, int heads, int nq, int nk, int blo
                                    int block_k, int list_heads);
 int bsa_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
                  const float* lse, int batch, int heads, int nq, int nk, int head_dim,
-                 int block_q, int block_k, const int* row_ptr, const int* col_idx,
-                 int list_heads, float scale, void* dq, void* dk, void* dv, void* ws,
-                 size_t ws_bytes, void* stream);
+                 int qkv_row_stride, int o_row_stride, int block_q, int block_k,
+                 const int* row_ptr, const int* col_idx, int list_heads, float scale, void* dq,
+                 void* dk, void* dv, void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
  * (d') Block-sparse attention forward that allocates nothing.
@@ -275,9 +295,9 @@ int bsa_attn_bwd(const void* q, const void* k, const void* v, const void* o, con
  * inside a host framework that owns every device allocation through its own
  * pre-reserved pool, or a serving loop where a cudaMalloc (which may
  * synchronise the device) is not permitted.  Same arguments and results as
- * bsa_attn_fwd, without ws / ws_bytes: the workspace is a fixed 8 MiB device
- * array inside libbsa.so, which every GPU that loads the library holds until
- * the process exits.
+ * bsa_attn_fwd with dense token rows (both row strides 0), without ws /
+ * ws_bytes: the workspace is a fixed 8 MiB device array inside libbsa.so,
+ * which every GPU that loads the library holds until the process exits.
  *   - Shapes whose bsa_attn_workspace_size() exceeds 8 MiB are rejected with
  *     BSA_ERR_WORKSPACE (see bsa_last_error_message()) before any work.
  *   - Arguments are checked as bsa_attn_fwd checks them, in the same order and

@@ -59,24 +59,31 @@ def test_status_strings_and_version(lib):
 
 def test_host_argument_validation_without_gpu(lib, no_gpu):
     # null pointers and bad shapes are rejected before anything touches CUDA
-    assert lib.bsa_tile_permute(None, None, 1, 2, 2, 2, 1, 1, 1, 256, 8, None) == 1
+    assert lib.bsa_tile_permute(None, None, 1, 2, 2, 2, 1, 1, 1, 256, 8, 0, 0, None) == 1
     assert lib.bsa_sta_mask(1, 1, 1, 1, 1, 1, 0, None, None) == 1
     assert lib.bsa_radial_mask(10, 4, 4, None, None) == 1
     assert lib.bsa_mask_compact(None, 4, 4, None, None, None) == 1
     fake = ctypes.c_void_p(16)
     # unsupported head_dim / block sizes -> BSA_ERR_UNSUPPORTED
-    args = [fake, fake, fake, 1, 2, 256, 256, 96, 128, 128, fake, fake, 1, 0.0, fake, fake, fake,
-            1 << 20, None]
+    # q k v B H nq nk d qkv_stride o_stride bq bk row_ptr col_idx list_heads scale o lse ws ws_bytes
+    args = [fake, fake, fake, 1, 2, 256, 256, 96, 0, 0, 128, 128, fake, fake, 1, 0.0, fake, fake,
+            fake, 1 << 20, None]
     assert lib.bsa_attn_fwd(*args) == 2
-    args[7], args[8] = 128, 192
+    args[7], args[10] = 128, 192
     assert lib.bsa_attn_fwd(*args) == 2
     # workspace too small -> BSA_ERR_WORKSPACE
-    args[8] = 128
-    args[17] = 16
+    args[10] = 128
+    args[19] = 16
     assert lib.bsa_attn_fwd(*args) == 3
     # list_heads must be 1 or batch*heads
-    args[12] = 3
+    args[14] = 3
     assert lib.bsa_attn_fwd(*args) == 1
+    # row strides: shorter than a row (2 heads x 128), or rows not 16-byte aligned
+    args[14] = 1
+    for i, val in ((8, 128), (8, 260), (9, 255)):
+        bad = list(args)
+        bad[i] = val
+        assert lib.bsa_attn_fwd(*bad) == 1, (i, val)
 
 
 def test_every_entry_rejects_bad_arguments_before_touching_cuda(lib, no_gpu):
@@ -86,12 +93,14 @@ def test_every_entry_rejects_bad_arguments_before_touching_cuda(lib, no_gpu):
     A = ctypes.c_void_p(16)          # 16-byte aligned stand-in; never dereferenced here
     U = ctypes.c_void_p(8)           # not 16-byte aligned
     INV, UNS, WS = 1, 2, 3
-    # backward: q k v o dO lse B H nq nk d bq bk row_ptr col_idx list_heads scale dq dk dv ws ws_bytes
-    bwd = [A, A, A, A, A, A, 1, 2, 256, 256, 128, 128, 128, A, A, 1, 0.0, A, A, A, A, 1 << 30, None]
-    assert lib.bsa_attn_bwd(*([None] * 6 + bwd[6:13] + [None, None] + bwd[15:17] + [None] * 4
-                               + bwd[21:])) == INV
-    for i, val, rc in ((10, 96, UNS), (11, 192, UNS), (21, 16, WS), (15, 3, INV), (0, U, INV),
-                       (20, U, INV)):
+    # backward: q k v o dO lse B H nq nk d qkv_rs o_rs bq bk row_ptr col_idx list_heads scale
+    #           dq dk dv ws ws_bytes
+    bwd = [A, A, A, A, A, A, 1, 2, 256, 256, 128, 0, 0, 128, 128, A, A, 1, 0.0, A, A, A, A, 1 << 30,
+           None]
+    assert lib.bsa_attn_bwd(*([None] * 6 + bwd[6:15] + [None, None] + bwd[17:19] + [None] * 4
+                               + bwd[23:])) == INV
+    for i, val, rc in ((10, 96, UNS), (13, 192, UNS), (23, 16, WS), (17, 3, INV), (0, U, INV),
+                       (22, U, INV), (11, 200, INV), (12, 260, INV)):
         args = list(bwd)
         args[i] = val
         assert lib.bsa_attn_bwd(*args) == rc, (i, val)
@@ -127,23 +136,25 @@ def test_every_entry_rejects_bad_arguments_before_touching_cuda(lib, no_gpu):
         if i == 9:
             args[10] = 4                                         # kb_begin > kb_end
         assert lib.bsa_nabla_select(*args) == rc, (i, val)
-    # NABLA mask (q k B H nq nk d block p scale kb_begin kb_end force mask near ws ws_bytes)
-    nm = [A, A, 1, 2, 1000, 1000, 128, 64, 0.9, 0.0, 0, 16, 0, A, None, A, 1 << 30, None]
-    for i, val, rc in ((7, 8, INV), (7, 72, INV), (16, 64, WS), (0, U, INV), (11, 17, INV),
-                       (6, 32, UNS)):
+    # NABLA mask (q k B H nq nk d row_stride block p scale kb_begin kb_end force mask near ws
+    #             ws_bytes)
+    nm = [A, A, 1, 2, 1000, 1000, 128, 0, 64, 0.9, 0.0, 0, 16, 0, A, None, A, 1 << 30, None]
+    for i, val, rc in ((8, 8, INV), (8, 72, INV), (17, 64, WS), (0, U, INV), (12, 17, INV),
+                       (6, 32, UNS), (7, 250, INV), (7, 260, INV)):
         args = list(nm)
         args[i] = val
         assert lib.bsa_nabla_mask(*args) == rc, (i, val)
-    # permutes: x y B T H W tT tH tW row_bytes n_pad
+    # permutes: x y B T H W tT tH tW row_bytes n_pad x_stride y_stride (bytes)
     for f in (lib.bsa_tile_permute, lib.bsa_tile_untile):
-        base = [A, ctypes.c_void_p(1 << 40), 1, 4, 8, 8, 4, 4, 4, 256, 256, None]
-        for i, val in ((9, 8), (9, 24), (10, 255), (1, A), (0, U), (6, 0)):
+        base = [A, ctypes.c_void_p(1 << 40), 1, 4, 8, 8, 4, 4, 4, 256, 256, 0, 0, None]
+        for i, val in ((9, 8), (9, 24), (10, 255), (1, A), (0, U), (6, 0), (11, 128), (12, 264)):
             args = list(base)
             args[i] = val
             assert f(*args) == INV, (f, i, val)
-    # fused permute + pooling: x y B T H W tT tH tW heads d n_pad block pooled
-    pp = [A, ctypes.c_void_p(1 << 40), 1, 4, 8, 8, 4, 4, 4, 2, 128, 256, 64, A, None]
-    for i, val in ((11, 250), (12, 96), (12, 2048), (10, 12), (1, A), (13, U)):
+    # fused permute + pooling: x y B T H W tT tH tW heads d n_pad block pooled x_rs y_rs
+    pp = [A, ctypes.c_void_p(1 << 40), 1, 4, 8, 8, 4, 4, 4, 2, 128, 256, 64, A, 0, 0, None]
+    for i, val in ((11, 250), (12, 96), (12, 2048), (10, 12), (1, A), (13, U), (14, 128),
+                   (15, 260)):
         args = list(pp)
         args[i] = val
         assert lib.bsa_tile_permute_pool(*args) == INV, (i, val)
@@ -241,7 +252,7 @@ def test_header_compiles_as_c_and_links(tmp_path, lib, no_gpu):
 #include <stdio.h>
 #include "bsa.h"
 int main(void) {
-  if (bsa_version() < 100) return 1;
+  if (bsa_version() < 200) return 1;
   if (bsa_sta_mask(1, 1, 1, 1, 1, 1, 0, NULL, NULL) != BSA_ERR_INVALID_ARG) return 2;
   if (bsa_attn_workspace_size(1, 1, 1, 1, 96, 128, 1) != 0) return 3;
   printf("%s\n", bsa_status_string(BSA_ERR_TIMEOUT));

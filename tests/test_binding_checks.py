@@ -34,3 +34,24 @@ def test_row_rule_of_the_permutes():
     assert "rows for" in B._row_problem((1, 100, 2, 64), 2, 1, 105, 256)
     assert "bytes" in B._row_problem((1, 105, 2, 32), 2, 1, 105, 256)
     assert "must be" in B._row_problem((3, 105, 2, 64), 2, 2, 105, 256)
+
+
+def test_row_stride_rule_of_strided_token_tensors():
+    # head slice of a [2, 700, 8, 64] tensor: rows 512 elements apart, batches 700 rows apart
+    full = torch.empty(2, 700, 8, 64, dtype=BF)
+    sl = full[:, :, 2:5]
+    assert B._stride_problem(tuple(sl.shape), tuple(sl.stride()), 700, 3 * 64, 8) is None
+    # Q of a fused [1, 300, 3, 4, 64] projection: rows 768 elements apart
+    qkv = torch.empty(1, 300, 3, 4, 64, dtype=BF)
+    q = qkv[:, :, 0]
+    assert B._stride_problem(tuple(q.shape), tuple(q.stride()), 300, 4 * 64, 8) is None
+    # a padded batch stride (rows per batch != n) is refused for several batches
+    pad = torch.empty(2, 704, 3, 64, dtype=BF)
+    assert "batch stride" in B._stride_problem(tuple(pad.shape), tuple(pad.stride()), 700,
+                                               3 * 64, 8)
+    # transposed heads (head_dim not innermost-contiguous) and rows that do not fit
+    tr = torch.empty(1, 100, 64, 4, dtype=BF).transpose(2, 3)
+    assert "contiguous" in B._stride_problem(tuple(tr.shape), tuple(tr.stride()), 100, 256, 8)
+    odd = torch.empty(1, 100, 260, dtype=BF)[:, :, :256].reshape(1, 100, 4, 64)
+    assert "multiple of 8" in B._stride_problem(tuple(odd.shape), tuple(odd.stride()), 100,
+                                                256, 8)
