@@ -46,3 +46,54 @@ def test_single_process_is_the_identity():
     import bench
     assert bench.max_over_ranks([3.0, 4.0]) == [3.0, 4.0]
     assert abs(bench.weak_scaling_value(1e12, 1, 10.0) - 100.0) < 1e-9
+
+
+def test_head_ranges_cover_every_head_once_and_balance():
+    from block_sparse_attention_tokens_b200.pipeline import head_range
+    for heads in (1, 2, 5, 12, 16, 24, 40):
+        for world in range(1, min(heads, 8) + 1):
+            ranges = [head_range(r, world, heads) for r in range(world)]
+            assert ranges[0][0] == 0 and ranges[-1][1] == heads
+            assert all(a[1] == b[0] for a, b in zip(ranges, ranges[1:]))
+            sizes = [h1 - h0 for h0, h1 in ranges]
+            assert min(sizes) >= 1 and max(sizes) - min(sizes) <= 1
+
+
+def _head_split_main(rank, world, port, out):
+    """Each rank evaluates the oracle's attention on its own heads only; the host
+    gathers the pieces (test-side reassembly; the library path has no exchange)."""
+    import datetime
+    import numpy as np
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    import oracle as O
+    from block_sparse_attention_tokens_b200.pipeline import head_range
+    rng = np.random.default_rng(5)                    # the same inputs on every rank
+    Bn, H, n, D, blk = 1, 5, 200, 16, 64
+    q, k, v = (rng.standard_normal((Bn, n, H, D)) for _ in range(3))
+    mask = (rng.random((H, 4, 4)) < 0.6).astype(np.uint8)
+    h0, h1 = head_range(rank, world, H)
+    o, lse = O.block_sparse_attention(q[:, :, h0:h1], k[:, :, h0:h1], v[:, :, h0:h1],
+                                      mask[h0:h1], blk, blk)
+    pieces = [None] * world
+    dist.all_gather_object(pieces, (h0, h1, o, lse))
+    o_all = np.concatenate([p[2] for p in sorted(pieces, key=lambda p: p[0])], axis=2)
+    lse_all = np.concatenate([p[3] for p in sorted(pieces, key=lambda p: p[0])], axis=1)
+    ref_o, ref_lse = O.block_sparse_attention(q, k, v, mask, blk, blk)
+    out[rank] = (bool(np.array_equal(o_all, ref_o)), bool(np.array_equal(lse_all, ref_lse)),
+                 (h0, h1))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_split_heads_and_reassemble_exactly():
+    world = 2
+    manager = mp.Manager()
+    out = manager.dict()
+    mp.spawn(_head_split_main, args=(world, _free_port(), out), nprocs=world, join=True)
+    assert out[0][2] == (0, 2) and out[1][2] == (2, 5)
+    for rank in range(world):
+        assert out[rank][0] and out[rank][1]
