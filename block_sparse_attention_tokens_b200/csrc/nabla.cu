@@ -12,9 +12,11 @@
 //   pool   : HBM-bound column sums.  One CTA per (tensor, batch, block, 1024-column
 //            chunk); each thread owns 8 adjacent bf16 columns (one 16-byte vector
 //            per token row) and accumulates in fp32 over the block's valid rows.
-//   select : one CTA per (batch, head, 8 query blocks).  Pooled keys stream
-//            through shared memory in tiles of 32 blocks; every thread forms one
-//            logit per tile.  Each warp then owns one query row: softmax
+//   select : one CTA per (batch, head, up to 8 query blocks: fewer when the key
+//            range is long, so that the rows' logits fit in shared memory).
+//            Pooled keys stream through shared memory in tiles of 32 blocks;
+//            every thread forms one (partial) logit per tile.  Each warp then
+//            owns one query row: softmax
 //            statistics, a 32-step radix search over the order-preserving integer
 //            image of the fp32 logits for the cut, ties resolved to the lower
 //            block index, and the row of mask bytes.
@@ -98,31 +100,40 @@ __device__ __forceinline__ int warp_isum(int v) {
   return v;
 }
 
-// grid: x = ceil(QB / kSelRows), y = heads, z = batch; 256 threads.
-// dynamic smem: qs[kSelRows][D] + ks[kSelTile][D+1] + z[kSelRows][nr] + e[kSelRows][nr]
+// grid: x = ceil(QB / rows), y = heads, z = batch; 256 threads (8 warps).
+// `rows` (1, 2, 4 or 8) query rows per CTA, chosen by the host so that the rows'
+// logits fit in shared memory: 8 for short key ranges, fewer for long ones.  In
+// the logit phase the 8 / rows warps of a row split head_dim and add their
+// partial dot products; in the selection phase warp r owns row r.
+// dynamic smem: qs[rows][D] + ks[kSelTile][D+1] + pz[8][32] + z[rows][nr] + e[rows][nr]
 template <int D>
 __global__ void __launch_bounds__(256) nabla_select_kernel(
     const float* __restrict__ qbar, const float* __restrict__ kbar, int heads, int qb_count,
     int kb_count, int kb_begin, int kb_end, float p, float scale, int force_outside,
     const uint8_t* __restrict__ base_mask, const uint8_t* __restrict__ key_allowed,
-    uint8_t* __restrict__ mask, int* __restrict__ near_count) {
+    uint8_t* __restrict__ mask, int* __restrict__ near_count, int rows) {
   extern __shared__ float smem[];
   const int nr = kb_end - kb_begin;
+  const int parts = kSelRows / rows;       // warps per row in the logit phase
   float* qs = smem;
-  float* ks = qs + kSelRows * D;
-  float* zs = ks + kSelTile * (D + 1);
-  float* es = zs + kSelRows * nr;
+  float* ks = qs + rows * D;
+  float* pz = ks + kSelTile * (D + 1);
+  float* zs = pz + kSelRows * 32;
+  float* es = zs + rows * nr;
   const int b = blockIdx.z, h = blockIdx.y;
-  const int q0 = blockIdx.x * kSelRows;
+  const int q0 = blockIdx.x * rows;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const float* qsrc = qbar + (static_cast<long long>(b) * heads + h) * qb_count * D;
   const float* ksrc = kbar + (static_cast<long long>(b) * heads + h) * kb_count * D;
 
-  for (int i = tid; i < kSelRows * D; i += blockDim.x) {
+  for (int i = tid; i < rows * D; i += blockDim.x) {
     const int r = i / D;
     qs[i] = (q0 + r < qb_count) ? qsrc[static_cast<long long>(q0 + r) * D + (i - r * D)] : 0.f;
   }
-  // logits z[r][c] = qbar[r] . kbar[kb_begin + c] * scale
+  // logits z[r][c] = qbar[r] . kbar[kb_begin + c] * scale; warp w forms the partial
+  // dot product of row w % rows over head_dim slice w / rows
+  const int lr = warp % rows, part = warp / rows;
+  const int j0 = part * (D / parts), j1 = j0 + D / parts;
   for (int t0 = 0; t0 < nr; t0 += kSelTile) {
     __syncthreads();
     for (int i = tid; i < kSelTile * D; i += blockDim.x) {
@@ -131,15 +142,26 @@ __global__ void __launch_bounds__(256) nabla_select_kernel(
           (t0 + c < nr) ? ksrc[static_cast<long long>(kb_begin + t0 + c) * D + j] : 0.f;
     }
     __syncthreads();
-    const float* qrow = qs + warp * D;
+    const float* qrow = qs + lr * D;
     const float* krow = ks + lane * (D + 1);
     float acc = 0.f;
 #pragma unroll 8
-    for (int j = 0; j < D; ++j) acc = fmaf(qrow[j], krow[j], acc);
-    if (t0 + lane < nr) zs[warp * nr + t0 + lane] = acc * scale;
+    for (int j = j0; j < j1; ++j) acc = fmaf(qrow[j], krow[j], acc);
+    if (parts == 1) {
+      if (t0 + lane < nr) zs[lr * nr + t0 + lane] = acc * scale;
+    } else {
+      pz[warp * 32 + lane] = acc;
+      __syncthreads();
+      if (part == 0 && t0 + lane < nr) {
+        float sum = 0.f;
+        for (int q = 0; q < parts; ++q) sum += pz[(q * rows + lr) * 32 + lane];
+        zs[lr * nr + t0 + lane] = sum * scale;
+      }
+    }
   }
   __syncthreads();
 
+  if (warp >= rows) return;
   const int qb = q0 + warp;
   if (qb >= qb_count) return;
   uint8_t* mrow = mask + ((static_cast<long long>(b) * heads + h) * qb_count + qb) * kb_count;
@@ -249,21 +271,32 @@ extern "C" size_t bsa_nabla_workspace_size(int batch, int heads, int nq, int nk,
 namespace bsa {
 namespace {
 
+// Shared memory of the selection kernel for `rows` query rows per CTA.
+size_t select_smem(int rows, int head_dim, int nr) {
+  return sizeof(float) * (static_cast<size_t>(rows) * head_dim +
+                          static_cast<size_t>(kSelTile) * (head_dim + 1) +
+                          static_cast<size_t>(kSelRows) * 32 + 2 * static_cast<size_t>(rows) * nr);
+}
+
+constexpr size_t kSelSmemLimit = 200 * 1024;
+
 int launch_select(const float* qbar, const float* kbar, int batch, int heads, int qb, int kb,
                   int head_dim, float p, float scale, int kb_begin, int kb_end, int force_outside,
                   const uint8_t* base_mask, const uint8_t* key_allowed, uint8_t* mask,
                   int* near_count, cudaStream_t st) {
   const int nr = kb_end - kb_begin;
-  const size_t smem = sizeof(float) * (static_cast<size_t>(kSelRows) * head_dim +
-                                       static_cast<size_t>(kSelTile) * (head_dim + 1) +
-                                       2 * static_cast<size_t>(kSelRows) * nr);
-  if (smem > 200 * 1024) return BSA_ERR_UNSUPPORTED;
+  // as many rows per CTA as the rows' logits allow (8 up to ~2,900 candidate key
+  // blocks at head_dim 128, 1 up to ~23,000)
+  int rows = kSelRows;
+  while (rows > 1 && select_smem(rows, head_dim, nr) > kSelSmemLimit) rows >>= 1;
+  const size_t smem = select_smem(rows, head_dim, nr);
+  if (smem > kSelSmemLimit) return BSA_ERR_UNSUPPORTED;
   if (scale <= 0.0f) scale = 1.0f / sqrtf(static_cast<float>(head_dim));
   if (near_count) {
     cudaError_t e = cudaMemsetAsync(near_count, 0, sizeof(int), st);
     if (e != cudaSuccess) return record_cuda_error(e);
   }
-  dim3 sgrid(ceil_div(qb, kSelRows), heads, batch);
+  dim3 sgrid(ceil_div(qb, rows), heads, batch);
   cudaError_t e;
   if (head_dim == 128) {
     e = cudaFuncSetAttribute(nabla_select_kernel<128>,
@@ -271,14 +304,14 @@ int launch_select(const float* qbar, const float* kbar, int batch, int heads, in
     if (e != cudaSuccess) return record_cuda_error(e);
     nabla_select_kernel<128><<<sgrid, 256, smem, st>>>(qbar, kbar, heads, qb, kb, kb_begin, kb_end,
                                                        p, scale, force_outside, base_mask, key_allowed, mask,
-                                                       near_count);
+                                                       near_count, rows);
   } else {
     e = cudaFuncSetAttribute(nabla_select_kernel<64>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return record_cuda_error(e);
     nabla_select_kernel<64><<<sgrid, 256, smem, st>>>(qbar, kbar, heads, qb, kb, kb_begin, kb_end,
                                                       p, scale, force_outside, base_mask, key_allowed, mask,
-                                                      near_count);
+                                                      near_count, rows);
   }
   return check_launch();
 }

@@ -333,3 +333,32 @@ def test_backward_column_sampling_is_exact_on_dk_dv():
         for qb in range(QB):
             if not mask[h, qb, wanted].any():
                 assert np.all(part[0][0, qb * bq:(qb + 1) * bq, h] == 0)
+
+
+def test_nabla_mask_at_long_key_ranges():
+    # 7,088 key blocks (453,600 tokens in 64-token blocks): a closed-form row --
+    # five blocks at logit 12, the rest at 0, so the five hold 5e^12 / (5e^12 + 7083)
+    # > 0.9 of the mass and no four of them reach 0.9 -- keeps exactly those five;
+    # random rows keep the shortest prefix reaching p (checked against the sorted
+    # probabilities directly)
+    KB, D, p = 7088, 16, 0.9
+    hot = np.array([3, 1000, 4096, 7000, KB - 1])
+    kbar = np.zeros((1, 1, KB, D))
+    kbar[0, 0, hot, 0] = 3.0
+    qbar = np.zeros((1, 1, 2, D))
+    qbar[0, 0, 0, 0] = 4.0
+    qbar[0, 0, 1] = np.random.default_rng(7).standard_normal(D)
+    kbar[0, 0, :, 1:] = np.random.default_rng(8).standard_normal((KB, D - 1))
+    kbar_hot_only = kbar.copy()
+    kbar_hot_only[0, 0, :, 1:] = 0.0
+    m, near = O.nabla_mask(qbar[:, :, :1], kbar_hot_only, p, 1.0)
+    assert np.array_equal(np.nonzero(m[0, 0, 0])[0], hot) and not near.any()
+    m, _ = O.nabla_mask(qbar[:, :, 1:], kbar, p, 0.3)
+    z = (kbar[0, 0] @ qbar[0, 0, 1]) * 0.3
+    pr = np.exp(z - z.max())
+    pr /= pr.sum()
+    kept = m[0, 0, 0] != 0
+    srt = np.sort(pr)[::-1]
+    k = int(kept.sum())
+    assert pr[kept].sum() >= p and srt[:k - 1].sum() < p
+    assert pr[kept].min() >= pr[~kept].max()
