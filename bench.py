@@ -63,17 +63,20 @@ def with_nominal(roofline: dict) -> dict:
 
 
 def choose_tensor_peak(peaks: dict, clocks: dict, timed_s: float):
-    """The bf16 peak a kernel timed in this run is held to: the burst figure
-    (a GEMM timed alone, at the maximum clock) when the timed region was short
-    (under 3 s) or the median SM clock stayed within 3 % of the maximum, else the
-    sustained figure (a seconds-long GEMM loop under the power cap)."""
+    """The bf16 peak a kernel timed in this run is held to: the burst figure (a GEMM
+    timed alone, at the maximum clock) when the median SM clock over the timed
+    region stayed within 3 % of the maximum, else the sustained figure (a
+    seconds-long GEMM loop under the power cap): a kernel that itself drove the
+    clock down under the power cap is compared with the GEMM under the same cap,
+    however short the region.  Without clock samples the burst figure is used."""
     mhz, mx = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
-    at_max = bool(mhz and mx and mhz >= 0.97 * mx)
-    if timed_s < 3.0 or at_max:
-        why = "timed region under 3 s" if timed_s < 3.0 else "median SM clock at its maximum"
-        return peaks["bf16_tflops"], "burst", why
+    if not (mhz and mx):
+        return peaks["bf16_tflops"], "burst", "no clock samples"
+    if mhz >= 0.97 * mx:
+        return peaks["bf16_tflops"], "burst", \
+            f"median SM clock {mhz:.0f} of {mx:.0f} MHz over {timed_s:.1f} s"
     return peaks["bf16_tflops_sustained"], "sustained", \
-        f"{timed_s:.1f} s timed region, median SM clock {mhz} of {mx} MHz"
+        f"median SM clock {mhz:.0f} of {mx:.0f} MHz over {timed_s:.1f} s (power cap)"
 
 
 def tensor_roofline(achieved: float, kernel_ms: float, peaks: dict, peak_kind: str,

@@ -49,16 +49,37 @@ namespace {
 constexpr int kThreads = 320;
 constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = 9;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // The fast path keeps the running max while a tile's P sum stays <= 2^12.
 constexpr float kFastSumLimit = 4096.0f;
-// Optional software 2^x (FMA pipe) for a quarter of the fast-path exponentials, to
-// relieve the MUFU (one exponential per 512 tensor FLOPs at head_dim 128); off by
-// default: it measured slower on the attention workloads.
+// Optional software 2^x (FMA pipe) for BSA_POLY_PAIRS of every 16 column pairs of
+// the fast path's exponentials, to relieve the MUFU (one exponential per 512 tensor
+// FLOPs at head_dim 128); 0 by default.  BSA_POLY_EXP2=1 is the older spelling of
+// 4 pairs in 16.
 #ifndef BSA_POLY_EXP2
 #define BSA_POLY_EXP2 0
 #endif
-constexpr bool kPolyExp2 = BSA_POLY_EXP2 != 0;
+#ifndef BSA_POLY_PAIRS
+#define BSA_POLY_PAIRS (BSA_POLY_EXP2 ? 4 : 0)
+#endif
+constexpr int kPolyPairs = BSA_POLY_PAIRS;
+static_assert(kPolyPairs >= 0 && kPolyPairs <= 16, "BSA_POLY_PAIRS is 0..16");
+// Pair i of a 16-pair chunk goes to the polynomial: spread evenly over the chunk.
+__device__ __forceinline__ constexpr bool poly_pair(int i) {
+  return kPolyPairs > 0 && (i * kPolyPairs) % 16 < kPolyPairs;
+}
+// Optional packed bf16 exponentials in the fast path (one MUFU operation per column
+// pair; the argument is rounded to bf16 first, P comes out as bf16 directly); off by
+// default.
+#ifndef BSA_EX2_BF16X2
+#define BSA_EX2_BF16X2 0
+#endif
+constexpr bool kEx2Bf16x2 = BSA_EX2_BF16X2 != 0;
+// Lazy-rescale threshold in log2 units (the running max in use may trail the true
+// one by up to this much, so fast-path P values stay below 2^threshold).
+#ifndef BSA_RESCALE_THRESHOLD
+#define BSA_RESCALE_THRESHOLD 8.0f
+#endif
+constexpr float kRescaleThreshold = BSA_RESCALE_THRESHOLD;  // log2 units
 
 // Optional phase timestamps (SM clock) of CTA 0 for latency analysis; compiled
 // only with -DBSA_TRACE and read back with bsa_trace_dump().
@@ -221,7 +242,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
+  if (warp >= 8) {
+  // third warpgroup (two warps): producer and MMA issuer
   if (warp == kLoadWarp) {
     // ------------------------------------------------------------ producer
     // Ring order (must match the MMA issuer): per unit, K of step 0 for each slot,
@@ -461,6 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(FINAL);
       mbar_wait_drain(FINAL, 0, p.status, p.timeout_ns);
     }
+  }
   } else {
     // ------------------------------------------------------------ softmax (8 warps)
     const int s = warp >> 2;                 // slot
@@ -537,7 +560,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                  __uint_as_float(cur[2 * i + 1])),
                                      sl2x2, negm);
               float2 pp;
-              if (kPolyExp2 && (i & 3) == 3) {
+              if constexpr (kEx2Bf16x2) {
+                if (!poly_pair(i)) {
+                  const uint32_t pb = fast_exp2_bf16x2(x);
+                  out[i] = pb;
+                  pp = make_float2(__uint_as_float(pb << 16), __uint_as_float(pb & 0xFFFF0000u));
+                  if (i & 1) lpb = fadd2(lpb, pp); else lpa = fadd2(lpa, pp);
+                  continue;
+                }
+              }
+              if (poly_pair(i)) {
                 pp = poly_exp2x2(x);
               } else {
                 pp.x = fast_exp2(x.x);

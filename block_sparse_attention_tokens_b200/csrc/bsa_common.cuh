@@ -209,9 +209,11 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, in
 
 // 2^x on the FMA/ALU pipes (no MUFU), for finite x <= 64: Cody-Waite style
 // reduction x = n + f with n = round(x) obtained by the 1.5 * 2^23 rounding
-// constant, f in [-0.5, 0.5]; 2^f by a cubic fitted here to 2^f on [-0.5, 0.5]
-// for least maximum relative error (max rel. error 7.8e-5, below the 2^-9
-// spacing of the bfloat16 values it feeds); the exponent n is added to the bit
+// constant, f in [-0.5, 0.5]; 2^f by a cubic minimax polynomial in the relative
+// error on [-0.5, 0.5] (coefficients from an iteratively reweighted
+// least-squares fit, Lawson's method; max rel. error 7.8e-5, below the 2^-9
+// spacing of the bfloat16 values it feeds -- tests/test_poly_exp2.py checks the
+// coefficients against 2^f in float64); the exponent n is added to the bit
 // pattern.  x is clamped at -125 so the result stays a normal float (>= 2^-125.5).
 __device__ __forceinline__ float poly_exp2(float x) {
   x = fmaxf(x, -125.0f);
@@ -284,6 +286,15 @@ __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x of two lanes as packed bf16 (x.x in the low half): the arguments are rounded
+// to bf16, then one packed MUFU operation.
+__device__ __forceinline__ uint32_t fast_exp2_bf16x2(float2 x) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(x.x, x.y);
+  uint32_t in = *reinterpret_cast<uint32_t*>(&h), out;
+  asm("ex2.approx.ftz.bf16x2 %0, %1;" : "=r"(out) : "r"(in));
+  return out;
 }
 
 }  // namespace bsa

@@ -51,8 +51,10 @@ def test_peak_choice_follows_the_run():
     at_max = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0}
     capped = {"sm_mhz": 1500.0, "sm_max_mhz": 1965.0}
     assert bench.choose_tensor_peak(peaks, at_max, 10.0)[:2] == (1600.0, "burst")
-    assert bench.choose_tensor_peak(peaks, capped, 1.0)[:2] == (1600.0, "burst")
+    assert bench.choose_tensor_peak(peaks, at_max, 1.0)[:2] == (1600.0, "burst")
+    assert bench.choose_tensor_peak(peaks, capped, 1.0)[:2] == (1400.0, "sustained")
     assert bench.choose_tensor_peak(peaks, capped, 10.0)[:2] == (1400.0, "sustained")
+    assert bench.choose_tensor_peak(peaks, {"sm_mhz": None}, 10.0)[:2] == (1600.0, "burst")
     r = bench.tensor_roofline(700.0, 20.0, peaks, "measured", capped, 10.0, attn_ms=20.0)
     assert r["frac"] == 0.5 and r["frac_of_burst"] == 700.0 / 1600.0
     assert r["kernel_ms_x_sm_mhz"] == 20.0 * 1500.0 and r["attn_ms"] == 20.0

@@ -103,9 +103,9 @@ def test_strided_views_equal_dense_copies_forward_and_backward(D, bq, bk):
     assert B.bsa_read_status(ws) == 0
     assert torch.equal(o_s, o_d) and torch.equal(lse_s, lse_d)
     assert torch.all(o_wide[:, :, :2] == 0) and torch.all(o_wide[:, :, H + 2:] == 0)
-    # backward: gradients into a fused dQKV buffer, dO a head slice of a wider tensor
-    do_wide = torch.randn(Bn, n, H + 1, D, generator=g).to(torch.bfloat16).cuda()
-    do = do_wide[:, :, 1:]
+    # backward: gradients into a fused dQKV buffer, dO a head slice of a tensor as wide as O's
+    do_wide = torch.randn(Bn, n, H + 3, D, generator=g).to(torch.bfloat16).cuda()
+    do = do_wide[:, :, 2:H + 2]                     # same row stride as o
     dqkv = torch.zeros_like(qkv)
     dq, dk, dv = (dqkv[:, :, i, 1:H + 1] for i in range(3))
     _, _, _, bws = B.bsa_attn_bwd(q, k, v, o_s, do, lse_s, rp, ci, bq, bk, Bn * H, dq=dq, dk=dk,
