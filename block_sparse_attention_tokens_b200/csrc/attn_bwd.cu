@@ -141,7 +141,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t FINAL = bar0 + 8u * (2 * C::NSTAGE + 6);
   auto UFULL = [&](int i) { return bar0 + 8u * (2 * C::NSTAGE + 7 + i); };
   auto UEMPTY = [&](int i) { return bar0 + 8u * (2 * C::NSTAGE + 11 + i); };
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + 8 * (2 * C::NSTAGE + 15));
+  // dQ pass only: S/dP of the current entry read by every compute warp (the next
+  // entry's S/dP may be issued), and dS buffer b read by its dQ MMAs (free to refill);
+  // PREADY(b) then signals "dS of the entry in buffer b written"
+  const uint32_t SREAD = bar0 + 8u * (2 * C::NSTAGE + 15);
+  auto DSFREE = [&](int b) { return bar0 + 8u * (2 * C::NSTAGE + 16 + b); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + 8 * (2 * C::NSTAGE + 18));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* unit_ring = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
@@ -158,6 +163,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(PREADY(1), 8);
     mbar_init(DONE, 1);
     mbar_init(FINAL, 1);
+    mbar_init(SREAD, 8);
+    mbar_init(DSFREE(0), 1);
+    mbar_init(DSFREE(1), 1);
     for (int i = 0; i < 4; ++i) {
       mbar_init(UFULL(i), 1);
       mbar_init(UEMPTY(i), 1 + 8);  // MMA thread + 8 compute warps
@@ -303,6 +311,30 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                    a0);
         }
       };
+      // dQ pass: dQ += dS K with dS from a double-buffered region of the free TMEM
+      // columns [384, 512), so S and dP of the next entry are issued as soon as the
+      // compute warps have read the current ones (SREAD), ahead of this entry's dQ
+      // MMAs; K stays resident until its dQ MMAs, V is released after dP.
+      uint32_t g_sd = 0, g_acc = 0;  // S/dP pairs issued / dQ accumulations issued (whole CTA)
+      auto issue_sd = [&](int sa, int sb) -> bool {
+        // S/dP TMEM may be overwritten once the previous entry's S/dP have been read
+        if (g_sd > 0 && !mbar_wait(SREAD, (g_sd - 1) & 1u, abort_flag, p.status, p.timeout_ns))
+          return false;
+        sd(sa, sb);
+        mma_commit(SFULL);
+        mma_commit(EMPTY(sb));
+        ++g_sd;
+        return true;
+      };
+      auto acc_dq = [&](int sa, bool first) {
+        tc_fence_after();
+        const uint32_t buf = g_acc & 1u;
+        const uint64_t dA = dColMN + static_cast<uint64_t>(sa * kTileUnits);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + 256, tmem + 384 + 64 * buf + 8 * kk, dA + static_cast<uint64_t>(kk * 128),
+                 idesc_ts, (first && kk == 0) ? 0u : 1u);
+      };
       for (int uk = 0; ok; ++uk) {
         const int slot = uk & 3;
         if (!mbar_wait(UFULL(slot), (uk >> 2) & 1, abort_flag, p.status, p.timeout_ns)) {
@@ -321,6 +353,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         rph ^= 1u;
         int sa = 0, sb = 0;
         if (!acquire(sa) || !acquire(sb)) { ok = false; break; }
+        if constexpr (!kDKV) {
+          if (!issue_sd(sa, sb)) { ok = false; break; }
+          if (it.n == 1) mma_commit(ROWEMPTY);
+          for (int j = 0; j < it.n && ok; ++j) {
+            int na = 0, nb = 0;
+            if (j + 1 < it.n) {
+              if (!acquire(na) || !acquire(nb) || !issue_sd(na, nb)) { ok = false; break; }
+              if (j + 2 == it.n) mma_commit(ROWEMPTY);
+            }
+            const uint32_t buf = g_acc & 1u;
+            if (!mbar_wait(PREADY(buf), (g_acc >> 1) & 1u, abort_flag, p.status, p.timeout_ns)) {
+              ok = false;
+              break;
+            }
+            acc_dq(sa, j == 0);
+            mma_commit(EMPTY(sa));
+            mma_commit(DSFREE(buf));
+            ++g_acc;
+            if (j == it.n - 1) mma_commit(DONE);
+            sa = na;
+          }
+          continue;
+        }
         sd(sa, sb);
         mma_commit(SFULL);
         if (it.n == 1) mma_commit(ROWEMPTY);
@@ -424,6 +479,59 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (threadIdx.x == 0) BSA_BTRACE_AT(gc, 1);
         sph ^= 1u;
         tc_fence_after();
+        if constexpr (!kDKV) {
+          // dS of this entry goes to buffer gc & 1 of the free TMEM columns; the
+          // buffer's previous dS must have been consumed by its dQ MMAs
+          const uint32_t buf = gc & 1u;
+          if (gc >= 2) {
+            ok = mbar_wait(DSFREE(buf), ((gc >> 1) - 1) & 1u, abort_flag, p.status, p.timeout_ns);
+            if (!ok) break;
+            tc_fence_after();
+          }
+          const uint32_t tD = tmem + lane_base + 384 + 64 * buf + 16 * cg;
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t tS = tmem + lane_base + 64u * h + 32u * cg;
+            const bool row_ok = (bits >> (rh * 2 + h)) & 1u;
+            uint32_t dpk[16];
+            uint32_t sr[32], dr[32];
+            if (row_ok) {
+              tmem_ld32x32b_x32_nowait(tS, sr);
+              tmem_ld32x32b_x32_nowait(tS + 128, dr);
+              tmem_wait_ld_x32(sr);
+              tmem_wait_ld_x32(dr);
+            }
+            if (h == 1) {  // S and dP of this entry are in registers: the next may be issued
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(SREAD);
+            }
+            if (!row_ok) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) dpk[i] = 0u;
+            } else {
+              const int cbase = 64 * h + 32 * cg;
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const int c = cbase + 2 * i;
+                const float2 a = ffma2(make_float2(__uint_as_float(sr[2 * i]),
+                                                   __uint_as_float(sr[2 * i + 1])), sl2, nlse);
+                float2 pr = make_float2(fast_exp2(a.x), fast_exp2(a.y));
+                if (c >= cvalid) pr.x = 0.f;
+                if (c + 1 >= cvalid) pr.y = 0.f;
+                const float2 ds = fmul2(pr, fsub2(make_float2(__uint_as_float(dr[2 * i]),
+                                                              __uint_as_float(dr[2 * i + 1])),
+                                                  dd));
+                __nv_bfloat162 hd = __floats2bfloat162_rn(ds.x, ds.y);
+                dpk[i] = *reinterpret_cast<uint32_t*>(&hd);
+              }
+            }
+            tmem_st32x32b_x16(tD + 32 * h, dpk);
+          }
+          asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(PREADY(buf));
+        } else {
         for (int h = 0; h < 2; ++h) {
           // this warp's 32 columns of the half; P and dS are packed into the first 16
           // columns of the same ranges of S and dP
@@ -477,6 +585,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           __syncwarp();
           if (threadIdx.x == 0) BSA_BTRACE_AT(gc, 2 + h);
           if (lane == 0) mbar_arrive(PREADY(h));
+        }
         }
         ++gc;
       }
