@@ -47,6 +47,13 @@ __device__ unsigned long long g_bsa_btrace[1 << 16];
 #endif
 
 constexpr int kBwdThreads = 320;
+// BSA_BWD_LOAD_ALL=1: the decoupled passes load S (and dP) of both 64-column halves
+// before computing either (one exposed load latency per entry, at the price of
+// more live registers); 0: one half at a time.
+#ifndef BSA_BWD_LOAD_ALL
+#define BSA_BWD_LOAD_ALL 0
+#endif
+constexpr bool kLoadAll = BSA_BWD_LOAD_ALL != 0;
 constexpr int kBwdLoadWarp = 8;
 constexpr int kBwdMmaWarp = 9;
 
@@ -89,6 +96,25 @@ struct BItem {
   const uint32_t* ent;
 };
 
+// Kernel passes.  kPassDKV: dK and dV together (two accumulators, P and dS written
+// over the S and dP columns, so each entry's accumulation precedes the next
+// entry's S and dP).  The decoupled passes hold one accumulator and put the
+// accumulation operand (dS or P, bf16) in a double-buffered region of the free
+// TMEM columns [384, 512), so the next entry's S (and dP) are issued as soon as
+// the current ones have been read:
+//   kPassDQ: rows = q-tiles,   S = Q K^T, dP = dO V^T, dQ += dS K
+//   kPassDK: rows = key tiles, S = K Q^T, dP = V dO^T, dK += dS Q
+//   kPassDV: rows = key tiles, S = K Q^T,              dV += P dO
+enum : int { kPassDKV = 0, kPassDQ = 1, kPassDK = 2, kPassDV = 3 };
+
+template <int kPass>
+struct PassTraits {
+  static constexpr bool kKeyRows = kPass != kPassDQ;      // items are key tiles
+  static constexpr bool kFused = kPass == kPassDKV;
+  static constexpr bool kHasDP = kPass != kPassDV;        // dP (and the second row operand)
+  static constexpr bool kAccColB = kPass == kPassDV;      // accumulate with colB (dO)
+};
+
 template <bool kDKV>
 __device__ __forceinline__ BItem get_bitem(const BwdParams& p, int it) {
   BItem r;
@@ -115,15 +141,21 @@ __device__ __forceinline__ BItem get_bitem(const BwdParams& p, int it) {
   return r;
 }
 
-// rowA / rowB: the item's fixed operands (kDKV: K, V; kDQ: Q, dO), 128-row tiles.
-// colA / colB: the per-step operands (kDKV: Q, dO; kDQ: K, V), 128-row tiles
-// streamed through the ring (colA then colB per kept entry).
-template <int D, bool kDKV>
+// rowA / rowB: the item's fixed operands (key-row passes: K, V; dQ pass: Q, dO;
+// the dV pass uses rowA only), 128-row tiles.  colA / colB: the per-step operands
+// (key-row passes: Q, dO; dQ pass: K, V), 128-row tiles streamed through the ring
+// (colA then colB per kept entry).
+template <int D, int kPass>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tmRowA, const __grid_constant__ CUtensorMap tmRowB,
                     const __grid_constant__ CUtensorMap tmColA, const __grid_constant__ CUtensorMap tmColB,
                     const BwdParams p) {
   using C = BwdCfg<D>;
+  using T = PassTraits<kPass>;
+  constexpr bool kDKV = T::kKeyRows;   // per-column LSE / Delta, transposed lists
+  constexpr int kRowTiles = T::kHasDP ? 2 : 1;
+  // ring order per entry: colB before colA when the accumulation holds colA
+  constexpr bool kLoadHeldLast = !T::kFused && !T::kAccColB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -141,9 +173,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t FINAL = bar0 + 8u * (2 * C::NSTAGE + 6);
   auto UFULL = [&](int i) { return bar0 + 8u * (2 * C::NSTAGE + 7 + i); };
   auto UEMPTY = [&](int i) { return bar0 + 8u * (2 * C::NSTAGE + 11 + i); };
-  // dQ pass only: S/dP of the current entry read by every compute warp (the next
-  // entry's S/dP may be issued), and dS buffer b read by its dQ MMAs (free to refill);
-  // PREADY(b) then signals "dS of the entry in buffer b written"
+  // decoupled passes: S (and dP) of the current entry read by every compute warp
+  // (the next entry's may be issued), and buffer b read by its accumulation MMAs
+  // (free to refill); PREADY(b) then signals "the entry's dS or P is in buffer b"
   const uint32_t SREAD = bar0 + 8u * (2 * C::NSTAGE + 15);
   auto DSFREE = [&](int b) { return bar0 + 8u * (2 * C::NSTAGE + 16 + b); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + 8 * (2 * C::NSTAGE + 18));
@@ -225,12 +257,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         row_filled = static_cast<int>(rph);
         rph ^= 1u;
-        mbar_expect_tx(ROWFULL, 2 * C::TILE_BYTES);
+        mbar_expect_tx(ROWFULL, kRowTiles * C::TILE_BYTES);
         for (int c = 0; c < C::KCH; ++c) {
           tma_load_4d(sRow + c * C::CHUNK_BYTES, &tmRowA, ROWFULL, 64 * c, it.h,
                       it.row_tile * kBM, it.b);
-          tma_load_4d(sRow + C::TILE_BYTES + c * C::CHUNK_BYTES, &tmRowB, ROWFULL, 64 * c, it.h,
-                      it.row_tile * kBM, it.b);
+          if (kRowTiles == 2)
+            tma_load_4d(sRow + C::TILE_BYTES + c * C::CHUNK_BYTES, &tmRowB, ROWFULL, 64 * c, it.h,
+                        it.row_tile * kBM, it.b);
         }
         // entry words read four ahead, so no load latency sits between two TMA issues
         uint32_t pf0 = __ldg(it.ent), pf1 = it.n > 1 ? __ldg(it.ent + 1) : 0u;
@@ -242,10 +275,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           pf2 = pf3;
           pf3 = j + 4 < it.n ? __ldg(it.ent + j + 4) : 0u;
           const int ct = static_cast<int>(ent & 0x0FFFFFFFu);
-          ok = load_col(&tmColA, it, ct);
+          // decoupled passes: the operand released early (after S / dP) first, the
+          // one the accumulation holds second -- in the ring the next entry's early
+          // operand then reuses the stage of an operand released an entry sooner,
+          // which gives the loads one more entry of lead
+          if (kLoadHeldLast) {
+            ok = load_col(&tmColB, it, ct);
+            ok = ok && load_col(&tmColA, it, ct);
+          } else {
+            ok = load_col(&tmColA, it, ct);
+            ok = ok && load_col(&tmColB, it, ct);
+          }
           BSA_BTRACE_AT(gl, 7);
           ++gl;
-          ok = ok && load_col(&tmColB, it, ct);
         }
       }
       for (int i = 0; i < C::NSTAGE; ++i)
@@ -285,11 +327,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               static_cast<uint64_t>((((kk >> 2) * C::CHUNK_BYTES) + (kk & 3) * 32) >> 4);
           mma_ss(tmem, dRowK + off, da + off, idesc_ss, kk > 0 ? 1u : 0u);
         }
+        if constexpr (T::kHasDP) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t off =
-              static_cast<uint64_t>((((kk >> 2) * C::CHUNK_BYTES) + (kk & 3) * 32) >> 4);
-          mma_ss(tmem + 128, dRowK + kTileUnits + off, db + off, idesc_ss, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off =
+                static_cast<uint64_t>((((kk >> 2) * C::CHUNK_BYTES) + (kk & 3) * 32) >> 4);
+            mma_ss(tmem + 128, dRowK + kTileUnits + off, db + off, idesc_ss, kk > 0 ? 1u : 0u);
+          }
         }
       };
       // one 64-column half of the accumulation: accA (+)= dS colA, accB (+)= P colB
@@ -322,14 +366,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           return false;
         sd(sa, sb);
         mma_commit(SFULL);
-        mma_commit(EMPTY(sb));
+        mma_commit(EMPTY(T::kAccColB ? sa : sb));   // the operand the accumulation does not read
         ++g_sd;
         return true;
       };
-      auto acc_dq = [&](int sa, bool first) {
+      // acc (+)= buffer . (colA or colB); `sacc` is the ring stage of that operand
+      auto acc_dq = [&](int sacc, bool first) {
         tc_fence_after();
         const uint32_t buf = g_acc & 1u;
-        const uint64_t dA = dColMN + static_cast<uint64_t>(sa * kTileUnits);
+        const uint64_t dA = dColMN + static_cast<uint64_t>(sacc * kTileUnits);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_ts(tmem + 256, tmem + 384 + 64 * buf + 8 * kk, dA + static_cast<uint64_t>(kk * 128),
@@ -352,14 +397,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         rph ^= 1u;
         int sa = 0, sb = 0;
-        if (!acquire(sa) || !acquire(sb)) { ok = false; break; }
-        if constexpr (!kDKV) {
+        if (kLoadHeldLast ? (!acquire(sb) || !acquire(sa)) : (!acquire(sa) || !acquire(sb))) {
+          ok = false;
+          break;
+        }
+        if constexpr (!T::kFused) {
           if (!issue_sd(sa, sb)) { ok = false; break; }
           if (it.n == 1) mma_commit(ROWEMPTY);
+          int sacc = T::kAccColB ? sb : sa;
           for (int j = 0; j < it.n && ok; ++j) {
             int na = 0, nb = 0;
             if (j + 1 < it.n) {
-              if (!acquire(na) || !acquire(nb) || !issue_sd(na, nb)) { ok = false; break; }
+              const bool got = kLoadHeldLast ? (acquire(nb) && acquire(na)) : (acquire(na) && acquire(nb));
+              if (!got || !issue_sd(na, nb)) { ok = false; break; }
               if (j + 2 == it.n) mma_commit(ROWEMPTY);
             }
             const uint32_t buf = g_acc & 1u;
@@ -367,12 +417,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               ok = false;
               break;
             }
-            acc_dq(sa, j == 0);
-            mma_commit(EMPTY(sa));
+            acc_dq(sacc, j == 0);
+            mma_commit(EMPTY(sacc));
             mma_commit(DSFREE(buf));
             ++g_acc;
             if (j == it.n - 1) mma_commit(DONE);
-            sa = na;
+            sacc = T::kAccColB ? nb : na;
           }
           continue;
         }
@@ -479,9 +529,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (threadIdx.x == 0) BSA_BTRACE_AT(gc, 1);
         sph ^= 1u;
         tc_fence_after();
-        if constexpr (!kDKV) {
-          // dS of this entry goes to buffer gc & 1 of the free TMEM columns; the
-          // buffer's previous dS must have been consumed by its dQ MMAs
+        if constexpr (!T::kFused) {
+          // dS (or P) of this entry goes to buffer gc & 1 of the free TMEM columns;
+          // the buffer's previous contents must have been consumed by their MMAs
           const uint32_t buf = gc & 1u;
           if (gc >= 2) {
             ok = mbar_wait(DSFREE(buf), ((gc >> 1) - 1) & 1u, abort_flag, p.status, p.timeout_ns);
@@ -489,6 +539,70 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tc_fence_after();
           }
           const uint32_t tD = tmem + lane_base + 384 + 64 * buf + 16 * cg;
+          if constexpr (kLoadAll) {
+          // S (and dP) of both halves are loaded at once: one load latency per
+          // entry, and the next entry's S / dP may be issued as soon as they are in
+          // registers
+          uint32_t sr[2][32], dr[2][32];
+          bool hok[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            hok[h] = (bits >> (rh * 2 + h)) & 1u;
+            const uint32_t tS = tmem + lane_base + 64u * h + 32u * cg;
+            if (hok[h]) {
+              tmem_ld32x32b_x32_nowait(tS, sr[h]);
+              if constexpr (T::kHasDP) tmem_ld32x32b_x32_nowait(tS + 128, dr[h]);
+            }
+          }
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            if (hok[h]) {
+              tmem_wait_ld_x32(sr[h]);
+              if constexpr (T::kHasDP) tmem_wait_ld_x32(dr[h]);
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(SREAD);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            uint32_t dpk[16];
+            if (!hok[h]) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) dpk[i] = 0u;
+            } else {
+              const int cbase = 64 * h + 32 * cg;
+              const float vl = h ? cl[1] : cl[0], vd = h ? cd[1] : cd[0];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const int c = cbase + 2 * i;
+                float2 nl = nlse, dv = dd;
+                if constexpr (T::kKeyRows) {  // per-column (query) statistics
+                  nl = make_float2(__shfl_sync(0xffffffffu, vl, 2 * i),
+                                   __shfl_sync(0xffffffffu, vl, 2 * i + 1));
+                  if constexpr (T::kHasDP)
+                    dv = make_float2(__shfl_sync(0xffffffffu, vd, 2 * i),
+                                     __shfl_sync(0xffffffffu, vd, 2 * i + 1));
+                }
+                const float2 a = ffma2(make_float2(__uint_as_float(sr[h][2 * i]),
+                                                   __uint_as_float(sr[h][2 * i + 1])), sl2, nl);
+                float2 pr = make_float2(fast_exp2(a.x), fast_exp2(a.y));
+                if constexpr (!T::kKeyRows) {   // dQ pass: ragged key tail
+                  if (c >= cvalid) pr.x = 0.f;
+                  if (c + 1 >= cvalid) pr.y = 0.f;
+                }
+                float2 val = pr;
+                if constexpr (T::kHasDP)
+                  val = fmul2(pr, fsub2(make_float2(__uint_as_float(dr[h][2 * i]),
+                                                    __uint_as_float(dr[h][2 * i + 1])),
+                                        dv));
+                __nv_bfloat162 hd = __floats2bfloat162_rn(val.x, val.y);
+                dpk[i] = *reinterpret_cast<uint32_t*>(&hd);
+              }
+            }
+            tmem_st32x32b_x16(tD + 32 * h, dpk);
+          }
+          } else {
           for (int h = 0; h < 2; ++h) {
             const uint32_t tS = tmem + lane_base + 64u * h + 32u * cg;
             const bool row_ok = (bits >> (rh * 2 + h)) & 1u;
@@ -496,9 +610,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             uint32_t sr[32], dr[32];
             if (row_ok) {
               tmem_ld32x32b_x32_nowait(tS, sr);
-              tmem_ld32x32b_x32_nowait(tS + 128, dr);
+              if constexpr (T::kHasDP) tmem_ld32x32b_x32_nowait(tS + 128, dr);
               tmem_wait_ld_x32(sr);
-              tmem_wait_ld_x32(dr);
+              if constexpr (T::kHasDP) tmem_wait_ld_x32(dr);
             }
             if (h == 1) {  // S and dP of this entry are in registers: the next may be issued
               tc_fence_before();
@@ -510,22 +624,36 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               for (int i = 0; i < 16; ++i) dpk[i] = 0u;
             } else {
               const int cbase = 64 * h + 32 * cg;
+              const float vl = h ? cl[1] : cl[0], vd = h ? cd[1] : cd[0];
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
                 const int c = cbase + 2 * i;
+                float2 nl = nlse, dv = dd;
+                if constexpr (T::kKeyRows) {  // per-column (query) statistics
+                  nl = make_float2(__shfl_sync(0xffffffffu, vl, 2 * i),
+                                   __shfl_sync(0xffffffffu, vl, 2 * i + 1));
+                  if constexpr (T::kHasDP)
+                    dv = make_float2(__shfl_sync(0xffffffffu, vd, 2 * i),
+                                     __shfl_sync(0xffffffffu, vd, 2 * i + 1));
+                }
                 const float2 a = ffma2(make_float2(__uint_as_float(sr[2 * i]),
-                                                   __uint_as_float(sr[2 * i + 1])), sl2, nlse);
+                                                   __uint_as_float(sr[2 * i + 1])), sl2, nl);
                 float2 pr = make_float2(fast_exp2(a.x), fast_exp2(a.y));
-                if (c >= cvalid) pr.x = 0.f;
-                if (c + 1 >= cvalid) pr.y = 0.f;
-                const float2 ds = fmul2(pr, fsub2(make_float2(__uint_as_float(dr[2 * i]),
-                                                              __uint_as_float(dr[2 * i + 1])),
-                                                  dd));
-                __nv_bfloat162 hd = __floats2bfloat162_rn(ds.x, ds.y);
+                if constexpr (!T::kKeyRows) {   // dQ pass: ragged key tail
+                  if (c >= cvalid) pr.x = 0.f;
+                  if (c + 1 >= cvalid) pr.y = 0.f;
+                }
+                float2 val = pr;
+                if constexpr (T::kHasDP)
+                  val = fmul2(pr, fsub2(make_float2(__uint_as_float(dr[2 * i]),
+                                                    __uint_as_float(dr[2 * i + 1])),
+                                        dv));
+                __nv_bfloat162 hd = __floats2bfloat162_rn(val.x, val.y);
                 dpk[i] = *reinterpret_cast<uint32_t*>(&hd);
               }
             }
             tmem_st32x32b_x16(tD + 32 * h, dpk);
+          }
           }
           asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
           tc_fence_before();
@@ -596,7 +724,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const long long orow_off =
           (static_cast<long long>(it.b) * nrows + grow) * p.out_stride + static_cast<long long>(it.h) * D;
       __nv_bfloat16* rowA = p.outA + orow_off;
-      __nv_bfloat16* rowB = kDKV ? p.outB + orow_off : nullptr;
+      __nv_bfloat16* rowB = T::kFused ? p.outB + orow_off : nullptr;
       if (it.n > 0) {
         ok = mbar_wait(DONE, dph, abort_flag, p.status, p.timeout_ns);
         if (!ok) break;
@@ -604,10 +732,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_after();
       }
 #pragma unroll 1
-      for (int pass = 0; pass < (kDKV ? 2 : 1); ++pass) {
+      for (int pass = 0; pass < (T::kFused ? 2 : 1); ++pass) {
         const uint32_t tacc = pass == 0 ? tA : tB;
         __nv_bfloat16* dst_row = pass == 0 ? rowA : rowB;
-        const float mul = pass == 0 ? p.scale : 1.0f;
+        // dK and dQ carry the softmax scale (S = scale * Q K^T); dV does not
+        const float mul = (pass == 0 && kPass != kPassDV) ? p.scale : 1.0f;
 #pragma unroll 1
         for (int c0 = cg * (D / 2); c0 < (cg + 1) * (D / 2); c0 += 32) {
           uint32_t ov[32];
@@ -770,19 +899,33 @@ BwdGeometry bwd_geometry(int batch, int heads, int nq, int nk, int block_q, int 
   return g;
 }
 
-template <int D, bool kDKV>
+template <int D, int kPass>
 int launch_bwd(const CUtensorMap& ra, const CUtensorMap& rb, const CUtensorMap& ca,
                const CUtensorMap& cb, const BwdParams& p, cudaStream_t st) {
   using C = BwdCfg<D>;
-  cudaError_t e = cudaFuncSetAttribute(attn_bwd_kernel<D, kDKV>,
+  cudaError_t e = cudaFuncSetAttribute(attn_bwd_kernel<D, kPass>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return record_cuda_error(e);
   int grid = device_sm_count();
   if (grid > p.total_items) grid = p.total_items;
   if (grid < 1) grid = 1;
-  attn_bwd_kernel<D, kDKV><<<grid, kBwdThreads, C::SMEM, st>>>(ra, rb, ca, cb, p);
+  attn_bwd_kernel<D, kPass><<<grid, kBwdThreads, C::SMEM, st>>>(ra, rb, ca, cb, p);
   return check_launch();
 }
+
+template <int kPass>
+int launch_bwd_d(int head_dim, const CUtensorMap& ra, const CUtensorMap& rb,
+                 const CUtensorMap& ca, const CUtensorMap& cb, const BwdParams& p,
+                 cudaStream_t st) {
+  return head_dim == 128 ? launch_bwd<128, kPass>(ra, rb, ca, cb, p, st)
+                         : launch_bwd<64, kPass>(ra, rb, ca, cb, p, st);
+}
+
+// BSA_BWD_SPLIT=1: three decoupled passes (dV, dK, dQ) instead of the fused dK/dV
+// pass and the decoupled dQ pass.
+#ifndef BSA_BWD_SPLIT
+#define BSA_BWD_SPLIT 0
+#endif
 
 }  // namespace
 }  // namespace bsa
@@ -841,8 +984,8 @@ extern "C" int bsa_attn_bwd(const void* q, const void* k, const void* v, const v
   float* lse2 = reinterpret_cast<float*>(wsb + g.lse_off);
   float* dvec = reinterpret_cast<float*>(wsb + g.dvec_off);
 
-  // status word + two unit counters
-  cudaError_t e = cudaMemsetAsync(status, 0, 3 * sizeof(int), st);
+  // status word + unit counters of the passes
+  cudaError_t e = cudaMemsetAsync(status, 0, 4 * sizeof(int), st);  // status + 3 unit counters
   if (e == cudaSuccess) e = cudaMemsetAsync(map, 0, g.lse_off - g.map_off, st);
   if (e != cudaSuccess) return record_cuda_error(e);
   int rc = launch_build_lists(row_ptr, col_idx, list_heads, g.fwd, nk, block_q, block_k, cnt,
@@ -885,21 +1028,30 @@ extern "C" int bsa_attn_bwd(const void* q, const void* k, const void* v, const v
   p.out_stride = qkv_rs;
   p.status = status;
   p.timeout_ns = 2000000000ULL;
-  // pass 1: dK, dV (rows = key tiles, columns = q-tiles)
+  // key-row passes (rows = key tiles, columns = q-tiles)
   p.total_items = batch * heads * g.KT;
-  p.outA = static_cast<__nv_bfloat16*>(dk);
-  p.outB = static_cast<__nv_bfloat16*>(dv);
-  p.unit_counter = status + 1;
-  rc = head_dim == 128 ? launch_bwd<128, true>(mk, mv, mq, mdo, p, st)
-                       : launch_bwd<64, true>(mk, mv, mq, mdo, p, st);
+  if (BSA_BWD_SPLIT) {
+    p.outA = static_cast<__nv_bfloat16*>(dv);
+    p.outB = nullptr;
+    p.unit_counter = status + 1;
+    rc = launch_bwd_d<kPassDV>(head_dim, mk, mv, mq, mdo, p, st);
+    if (rc != BSA_OK) return rc;
+    p.outA = static_cast<__nv_bfloat16*>(dk);
+    p.unit_counter = status + 3;
+    rc = launch_bwd_d<kPassDK>(head_dim, mk, mv, mq, mdo, p, st);
+  } else {
+    p.outA = static_cast<__nv_bfloat16*>(dk);
+    p.outB = static_cast<__nv_bfloat16*>(dv);
+    p.unit_counter = status + 1;
+    rc = launch_bwd_d<kPassDKV>(head_dim, mk, mv, mq, mdo, p, st);
+  }
   if (rc != BSA_OK) return rc;
-  // pass 2: dQ (rows = q-tiles, columns = key tiles)
+  // dQ pass (rows = q-tiles, columns = key tiles)
   p.total_items = batch * heads * g.fwd.QT;
   p.outA = static_cast<__nv_bfloat16*>(dq);
   p.outB = nullptr;
   p.unit_counter = status + 2;
-  return head_dim == 128 ? launch_bwd<128, false>(mq, mdo, mk, mv, p, st)
-                         : launch_bwd<64, false>(mq, mdo, mk, mv, p, st);
+  return launch_bwd_d<kPassDQ>(head_dim, mq, mdo, mk, mv, p, st);
 }
 
 #ifdef BSA_TRACE
