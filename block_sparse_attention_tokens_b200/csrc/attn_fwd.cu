@@ -53,8 +53,10 @@ constexpr int kMmaWarp = 9;
 constexpr float kFastSumLimit = 4096.0f;
 // Optional software 2^x (FMA pipe) for BSA_POLY_PAIRS of every 16 column pairs of
 // the fast path's exponentials, to relieve the MUFU (one exponential per 512 tensor
-// FLOPs at head_dim 128); 0 by default.  BSA_POLY_EXP2=1 is the older spelling of
-// 4 pairs in 16.
+// FLOPs at head_dim 128); 0 by default: the FMA pipe's 128 lanes per SM clock
+// spend about as many cycles on one polynomial exponential as the MUFU does (16
+// per SM clock), and 2, 4 and 6 pairs in 16 measured 3-7 % slower on the radial
+// and Sliding-Tile workloads.  BSA_POLY_EXP2=1 is the older spelling of 4 in 16.
 #ifndef BSA_POLY_EXP2
 #define BSA_POLY_EXP2 0
 #endif
@@ -67,13 +69,6 @@ static_assert(kPolyPairs >= 0 && kPolyPairs <= 16, "BSA_POLY_PAIRS is 0..16");
 __device__ __forceinline__ constexpr bool poly_pair(int i) {
   return kPolyPairs > 0 && (i * kPolyPairs) % 16 < kPolyPairs;
 }
-// Optional packed bf16 exponentials in the fast path (one MUFU operation per column
-// pair; the argument is rounded to bf16 first, P comes out as bf16 directly); off by
-// default.
-#ifndef BSA_EX2_BF16X2
-#define BSA_EX2_BF16X2 0
-#endif
-constexpr bool kEx2Bf16x2 = BSA_EX2_BF16X2 != 0;
 // Lazy-rescale threshold in log2 units (the running max in use may trail the true
 // one by up to this much, so fast-path P values stay below 2^threshold).
 #ifndef BSA_RESCALE_THRESHOLD
@@ -391,7 +386,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       // O_s (+)= P_s V once slot s's softmax has published P.
       auto pv = [&](int s, int stage, int step) -> bool {
         if (!mbar_wait(PREADY(s), pph[s], abort_flag, p.status, p.timeout_ns)) return false;
-        pph[s] ^= 1u;
         tc_fence_after();
         const uint64_t db = dv0 + static_cast<uint64_t>(stage * kTileUnits);
         const uint32_t dt = tmem + 256 + s * 128;
@@ -401,6 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < kBN / 16; ++kk)
           mma_ts(dt, ta + kk * 8, db + static_cast<uint64_t>(kk * (16 * 128 / 16)), idesc_pv,
                  kk > 0 ? 1u : acc0);
+        pph[s] ^= 1u;
         return true;
       };
       for (int uk = 0; ok; ++uk) {
@@ -560,15 +555,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                  __uint_as_float(cur[2 * i + 1])),
                                      sl2x2, negm);
               float2 pp;
-              if constexpr (kEx2Bf16x2) {
-                if (!poly_pair(i)) {
-                  const uint32_t pb = fast_exp2_bf16x2(x);
-                  out[i] = pb;
-                  pp = make_float2(__uint_as_float(pb << 16), __uint_as_float(pb & 0xFFFF0000u));
-                  if (i & 1) lpb = fadd2(lpb, pp); else lpa = fadd2(lpa, pp);
-                  continue;
-                }
-              }
               if (poly_pair(i)) {
                 pp = poly_exp2x2(x);
               } else {

@@ -288,13 +288,5 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// 2^x of two lanes as packed bf16 (x.x in the low half): the arguments are rounded
-// to bf16, then one packed MUFU operation.
-__device__ __forceinline__ uint32_t fast_exp2_bf16x2(float2 x) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(x.x, x.y);
-  uint32_t in = *reinterpret_cast<uint32_t*>(&h), out;
-  asm("ex2.approx.ftz.bf16x2 %0, %1;" : "=r"(out) : "r"(in));
-  return out;
-}
 
 }  // namespace bsa
