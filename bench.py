@@ -194,18 +194,31 @@ def cpu_cores() -> int:
         return os.cpu_count() or 1
 
 
-def oracle_workload_mask(w, q, k):
+def oracle_head_perms(w, q, k):
+    """Token order of every head in the path, by the oracle: None (raster order),
+    the workload's tile order, or (per-head slicing) the tile order of the shape the
+    oracle's SICS scheme picks for the head."""
+    import oracle as O
+    if w.mask == "spade":
+        from block_sparse_attention_tokens_b200.configs import sics_menu
+        menu = sics_menu(w.block)
+        _, choice = O.sics_scheme(q.double().numpy(), k.double().numpy(), w.grid, menu)
+        return [O.tile_order(w.grid, menu[int(choice[0, h])]) for h in range(w.heads)]
+    if w.tile is not None:
+        return [O.tile_order(w.grid, w.tile)] * w.heads
+    return [None] * w.heads
+
+
+def oracle_workload_mask(w, q, k, perms=None):
     """The oracle's own block mask of the workload, [Hm, QB, KB] uint8 (Hm = 1 for
     the static masks, batch * heads otherwise), from the raster-order bf16 inputs:
     the Sliding-Tile window, the radial rule, NABLA (per-head pooled means of the
-    tile-ordered Q and K), NABLA united with the window, or the autoregressive
-    composition."""
+    tile-ordered Q and K), NABLA united with the window, NABLA over per-head slices,
+    or the autoregressive composition.  perms: oracle_head_perms (computed if None)."""
     import numpy as np
     import oracle as O
     QB, KB = math.ceil(w.nq / w.block), math.ceil(w.nk / w.block)
     if w.tile is not None:
-        perm = O.tile_order(w.grid, w.tile)
-        n_pad = QB * w.block
         tg = tuple(math.ceil(g / t) for g, t in zip(w.grid, w.tile))
     if w.mask == "sta":
         return O.sta_tile_mask(tg, w.window)[None]
@@ -213,19 +226,22 @@ def oracle_workload_mask(w, q, k):
         return O.radial_block_mask_fast(w.nk, w.tokens_per_frame, w.block)[None]
     D = w.head_dim
     scale = 1.0 / math.sqrt(D)
+    if perms is None:
+        perms = oracle_head_perms(w, q, k)
+    n_pad = QB * w.block
     qbar = np.zeros((w.batch, w.heads, QB, D))
     kbar = np.zeros((w.batch, w.heads, KB, D))
     for h in range(w.heads):
         qh = q[:, :, h:h + 1].double().numpy()
         kh = k[:, :, h:h + 1].double().numpy()
-        if w.tile is not None:
-            qh, kh = O.tile_permute(qh, perm, n_pad), O.tile_permute(kh, perm, n_pad)
+        if perms[h] is not None:
+            qh, kh = O.tile_permute(qh, perms[h], n_pad), O.tile_permute(kh, perms[h], n_pad)
         else:
             qh = np.concatenate([qh, np.zeros((w.batch, QB * w.block - w.nq, 1, D))], axis=1)
             kh = np.concatenate([kh, np.zeros((w.batch, KB * w.block - w.nk, 1, D))], axis=1)
         qbar[:, h] = O.nabla_pool(qh, w.block, w.nq)[:, 0]
         kbar[:, h] = O.nabla_pool(kh, w.block, w.nk)[:, 0]
-    if w.mask == "nabla":
+    if w.mask in ("nabla", "spade"):
         m, _ = O.nabla_mask(qbar, kbar, w.p, scale)
     elif w.mask == "nabla_sta":
         m, _ = O.nabla_sta_mask(qbar, kbar, w.p, scale, O.sta_tile_mask(tg, w.window))
@@ -257,14 +273,14 @@ class OracleSample:
         self.w, self.O, self.np = w, O, np
         t0 = time.perf_counter()
         self.q, self.k, self.v = q, k, v
-        self.perm = O.tile_order(w.grid, w.tile) if w.tile is not None else None
-        self.mask = oracle_workload_mask(w, q, k)
+        self.perms = oracle_head_perms(w, q, k)
+        self.mask = oracle_workload_mask(w, q, k, self.perms)
         self.setup_s = time.perf_counter() - t0
         self.rng = np.random.default_rng(7)
 
     def path_rows(self, t, rows, h):
         """float64 [B, len(rows), 1, D] of tensor t at path-order rows, head h."""
-        idx = rows if self.perm is None else self.perm[rows]
+        idx = rows if self.perms[h] is None else self.perms[h][rows]
         return t[:, self.np.asarray(idx), h:h + 1].double().numpy()
 
     def gather(self, qb, h):
@@ -576,13 +592,18 @@ def permute_bandwidth(w, plan, stage_ms: dict, hbm_peak: float):
         return None
     row = w.heads * w.head_dim * 2
     n, n_pad = w.n_tokens, plan.n_pad
+    permute_bytes = 3 * w.batch * (n + n_pad) * row
+    if w.mask == "spade":
+        # the stage also runs the SICS scheme: Q and K read once per menu shape
+        permute_bytes += 2 * len(plan.menu) * w.batch * n * row
     out = {}
-    for name, nbytes in (("permute", 3 * w.batch * (n + n_pad) * row),
-                         ("untile", 2 * w.batch * n * row)):
+    for name, nbytes in (("permute", permute_bytes), ("untile", 2 * w.batch * n * row)):
         ms = stage_ms[name]
         gbs = nbytes / (ms * 1e-3) / 1e9 if ms > 0 else None
         out[name] = {"bytes": nbytes, "gb_s": gbs,
                      "frac_of_hbm": gbs / hbm_peak if gbs else None}
+    if w.mask == "spade":
+        out["permute"]["stage"] = "SICS scheme + per-head permute of Q, K (pooled), V"
     return out
 
 

@@ -28,6 +28,7 @@ EXPORTS = [
     "bsa_wait_selftest", "bsa_attn_bwd_workspace_size", "bsa_attn_bwd", "bsa_sics_blocks",
     "bsa_sics_workspace_size", "bsa_sics_scheme", "bsa_kv_write", "bsa_block_pool",
     "bsa_kv_resident_blocks", "bsa_kv_page_scores", "bsa_kv_keep_pages", "bsa_attn_fwd_paged",
+    "bsa_scheme_permute", "bsa_scheme_untile",
 ]
 
 
@@ -72,14 +73,18 @@ def load_library(path: str = _LIB_PATH) -> ctypes.CDLL:
         "bsa_attn_bwd_workspace_size": (c_size, [c_int] * 7),
         "bsa_attn_bwd": (c_int, [c_void] * 6 + [c_int] * 9 + [c_void, c_void, c_int, c_float]
                          + [c_void] * 4 + [c_size, c_void]),
-        "bsa_sics_blocks": (c_int, [c_void] + [c_int] * 9 + [c_void, c_void]),
+        "bsa_sics_blocks": (c_int, [c_void] + [c_int] * 10 + [c_void, c_void]),
         "bsa_sics_workspace_size": (c_size, [c_int] * 5 + [c_void, c_int]),
-        "bsa_sics_scheme": (c_int, [c_void, c_void] + [c_int] * 6 + [c_void, c_int]
+        "bsa_sics_scheme": (c_int, [c_void, c_void] + [c_int] * 7 + [c_void, c_int]
                             + [c_void] * 3 + [c_size, c_void]),
         "bsa_read_status": (c_int, [c_void, ctypes.POINTER(c_int), c_void]),
         "bsa_wait_selftest": (c_int, [c_void, ctypes.c_ulonglong, c_void]),
         "bsa_tile_permute_pool": (c_int, [c_void, c_void] + [c_int] * 11 + [c_void, c_int, c_int,
                                                                              c_void]),
+        "bsa_scheme_permute": (c_int, [c_void, c_void] + [c_int] * 4 + [c_void, c_int, c_void]
+                               + [c_int] * 4 + [c_void, c_int, c_int, c_void, c_void]),
+        "bsa_scheme_untile": (c_int, [c_void, c_void] + [c_int] * 4 + [c_void, c_int, c_void]
+                              + [c_int] * 5 + [c_void, c_void]),
         "bsa_nabla_select": (c_int, [c_void, c_void] + [c_int] * 5 + [c_float, c_float]
                              + [c_int] * 3 + [c_void] * 5),
         "bsa_kv_write": (c_int, [c_void] + [c_int] * 5 + [c_void, c_int, c_void, c_int, c_void,
@@ -345,6 +350,60 @@ def bsa_tile_permute_pool(x: torch.Tensor, grid: Tuple[int, int, int],
     return y, pooled
 
 
+def _choice(choice: torch.Tensor, batch: int, heads: int):
+    _cuda(choice, "choice")
+    if choice.dtype != torch.int32 or choice.numel() != batch * heads or not choice.is_contiguous():
+        raise ValueError(f"choice: expected contiguous int32 [{batch}, {heads}], got "
+                         f"{choice.dtype} {tuple(choice.shape)}")
+
+
+def bsa_scheme_permute(x: torch.Tensor, grid: Tuple[int, int, int], shapes, choice: torch.Tensor,
+                       n_pad: int, block: int = 0, y: Optional[torch.Tensor] = None,
+                       pooled: Optional[torch.Tensor] = None, pool: bool = False,
+                       device_status: Optional[torch.Tensor] = None):
+    """Tile permute with the slice shape shapes[choice[b, h]] per (batch, head).
+    x [B, N, H, D] bf16 raster -> y [B, n_pad, H, D] (per-head tile order, zero
+    tail); with ``pool`` (or a ``pooled`` buffer) also the per-block means
+    [B, H, n_pad / block, D] fp32.  x and y may be head slices of wider tensors.
+    Returns (y, pooled or None)."""
+    B, _, H, D = x.shape
+    xs = _strided_tokens(x, "x", B, grid[0] * grid[1] * grid[2], H, D)
+    _choice(choice, B, H)
+    if y is None:
+        y = torch.empty((B, n_pad, H, D), dtype=x.dtype, device=x.device)
+    ys = _strided_tokens(y, "y", B, n_pad, H, D)
+    if pooled is None and pool:
+        pooled = torch.empty((B, H, n_pad // max(block, 1), D), dtype=torch.float32,
+                             device=x.device)
+    if pooled is not None:
+        _buffer(pooled, "pooled", torch.float32, B * H * (n_pad // max(block, 1)) * D)
+    arr, n = _shape_array(shapes)
+    _check(load_library().bsa_scheme_permute(_ptr(x), _ptr(y), B, *grid, arr, n, _ptr(choice),
+                                             H, D, n_pad, block, _ptr(pooled), xs, ys,
+                                             _ptr(device_status), _stream()),
+           "bsa_scheme_permute")
+    return y, pooled
+
+
+def bsa_scheme_untile(y: torch.Tensor, grid: Tuple[int, int, int], shapes, choice: torch.Tensor,
+                      x: Optional[torch.Tensor] = None,
+                      device_status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Inverse of bsa_scheme_permute: y [B, n_pad, H, D] -> x [B, N, H, D] raster (either
+    may be a head slice of a wider tensor)."""
+    B, n_pad, H, D = y.shape
+    N = grid[0] * grid[1] * grid[2]
+    ys = _strided_tokens(y, "y", B, n_pad, H, D)
+    _choice(choice, B, H)
+    if x is None:
+        x = torch.empty((B, N, H, D), dtype=y.dtype, device=y.device)
+    xs = _strided_tokens(x, "x", B, N, H, D)
+    arr, n = _shape_array(shapes)
+    _check(load_library().bsa_scheme_untile(_ptr(y), _ptr(x), B, *grid, arr, n, _ptr(choice), H,
+                                            D, n_pad, ys, xs, _ptr(device_status), _stream()),
+           "bsa_scheme_untile")
+    return x
+
+
 # --------------------------------------------------------------------------- (b)
 
 def bsa_sta_mask(tile_grid: Tuple[int, int, int], window: Tuple[int, int, int], shift: int = 0,
@@ -581,15 +640,15 @@ def _n_tiles(grid, tile) -> int:
 
 def bsa_sics_blocks(x: torch.Tensor, grid, tile, out: Optional[torch.Tensor] = None):
     """SICS of every tile of shape `tile` per head.  x: [B, T*H*W, heads, D] bf16 in
-    raster order.  Returns out [B, heads, n_tiles] float32."""
-    _cuda(x, "x")
+    raster order (may be a head slice of a wider tensor).  Returns out [B, heads, n_tiles]
+    float32."""
     B, _, Hh, D = x.shape
-    _tokens(x, "x", B, grid[0] * grid[1] * grid[2], Hh, D)
+    xs = _strided_tokens(x, "x", B, grid[0] * grid[1] * grid[2], Hh, D)
     if out is None:
         out = torch.empty((B, Hh, _n_tiles(grid, tile)), dtype=torch.float32, device=x.device)
     _buffer(out, "out", torch.float32, B * Hh * _n_tiles(grid, tile))
-    _check(load_library().bsa_sics_blocks(_ptr(x), B, *grid, *tile, Hh, D, _ptr(out), _stream()),
-           "bsa_sics_blocks")
+    _check(load_library().bsa_sics_blocks(_ptr(x), B, *grid, *tile, Hh, D, xs, _ptr(out),
+                                          _stream()), "bsa_sics_blocks")
     return out
 
 
@@ -608,11 +667,10 @@ def bsa_sics_scheme(q: torch.Tensor, k: torch.Tensor, grid, shapes,
                     ws: Optional[torch.Tensor] = None):
     """Per-head slicing choice from a shape menu.  Returns (scores [B, H, n_shapes]
     float32, choice [B, H] int32, ws)."""
-    _cuda(q, "q")
     B, _, Hh, D = q.shape
     N = grid[0] * grid[1] * grid[2]
-    _tokens(q, "q", B, N, Hh, D)
-    _tokens(k, "k", B, N, Hh, D)
+    rs = _shared_stride([(q, "q", _strided_tokens(q, "q", B, N, Hh, D)),
+                         (k, "k", _strided_tokens(k, "k", B, N, Hh, D))])
     arr, n = _shape_array(shapes)
     if scores is None:
         scores = torch.empty((B, Hh, n), dtype=torch.float32, device=q.device)
@@ -624,7 +682,7 @@ def bsa_sics_scheme(q: torch.Tensor, k: torch.Tensor, grid, shapes,
         ws = torch.empty(max(1, bsa_sics_workspace_size(B, Hh, grid, shapes)), dtype=torch.uint8,
                          device=q.device)
     _cuda(ws, "ws")
-    _check(load_library().bsa_sics_scheme(_ptr(q), _ptr(k), B, *grid, Hh, D, arr, n,
+    _check(load_library().bsa_sics_scheme(_ptr(q), _ptr(k), B, *grid, Hh, D, rs, arr, n,
                                           _ptr(scores), _ptr(choice), _ptr(ws), _nbytes(ws),
                                           _stream()), "bsa_sics_scheme")
     return scores, choice, ws

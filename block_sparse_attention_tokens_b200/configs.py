@@ -94,6 +94,13 @@ EXTRA = [
     Workload(name="nabla_sta_480p", index=5, batch=1, heads=40, head_dim=128,
              grid=(20, 32, 52), block=64, mask="nabla_sta", tile=(4, 4, 4), window=(3, 3, 5),
              p=0.9, strength_range=(0.5, 3.0)),
+    # SPADE-style per-head slicing on the 480p grid: SICS picks one of the 64-token
+    # slice shapes per head, Q/K/V are permuted head by head with it, then the
+    # NABLA mask over those slices.  Per-head axis stretches make the heads'
+    # features vary along different axes, so the choices differ between heads.
+    Workload(name="spade_480p", index=6, batch=1, heads=40, head_dim=128, grid=(21, 30, 52),
+             block=64, mask="spade", p=0.9, strength_range=(1.0, 3.0),
+             extra={"axis_stretch": 6.0}),
 ]
 
 BY_NAME = {w.name: w for w in WORKLOADS + EXTRA}

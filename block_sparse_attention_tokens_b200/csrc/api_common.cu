@@ -48,7 +48,7 @@ extern "C" const char* bsa_status_string(int status) {
 
 extern "C" const char* bsa_last_error_message(void) { return bsa::g_last_error; }
 
-extern "C" int bsa_version(void) { return 200; }
+extern "C" int bsa_version(void) { return 201; }
 
 extern "C" int bsa_read_status(void* ws, int* status, void* stream) {
   BSA_NVTX_RANGE("bsa_read_status");

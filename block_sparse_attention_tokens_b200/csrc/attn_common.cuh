@@ -273,16 +273,6 @@ int make_map(CUtensorMap* map, const void* base, int B, int N, int H, int D, lon
 
 bool block_ok(int blk) { return blk == 64 || (blk >= 128 && blk % 128 == 0); }
 
-// Row stride (elements) of a token tensor: 0 selects the dense heads * head_dim;
-// otherwise it must hold a whole row and keep every row 16-byte aligned (the TMA
-// maps need strides in multiples of 16 bytes).  Returns -1 if invalid.
-long long token_row_stride(int row_stride, int heads, int head_dim) {
-  const long long dense = static_cast<long long>(heads) * head_dim;
-  if (row_stride == 0) return dense;
-  if (row_stride < dense || (row_stride % 8) != 0) return -1;
-  return row_stride;
-}
-
 struct Geometry {
   int QB, KB, QT, LR, expand;
   long long nnz_cap, entries_cap;

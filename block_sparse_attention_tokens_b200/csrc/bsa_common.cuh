@@ -30,6 +30,16 @@ inline int check_launch() {
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Row stride (elements) of a token tensor: 0 selects the dense heads * head_dim;
+// otherwise it must hold a whole row and keep every row 16-byte aligned (the TMA
+// maps need strides in multiples of 16 bytes).  Returns -1 if invalid.
+inline long long token_row_stride(int row_stride, int heads, int head_dim) {
+  const long long dense = static_cast<long long>(heads) * head_dim;
+  if (row_stride == 0) return dense;
+  if (row_stride < dense || (row_stride % 8) != 0) return -1;
+  return row_stride;
+}
+
 template <typename T>
 __host__ __device__ __forceinline__ T ceil_div(T a, T b) { return (a + b - 1) / b; }
 

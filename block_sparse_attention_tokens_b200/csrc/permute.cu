@@ -220,6 +220,160 @@ int permute_common(bool forward, const void* src, void* dst, int batch, int T, i
   return check_launch();
 }
 
+// ---------------------------------------------------------------------------
+// Per-(batch, head) slicing (SPADE summary, solution parts 1 and 3): every head
+// of every batch is cut with the slice shape it chose from a menu, so the token
+// order differs from head to head.  One CTA per (run of output rows, head, batch)
+// moves that head's head_dim columns of each row; 16-byte vectors, head_dim / 8
+// threads per row, 128 / (head_dim / 8) rows per pass, four passes in flight.
+// ---------------------------------------------------------------------------
+constexpr int kMaxShapes = 8;
+constexpr int kSchemeThreads = 128;
+constexpr int kSchemeRows = 1024;   // upper bound on the rows one CTA handles
+
+struct ShapeMenu {
+  int n;
+  int t[kMaxShapes][3];
+};
+
+__device__ __forceinline__ bool menu_geo(const ShapeMenu& m, int c, int T, int H, int W,
+                                         PermGeo& g) {
+  if (c < 0 || c >= m.n) return false;
+  g = PermGeo{T, H, W, m.t[c][0], m.t[c][1], m.t[c][2]};
+  return true;
+}
+
+// Forward: raster x -> per-head tile order y (zero tail), optionally with the
+// per-block means of the moved rows (pooled [B, heads, n_pad / rb, head_dim]).
+// A (batch, head) whose choice is outside the menu gets zero rows and zero means
+// and BSA_ERR_INVALID_ARG in *status.
+template <bool kPool>
+__global__ void __launch_bounds__(kSchemeThreads) scheme_permute_kernel(
+    const uint4* __restrict__ src, uint4* __restrict__ dst, int n, int n_pad, int rb,
+    long long svpr, long long dvpr, int heads, int head_dim, int T, int H, int W,
+    const ShapeMenu menu, const int* __restrict__ choice, float* __restrict__ pooled,
+    int* status) {
+  const int blk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const long long p0 = static_cast<long long>(blk) * rb;
+  const int rows_here = static_cast<int>(min(static_cast<long long>(rb), n_pad - p0));
+  PermGeo g;
+  const bool good = menu_geo(menu, __ldg(choice + b * heads + h), T, H, W, g);
+  if (!good && threadIdx.x == 0) set_status(status, BSA_ERR_INVALID_ARG);
+  const int rows_valid =
+      good ? static_cast<int>(max(0LL, min(static_cast<long long>(rows_here), n - p0))) : 0;
+  __shared__ int src_row[kSchemeRows];
+  __shared__ float red[kSchemeThreads * 8];
+  for (int r = threadIdx.x; r < rows_valid; r += kSchemeThreads) src_row[r] = tile_token(p0 + r, g);
+  __syncthreads();
+  const int vph = head_dim / 8;                // 16-byte vectors of one head row
+  const int rp = kSchemeThreads / vph;         // rows per pass
+  const int v = threadIdx.x % vph, rg = threadIdx.x / vph;
+  const uint4* sb = src + static_cast<long long>(b) * n * svpr + static_cast<long long>(h) * vph + v;
+  uint4* db = dst + (static_cast<long long>(b) * n_pad + p0) * dvpr + static_cast<long long>(h) * vph + v;
+  float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  auto add = [&](const uint4& x) {
+    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&x);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __bfloat1622float2(h2[e]);
+      acc[2 * e] += f.x;
+      acc[2 * e + 1] += f.y;
+    }
+  };
+  if (rg < rp) {
+    int r = rg;
+    for (; r + 3 * rp < rows_valid; r += 4 * rp) {
+      uint4 x[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) x[u] = __ldg(sb + static_cast<long long>(src_row[r + u * rp]) * svpr);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        db[static_cast<long long>(r + u * rp) * dvpr] = x[u];
+        if (kPool) add(x[u]);
+      }
+    }
+    for (; r < rows_valid; r += rp) {
+      const uint4 x = __ldg(sb + static_cast<long long>(src_row[r]) * svpr);
+      db[static_cast<long long>(r) * dvpr] = x;
+      if (kPool) add(x);
+    }
+    for (; r < rows_here; r += rp) db[static_cast<long long>(r) * dvpr] = make_uint4(0, 0, 0, 0);
+  }
+  if constexpr (kPool) {
+    if (rg < rp) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) red[rg * head_dim + v * 8 + e] = acc[e];
+    }
+    __syncthreads();
+    const float inv = rows_valid > 0 ? 1.0f / static_cast<float>(rows_valid) : 0.f;
+    float* out = pooled + ((static_cast<long long>(b) * heads + h) * (n_pad / rb) + blk) * head_dim;
+    for (int col = threadIdx.x; col < head_dim; col += kSchemeThreads) {
+      float s = 0.f;
+      for (int q = 0; q < rp; ++q) s += red[q * head_dim + col];
+      out[col] = s * inv;
+    }
+  }
+}
+
+// Inverse: tile-order y (per-head order) -> raster x.  One CTA per (run of rb
+// tile-order positions < n, head, batch).  A (batch, head) with a choice outside
+// the menu gets zero rows in x (same positions, read as raster rows) and
+// BSA_ERR_INVALID_ARG in *status.
+__global__ void __launch_bounds__(kSchemeThreads) scheme_untile_kernel(
+    const uint4* __restrict__ src, uint4* __restrict__ dst, int n, int n_pad, int rb,
+    long long svpr, long long dvpr, int heads, int head_dim, int T, int H, int W,
+    const ShapeMenu menu, const int* __restrict__ choice, int* status) {
+  const int blk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const long long p0 = static_cast<long long>(blk) * rb;
+  const int rows = static_cast<int>(min(static_cast<long long>(rb), n - p0));
+  PermGeo g;
+  const bool good = menu_geo(menu, __ldg(choice + b * heads + h), T, H, W, g);
+  if (!good && threadIdx.x == 0) set_status(status, BSA_ERR_INVALID_ARG);
+  __shared__ int dst_row[kSchemeRows];
+  for (int r = threadIdx.x; r < rows; r += kSchemeThreads)
+    dst_row[r] = good ? tile_token(p0 + r, g) : static_cast<int>(p0 + r);
+  __syncthreads();
+  const int vph = head_dim / 8;
+  const int rp = kSchemeThreads / vph;
+  const int v = threadIdx.x % vph, rg = threadIdx.x / vph;
+  if (rg >= rp) return;
+  const uint4* sb = src + (static_cast<long long>(b) * n_pad + p0) * svpr + static_cast<long long>(h) * vph + v;
+  uint4* db = dst + static_cast<long long>(b) * n * dvpr + static_cast<long long>(h) * vph + v;
+  int r = rg;
+  for (; r + 3 * rp < rows; r += 4 * rp) {
+    uint4 x[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      x[u] = good ? __ldg(sb + static_cast<long long>(r + u * rp) * svpr) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) db[static_cast<long long>(dst_row[r + u * rp]) * dvpr] = x[u];
+  }
+  for (; r < rows; r += rp)
+    db[static_cast<long long>(dst_row[r]) * dvpr] =
+        good ? __ldg(sb + static_cast<long long>(r) * svpr) : make_uint4(0, 0, 0, 0);
+}
+
+// Host checks shared by the two scheme entry points; fills the menu.
+int scheme_args(const void* a, const void* b, int batch, int T, int H, int W, const int* shapes,
+                int n_shapes, const int* choice, int heads, int head_dim, int n_pad,
+                ShapeMenu& menu) {
+  if (!a || !b || !shapes || !choice) return BSA_ERR_INVALID_ARG;
+  if (batch < 1 || T < 1 || H < 1 || W < 1 || heads < 1 || head_dim < 8 || (head_dim % 8) != 0)
+    return BSA_ERR_INVALID_ARG;
+  if (n_shapes < 1 || n_shapes > kMaxShapes) return BSA_ERR_INVALID_ARG;
+  if (head_dim > 8 * kSchemeThreads) return BSA_ERR_UNSUPPORTED;
+  const long long n = static_cast<long long>(T) * H * W;
+  if (n > 0x7fffffffLL || n_pad < n) return BSA_ERR_INVALID_ARG;
+  if (!aligned16(a) || !aligned16(b) || (reinterpret_cast<uintptr_t>(choice) & 3u) != 0)
+    return BSA_ERR_INVALID_ARG;
+  menu.n = n_shapes;
+  for (int i = 0; i < kMaxShapes; ++i)
+    for (int j = 0; j < 3; ++j) menu.t[i][j] = i < n_shapes ? shapes[3 * i + j] : 1;
+  for (int i = 0; i < n_shapes; ++i)
+    if (menu.t[i][0] < 1 || menu.t[i][1] < 1 || menu.t[i][2] < 1) return BSA_ERR_INVALID_ARG;
+  return BSA_OK;
+}
+
 }  // namespace
 }  // namespace bsa
 
@@ -265,4 +419,69 @@ extern "C" int bsa_tile_untile(const void* y, void* x, int batch, int T, int H, 
   BSA_NVTX_RANGE("bsa_tile_untile");
   return bsa::permute_common(false, y, x, batch, T, H, W, tT, tH, tW, row_bytes, n_pad,
                              y_row_stride_bytes, x_row_stride_bytes, stream);
+}
+
+extern "C" int bsa_scheme_permute(const void* x, void* y, int batch, int T, int H, int W,
+                                  const int* shapes, int n_shapes, const int* choice, int heads,
+                                  int head_dim, int n_pad, int block, float* pooled,
+                                  int x_row_stride, int y_row_stride, int* device_status,
+                                  void* stream) {
+  BSA_NVTX_RANGE("bsa_scheme_permute");
+  using namespace bsa;
+  ShapeMenu menu;
+  const int rc = scheme_args(x, y, batch, T, H, W, shapes, n_shapes, choice, heads, head_dim,
+                             n_pad, menu);
+  if (rc != BSA_OK) return rc;
+  if (pooled) {
+    if (block < 1 || block > kSchemeRows || (n_pad % block) != 0 || !aligned16(pooled))
+      return BSA_ERR_INVALID_ARG;
+  } else if (block < 0 || block > kSchemeRows) {
+    return BSA_ERR_INVALID_ARG;
+  }
+  const int rb = block > 0 ? block : 64;
+  const long long n = static_cast<long long>(T) * H * W;
+  const long long row_bytes = static_cast<long long>(heads) * head_dim * 2;
+  const long long xs = row_stride_bytes(2LL * x_row_stride, row_bytes);
+  const long long ys = row_stride_bytes(2LL * y_row_stride, row_bytes);
+  if (x_row_stride < 0 || y_row_stride < 0 || xs < 0 || ys < 0) return BSA_ERR_INVALID_ARG;
+  if (spans_overlap(x, batch * n, xs, y, batch * static_cast<long long>(n_pad), ys, row_bytes))
+    return BSA_ERR_INVALID_ARG;
+  dim3 grid(static_cast<unsigned>(ceil_div<long long>(n_pad, rb)), heads, batch);
+  if (grid.y > 65535u || grid.z > 65535u) return BSA_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (pooled)
+    scheme_permute_kernel<true><<<grid, kSchemeThreads, 0, st>>>(
+        static_cast<const uint4*>(x), static_cast<uint4*>(y), static_cast<int>(n), n_pad, rb,
+        xs / 16, ys / 16, heads, head_dim, T, H, W, menu, choice, pooled, device_status);
+  else
+    scheme_permute_kernel<false><<<grid, kSchemeThreads, 0, st>>>(
+        static_cast<const uint4*>(x), static_cast<uint4*>(y), static_cast<int>(n), n_pad, rb,
+        xs / 16, ys / 16, heads, head_dim, T, H, W, menu, choice, nullptr, device_status);
+  return check_launch();
+}
+
+extern "C" int bsa_scheme_untile(const void* y, void* x, int batch, int T, int H, int W,
+                                 const int* shapes, int n_shapes, const int* choice, int heads,
+                                 int head_dim, int n_pad, int y_row_stride, int x_row_stride,
+                                 int* device_status, void* stream) {
+  BSA_NVTX_RANGE("bsa_scheme_untile");
+  using namespace bsa;
+  ShapeMenu menu;
+  const int rc = scheme_args(y, x, batch, T, H, W, shapes, n_shapes, choice, heads, head_dim,
+                             n_pad, menu);
+  if (rc != BSA_OK) return rc;
+  const long long n = static_cast<long long>(T) * H * W;
+  const long long row_bytes = static_cast<long long>(heads) * head_dim * 2;
+  const long long ys = row_stride_bytes(2LL * y_row_stride, row_bytes);
+  const long long xs = row_stride_bytes(2LL * x_row_stride, row_bytes);
+  if (x_row_stride < 0 || y_row_stride < 0 || xs < 0 || ys < 0) return BSA_ERR_INVALID_ARG;
+  if (spans_overlap(y, batch * static_cast<long long>(n_pad), ys, x, batch * n, xs, row_bytes))
+    return BSA_ERR_INVALID_ARG;
+  constexpr int rb = 128;
+  dim3 grid(static_cast<unsigned>(ceil_div<long long>(n, rb)), heads, batch);
+  if (grid.y > 65535u || grid.z > 65535u) return BSA_ERR_UNSUPPORTED;
+  scheme_untile_kernel<<<grid, kSchemeThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(y), static_cast<uint4*>(x), static_cast<int>(n), n_pad, rb,
+      ys / 16, xs / 16, heads, head_dim, T, H, W, menu, choice, device_status);
+  return check_launch();
 }

@@ -37,6 +37,7 @@ SicsGrid sics_grid(int T, int H, int W, int tT, int tH, int tW) {
 // CTAs of segment s are blockIdx.x in [first[s], first[s + 1]), one per tile.
 struct SicsSegments {
   int n;
+  long long row_vec;  // token row stride in 16-byte vectors (>= heads * head_dim / 8)
   int first[2 * kMaxShapes + 1];
   SicsGrid g[2 * kMaxShapes];
   const uint4* x[2 * kMaxShapes];
@@ -56,9 +57,9 @@ __global__ void __launch_bounds__(1024) sics_kernel(const __grid_constant__ Sics
   const SicsGrid& g = sg.g[seg];
   const uint4* __restrict__ x = sg.x[seg];
   const int tile = blockIdx.x - sg.first[seg], b = blockIdx.y;
-  const int row_vec = heads * G;  // 16-byte vectors per token row
+  const long long row_vec = sg.row_vec;   // 16-byte vectors from one token row to the next
   const int j = threadIdx.x;
-  const bool active = j < row_vec;
+  const bool active = j < heads * G;
   const int a = tile / (g.nH * g.nW);
   const int rem = tile - a * (g.nH * g.nW);
   const int bb = rem / g.nW, c = rem - bb * g.nW;
@@ -202,14 +203,18 @@ double pairs_of(int T, int H, int W, int tT, int tH, int tW) {
 }  // namespace bsa
 
 extern "C" int bsa_sics_blocks(const void* x, int batch, int T, int H, int W, int tT, int tH,
-                               int tW, int heads, int head_dim, float* out, void* stream) {
+                               int tW, int heads, int head_dim, int row_stride, float* out,
+                               void* stream) {
   BSA_NVTX_RANGE("bsa_sics_blocks");
   using namespace bsa;
   if (!x || !out || !aligned16(x)) return BSA_ERR_INVALID_ARG;
   int rc = check_sics_args(batch, T, H, W, heads, head_dim);
   if (rc != BSA_OK) return rc;
   if ((rc = check_shape(T, H, W, tT, tH, tW)) != BSA_OK) return rc;
+  const long long rs = token_row_stride(row_stride, heads, head_dim);
+  if (rs < 0) return BSA_ERR_INVALID_ARG;
   SicsSegments sg;
+  sg.row_vec = rs / 8;
   sg.n = 1;
   sg.g[0] = sics_grid(T, H, W, tT, tH, tW);
   sg.x[0] = static_cast<const uint4*>(x);
@@ -233,9 +238,9 @@ extern "C" size_t bsa_sics_workspace_size(int batch, int heads, int T, int H, in
 }
 
 extern "C" int bsa_sics_scheme(const void* q, const void* k, int batch, int T, int H, int W,
-                               int heads, int head_dim, const int* shapes, int n_shapes,
-                               float* scores, int* choice, void* ws, size_t ws_bytes,
-                               void* stream) {
+                               int heads, int head_dim, int row_stride, const int* shapes,
+                               int n_shapes, float* scores, int* choice, void* ws,
+                               size_t ws_bytes, void* stream) {
   BSA_NVTX_RANGE("bsa_sics_scheme");
   using namespace bsa;
   if (!q || !k || !shapes || !scores || !choice || !ws || !aligned16(q) || !aligned16(k))
@@ -246,6 +251,8 @@ extern "C" int bsa_sics_scheme(const void* q, const void* k, int batch, int T, i
   for (int s = 0; s < n_shapes; ++s)
     if ((rc = check_shape(T, H, W, shapes[3 * s], shapes[3 * s + 1], shapes[3 * s + 2])) != BSA_OK)
       return rc;
+  const long long rs = token_row_stride(row_stride, heads, head_dim);
+  if (rs < 0) return BSA_ERR_INVALID_ARG;
   const size_t need = bsa_sics_workspace_size(batch, heads, T, H, W, shapes, n_shapes);
   if (ws_bytes < need) return BSA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -255,6 +262,7 @@ extern "C" int bsa_sics_scheme(const void* q, const void* k, int batch, int T, i
   SicsMenu m;
   m.n = n_shapes;
   SicsSegments sg;
+  sg.row_vec = rs / 8;
   sg.n = 2 * n_shapes;
   long long off = 0, ctas = 0;
   for (int s = 0; s < n_shapes; ++s) {

@@ -4,6 +4,8 @@ A ``Plan`` owns the device buffers of one workload and runs the whole path with
 ``step(q, k, v)``: tile permute of Q/K/V, block-mask generation (Sliding-Tile,
 radial, NABLA or the autoregressive anchor/recent/NABLA composition), CSR
 compaction, the block-sparse attention forward and the inverse permute of O.
+The ``spade`` family first picks a slice shape per head by SICS and permutes each
+head with its own shape before the NABLA mask.
 Every step is a libbsa kernel; this module only allocates and orders calls.
 """
 from __future__ import annotations
@@ -15,7 +17,7 @@ from typing import Optional, Tuple
 import torch
 
 from . import binding as B
-from .configs import Workload
+from .configs import Workload, sics_menu
 
 
 def ceil_div(a: int, b: int) -> int:
@@ -60,7 +62,7 @@ class Plan:
         Hh, D, Bt = self.h1 - self.h0, w.head_dim, w.batch
         self.heads = Hh
         self.nq, self.nk = w.nq, w.nk
-        self.permuted = w.tile is not None
+        self.permuted = w.tile is not None or w.mask == "spade"
         if self.permuted:
             self.n_pad = ceil_div(w.n_tokens, w.block) * w.block
             self.qp = torch.empty((Bt, self.n_pad, Hh, D), dtype=torch.bfloat16, device=device)
@@ -79,7 +81,15 @@ class Plan:
             self.nabla_ws = torch.empty(
                 B.bsa_nabla_workspace_size(Bt, Hh, self.nq, self.nk, D, w.block),
                 dtype=torch.uint8, device=device)
-        if w.mask in ("nabla", "nabla_sta"):
+        if w.mask == "spade":
+            # per-head slice shapes chosen by SICS from the menu of the block size
+            self.menu = sics_menu(w.block)
+            self.scores = torch.empty((Bt, Hh, len(self.menu)), dtype=torch.float32, device=device)
+            self.choice = torch.empty((Bt, Hh), dtype=torch.int32, device=device)
+            self.sics_ws = torch.empty(max(1, B.bsa_sics_workspace_size(Bt, Hh, w.grid, self.menu)),
+                                       dtype=torch.uint8, device=device)
+            self.scheme_status = torch.zeros(1, dtype=torch.int32, device=device)
+        if w.mask in ("nabla", "nabla_sta", "spade"):
             # block means come out of the fused permute of Q and K
             self.qbar = torch.empty((Bt, Hh, self.QB, D), dtype=torch.float32, device=device)
             self.kbar = torch.empty((Bt, Hh, self.KB, D), dtype=torch.float32, device=device)
@@ -123,6 +133,14 @@ class Plan:
                                     pooled=self.kbar)
             B.bsa_tile_permute(v, w.grid, w.tile, self.n_pad, y=self.vp)
             return
+        if w.mask == "spade":
+            B.bsa_sics_scheme(q, k, w.grid, self.menu, scores=self.scores, choice=self.choice,
+                              ws=self.sics_ws)
+            for src, dst, pooled in ((q, self.qp, self.qbar), (k, self.kp, self.kbar),
+                                     (v, self.vp, None)):
+                B.bsa_scheme_permute(src, w.grid, self.menu, self.choice, self.n_pad, w.block,
+                                     y=dst, pooled=pooled, device_status=self.scheme_status)
+            return
         for src, dst in ((q, self.qp), (k, self.kp), (v, self.vp)):
             B.bsa_tile_permute(src, w.grid, w.tile, self.n_pad, y=dst)
 
@@ -132,7 +150,7 @@ class Plan:
             B.bsa_sta_mask(self.tile_grid, w.window, 0, mask=self.mask)
         elif w.mask == "radial":
             B.bsa_radial_mask(self.nk, w.tokens_per_frame, w.block, mask=self.mask)
-        elif w.mask == "nabla":
+        elif w.mask in ("nabla", "spade"):
             B.bsa_nabla_select(self.qbar, self.kbar, w.p, mask=self.mask, near_count=self.near)
         elif w.mask == "nabla_sta":
             B.bsa_sta_mask(self.tile_grid, w.window, 0, mask=self.base_mask)
@@ -160,6 +178,10 @@ class Plan:
                        nq=self.nq, nk=self.nk, o=out, lse=self.lse, ws=self.attn_ws)
 
     def untile(self):
+        if self.w.mask == "spade":
+            B.bsa_scheme_untile(self.op, self.w.grid, self.menu, self.choice,
+                                x=self._mine(self.out), device_status=self.scheme_status)
+            return
         B.bsa_tile_untile(self.op, self.w.grid, self.w.tile, x=self._mine(self.out))
 
     def step(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
@@ -189,6 +211,8 @@ class Plan:
         n = 0
         if self.permuted:
             n += 3 + 1                   # permute Q, K, V and untile O
+        if self.w.mask == "spade":
+            n += 2                       # SICS of every (tensor, shape) tile + the per-head pick
         n += {"nabla": 1, "nabla_sta": 2, "ar": 2}.get(self.w.mask, 1)   # mask kernels
         n += 3                           # compact: count, scan, fill
         n += 2                           # kept-list build + attention

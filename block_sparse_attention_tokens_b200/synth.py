@@ -10,10 +10,14 @@ Recipe (one call per workload, ``numpy.random.default_rng(seed)``, seed = 1000 +
 2. ``phi``    (16,)    ~ U[0, 2*pi)         their phases
 3. per-head strength s_h: fixed, or U(lo, hi) drawn in head order
 4. ``W_q[h]`` (16, D)  ~ N(0, 1/16) for h = 0..H-1, then ``W_k[h]`` likewise
+4b. only with an axis stretch r: ``a[h]`` (H, 3) = exp(U(-ln r, ln r)), per-head
+    scales of the (t, h, w) coordinates (heads whose features vary fastest along
+    different axes)
 5. noise for Q, then K, then V: standard normal float32 of shape (B, N, H, D)
 
 Position features: token i of a T x H x W grid in raster order sits at
-x = (t/(T-1), h/(H-1), w/(W-1)) (0 on an axis of length 1) and F(x) = cos(omega x + phi).
+x = (t/(T-1), h/(H-1), w/(W-1)) (0 on an axis of length 1) and F(x) = cos(omega x + phi)
+(with a stretch: F_h(x) = cos(omega (a[h] * x) + phi)).
 Q = noise + s_h * F(x) W_q[h], K = noise + s_h * F(x) W_k[h], V = noise (iid N(0,1)).
 The float32 values are rounded to bfloat16 (round to nearest even).  Tokens are
 returned in raster order, layout [B, N, H, D].
@@ -51,7 +55,8 @@ def generate(batch: int, heads: int, head_dim: int, grid: Tuple[int, int, int], 
              strength: Optional[float] = None,
              strength_range: Optional[Tuple[float, float]] = None,
              iid: bool = False,
-             q_token_ids: Optional[np.ndarray] = None):
+             q_token_ids: Optional[np.ndarray] = None,
+             axis_stretch: Optional[float] = None):
     """Draw (Q, K, V) as bfloat16 CPU tensors [B, N, H, D] following the module recipe.
 
     ``q_token_ids`` selects the raster positions of the query tokens (default: all
@@ -75,12 +80,19 @@ def generate(batch: int, heads: int, head_dim: int, grid: Tuple[int, int, int], 
         s = np.zeros(heads)
     wq = np.stack([rng.normal(0.0, 0.25, size=(N_FEATURES, head_dim)) for _ in range(heads)])
     wk = np.stack([rng.normal(0.0, 0.25, size=(N_FEATURES, head_dim)) for _ in range(heads)])
+    stretch = None
+    if axis_stretch is not None:
+        lr = math.log(axis_stretch)
+        stretch = np.exp(rng.uniform(-lr, lr, size=(heads, 3)))
 
     def with_features(noise: np.ndarray, ids: np.ndarray, w: np.ndarray) -> np.ndarray:
         if iid:
             return noise
-        feats = np.cos(raster_positions(grid, ids) @ omega.T + phi)       # (n, 16)
+        pos = raster_positions(grid, ids)
+        feats = np.cos(pos @ omega.T + phi)                                 # (n, 16)
         for h in range(heads):
+            if stretch is not None:
+                feats = np.cos((pos * stretch[h]) @ omega.T + phi)
             add = (feats @ (s[h] * w[h])).astype(np.float32)               # (n, D)
             noise[:, :, h, :] += add[None, :, :]
         return noise
@@ -94,7 +106,7 @@ def generate(batch: int, heads: int, head_dim: int, grid: Tuple[int, int, int], 
     v = rng.standard_normal((batch, n, heads, head_dim), dtype=np.float32)
     vt = _to_bf16(v)
     del v
-    return qt, kt, vt, {"strength": s, "omega": omega, "phi": phi}
+    return qt, kt, vt, {"strength": s, "omega": omega, "phi": phi, "stretch": stretch}
 
 
 def workload_inputs(w: "_configs.Workload"):
@@ -104,7 +116,8 @@ def workload_inputs(w: "_configs.Workload"):
         n = w.n_tokens
         q_ids = np.arange(n - w.nq, n, dtype=np.int64)
     return generate(w.batch, w.heads, w.head_dim, w.grid, w.seed, strength=w.strength,
-                    strength_range=w.strength_range, iid=w.iid, q_token_ids=q_ids)
+                    strength_range=w.strength_range, iid=w.iid, q_token_ids=q_ids,
+                    axis_stretch=w.extra.get("axis_stretch"))
 
 
 def grad_output(w: "_configs.Workload", seed_offset: int = 500) -> torch.Tensor:

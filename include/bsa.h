@@ -119,6 +119,44 @@ int bsa_tile_permute_pool(const void* x, void* y, int batch, int T, int H, int W
                           float* pooled, int x_row_stride, int y_row_stride, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * (a'') Tile permute with a slice shape per (batch, head).
+ * Source: SPADE summary (gist.science/ja/paper/2608.03335), solution part 1 (a
+ * menu of ways to cut the T x H x W cube, the best one picked for the video),
+ * part 2 (the pick by SICS, bsa_sics_scheme) and part 3 (head-wise sparse
+ * attention on the result).
+ *
+ * Head h of batch b is permuted like bsa_tile_permute with the tile
+ * shapes[choice[b * heads + h]], so each head of y has its own token order; the
+ * attention, masks and compaction then run on y unchanged (they are per head).
+ *   shapes : HOST int array [n_shapes][3] (tT, tH, tW), 1 <= n_shapes <= 8,
+ *            e.g. the menu given to bsa_sics_scheme.
+ *   choice : DEVICE int32 [batch][heads] (4-byte aligned), e.g. bsa_sics_scheme's
+ *            choice output.
+ *            An entry outside [0, n_shapes) is not a host error (the host does
+ *            not read it): that head's rows of y (and its pooled means) are
+ *            zero and BSA_ERR_INVALID_ARG is written to *device_status (a device
+ *            int, may be NULL, not cleared by the call).
+ *   x, y   : bf16 [batch, N, heads, head_dim] raster / [batch, n_pad, heads,
+ *            head_dim] in per-head tile order, zero tail; row strides in
+ *            elements as in bsa_tile_permute_pool.  head_dim a multiple of 8,
+ *            at most 1024.
+ *   pooled : optional (NULL: no pooling) float32 [batch, heads, n_pad / block,
+ *            head_dim], the mean of every `block` consecutive rows of y per head
+ *            over the rows that hold tokens; n_pad a multiple of block, block <=
+ *            1024.  Without pooled, block only sets the rows per CTA (0 = 64).
+ * bsa_scheme_untile: the inverse, y (per-head tile order) -> x (raster); the
+ *   zero tail of y is not read.  A head with a choice outside the menu gets zero
+ *   rows in x and the same device status.
+ * ------------------------------------------------------------------------- */
+int bsa_scheme_permute(const void* x, void* y, int batch, int T, int H, int W,
+                       const int* shapes, int n_shapes, const int* choice, int heads,
+                       int head_dim, int n_pad, int block, float* pooled, int x_row_stride,
+                       int y_row_stride, int* device_status, void* stream);
+int bsa_scheme_untile(const void* y, void* x, int batch, int T, int H, int W, const int* shapes,
+                      int n_shapes, const int* choice, int heads, int head_dim, int n_pad,
+                      int y_row_stride, int x_row_stride, int* device_status, void* stream);
+
+/* ---------------------------------------------------------------------------
  * (b1) Sliding Tile Attention mask.
  * Source: STA explainer (aibr.jp/archives/60739), sections 2-3: each query tile
  * attends to a window of neighbouring tiles; the window is counted in tiles.
@@ -332,7 +370,9 @@ int bsa_attn_fwd_noalloc(const void* q, const void* k, const void* v, int batch,
  *     out[b][h][tile] = sum over ordered token pairs (i, j) of the tile of
  *                       cos(x[b, i, h, :], x[b, j, h, :])   (i == j included;
  *                       a zero vector contributes 0).
- *   x : [batch, T*H*W, heads, head_dim] bf16, raster token order, 16-byte aligned
+ *   x : [batch, T*H*W, heads, head_dim] bf16, raster token order, 16-byte aligned;
+ *       row_stride: token row stride in elements (0 = heads * head_dim), as in the
+ *       conventions above (bsa_sics_scheme: shared by q and k)
  *   out : float32 [batch][heads][ceil(T/tT)*ceil(H/tH)*ceil(W/tW)], written
  *   head_dim in {64, 128}; heads * head_dim <= 8192; tT*tH*tW <= 4096 tokens.
  *
@@ -348,12 +388,12 @@ int bsa_attn_fwd_noalloc(const void* q, const void* k, const void* v, int batch,
  * range), BSA_ERR_WORKSPACE.
  * ------------------------------------------------------------------------- */
 int bsa_sics_blocks(const void* x, int batch, int T, int H, int W, int tT, int tH, int tW,
-                    int heads, int head_dim, float* out, void* stream);
+                    int heads, int head_dim, int row_stride, float* out, void* stream);
 size_t bsa_sics_workspace_size(int batch, int heads, int T, int H, int W, const int* shapes,
                                int n_shapes);
 int bsa_sics_scheme(const void* q, const void* k, int batch, int T, int H, int W, int heads,
-                    int head_dim, const int* shapes, int n_shapes, float* scores, int* choice,
-                    void* ws, size_t ws_bytes, void* stream);
+                    int head_dim, int row_stride, const int* shapes, int n_shapes,
+                    float* scores, int* choice, void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
  * (g) Paged KV cache with persistent anchors (autoregressive chunk decoding).

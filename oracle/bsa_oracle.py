@@ -86,6 +86,35 @@ def tile_untile(y: np.ndarray, perm: np.ndarray) -> np.ndarray:
     return x
 
 
+def scheme_permute(x: np.ndarray, grid: Tuple[int, int, int], shapes, choice: np.ndarray,
+                   n_pad: int) -> np.ndarray:
+    """Per-head slicing (SPADE summary, solution parts 1 and 3): head h of batch b
+    is put in the tile order of the slice shape shapes[choice[b, h]].
+
+    x: [B, N, H, D] raster; returns y [B, n_pad, H, D], rows N.. zero.
+    y[b, p, h] = x[b, perm_bh[p], h] with perm_bh = tile_order(grid, shape of (b, h)).
+    """
+    Bt, n, H = x.shape[0], x.shape[1], x.shape[2]
+    y = np.zeros((Bt, n_pad) + x.shape[2:], dtype=x.dtype)
+    for b in range(Bt):
+        for h in range(H):
+            perm = tile_order(grid, tuple(shapes[int(choice[b, h])]))
+            y[b, :n, h] = x[b, perm, h]
+    return y
+
+
+def scheme_untile(y: np.ndarray, grid: Tuple[int, int, int], shapes, choice: np.ndarray) -> np.ndarray:
+    """Inverse of scheme_permute: x[b, perm_bh[p], h] = y[b, p, h] for p < N."""
+    n = grid[0] * grid[1] * grid[2]
+    Bt, H = y.shape[0], y.shape[2]
+    x = np.empty((Bt, n) + y.shape[2:], dtype=y.dtype)
+    for b in range(Bt):
+        for h in range(H):
+            perm = tile_order(grid, tuple(shapes[int(choice[b, h])]))
+            x[b, perm, h] = y[b, :n, h]
+    return x
+
+
 # ---------------------------------------------------------------------------
 # 2. Sliding Tile Attention mask
 # ---------------------------------------------------------------------------

@@ -158,17 +158,37 @@ def test_every_entry_rejects_bad_arguments_before_touching_cuda(lib, no_gpu):
         args = list(pp)
         args[i] = val
         assert lib.bsa_tile_permute_pool(*args) == INV, (i, val)
-    # SICS: blocks (x B T H W tT tH tW heads d out) and scheme
-    sb = [A, 1, 4, 8, 8, 4, 4, 4, 2, 128, A, None]
-    for i, val, rc in ((9, 96, UNS), (5, 300, UNS), (8, 200, UNS), (0, U, INV), (2, 0, INV)):
+    # per-head slicing: x y B T H W shapes n_shapes choice heads d n_pad block pooled x_rs y_rs
+    # status  (untile: y x B T H W shapes n_shapes choice heads d n_pad y_rs x_rs status)
+    menu = (ctypes.c_int * 6)(4, 4, 4, 1, 8, 8)
+    bad_menu = (ctypes.c_int * 6)(4, 4, 4, 1, 0, 8)
+    Y = ctypes.c_void_p(1 << 40)
+    sp = [A, Y, 1, 4, 8, 8, menu, 2, A, 2, 128, 256, 64, A, 0, 0, None, None]
+    for i, val, rc in ((6, None, INV), (7, 0, INV), (7, 9, INV), (6, bad_menu, INV), (8, None, INV),
+                       (8, ctypes.c_void_p(18), INV), (10, 12, INV), (10, 2048, UNS), (11, 255, INV), (12, 48, INV),
+                       (12, 2048, INV), (13, U, INV), (14, 250, INV), (15, 260, INV), (1, A, INV)):
+        args = list(sp)
+        args[i] = val
+        assert lib.bsa_scheme_permute(*args) == rc, (i, val)
+    su = [A, Y, 1, 4, 8, 8, menu, 2, A, 2, 128, 256, 0, 0, None, None]
+    for i, val, rc in ((6, None, INV), (7, 9, INV), (8, None, INV), (11, 255, INV),
+                       (12, 250, INV), (13, 260, INV), (1, A, INV), (10, 2048, UNS)):
+        args = list(su)
+        args[i] = val
+        assert lib.bsa_scheme_untile(*args) == rc, (i, val)
+    # SICS: blocks (x B T H W tT tH tW heads d row_stride out) and scheme
+    sb = [A, 1, 4, 8, 8, 4, 4, 4, 2, 128, 0, A, None]
+    for i, val, rc in ((9, 96, UNS), (5, 300, UNS), (8, 200, UNS), (0, U, INV), (2, 0, INV),
+                       (10, 128, INV), (10, 260, INV)):
         args = list(sb)
         args[i] = val
         assert lib.bsa_sics_blocks(*args) == rc, (i, val)
     shapes = (ctypes.c_int * 6)(4, 4, 4, 1, 8, 8)
     need = lib.bsa_sics_workspace_size(1, 2, 4, 8, 8, shapes, 2)
     assert need == 4 * 2 * 1 * 2 * (4 + 4)
-    sch = [A, A, 1, 4, 8, 8, 2, 128, shapes, 2, A, A, A, need, None]
-    for i, val, rc in ((9, 0, INV), (9, 17, INV), (13, need - 4, WS), (1, U, INV)):
+    sch = [A, A, 1, 4, 8, 8, 2, 128, 0, shapes, 2, A, A, A, need, None]
+    for i, val, rc in ((10, 0, INV), (10, 17, INV), (14, need - 4, WS), (1, U, INV),
+                       (8, 200, INV)):
         args = list(sch)
         args[i] = val
         assert lib.bsa_sics_scheme(*args) == rc, (i, val)

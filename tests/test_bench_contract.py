@@ -34,7 +34,7 @@ def test_reference_arm_prints_one_contract_line(pass_):
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
 
 
-@pytest.mark.parametrize("workload", ["nabla_480p", "ar_decode"])
+@pytest.mark.parametrize("workload", ["nabla_480p", "ar_decode", "spade_480p"])
 def test_reference_arm_on_dynamic_masks(workload):
     # the oracle builds its own NABLA / autoregressive mask (untimed) and is timed
     # on sampled query blocks (two heads keep the CPU run short)

@@ -35,6 +35,8 @@ SMALL = [
       mask="ar", p=0.85, strength=1.5, q_frames=3, anchor_frames=3, recent_frames=6),
     W(name="nabla_sta_small", index=15, batch=1, heads=2, head_dim=128, grid=(8, 8, 12), block=64,
       mask="nabla_sta", tile=(4, 4, 4), window=(3, 3, 3), p=0.9, strength_range=(0.5, 3.0)),
+    W(name="spade_small", index=16, batch=1, heads=4, head_dim=128, grid=(6, 10, 12), block=64,
+      mask="spade", p=0.9, strength_range=(1.0, 3.0), extra={"axis_stretch": 6.0}),
 ]
 
 
@@ -59,12 +61,15 @@ def test_head_halves_equal_the_whole_and_the_oracle(w):
     assert torch.equal(out, o_ref), "head halves differ from the whole call"
     assert torch.equal(torch.cat(lses, dim=1), lse_ref)
     # the oracle on sampled rows of the first head of each half (path token order)
-    from tests.test_gpu_workloads import oracle_mask
+    from tests.test_gpu_workloads import check_spade_choice, head_perms, oracle_mask
+    if w.mask == "spade":
+        check_spade_choice(w, whole, q, k)
     ref_mask, near = oracle_mask(w, whole, q, k)
     op = (whole.op if whole.permuted else whole.o).cpu()
     rows = np.unique(np.r_[0, w.nq - 1, np.random.default_rng(w.seed).integers(0, w.nq, 24)])
-    perm = O.tile_order(w.grid, w.tile) if whole.permuted else None
+    perms = head_perms(w, whole)
     for h in (0, head_range(1, 2, w.heads)[0]):
+        perm = perms[h]
         hm = 0 if ref_mask.shape[0] == 1 else h
         keep = rows if near is None else rows[~near[hm, rows // w.block]]
         qh, kh, vh = (to64(t[:, :, h:h + 1]) for t in (q, k, v))

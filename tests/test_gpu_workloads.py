@@ -33,6 +33,31 @@ def sample_rows_in_blocks(blocks, block, n_valid, per_block, seed):
     return np.array(sorted(rows), dtype=np.int64)
 
 
+def head_perms(w, plan):
+    """Token order of every head in the path (None: raster order).  The spade family's
+    per-head shapes are the plan's SICS choice, which tests/test_gpu_sics.py and
+    check_spade_choice hold to the oracle's."""
+    if not plan.permuted:
+        return [None] * w.heads
+    if w.mask == "spade":
+        choice = plan.choice.cpu().numpy()
+        return [O.tile_order(w.grid, plan.menu[int(choice[0, h])]) for h in range(w.heads)]
+    perm = O.tile_order(w.grid, w.tile)
+    return [perm] * w.heads
+
+
+def check_spade_choice(w, plan, q, k):
+    """The plan's per-head slice choice against the oracle's SICS scheme (near ties
+    may go either way)."""
+    rs, rc = O.sics_scheme(to64(q), to64(k), w.grid, plan.menu)
+    choice = plan.choice.cpu().numpy()
+    for h in range(w.heads):
+        order = np.argsort(-rs[0, h], kind="stable")
+        near = [s for s in range(rs.shape[2]) if rs[0, h, order[0]] - rs[0, h, s] < 1e-4]
+        assert choice[0, h] == rc[0, h] or choice[0, h] in near, h
+    return choice
+
+
 def oracle_mask(w, plan, q, k):
     """The oracle's own block mask for the workload ([Hm, QB, KB] plus near flags)."""
     if w.mask == "sta":
@@ -41,16 +66,16 @@ def oracle_mask(w, plan, q, k):
         return O.radial_block_mask_fast(w.nk, w.tokens_per_frame, w.block)[None], None
     D = w.head_dim
     scale = 1.0 / math.sqrt(D)
-    if w.mask in ("nabla", "nabla_sta"):
-        perm = O.tile_order(w.grid, w.tile)
+    if w.mask in ("nabla", "nabla_sta", "spade"):
+        perms = head_perms(w, plan)
         qbar = np.zeros((w.batch, w.heads, plan.QB, D))
         kbar = np.zeros((w.batch, w.heads, plan.KB, D))
         for h in range(w.heads):
-            qh = O.tile_permute(to64(q[:, :, h:h + 1]), perm, plan.n_pad)
-            kh = O.tile_permute(to64(k[:, :, h:h + 1]), perm, plan.n_pad)
+            qh = O.tile_permute(to64(q[:, :, h:h + 1]), perms[h], plan.n_pad)
+            kh = O.tile_permute(to64(k[:, :, h:h + 1]), perms[h], plan.n_pad)
             qbar[:, h] = O.nabla_pool(qh, w.block, w.nq)[:, 0]
             kbar[:, h] = O.nabla_pool(kh, w.block, w.nk)[:, 0]
-        if w.mask == "nabla":
+        if w.mask in ("nabla", "spade"):
             m, near = O.nabla_mask(qbar, kbar, w.p, scale)
         else:
             m, near = O.nabla_sta_mask(qbar, kbar, w.p, scale,
@@ -81,6 +106,10 @@ def test_workload_path(name):
     from block_sparse_attention_tokens_b200 import binding as B
     assert B.bsa_read_status(plan.attn_ws) == 0
 
+    if w.mask == "spade":
+        check_spade_choice(w, plan, q, k)
+        assert int(plan.scheme_status.item()) == 0
+
     # --- mask: bit-exact against the oracle's own mask
     ref_mask, near = oracle_mask(w, plan, q, k)
     gpu_mask = plan.mask.cpu().numpy().reshape(-1, plan.QB, plan.KB)
@@ -93,7 +122,7 @@ def test_workload_path(name):
         skip_rows = differs
 
     # --- attention on sampled rows (path token order) against the oracle
-    perm = O.tile_order(w.grid, w.tile) if plan.permuted else None
+    perms = head_perms(w, plan)
     blocks = sample_blocks(plan.QB, 6 if w.nk > 200000 else 12, seed=w.seed)
     rows = sample_rows_in_blocks(blocks, w.block, w.nq, 6, seed=w.seed + 1)
     op = (plan.op if plan.permuted else plan.o).cpu()
@@ -104,9 +133,9 @@ def test_workload_path(name):
         if keep_rows.size == 0:
             continue
         if plan.permuted:
-            qh = O.tile_permute(to64(q[:, :, h:h + 1]), perm, plan.n_pad)
-            kh = O.tile_permute(to64(k[:, :, h:h + 1]), perm, plan.n_pad)
-            vh = O.tile_permute(to64(v[:, :, h:h + 1]), perm, plan.n_pad)
+            qh = O.tile_permute(to64(q[:, :, h:h + 1]), perms[h], plan.n_pad)
+            kh = O.tile_permute(to64(k[:, :, h:h + 1]), perms[h], plan.n_pad)
+            vh = O.tile_permute(to64(v[:, :, h:h + 1]), perms[h], plan.n_pad)
             qh, kh, vh = qh[:, :w.nq], kh[:, :w.nk], vh[:, :w.nk]
         else:
             qh, kh, vh = to64(q[:, :, h:h + 1]), to64(k[:, :, h:h + 1]), to64(v[:, :, h:h + 1])
@@ -120,4 +149,6 @@ def test_workload_path(name):
     if plan.permuted:
         ob = o.cpu().view(torch.int16).numpy()
         opb = op.view(torch.int16).numpy()
-        assert np.array_equal(ob[:, perm[rows[rows < w.nq]]], opb[:, rows[rows < w.nq]])
+        r = rows[rows < w.nq]
+        for h in range(w.heads):
+            assert np.array_equal(ob[:, perms[h][r], h], opb[:, r, h]), h

@@ -23,6 +23,7 @@ from oracle import bsa_oracle as M
 from tests import test_oracle_masks as TM
 from tests import test_oracle_nabla_attention as TN
 from tests import test_oracle_paged as TP
+from tests import test_oracle_scheme as TSC
 from tests import test_oracle_sics as TS
 
 
@@ -74,6 +75,26 @@ MUTANTS = [
     Mutant("tile_untile/forward-permutation", "tile_untile",
            "x[:, perm] = y[:, :n]", "x[:] = y[:, perm]",
            [pin(TM.test_permute_untile_roundtrip_and_zero_tail)]),
+    Mutant("scheme_permute/choice-transposed", "scheme_permute",
+           "perm = tile_order(grid, tuple(shapes[int(choice[b, h])]))",
+           "perm = tile_order(grid, tuple(shapes[int(choice.reshape(-1)[h * Bt + b])]))",
+           [pin(TSC.test_scheme_permute_golden_mixed_choices)]),
+    Mutant("scheme_permute/first-head-shape-for-all", "scheme_permute",
+           "perm = tile_order(grid, tuple(shapes[int(choice[b, h])]))",
+           "perm = tile_order(grid, tuple(shapes[int(choice[b, 0])]))",
+           [pin(TSC.test_scheme_permute_golden_mixed_choices)]),
+    Mutant("scheme_permute/inverse-permutation", "scheme_permute",
+           "y[b, :n, h] = x[b, perm, h]", "y[b, perm, h] = x[b, :, h]",
+           [pin(TSC.test_scheme_permute_golden_mixed_choices),
+            pin(TSC.test_scheme_roundtrip_random_choices)]),
+    Mutant("scheme_untile/forward-permutation", "scheme_untile",
+           "x[b, perm, h] = y[b, :n, h]", "x[b, :, h] = y[b, perm, h]",
+           [pin(TSC.test_scheme_untile_golden_mixed_choices),
+            pin(TSC.test_scheme_roundtrip_random_choices)]),
+    Mutant("scheme_untile/batch-0-choice", "scheme_untile",
+           "perm = tile_order(grid, tuple(shapes[int(choice[b, h])]))",
+           "perm = tile_order(grid, tuple(shapes[int(choice[0, h])]))",
+           [pin(TSC.test_scheme_untile_golden_mixed_choices)]),
 
     # ------------------------------------------------------------ Sliding-Tile window
     Mutant("sta/exclusive-upper-edge", "sta_axis_keep",
