@@ -100,12 +100,58 @@ __device__ __forceinline__ int warp_isum(int v) {
   return v;
 }
 
+// The cut of one row's top-p selection: the largest order key v whose mass
+// F(v) = sum of e_c over the keys >= v reaches target, found bit by bit from the
+// top.  Each lane sums its entries c = lane, lane + 32, ... in that order, so the
+// register and shared-memory forms give the same sums.
+template <int NREG>
+__device__ __forceinline__ uint32_t radix_cut_regs(const float* z, const float* e, int nr,
+                                                   int lane, float target) {
+  uint32_t kr[NREG];
+  float er[NREG];
+#pragma unroll
+  for (int i = 0; i < NREG; ++i) {
+    const int c = lane + 32 * i;
+    kr[i] = c < nr ? order_key(z[c]) : 0u;   // 0 is below every candidate (>= 1)
+    er[i] = c < nr ? e[c] : 0.f;
+  }
+  uint32_t v = 0;
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t cand = v | (1u << bit);
+    float f = 0.f;
+#pragma unroll
+    for (int i = 0; i < NREG; ++i)
+      if (kr[i] >= cand) f += er[i];
+    f = warp_sum(f);
+    if (f >= target) v = cand;
+  }
+  return v;
+}
+
+__device__ __forceinline__ uint32_t radix_cut_smem(const float* z, const float* e, int nr,
+                                                   int lane, float target) {
+  uint32_t v = 0;
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t cand = v | (1u << bit);
+    float f = 0.f;
+    for (int c = lane; c < nr; c += 32)
+      if (order_key(z[c]) >= cand) f += e[c];
+    f = warp_sum(f);
+    if (f >= target) v = cand;
+  }
+  return v;
+}
+
 // grid: x = ceil(QB / rows), y = heads, z = batch; 256 threads (8 warps).
 // `rows` (1, 2, 4 or 8) query rows per CTA, chosen by the host so that the rows'
 // logits fit in shared memory: 8 for short key ranges, fewer for long ones.  In
-// the logit phase the 8 / rows warps of a row split head_dim and add their
-// partial dot products; in the selection phase warp r owns row r.
-// dynamic smem: qs[rows][D] + ks[kSelTile][D+1] + pz[8][32] + z[rows][nr] + e[rows][nr]
+// the logit phase the 8 warps split head_dim: warp w forms, for every row of the
+// CTA and the 32 key blocks of a tile (one per lane), the partial dot product over
+// its D / 8 columns -- the query values as 16-byte broadcast loads, the key values
+// from a transposed tile -- and the partials are added in warp order.  In the
+// selection phase warp r owns row r.
+// dynamic smem: qs[rows][D] + ks[D][kSelTile + 1] + pz[8][rows][32] + z[rows][nr]
+//               + e[rows][nr]
 template <int D>
 __global__ void __launch_bounds__(256) nabla_select_kernel(
     const float* __restrict__ qbar, const float* __restrict__ kbar, int heads, int qb_count,
@@ -114,11 +160,12 @@ __global__ void __launch_bounds__(256) nabla_select_kernel(
     uint8_t* __restrict__ mask, int* __restrict__ near_count, int rows) {
   extern __shared__ float smem[];
   const int nr = kb_end - kb_begin;
-  const int parts = kSelRows / rows;       // warps per row in the logit phase
+  constexpr int kKs = kSelTile + 1;        // transposed key tile row (conflict-free)
+  constexpr int DW = D / kSelRows;         // head_dim columns per warp
   float* qs = smem;
   float* ks = qs + rows * D;
-  float* pz = ks + kSelTile * (D + 1);
-  float* zs = pz + kSelRows * 32;
+  float* pz = ks + D * kKs;
+  float* zs = pz + kSelRows * rows * 32;
   float* es = zs + rows * nr;
   const int b = blockIdx.z, h = blockIdx.y;
   const int q0 = blockIdx.x * rows;
@@ -130,32 +177,45 @@ __global__ void __launch_bounds__(256) nabla_select_kernel(
     const int r = i / D;
     qs[i] = (q0 + r < qb_count) ? qsrc[static_cast<long long>(q0 + r) * D + (i - r * D)] : 0.f;
   }
-  // logits z[r][c] = qbar[r] . kbar[kb_begin + c] * scale; warp w forms the partial
-  // dot product of row w % rows over head_dim slice w / rows
-  const int lr = warp % rows, part = warp / rows;
-  const int j0 = part * (D / parts), j1 = j0 + D / parts;
+  // logits z[r][c] = qbar[r] . kbar[kb_begin + c] * scale
+  const int j0 = warp * DW;
   for (int t0 = 0; t0 < nr; t0 += kSelTile) {
-    __syncthreads();
+    __syncthreads();   // the previous tile's keys and partials are consumed
     for (int i = tid; i < kSelTile * D; i += blockDim.x) {
       const int c = i / D, j = i - c * D;
-      ks[c * (D + 1) + j] =
+      ks[j * kKs + c] =
           (t0 + c < nr) ? ksrc[static_cast<long long>(kb_begin + t0 + c) * D + j] : 0.f;
     }
     __syncthreads();
-    const float* qrow = qs + lr * D;
-    const float* krow = ks + lane * (D + 1);
-    float acc = 0.f;
-#pragma unroll 8
-    for (int j = j0; j < j1; ++j) acc = fmaf(qrow[j], krow[j], acc);
-    if (parts == 1) {
-      if (t0 + lane < nr) zs[lr * nr + t0 + lane] = acc * scale;
-    } else {
-      pz[warp * 32 + lane] = acc;
-      __syncthreads();
-      if (part == 0 && t0 + lane < nr) {
+    float acc[kSelRows];
+#pragma unroll
+    for (int r = 0; r < kSelRows; ++r) acc[r] = 0.f;
+#pragma unroll
+    for (int j = j0; j < j0 + DW; j += 4) {
+      const float k0 = ks[j * kKs + lane], k1 = ks[(j + 1) * kKs + lane];
+      const float k2 = ks[(j + 2) * kKs + lane], k3 = ks[(j + 3) * kKs + lane];
+#pragma unroll
+      for (int r = 0; r < kSelRows; ++r) {
+        if (r < rows) {
+          const float4 qv = *reinterpret_cast<const float4*>(qs + r * D + j);
+          acc[r] = fmaf(qv.x, k0, acc[r]);
+          acc[r] = fmaf(qv.y, k1, acc[r]);
+          acc[r] = fmaf(qv.z, k2, acc[r]);
+          acc[r] = fmaf(qv.w, k3, acc[r]);
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < kSelRows; ++r)
+      if (r < rows) pz[(warp * rows + r) * 32 + lane] = acc[r];
+    __syncthreads();
+    for (int i = tid; i < rows * 32; i += blockDim.x) {
+      const int r = i >> 5, c = i & 31;
+      if (t0 + c < nr) {
         float sum = 0.f;
-        for (int q = 0; q < parts; ++q) sum += pz[(q * rows + lr) * 32 + lane];
-        zs[lr * nr + t0 + lane] = sum * scale;
+#pragma unroll
+        for (int w = 0; w < kSelRows; ++w) sum += pz[(w * rows + r) * 32 + c];
+        zs[r * nr + t0 + c] = sum * scale;
       }
     }
   }
@@ -205,15 +265,15 @@ __global__ void __launch_bounds__(256) nabla_select_kernel(
   }
   const float target = p * tot;
   // largest v with F(v) = sum_{key_c >= v} e_c >= target
-  uint32_t v = 0;
-  for (int bit = 31; bit >= 0; --bit) {
-    const uint32_t cand = v | (1u << bit);
-    float f = 0.f;
-    for (int c = lane; c < nr; c += 32)
-      if (order_key(z[c]) >= cand) f += e[c];
-    f = warp_sum(f);
-    if (f >= target) v = cand;
-  }
+  uint32_t v;
+  if (nr <= 32 * 4)
+    v = radix_cut_regs<4>(z, e, nr, lane, target);
+  else if (nr <= 32 * 16)
+    v = radix_cut_regs<16>(z, e, nr, lane, target);
+  else if (nr <= 32 * 48)
+    v = radix_cut_regs<48>(z, e, nr, lane, target);
+  else
+    v = radix_cut_smem(z, e, nr, lane, target);
   // mass strictly above the cut, the tied value, and the largest value below it
   float f_gt = 0.f, e_eq = 0.f, e_below = 0.f;
   int n_eq = 0;
@@ -274,8 +334,9 @@ namespace {
 // Shared memory of the selection kernel for `rows` query rows per CTA.
 size_t select_smem(int rows, int head_dim, int nr) {
   return sizeof(float) * (static_cast<size_t>(rows) * head_dim +
-                          static_cast<size_t>(kSelTile) * (head_dim + 1) +
-                          static_cast<size_t>(kSelRows) * 32 + 2 * static_cast<size_t>(rows) * nr);
+                          static_cast<size_t>(head_dim) * (kSelTile + 1) +
+                          static_cast<size_t>(kSelRows) * rows * 32 +
+                          2 * static_cast<size_t>(rows) * nr);
 }
 
 constexpr size_t kSelSmemLimit = 200 * 1024;
