@@ -102,10 +102,35 @@ __device__ __forceinline__ int warp_isum(int v) {
 
 // The cut of one row's top-p selection: the largest order key v whose mass
 // F(v) = sum of e_c over the keys >= v reaches target, found bit by bit from the
-// top.  (Holding the row's keys and values in registers instead was measured: the
-// extra registers cost occupancy and the NABLA step's selection got slower.)
-__device__ __forceinline__ uint32_t radix_cut(const float* z, const float* e, int nr,
+// top.  Each lane sums its entries c = lane, lane + 32, ... in that order, so the
+// register form (rows of up to 512 candidates, the keys and values held by the
+// lanes) and the shared-memory form give the same sums.
+template <int NREG>
+__device__ __forceinline__ uint32_t radix_cut_regs(const float* z, const float* e, int nr,
                                                    int lane, float target) {
+  uint32_t kr[NREG];
+  float er[NREG];
+#pragma unroll
+  for (int i = 0; i < NREG; ++i) {
+    const int c = lane + 32 * i;
+    kr[i] = c < nr ? order_key(z[c]) : 0u;   // 0 is below every candidate (>= 1)
+    er[i] = c < nr ? e[c] : 0.f;
+  }
+  uint32_t v = 0;
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t cand = v | (1u << bit);
+    float f = 0.f;
+#pragma unroll
+    for (int i = 0; i < NREG; ++i)
+      if (kr[i] >= cand) f += er[i];
+    f = warp_sum(f);
+    if (f >= target) v = cand;
+  }
+  return v;
+}
+
+__device__ __forceinline__ uint32_t radix_cut(const float* z, const float* e, int nr,
+                                              int lane, float target) {
   uint32_t v = 0;
   for (int bit = 31; bit >= 0; --bit) {
     const uint32_t cand = v | (1u << bit);
@@ -241,7 +266,8 @@ __global__ void __launch_bounds__(256) nabla_select_kernel(
   }
   const float target = p * tot;
   // largest v with F(v) = sum_{key_c >= v} e_c >= target
-  const uint32_t v = radix_cut(z, e, nr, lane, target);
+  const uint32_t v = nr <= 32 * 16 ? radix_cut_regs<16>(z, e, nr, lane, target)
+                                   : radix_cut(z, e, nr, lane, target);
   // mass strictly above the cut, the tied value, and the largest value below it
   float f_gt = 0.f, e_eq = 0.f, e_below = 0.f;
   int n_eq = 0;
