@@ -37,6 +37,9 @@ SMALL = [
       mask="nabla_sta", tile=(4, 4, 4), window=(3, 3, 3), p=0.9, strength_range=(0.5, 3.0)),
     W(name="spade_small", index=16, batch=1, heads=4, head_dim=128, grid=(6, 10, 12), block=64,
       mask="spade", p=0.9, strength_range=(1.0, 3.0), extra={"axis_stretch": 6.0}),
+    # 128-token slices (2x8x8, 1x8x16, 4x4x8, 32x2x2) on a ragged grid, head_dim 64
+    W(name="spade128_small", index=17, batch=1, heads=3, head_dim=64, grid=(9, 12, 20), block=128,
+      mask="spade", p=0.85, strength_range=(1.0, 3.0), extra={"axis_stretch": 6.0}),
 ]
 
 
