@@ -86,6 +86,25 @@ def test_large_logits_exercise_rescaling():
     run_case(1, 1, nq, nk, D, 128, 128, mask, 1, seed=0, qkv=(q, k, v))
 
 
+@pytest.mark.parametrize("D", [64, 128])
+def test_second_half_of_a_tile_jumps_above_the_running_max(D):
+    # In every key tile after the first the keys of its second half (64..127) score
+    # far above everything before them while its first half stays low: a tile's first
+    # half passes the fast path's bound against the running max and its second half
+    # does not, so the max moves in the middle of a tile.
+    nq, nk = 256, 4 * 128
+    g = torch.Generator().manual_seed(21)
+    q = (torch.randn(1, nq, 1, D, generator=g) * 0.1 + 1.0).to(torch.bfloat16)
+    k = torch.randn(1, nk, 1, D, generator=g) * 0.1
+    level = torch.zeros(nk)
+    for t in range(1, 4):
+        level[128 * t + 64:128 * (t + 1)] = 1.2 * t     # scores jump by ~1.2 t * sqrt(D)
+    k = (k + level.view(1, nk, 1, 1)).to(torch.bfloat16)
+    v = torch.randn(1, nk, 1, D, generator=g).to(torch.bfloat16)
+    mask = np.ones((1, 2, 4), np.uint8)
+    run_case(1, 1, nq, nk, D, 128, 128, mask, 1, seed=0, qkv=(q, k, v))
+
+
 def test_all_masked_everywhere():
     mask = np.zeros((1, 3, 3), np.uint8)
     run_case(1, 2, 300, 300, 128, 128, 128, mask, 1, seed=2)
