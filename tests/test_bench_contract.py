@@ -116,3 +116,15 @@ def test_permute_bandwidth_counts_the_algorithmic_bytes():
     assert abs(got["permute"]["gb_s"] - 3 * 2 * 115200 * row / 0.714e-3 / 1e9) < 1e-6
     assert 0.9 < got["permute"]["frac_of_hbm"] < 0.92
     assert bench.permute_bandwidth(w, SimpleNamespace(permuted=False), {}, 6543.4) is None
+
+
+def test_committed_profiles_describe_the_current_kernel_sources():
+    # every ncu summary bench.py reads its DRAM traffic from was captured on the
+    # kernel sources as they are now (the summary's source hash matches), so the
+    # bench line's roofline carries that traffic instead of null
+    sys.path.insert(0, ROOT)
+    import bench
+    for workload, kind in (("radial_long", "attn_fwd"), ("sta_720p", "attn_fwd"),
+                           ("nabla_480p", "attn_fwd"), ("sta_720p", "attn_bwd"),
+                           ("nabla_480p", "sics")):
+        assert bench.profiled_traffic(workload, kind) is not None, (workload, kind)
