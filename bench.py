@@ -670,9 +670,10 @@ def run_backward(args, w):
                                                    w.block, plan.list_heads),
                      dtype=torch.uint8, device=dev)
 
-    def bwd(q_, k_, v_, o_, do_, lse_, rp_, ci_):
+    def bwd(q_, k_, v_, o_, do_, lse_, rp_, ci_, outs=None):
+        dq_, dk_, dv_ = (dq, dk, dv) if outs is None else outs
         B.bsa_attn_bwd(q_, k_, v_, o_, do_, lse_, rp_, ci_, w.block, w.block, plan.list_heads,
-                       nq=plan.nq, nk=plan.nk, dq=dq, dk=dk, dv=dv, ws=ws)
+                       nq=plan.nq, nk=plan.nk, dq=dq_, dk=dk_, dv=dv_, ws=ws)
 
     def barrier():
         if world > 1:
@@ -708,31 +709,60 @@ def run_backward(args, w):
 
     # end to end through the public API: every step copies its inputs from pinned
     # host memory (Q, K, V, O, dO in the path's token order, LSE, the kept lists),
-    # runs the backward and copies dQ, dK, dV back, all on one stream
+    # runs the backward and copies dQ, dK, dV back.  Steps are pipelined as a
+    # training loop would run them: the input copy of step i+1 (copy stream) and the
+    # output copy of step i-1 (out stream) overlap the backward of step i; inputs
+    # and outputs are double-buffered.
     e2e = None
     if not args.no_e2e:
         host_in = [t_.detach().to("cpu").pin_memory() for t_ in args_dev]
-        dev_in = [torch.empty_like(t_) for t_ in args_dev]
+        dev_in = [[torch.empty_like(t_) for t_ in args_dev] for _ in range(2)]
+        dev_out = [tuple(torch.empty_like(t_) for t_ in (dq, dk, dv)) for _ in range(2)]
         host_out = [torch.empty(t_.shape, dtype=t_.dtype).pin_memory() for t_ in (dq, dk, dv)]
         e_steps = max(3, args.steps // 2)
+        total = 2 + e_steps
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_in = [torch.cuda.Event() for _ in range(total)]
+        ev_done = [torch.cuda.Event() for _ in range(total)]
+        ev_out = [torch.cuda.Event() for _ in range(total)]
+
+        def h2d(i):
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(ev_done[i - 2])      # inputs of step i-2 consumed
+                for dst, src in zip(dev_in[i % 2], host_in):
+                    dst.copy_(src, non_blocking=True)
+                ev_in[i].record(s_in)
+
         barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(e_steps):
-            for dst, src in zip(dev_in, host_in):
-                dst.copy_(src, non_blocking=True)
-            bwd(*dev_in)
-            for dst, src in zip(host_out, (dq, dk, dv)):
-                dst.copy_(src, non_blocking=True)
+        h2d(0)
+        for i in range(total):
+            if i == 2:
+                e0.record(stream)
+            if i + 1 < total:
+                h2d(i + 1)
+            stream.wait_event(ev_in[i])
+            if i >= 2:
+                stream.wait_event(ev_out[i - 2])         # these outputs copied out (step i-2)
+            bwd(*dev_in[i % 2], outs=dev_out[i % 2])
+            ev_done[i].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_done[i])
+                for dst, src in zip(host_out, dev_out[i % 2]):
+                    dst.copy_(src, non_blocking=True)
+                ev_out[i].record(s_out)
+        stream.wait_event(ev_out[total - 1])
         e1.record(stream)
         barrier()
+        # time from the start of step 2 to the end of the last output copy, per step
         e_ms = max_over_ranks([e0.elapsed_time(e1) / e_steps], dev)[0]
         h2d, d2h = sum_over_ranks(
             [sum(t_.numel() * t_.element_size() for t_ in host_in),
              sum(t_.numel() * t_.element_size() for t_ in host_out)], dev)
         e2e = {"value": job_value(flops_all, e_ms), "unit": "TFLOP/s",
                "ms_per_step": e_ms, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "note": "pinned host buffers; copies and the backward serialised on one stream"}
+               "note": "pinned host buffers; copies of neighbouring steps overlap the backward"}
 
     peaks, peak_kind = load_peaks()
     achieved = flops_all / world / (ms * 1e-3) / 1e12
@@ -1124,13 +1154,14 @@ def main():
     # ---- end to end through the public API: pinned host inputs in, O back to host.
     # Steps are pipelined the way a serving loop would run them: the host->device
     # copy of step i+1 (copy stream) and the device->host copy of O of step i-1
-    # (out stream) overlap the path of step i (compute stream); device inputs are
-    # double-buffered.  Every step still moves all of its inputs and its output.
+    # (out stream) overlap the path of step i (compute stream); device inputs and O
+    # are double-buffered.  Every step still moves all of its inputs and its output.
     e2e = None
     if not args.no_e2e:
         qp, kp, vp = (t_.pin_memory() for t_ in (q_h, k_h, v_h))
         o_host = torch.empty(plan.o.shape, dtype=plan.o.dtype).pin_memory()
         bufs = [tuple(torch.empty_like(t_) for t_ in (q, k, v)) for _ in range(2)]
+        o_bufs = [plan.o, torch.empty_like(plan.o)]
         s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
         e2e_steps = max(3, args.steps // 2)
         total = 2 + e2e_steps
@@ -1158,23 +1189,25 @@ def main():
             stream.wait_event(ev_in[i])
             qd, kd, vd = bufs[i % 2]
             plan._q, plan._k, plan._v = qd, kd, vd
+            plan.set_output(o_bufs[i % 2])
             if plan.permuted:
                 plan.permute_inputs(qd, kd, vd)
             plan.build_mask()
             plan.compact()
-            if i >= 1 and not plan.permuted:
-                stream.wait_event(ev_out[i - 1])         # O of step i-1 copied out
+            if i >= 2 and not plan.permuted:
+                stream.wait_event(ev_out[i - 2])         # this O buffer copied out (step i-2)
             plan.attention()
             if plan.permuted:
-                if i >= 1:
-                    stream.wait_event(ev_out[i - 1])     # O of step i-1 copied out
+                if i >= 2:
+                    stream.wait_event(ev_out[i - 2])     # this O buffer copied out (step i-2)
                 plan.untile()
             ev_done[i].record(stream)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev_done[i])
-                o_host.copy_(plan.o, non_blocking=True)
+                o_host.copy_(o_bufs[i % 2], non_blocking=True)
                 ev_out[i].record(s_out)
         stream.wait_event(ev_out[total - 1])
+        plan.set_output(None)
         e1.record(stream)
         barrier()
         # time from the start of step 2 to the end of the last output copy, per step
