@@ -1080,19 +1080,35 @@ def main():
     import torch.distributed as dist
     from block_sparse_attention_tokens_b200 import binding as B
     from block_sparse_attention_tokens_b200 import synth
-    from block_sparse_attention_tokens_b200.pipeline import Plan, effective_flops, head_range
+    from block_sparse_attention_tokens_b200.pipeline import (Plan, effective_flops, head_range,
+                                                             qblock_range)
 
     world, rank, dev = setup_ranks()
 
     # inputs: the workload's seeded Q, K, V; with N ranks each rank takes its range
     # of heads (masks are per head and every head is independent, so nothing is
-    # exchanged) and holds only those heads, as after a head-parallel projection
+    # exchanged) and holds only those heads, as after a head-parallel projection.
+    # A raster-order workload whose heads do not split evenly (12 radial heads over
+    # 8 GPUs) splits its query blocks instead: each rank takes every head of its
+    # query rows, against all keys -- again with no exchange.
     q_all, k_all, v_all, _ = synth.workload_inputs(w)
-    h0, h1 = head_range(rank, world, w.heads)
-    q_h, k_h, v_h = (t_[:, :, h0:h1].contiguous() for t_ in (q_all, k_all, v_all))
+    split_q = (world > 1 and w.heads % world != 0 and w.tile is None
+               and w.mask in ("sta", "radial", "ar"))
+    if split_q:
+        qb0, qb1 = qblock_range(rank, world, math.ceil(w.nq / w.block),
+                                granule=max(1, 128 // w.block))
+        q_h = q_all[:, qb0 * w.block:min(w.nq, qb1 * w.block)].contiguous()
+        k_h, v_h = k_all, v_all
+        plan_kw = {"qblocks": (qb0, qb1)}
+        split_text = f"query blocks split over {world} GPU(s), no data-path collective"
+    else:
+        h0, h1 = head_range(rank, world, w.heads)
+        q_h, k_h, v_h = (t_[:, :, h0:h1].contiguous() for t_ in (q_all, k_all, v_all))
+        plan_kw = {"heads": (h0, h1)}
+        split_text = f"heads split over {world} GPU(s), no data-path collective"
     del q_all, k_all, v_all
     q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
-    plan = Plan(w, dev, heads=(h0, h1))
+    plan = Plan(w, dev, **plan_kw)
 
     def barrier():
         if world > 1:
@@ -1241,7 +1257,7 @@ def main():
 
     if rank == 0:
         cfg = workload_config(w)
-        cfg["parallelism"] = f"heads split over {world} GPU(s), no data-path collective"
+        cfg["parallelism"] = split_text
         line = {"metric": FWD_METRIC,
                 "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
                 "warmup": max(3, args.warmup), "ms_per_step": ms_per_step,

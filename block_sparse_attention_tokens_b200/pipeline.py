@@ -34,6 +34,21 @@ def ar_block_ranges(n_tokens_k: int, tokens_per_frame: int, block: int, anchor_f
     return a_end, max(r_begin, a_end)
 
 
+def qblock_range(rank: int, world: int, qblocks: int, granule: int = 1) -> Tuple[int, int]:
+    """Query blocks [b0, b1) of rank `rank` when `world` ranks share `qblocks` query
+    blocks of every head: the rows of the attention are independent given K and V,
+    so a workload with too few heads to split evenly splits its query blocks
+    instead, with no exchange.  The blocks go out in units of `granule` (the blocks
+    of one 128-row attention q-tile, 128 // block for blocks under 128 tokens), so
+    the ranks' q-tiles are the whole call's and the results bit-identical to it.
+    Contiguous, every block once, unit counts within one."""
+    if world < 1 or not 0 <= rank < world or granule < 1:
+        raise ValueError(f"rank {rank} of {world}, granule {granule}")
+    units = -(-qblocks // granule)
+    u0, u1 = rank * units // world, (rank + 1) * units // world
+    return min(qblocks, u0 * granule), min(qblocks, u1 * granule)
+
+
 def head_range(rank: int, world: int, heads: int) -> Tuple[int, int]:
     """Heads [h0, h1) of rank `rank` when `world` ranks share `heads` heads: every
     (batch, head) row of the attention is independent given Q, K, V and the masks
@@ -50,10 +65,17 @@ class Plan:
     ``heads=(h0, h1)`` restricts the plan to that range of the workload's heads (a
     rank's share when the heads are split over GPUs).  ``step`` then takes either
     the whole-head tensors [B, N, H, D] -- the range is read in place through the
-    library's token-row stride -- or tensors holding only the range's heads."""
+    library's token-row stride -- or tensors holding only the range's heads.
+
+    ``qblocks=(b0, b1)`` (raster-order workloads only) restricts it to those query
+    blocks: the plan's queries are rows [b0 * block, min(nq, b1 * block)) of every
+    head, against all keys.  ``step`` takes Q with either all of the workload's
+    query rows (the range is read in place) or only the range's, and writes O and
+    LSE for the range (into the range's rows of a whole-O ``out``)."""
 
     def __init__(self, w: Workload, device: torch.device = torch.device("cuda"),
-                 heads: Optional[Tuple[int, int]] = None):
+                 heads: Optional[Tuple[int, int]] = None,
+                 qblocks: Optional[Tuple[int, int]] = None):
         self.w = w
         self.dev = device
         self.h0, self.h1 = (0, w.heads) if heads is None else heads
@@ -63,6 +85,17 @@ class Plan:
         self.heads = Hh
         self.nq, self.nk = w.nq, w.nk
         self.permuted = w.tile is not None or w.mask == "spade"
+        qb_all = ceil_div(w.nq, w.block)
+        self.qb0, self.qb1 = (0, qb_all) if qblocks is None else qblocks
+        if not 0 <= self.qb0 < self.qb1 <= qb_all:
+            raise ValueError(f"query-block range {qblocks} of {qb_all} blocks")
+        if (self.qb0, self.qb1) != (0, qb_all):
+            if self.permuted:
+                raise ValueError("a query-block range needs a raster-order workload")
+            if w.mask not in ("sta", "radial", "ar"):
+                raise ValueError(f"no query-block range for the {w.mask} mask")
+        self.q0 = self.qb0 * w.block                      # first query row of the plan
+        self.nq = min(w.nq, self.qb1 * w.block) - self.q0
         if self.permuted:
             self.n_pad = ceil_div(w.n_tokens, w.block) * w.block
             self.qp = torch.empty((Bt, self.n_pad, Hh, D), dtype=torch.bfloat16, device=device)
@@ -72,7 +105,9 @@ class Plan:
         self.QB, self.KB = ceil_div(self.nq, w.block), ceil_div(self.nk, w.block)
         if w.mask in ("sta", "radial"):
             self.list_heads = 1
-            self.mask = torch.empty((self.QB, self.KB), dtype=torch.uint8, device=device)
+            # static masks are built whole; the plan's query blocks are a row range
+            self.mask_all = torch.empty((qb_all, self.KB), dtype=torch.uint8, device=device)
+            self.mask = self.mask_all[self.qb0:self.qb1]
         else:
             self.list_heads = Bt * Hh
             self.mask = torch.empty((Bt, Hh, self.QB, self.KB), dtype=torch.uint8, device=device)
@@ -122,6 +157,17 @@ class Plan:
         raise ValueError(f"tensor with {t.shape[2]} heads for a plan of heads "
                          f"[{self.h0}, {self.h1}) of {self.w.heads}")
 
+    def _rows(self, t: torch.Tensor) -> torch.Tensor:
+        """This plan's query rows of a query-side tensor [B, rows, H, D]: a row view
+        of one holding all of the workload's query rows, or the tensor itself when
+        it holds only the plan's."""
+        if t.shape[1] == self.nq:
+            return t
+        if t.shape[1] == self.w.nq:
+            return t[:, self.q0:self.q0 + self.nq]
+        raise ValueError(f"tensor with {t.shape[1]} query rows for a plan of rows "
+                         f"[{self.q0}, {self.q0 + self.nq}) of {self.w.nq}")
+
     def permute_inputs(self, q, k, v):
         w = self.w
         q, k, v = self._mine(q), self._mine(k), self._mine(v)
@@ -147,9 +193,9 @@ class Plan:
     def build_mask(self):
         w = self.w
         if w.mask == "sta":
-            B.bsa_sta_mask(self.tile_grid, w.window, 0, mask=self.mask)
+            B.bsa_sta_mask(self.tile_grid, w.window, 0, mask=self.mask_all)
         elif w.mask == "radial":
-            B.bsa_radial_mask(self.nk, w.tokens_per_frame, w.block, mask=self.mask)
+            B.bsa_radial_mask(self.nk, w.tokens_per_frame, w.block, mask=self.mask_all)
         elif w.mask in ("nabla", "spade"):
             B.bsa_nabla_select(self.qbar, self.kbar, w.p, mask=self.mask, near_count=self.near)
         elif w.mask == "nabla_sta":
@@ -158,7 +204,8 @@ class Plan:
                                mask=self.mask, near_count=self.near)
         elif w.mask == "ar":
             a_end, r_begin = self.kb_range
-            B.bsa_nabla_mask(self._mine(self._q), self._mine(self._k), w.block, w.p, 0.0, a_end,
+            B.bsa_nabla_mask(self._rows(self._mine(self._q)), self._mine(self._k), w.block, w.p,
+                             0.0, a_end,
                              r_begin, 1, nq=self.nq, nk=self.nk, mask=self.mask,
                              near_count=self.near, ws=self.nabla_ws)
         else:
@@ -172,8 +219,8 @@ class Plan:
         if self.permuted:
             q, k, v, out = self.qp, self.kp, self.vp, self.op
         else:
-            q, k, v = self._mine(self._q), self._mine(self._k), self._mine(self._v)
-            out = self._mine(self.out)
+            q, k, v = self._rows(self._mine(self._q)), self._mine(self._k), self._mine(self._v)
+            out = self._rows(self._mine(self.out))
         B.bsa_attn_fwd(q, k, v, self.row_ptr, self.col_idx, w.block, w.block, self.list_heads,
                        nq=self.nq, nk=self.nk, o=out, lse=self.lse, ws=self.attn_ws)
 
@@ -201,10 +248,11 @@ class Plan:
         return self.out, self.lse
 
     def set_output(self, out: Optional[torch.Tensor] = None):
-        """Where the next steps write O: a whole-head tensor (this plan's heads of
-        it), or the plan's own buffer (None)."""
+        """Where the next steps write O: a whole-head (and, with a query-block range,
+        whole-row) tensor -- this plan's heads and rows of it -- or the plan's own
+        buffer (None)."""
         self.out = self.o if out is None else out
-        self._mine(self.out)
+        self._rows(self._mine(self.out))
 
     def kernel_launches_per_step(self) -> int:
         """libbsa kernels one step launches (for the benchmark's launch count)."""

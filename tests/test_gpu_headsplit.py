@@ -146,3 +146,38 @@ def test_strided_nabla_mask_and_permutes_equal_dense_copies():
     back = torch.zeros(1, w.n_tokens, 6, 128, dtype=torch.bfloat16, device="cuda")
     B.bsa_tile_untile(y_s, w.grid, w.tile, x=back[:, :, 2:5])
     assert torch.equal(back[:, :, 2:5], qs) and torch.all(back[:, :, :2] == 0)
+
+
+@pytest.mark.parametrize("name", ["radial_small", "ar_small"])
+def test_query_block_halves_equal_the_whole(name):
+    # the split for raster-order workloads whose heads do not divide over the ranks:
+    # each of two plans takes half of the query blocks of every head (all keys),
+    # reading its rows of Q and writing its rows of O in place
+    from block_sparse_attention_tokens_b200.pipeline import qblock_range
+    w = next(x for x in SMALL if x.name == name)
+    q, k, v, _ = synth.workload_inputs(w)
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    whole = Plan(w)
+    o_ref, lse_ref = whole.step(qc, kc, vc)
+    o_ref, lse_ref = o_ref.clone(), lse_ref.clone()
+    QB = math.ceil(w.nq / w.block)
+    out = torch.full_like(o_ref, float("nan"))
+    lses = []
+    for r in range(2):
+        b0, b1 = qblock_range(r, 2, QB, granule=max(1, 128 // w.block))
+        part = Plan(w, qblocks=(b0, b1))
+        part.step(qc, kc, vc, out=out)
+        torch.cuda.synchronize()
+        assert B.bsa_read_status(part.attn_ws) == 0
+        assert part.nq == min(w.nq, b1 * w.block) - b0 * w.block
+        if whole.list_heads > 1:
+            assert torch.equal(part.mask, whole.mask[:, :, b0:b1]), "per-head masks differ"
+        lses.append(part.lse.clone())
+    assert torch.equal(out, o_ref), "query-block halves differ from the whole call"
+    assert torch.equal(torch.cat(lses, dim=2), lse_ref)
+
+
+def test_query_block_range_needs_a_raster_workload():
+    w = next(x for x in SMALL if x.name == "sta_small")
+    with pytest.raises(ValueError):
+        Plan(w, qblocks=(0, 1))

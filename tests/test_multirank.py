@@ -97,3 +97,66 @@ def test_two_gloo_ranks_split_heads_and_reassemble_exactly():
     assert out[0][2] == (0, 2) and out[1][2] == (2, 5)
     for rank in range(world):
         assert out[rank][0] and out[rank][1]
+
+
+def test_query_block_ranges_cover_every_block_once_and_balance():
+    from block_sparse_attention_tokens_b200.pipeline import qblock_range
+    for granule in (1, 2):
+        for qblocks in (1, 3, 37, 3544):
+            units = -(-qblocks // granule)
+            for world in range(1, min(units, 8) + 1):
+                ranges = [qblock_range(r, world, qblocks, granule) for r in range(world)]
+                assert ranges[0][0] == 0 and ranges[-1][1] == qblocks
+                assert all(a[1] == b[0] for a, b in zip(ranges, ranges[1:]))
+                assert all(b0 % granule == 0 for b0, _ in ranges)     # q-tile aligned
+                sizes = [-(-(b1 - b0) // granule) for b0, b1 in ranges]
+                assert min(sizes) >= 1 and max(sizes) - min(sizes) <= 1
+
+
+def test_query_block_split_is_chosen_when_heads_do_not_divide():
+    # the radial workload (12 heads) over 8 ranks: query blocks; 24 STA heads over 8
+    # ranks (tile-ordered anyway): heads
+    from block_sparse_attention_tokens_b200 import configs
+    w = configs.get("radial_long")
+    assert w.heads % 8 != 0 and w.tile is None and w.mask == "radial"
+    assert configs.get("sta_720p").heads % 8 == 0
+
+
+def _qblock_split_main(rank, world, port, out):
+    """Each rank evaluates the oracle's attention on its own query blocks of every
+    head (all keys); the host gathers the rows (test-side reassembly)."""
+    import datetime
+    import numpy as np
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    import oracle as O
+    from block_sparse_attention_tokens_b200.pipeline import qblock_range
+    rng = np.random.default_rng(6)                    # the same inputs on every rank
+    Bn, H, n, D, blk = 1, 3, 300, 16, 64
+    q, k, v = (rng.standard_normal((Bn, n, H, D)) for _ in range(3))
+    QB = -(-n // blk)
+    mask = (rng.random((1, QB, QB)) < 0.6).astype(np.uint8)
+    b0, b1 = qblock_range(rank, world, QB)
+    r0, r1 = b0 * blk, min(n, b1 * blk)
+    o, lse = O.block_sparse_attention(q[:, r0:r1], k, v, mask[:, b0:b1], blk, blk)
+    pieces = [None] * world
+    dist.all_gather_object(pieces, (r0, o, lse))
+    pieces = sorted(pieces, key=lambda p: p[0])
+    o_all = np.concatenate([p[1] for p in pieces], axis=1)
+    lse_all = np.concatenate([p[2] for p in pieces], axis=2)
+    ref_o, ref_lse = O.block_sparse_attention(q, k, v, mask, blk, blk)
+    out[rank] = (bool(np.array_equal(o_all, ref_o)), bool(np.array_equal(lse_all, ref_lse)))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_split_query_blocks_and_reassemble_exactly():
+    world = 2
+    manager = mp.Manager()
+    out = manager.dict()
+    mp.spawn(_qblock_split_main, args=(world, _free_port(), out), nprocs=world, join=True)
+    for rank in range(world):
+        assert out[rank] == (True, True)
