@@ -1235,7 +1235,7 @@ def main():
         e2e = {"value": job_value(flops_all, e_ms.item()), "unit": "TFLOP/s",
                "ms_per_step": e_ms.item(), "h2d_bytes_per_step": h2d_bytes,
                "d2h_bytes_per_step": d2h_bytes,
-               "note": "pinned host buffers (each rank its heads); copies of neighbouring steps "
+               "note": "pinned host buffers (each rank its share of Q, K, V); copies of neighbouring steps "
                        "overlap compute"}
 
     peaks, peak_kind = load_peaks()
