@@ -352,18 +352,26 @@ int launch_select(const float* qbar, const float* kbar, int batch, int heads, in
     if (e != cudaSuccess) return record_cuda_error(e);
   }
   dim3 sgrid(ceil_div(qb, rows), heads, batch);
-  cudaError_t e;
-  if (head_dim == 128) {
-    e = cudaFuncSetAttribute(nabla_select_kernel<128>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  // the shared-memory cap is raised to the selection's limit once per device (not
+  // per launch, so that a launch can be captured into a CUDA graph)
+  static bool attr_done[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || !attr_done[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(nabla_select_kernel<128>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kSelSmemLimit));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(nabla_select_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(kSelSmemLimit));
     if (e != cudaSuccess) return record_cuda_error(e);
+    if (dev >= 0 && dev < 64) attr_done[dev] = true;
+  }
+  if (head_dim == 128) {
     nabla_select_kernel<128><<<sgrid, 256, smem, st>>>(qbar, kbar, heads, qb, kb, kb_begin, kb_end,
                                                        p, scale, force_outside, base_mask, key_allowed, mask,
                                                        near_count, rows);
   } else {
-    e = cudaFuncSetAttribute(nabla_select_kernel<64>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return record_cuda_error(e);
     nabla_select_kernel<64><<<sgrid, 256, smem, st>>>(qbar, kbar, heads, qb, kb, kb_begin, kb_end,
                                                       p, scale, force_outside, base_mask, key_allowed, mask,
                                                       near_count, rows);

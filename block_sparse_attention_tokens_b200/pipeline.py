@@ -247,6 +247,21 @@ class Plan:
             self.untile()
         return self.out, self.lse
 
+    def capture(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                out: Optional[torch.Tensor] = None) -> "torch.cuda.CUDAGraph":
+        """Records one ``step`` on these tensors into a CUDA graph and returns it.
+        ``graph.replay()`` then re-runs the whole path -- every launch of the step,
+        with no host work between them -- on whatever the same tensors hold; new
+        inputs are copied into q, k, v in place.  One eager step runs first, outside
+        the capture, so that every one-time setup of the library (kernel attributes,
+        symbol addresses) is done before it."""
+        self.step(q, k, v, out=out)
+        torch.cuda.synchronize(self.dev)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            self.step(q, k, v, out=out)
+        return graph
+
     def set_output(self, out: Optional[torch.Tensor] = None):
         """Where the next steps write O: a whole-head (and, with a query-block range,
         whole-row) tensor -- this plan's heads and rows of it -- or the plan's own
