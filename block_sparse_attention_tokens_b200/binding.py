@@ -350,6 +350,12 @@ def bsa_tile_permute_pool(x: torch.Tensor, grid: Tuple[int, int, int],
     return y, pooled
 
 
+def _status(device_status: Optional[torch.Tensor]):
+    """The optional one-word error status a kernel writes on the device."""
+    if device_status is not None:
+        _buffer(device_status, "device_status", torch.int32, 1)
+
+
 def _choice(choice: torch.Tensor, batch: int, heads: int):
     _cuda(choice, "choice")
     if choice.dtype != torch.int32 or choice.numel() != batch * heads or not choice.is_contiguous():
@@ -366,6 +372,7 @@ def bsa_scheme_permute(x: torch.Tensor, grid: Tuple[int, int, int], shapes, choi
     tail); with ``pool`` (or a ``pooled`` buffer) also the per-block means
     [B, H, n_pad / block, D] fp32.  x and y may be head slices of wider tensors.
     Returns (y, pooled or None)."""
+    _status(device_status)
     B, _, H, D = x.shape
     xs = _strided_tokens(x, "x", B, grid[0] * grid[1] * grid[2], H, D)
     _choice(choice, B, H)
@@ -390,6 +397,7 @@ def bsa_scheme_untile(y: torch.Tensor, grid: Tuple[int, int, int], shapes, choic
                       device_status: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Inverse of bsa_scheme_permute: y [B, n_pad, H, D] -> x [B, N, H, D] raster (either
     may be a head slice of a wider tensor)."""
+    _status(device_status)
     B, n_pad, H, D = y.shape
     N = grid[0] * grid[1] * grid[2]
     ys = _strided_tokens(y, "y", B, n_pad, H, D)
@@ -584,8 +592,7 @@ def bsa_attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         lse = torch.empty((B, H, nq), dtype=torch.float32, device=q.device)
     _tokens(o, "o", B, nq, H, D)
     _buffer(lse, "lse", torch.float32, B * H * nq)
-    if device_status is not None:
-        _buffer(device_status, "device_status", torch.int32, 1)
+    _status(device_status)
     _check(load_library().bsa_attn_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), B, H, nq, nk, D,
                                                block_q, block_k, _ptr(row_ptr), _ptr(col_idx),
                                                list_heads, float(scale), _ptr(o), _ptr(lse),
@@ -703,8 +710,7 @@ def bsa_kv_write(src: torch.Tensor, first_token: int, page_table: torch.Tensor,
     _tokens(src, "src", B, n_new, H, D)
     _table(page_table, "page_table", B)
     _pool(pool, "pool", H, D)
-    if device_status is not None:
-        _buffer(device_status, "device_status", torch.int32, 1)
+    _status(device_status)
     _check(load_library().bsa_kv_write(_ptr(src), B, n_new, H, D, int(first_token),
                                        _ptr(page_table), page_table.shape[1], _ptr(pool),
                                        pool.shape[0], _ptr(device_status), _stream()),

@@ -55,3 +55,19 @@ def test_row_stride_rule_of_strided_token_tensors():
     odd = torch.empty(1, 100, 260, dtype=BF)[:, :, :256].reshape(1, 100, 4, 64)
     assert "multiple of 8" in B._stride_problem(tuple(odd.shape), tuple(odd.stride()), 100,
                                                 256, 8)
+
+
+def test_device_status_must_be_one_int32_word_on_the_gpu():
+    # refused before any argument reaches the library: a host tensor would be a
+    # host pointer written by a kernel
+    import pytest
+    x = torch.zeros(1, 8, 1, 8, dtype=BF)
+    choice = torch.zeros(1, 1, dtype=torch.int32)
+    host_status = torch.zeros(1, dtype=torch.int32)
+    with pytest.raises(ValueError, match="device_status"):
+        B.bsa_scheme_permute(x, (2, 2, 2), [(1, 1, 1)], choice, 8, device_status=host_status)
+    with pytest.raises(ValueError, match="device_status"):
+        B.bsa_scheme_untile(x, (2, 2, 2), [(1, 1, 1)], choice, device_status=host_status)
+    with pytest.raises(ValueError, match="device_status"):
+        B._status(torch.zeros(1, dtype=torch.int64))
+    B._status(None)
